@@ -1,0 +1,254 @@
+"""CPU oracle for tile-routed mixed-precision causal attention.
+
+TEST INFRASTRUCTURE ONLY: the test-suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The product path (the CUDA
+library and its Python binding) never imports this package, and this package
+never imports the product.  All arithmetic lives in ``tra_oracle.c`` (plain C,
+fp64, IEEE fp32 for the quantiser); this module only compiles it with gcc and
+marshals numpy arrays.
+
+Sources (page titles): "TriAttention: Unified Sparse Mixed-Precision Attention
+for Long-Context LLM Inference" (abstract), "TileMix: Tile-Centric
+Mixed-Precision Attention for LLM Inference Acceleration" (abstract),
+"HyQuant Uses Hybrid Precision to Compress LLM Attention" ("How HyQuant works").
+Each C function cites the sentence it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tra_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+TILE = 64
+INT4, INT8, BF16 = 1, 2, 3
+
+
+def build(force: bool = False) -> str:
+    """Compile tra_oracle.c into liboracle.so next to it (gcc, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([
+            "gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+            "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            L = ctypes.c_int64
+            D = ctypes.c_double
+            lib.orc_num_tiles.argtypes = [P, I]
+            lib.orc_num_tiles.restype = L
+            lib.orc_quantize.argtypes = [P, P, I, I, I, P, P, P, P]
+            lib.orc_quantize.restype = I
+            lib.orc_lists_boundary.argtypes = [P, I, I, P, P, P, P]
+            lib.orc_lists_boundary.restype = L
+            lib.orc_lists_bitmask.argtypes = [P, I, I, P, I, I, P, P]
+            lib.orc_lists_bitmask.restype = L
+            lib.orc_lists_decode.argtypes = [P, I, I, I, I, P, P, P, P]
+            lib.orc_lists_decode.restype = L
+            lib.orc_int_tile.argtypes = [I, I, P, P, P, P, P]
+            lib.orc_int_tile.restype = I
+            lib.orc_prefill_rows.argtypes = [P, P, P, P, I, I, I, I,
+                                             P, P, P, P, P, P, P, P,
+                                             P, P, D, I, P, P, P]
+            lib.orc_prefill_rows.restype = I
+            lib.orc_decode_step.argtypes = [P, P, I, I, I, I,
+                                            P, P, P, P, P, P, P, P,
+                                            P, P, P, P, P, I, D, P]
+            lib.orc_decode_step.restype = I
+            _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def num_tiles(cu_seqlens) -> int:
+    cu = _c(cu_seqlens, np.int32)
+    return int(_load().orc_num_tiles(_p(cu), len(cu) - 1))
+
+
+def quantize(x_bits, cu_seqlens, want8=True, want4=True):
+    """Per-(head, 64-token tile) symmetric quantisation of one tensor.
+
+    x_bits: uint16 bf16 bit patterns [ntok, H, d].  Returns (x8, x4, s8, s4)
+    with x8 int8 [H, ntiles, 64, d], x4 uint8 [H, ntiles, 64, d/2] (two INT4
+    codes per byte, even channel in the low nibble), s8/s4 float32 [H, ntiles].
+    """
+    x = _c(x_bits, np.uint16)
+    cu = _c(cu_seqlens, np.int32)
+    ntok, H, d = x.shape
+    nt = num_tiles(cu)
+    x8 = np.zeros((H, nt, TILE, d), np.int8) if want8 else None
+    x4 = np.zeros((H, nt, TILE, d // 2), np.uint8) if want4 else None
+    s8 = np.zeros((H, nt), np.float32) if want8 else None
+    s4 = np.zeros((H, nt), np.float32) if want4 else None
+    rc = _load().orc_quantize(_p(x), _p(cu), len(cu) - 1, H, d, _p(x8), _p(x4), _p(s8), _p(s4))
+    if rc != 0:
+        raise ValueError("oracle quantize failed")
+    return x8, x4, s8, s4
+
+
+def lists_boundary(cu_seqlens, b1, b2):
+    """Precision-grouped traversal rows (h, q-tile) from two diagonal boundaries."""
+    cu = _c(cu_seqlens, np.int32)
+    b1 = _c(b1, np.int32)
+    b2 = _c(b2, np.int32)
+    lib = _load()
+    B, Hq = len(cu) - 1, len(b1)
+    nnz = lib.orc_lists_boundary(_p(cu), B, Hq, _p(b1), _p(b2), None, None)
+    if nnz < 0:
+        raise ValueError("invalid boundaries")
+    row_ptr = np.zeros(Hq * num_tiles(cu) + 1, np.int32)
+    entries = np.zeros(max(nnz, 1), np.uint32)
+    lib.orc_lists_boundary(_p(cu), B, Hq, _p(b1), _p(b2), _p(row_ptr), _p(entries))
+    return row_ptr, entries[:nnz]
+
+
+def lists_bitmask(cu_seqlens, bitmask, G):
+    """Traversal rows from a packed bitmask [Hq, ntiles, W] (1 -> BF16, 0 -> INT8)."""
+    cu = _c(cu_seqlens, np.int32)
+    bm = _c(bitmask, np.uint32)
+    Hq, _, W = bm.shape
+    lib = _load()
+    B = len(cu) - 1
+    nnz = lib.orc_lists_bitmask(_p(cu), B, Hq, _p(bm), G, W, None, None)
+    if nnz < 0:
+        raise ValueError("invalid bitmask policy")
+    row_ptr = np.zeros(Hq * num_tiles(cu) + 1, np.int32)
+    entries = np.zeros(max(nnz, 1), np.uint32)
+    lib.orc_lists_bitmask(_p(cu), B, Hq, _p(bm), G, W, _p(row_ptr), _p(entries))
+    return row_ptr, entries[:nnz]
+
+
+def lists_decode(cu_seqlens, Hq, Hkv, b1=None, b2=None):
+    """Decode-cache rows (b, kv-head); boundary mode if b1/b2 given, else all INT8."""
+    cu = _c(cu_seqlens, np.int32)
+    mode = 1 if b1 is None else 0
+    b1a = _c(b1 if b1 is not None else np.zeros(Hq), np.int32)
+    b2a = _c(b2 if b2 is not None else np.zeros(Hq), np.int32)
+    lib = _load()
+    B = len(cu) - 1
+    nnz = lib.orc_lists_decode(_p(cu), B, Hq, Hkv, mode, _p(b1a), _p(b2a), None, None)
+    if nnz < 0:
+        raise ValueError("invalid decode policy")
+    row_ptr = np.zeros(B * Hkv + 1, np.int32)
+    entries = np.zeros(max(nnz, 1), np.uint32)
+    lib.orc_lists_decode(_p(cu), B, Hq, Hkv, mode, _p(b1a), _p(b2a), _p(row_ptr), _p(entries))
+    return row_ptr, entries[:nnz]
+
+
+def int_tile(prec, q8t=None, q4t=None, k8t=None, k4t=None, d=None):
+    """Raw int32 Q-code * K-code^T of one 64x64 tile (no masking)."""
+    out = np.zeros((TILE, TILE), np.int32)
+    if prec == INT8:
+        q8t = _c(q8t, np.int8); k8t = _c(k8t, np.int8); d = q8t.shape[-1]
+    else:
+        q4t = _c(q4t, np.uint8); k4t = _c(k4t, np.uint8); d = 2 * q4t.shape[-1]
+    rc = _load().orc_int_tile(prec, d, _p(q8t), _p(q4t), _p(k8t), _p(k4t), _p(out))
+    if rc != 0:
+        raise ValueError("bad precision")
+    return out
+
+
+class Quantised:
+    """Oracle-side quantised tensors of one prefill (its own, never the GPU's)."""
+
+    def __init__(self, q_bits, k_bits, v_bits, cu_seqlens):
+        none = (None, None, None, None)
+        self.q8, self.q4, self.sq8, self.sq4 = (
+            quantize(q_bits, cu_seqlens) if q_bits is not None else none)
+        self.k8, self.k4, self.sk8, self.sk4 = (
+            quantize(k_bits, cu_seqlens) if k_bits is not None else none)
+        self.v8, self.v4, self.sv8, self.sv4 = (
+            quantize(v_bits, cu_seqlens) if v_bits is not None else none)
+
+
+def prefill_rows(q_bits, k_bits, v_bits, cu_seqlens, qz: Quantised, row_ptr, entries,
+                 rows, scale=None):
+    """fp64 output [len(rows), 64, d] and lse [len(rows), 64] for traversal rows."""
+    q = _c(q_bits, np.uint16); k = _c(k_bits, np.uint16); v = _c(v_bits, np.uint16)
+    cu = _c(cu_seqlens, np.int32)
+    _, Hq, d = q.shape
+    Hkv = k.shape[1]
+    rows = _c(rows, np.int64)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.zeros((len(rows), TILE, d), np.float64)
+    lse = np.zeros((len(rows), TILE), np.float64)
+    rp = _c(row_ptr, np.int32); en = _c(entries, np.uint32)
+    rc = _load().orc_prefill_rows(
+        _p(q), _p(k), _p(v), _p(cu), len(cu) - 1, Hq, Hkv, d,
+        _p(qz.q8), _p(qz.q4), _p(qz.sq8), _p(qz.sq4),
+        _p(qz.k8), _p(qz.k4), _p(qz.sk8), _p(qz.sk4),
+        _p(rp), _p(en), float(scale), len(rows), _p(rows), _p(out), _p(lse))
+    if rc != 0:
+        raise ValueError(f"oracle prefill failed ({rc})")
+    return out, lse
+
+
+def gather_rows(out_rows, cu_seqlens, rows, Hq):
+    """Scatter per-row oracle output [nrows, 64, d] into token order for one head.
+
+    Returns a dict {(h, token): vector} for the valid tokens of each row.
+    """
+    cu = np.asarray(cu_seqlens, np.int64)
+    nt = [(int(cu[b + 1] - cu[b]) + TILE - 1) // TILE for b in range(len(cu) - 1)]
+    off = np.concatenate([[0], np.cumsum(nt)])
+    ntiles = int(off[-1])
+    res = {}
+    for i, row in enumerate(rows):
+        h, gq = divmod(int(row), ntiles)
+        b = int(np.searchsorted(off, gq, side="right") - 1)
+        qt = gq - off[b]
+        T = int(cu[b + 1] - cu[b])
+        for r in range(TILE):
+            t = qt * TILE + r
+            if t < T:
+                res[(h, int(cu[b]) + t)] = out_rows[i, r]
+    return res
+
+
+def decode_step(qd_bits, cu_seqlens, Hkv, cache: Quantised, row_ptr, entries,
+                k_tail_bits, v_tail_bits, tail_len, scale=None):
+    """fp64 decode output [B, Hq, d]; the tails already hold the new token."""
+    qd = _c(qd_bits, np.uint16)
+    cu = _c(cu_seqlens, np.int32)
+    B, Hq, d = qd.shape
+    kt = _c(k_tail_bits, np.uint16); vt = _c(v_tail_bits, np.uint16)
+    cap = kt.shape[2]
+    tl = _c(tail_len, np.int32)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.zeros((B, Hq, d), np.float64)
+    rp = _c(row_ptr, np.int32); en = _c(entries, np.uint32)
+    rc = _load().orc_decode_step(
+        _p(qd), _p(cu), B, Hq, Hkv, d,
+        _p(cache.k8), _p(cache.k4), _p(cache.sk8), _p(cache.sk4),
+        _p(cache.v8), _p(cache.v4), _p(cache.sv8), _p(cache.sv4),
+        _p(rp), _p(en), _p(kt), _p(vt), _p(tl), cap, float(scale), _p(out))
+    if rc != 0:
+        raise ValueError("oracle decode failed")
+    return out

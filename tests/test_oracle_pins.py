@@ -1,0 +1,459 @@
+"""Pins for the CPU oracle against facts that do not come from the oracle itself.
+
+Each test checks the oracle against something the pages or mathematics fix:
+hand-worked quantisation examples, closed-form list counts, textbook dense
+causal softmax attention (the all-BF16 policy), block-local attention
+(b1 = b2 = 1), dense attention over dequantised INT8 scores (b1 = b2 >= tiles),
+a per-(query, key) brute force of the routing rule, and probability rows that
+sum to one.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tile_routed_mixed_causal_b200 import workloads as wl
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+T = 64
+
+
+def bits_of(x: np.ndarray) -> np.ndarray:
+    return wl.bf16_bits(torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16))
+
+
+def val_of(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def read_golden(name):
+    rows = []
+    with open(os.path.join(GOLD, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([c.strip() for c in line.split("|")])
+    return rows
+
+
+# --------------------------------------------------------------------------- quantiser
+@pytest.mark.parametrize("row", read_golden("quant_examples.txt"))
+def test_quant_hand_examples(row):
+    fmt, vals, codes, scale = row
+    vals = [float(x) for x in vals.split()]
+    codes = [int(x) for x in codes.split()]
+    d = 64
+    x = np.zeros((T, 1, d), np.float32)
+    x[0, 0, :len(vals)] = vals
+    x8, x4, s8, s4 = oracle.quantize(bits_of(x), [0, T])
+    if fmt == "int8":
+        got = x8[0, 0, 0, :len(vals)].tolist()
+        s = s8[0, 0]
+    else:
+        c = x4[0, 0, 0]
+        nib = np.stack([c & 0xF, c >> 4], -1).reshape(-1).astype(np.int32)
+        got = np.where(nib >= 8, nib - 16, nib)[:len(vals)].tolist()
+        s = s4[0, 0]
+    assert got == codes
+    if scale != "-":
+        assert s == np.float32(float(scale))
+
+
+@pytest.mark.parametrize("row", read_golden("int4_packing.txt"))
+def test_int4_packing(row):
+    pair, byte = row
+    ce, co = [int(x) for x in pair.split()]
+    d = 64
+    x = np.zeros((T, 1, d), np.float32)
+    x[0, 0, 0], x[0, 0, 1] = ce, co
+    x[1, 0, 0] = 7.0          # amax 7 -> INT4 scale exactly 1
+    _, x4, _, s4 = oracle.quantize(bits_of(x), [0, T])
+    assert s4[0, 0] == 1.0
+    assert x4[0, 0, 0, 0] == int(byte, 16)
+
+
+def test_quant_invariants_random():
+    """Scale = fl32(amax/qmax); |code| <= qmax; amax maps to +-qmax; |x/s - code| <= 1/2;
+    padded rows and all-zero tiles give code 0; scales are per (head, tile)."""
+    rng = np.random.default_rng(7)
+    lengths = [100, 64, 1, 130]
+    ntok, H, d = sum(lengths), 3, 64
+    x = rng.standard_normal((ntok, H, d)).astype(np.float32) * rng.uniform(0.01, 50, size=(1, H, 1))
+    x[100:164, 1, :] = 0.0       # an all-zero tile (sequence 1, head 1)
+    bits = bits_of(x)
+    xv = val_of(bits)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    x8, x4, s8, s4 = oracle.quantize(bits, cu)
+    nt = oracle.num_tiles(cu)
+    assert nt == sum((L + 63) // 64 for L in lengths)
+    gt = 0
+    for b, L in enumerate(lengths):
+        for t in range((L + 63) // 64):
+            for h in range(H):
+                rows = xv[cu[b] + t * 64: cu[b] + min(L, t * 64 + 64), h, :]
+                amax = np.float32(np.abs(rows).max())
+                assert s8[h, gt] == np.float32(amax / np.float32(127.0))
+                assert s4[h, gt] == np.float32(amax / np.float32(7.0))
+                n = rows.shape[0]
+                c8 = x8[h, gt, :n].astype(np.int64)
+                nib = np.stack([x4[h, gt, :n] & 0xF, x4[h, gt, :n] >> 4], -1).reshape(n, d).astype(np.int64)
+                c4 = np.where(nib >= 8, nib - 16, nib)
+                assert np.all(np.abs(c8) <= 127) and np.all(np.abs(c4) <= 7)
+                assert np.all(x8[h, gt, n:] == 0) and np.all(x4[h, gt, n:] == 0)
+                if amax == 0:
+                    assert np.all(c8 == 0) and np.all(c4 == 0)
+                    continue
+                assert np.abs(c8).max() == 127 and np.abs(c4).max() == 7
+                r8 = rows.astype(np.float32) / s8[h, gt]
+                r4 = rows.astype(np.float32) / s4[h, gt]
+                assert np.all(np.abs(r8 - c8) <= 0.5 + 1e-6)
+                assert np.all(np.abs(r4 - c4) <= 0.5 + 1e-6)
+            gt += 1
+
+
+# --------------------------------------------------------------------------- traversal lists
+def _decode_entries(e):
+    return (e >> 28).astype(np.int64), (e & 0x0FFFFFFF).astype(np.int64)
+
+
+@pytest.mark.parametrize("lengths,b1,b2", [
+    ([256], [1, 1], [3, 3]),
+    ([1000, 1, 64, 65, 700], [1, 2, 3, 1], [1, 5, 3, 40]),
+])
+def test_lists_boundary_closed_form(lengths, b1, b2):
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    rp, en = oracle.lists_boundary(cu, b1, b2)
+    prec, kt = _decode_entries(en)
+    nts = [(L + 63) // 64 for L in lengths]
+    row = 0
+    nnz = 0
+    for h in range(len(b1)):
+        for nt in nts:
+            for qt in range(nt):
+                n = min(qt + 1, b2[h])
+                n8 = min(qt + 1, b1[h])
+                s, e = rp[row], rp[row + 1]
+                assert e - s == n
+                # INT4 block first: the n - n8 tiles qt-b2+1 .. qt-b1, ascending
+                assert list(prec[s:s + n - n8]) == [1] * (n - n8)
+                assert list(kt[s:s + n - n8]) == list(range(qt - n + 1, qt - n8 + 1))
+                # then INT8: qt-n8+1 .. qt ascending; the diagonal is last
+                assert list(prec[s + n - n8:e]) == [2] * n8
+                assert list(kt[s + n - n8:e]) == list(range(qt - n8 + 1, qt + 1))
+                nnz += n
+                row += 1
+    assert rp[-1] == nnz == len(en)
+
+
+def test_lists_bitmask_closed_form():
+    lengths = [64 * 37, 5, 64 * 9 + 3]
+    G = 3
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    nts = [(L + 63) // 64 for L in lengths]
+    Hq = 2
+    rng = np.random.default_rng(3)
+    W = 1
+    bm = rng.integers(0, 2**32, size=(Hq, sum(nts), W), dtype=np.uint64).astype(np.uint32)
+    rp, en = oracle.lists_bitmask(cu, bm, G)
+    prec, kt = _decode_entries(en)
+    row = 0
+    for h in range(Hq):
+        gt = 0
+        for nt in nts:
+            for qt in range(nt):
+                word = int(bm[h, gt + qt, 0])
+                hi = [j for j in range(qt + 1) if (word >> (j // G)) & 1]
+                lo = [j for j in range(qt + 1) if not (word >> (j // G)) & 1]
+                s, e = rp[row], rp[row + 1]
+                assert e - s == qt + 1              # dense connectivity: no skips
+                assert list(kt[s:e]) == lo + hi
+                assert list(prec[s:e]) == [2] * len(lo) + [3] * len(hi)
+                row += 1
+            gt += nt
+
+
+def test_lists_decode_closed_form():
+    lengths = [64 * 20, 64 * 7 + 5]
+    Hq, Hkv = 4, 2
+    b1 = [2, 5, 1, 1]
+    b2 = [3, 9, 1, 4]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    rp, en = oracle.lists_decode(cu, Hq, Hkv, b1, b2)
+    prec, kt = _decode_entries(en)
+    row = 0
+    for L in lengths:
+        nt = (L + 63) // 64
+        for kvh in range(Hkv):
+            hs = range(kvh * 2, kvh * 2 + 2)
+            B1 = max(b1[h] for h in hs)
+            B2 = max(b2[h] for h in hs)
+            n8 = min(nt, B1)
+            n = min(nt, B2)
+            s, e = rp[row], rp[row + 1]
+            assert e - s == n
+            assert list(kt[s:e]) == list(range(nt - n, nt - n8)) + list(range(nt - n8, nt))
+            assert list(prec[s:e]) == [1] * (n - n8) + [2] * n8
+            row += 1
+    # bitmask mode: every prefill tile is cached as INT8
+    rp, en = oracle.lists_decode(cu, Hq, Hkv)
+    assert rp[-1] == Hkv * sum((L + 63) // 64 for L in lengths)
+    assert np.all((en >> 28) == 2)
+
+
+def test_policy_storage_independent_of_length():
+    """Two int32 boundaries per head: 8 * Hq bytes at every context length."""
+    sizes = set()
+    for T in (256, 8192, 32768, 131072):
+        w = wl.custom("p", [T], 32, 8, 128, 0, "boundary", b1=np.ones(32), b2=np.full(32, 3))
+        sizes.add(w.b1.nbytes + w.b2.nbytes)
+    assert sizes == {8 * 32}
+
+
+# --------------------------------------------------------------------------- integer tiles
+def test_int_tile_matches_integer_matmul():
+    rng = np.random.default_rng(11)
+    for d in (64, 128):
+        q8 = rng.integers(-127, 128, size=(T, d)).astype(np.int8)
+        k8 = rng.integers(-127, 128, size=(T, d)).astype(np.int8)
+        ref = q8.astype(np.int64) @ k8.astype(np.int64).T
+        assert np.array_equal(oracle.int_tile(oracle.INT8, q8t=q8, k8t=k8), ref)
+        q4c = rng.integers(-7, 8, size=(T, d))
+        k4c = rng.integers(-7, 8, size=(T, d))
+        pack = lambda c: ((c[:, 0::2] & 0xF) | ((c[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+        ref4 = q4c.astype(np.int64) @ k4c.astype(np.int64).T
+        assert np.array_equal(oracle.int_tile(oracle.INT4, q4t=pack(q4c), k4t=pack(k4c)), ref4)
+
+
+# --------------------------------------------------------------------------- prefill
+def _dense_causal(qv, kv, vv, cu, Hq, Hkv, scores_fn=None):
+    """Textbook causal softmax attention per sequence and head, fp64."""
+    d = qv.shape[-1]
+    out = np.zeros_like(qv)
+    grp = Hq // Hkv
+    for b in range(len(cu) - 1):
+        s0, s1 = cu[b], cu[b + 1]
+        L = s1 - s0
+        for h in range(Hq):
+            if scores_fn is None:
+                S = qv[s0:s1, h] @ kv[s0:s1, h // grp].T / np.sqrt(d)
+            else:
+                S = scores_fn(b, h)
+            mask = np.tril(np.ones((L, L), bool))
+            S = np.where(mask, S, -np.inf)
+            P = np.exp(S - S.max(1, keepdims=True))
+            P /= P.sum(1, keepdims=True)
+            out[s0:s1, h] = P @ vv[s0:s1, h // grp]
+    return out
+
+
+def _run_oracle_all_rows(w: wl.Workload, q, k, v, cu):
+    qz = oracle.Quantised(q, k, None, cu)
+    if w.mode == "boundary":
+        rp, en = oracle.lists_boundary(cu, w.b1, w.b2)
+    else:
+        rp, en = oracle.lists_bitmask(cu, w.bitmask, w.G)
+    rows = np.arange(len(rp) - 1)
+    out, lse = oracle.prefill_rows(q, k, v, cu, qz, rp, en, rows)
+    res = oracle.gather_rows(out, cu, rows, w.Hq)
+    full = np.zeros((cu[-1], w.Hq, q.shape[-1]))
+    for (h, t), vec in res.items():
+        full[t, h] = vec
+    return full, qz, lse
+
+
+def _inputs(w):
+    t = wl.make_inputs(w, "cpu")
+    return tuple(wl.bf16_bits(t[n]) for n in ("q", "k", "v"))
+
+
+def _dequant_tokens(codes8, s8, cu, d, H):
+    """Token-major dequantised values [ntok, H, d] from tile-major INT8 codes."""
+    ntok = cu[-1]
+    out = np.zeros((ntok, H, d))
+    gt = 0
+    for b in range(len(cu) - 1):
+        L = cu[b + 1] - cu[b]
+        for t in range((L + 63) // 64):
+            n = min(64, L - t * 64)
+            for h in range(H):
+                out[cu[b] + t * 64: cu[b] + t * 64 + n, h] = codes8[h, gt, :n].astype(np.float64) * s8[h, gt]
+            gt += 1
+    return out
+
+
+def _unpack4(x4):
+    nib = np.stack([x4 & 0xF, x4 >> 4], -1).reshape(*x4.shape[:-1], -1).astype(np.int64)
+    return np.where(nib >= 8, nib - 16, nib)
+
+
+def test_prefill_all_bf16_is_dense_attention():
+    """All-BF16 bitmask == textbook dense causal attention (GQA, varlen, ragged)."""
+    w = wl.custom("allbf16", [130, 64, 1, 200], 4, 2, 64, 5, "bitmask", G=2, p_bf16=1.0)
+    q, k, v = _inputs(w)
+    cu = w.cu_seqlens
+    got, _, _ = _run_oracle_all_rows(w, q, k, v, cu)
+    ref = _dense_causal(val_of(q), val_of(k), val_of(v), cu, w.Hq, w.Hkv)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_prefill_block_local():
+    """b1 = b2 = 1: each query sees only its own tile's causal keys, INT8 scores."""
+    w = wl.custom("local", [200, 64], 2, 1, 64, 6, "boundary", b1=[1, 1], b2=[1, 1])
+    q, k, v = _inputs(w)
+    cu = w.cu_seqlens
+    got, qz, _ = _run_oracle_all_rows(w, q, k, v, cu)
+    qd = _dequant_tokens(qz.q8, qz.sq8, cu, 64, w.Hq)
+    kd = _dequant_tokens(qz.k8, qz.sk8, cu, 64, w.Hkv)
+    vv = val_of(v)
+    ref = np.zeros_like(got)
+    for b in range(len(cu) - 1):
+        for t0 in range(cu[b], cu[b + 1], 64):
+            t1 = min(t0 + 64, cu[b + 1])
+            L = t1 - t0
+            for h in range(w.Hq):
+                S = qd[t0:t1, h] @ kd[t0:t1, 0].T / 8.0
+                S = np.where(np.tril(np.ones((L, L), bool)), S, -np.inf)
+                P = np.exp(S - S.max(1, keepdims=True))
+                P /= P.sum(1, keepdims=True)
+                ref[t0:t1, h] = P @ vv[t0:t1, 0]
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_prefill_all_int8_is_dense_over_dequantised_scores():
+    """b1 = b2 >= tiles: every causal tile in INT8, none skipped."""
+    w = wl.custom("int8", [300, 90], 2, 2, 64, 8, "boundary", b1=[5, 9], b2=[5, 9])
+    q, k, v = _inputs(w)
+    cu = w.cu_seqlens
+    got, qz, _ = _run_oracle_all_rows(w, q, k, v, cu)
+    qd = _dequant_tokens(qz.q8, qz.sq8, cu, 64, w.Hq)
+    kd = _dequant_tokens(qz.k8, qz.sk8, cu, 64, w.Hkv)
+    ref = _dense_causal(qd, kd, val_of(v), cu, w.Hq, w.Hkv)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def _brute_force_prefill(w, q, k, v, qz):
+    """Per (query, key) pair: pick the precision by the boundary/bitmask rule directly."""
+    cu = w.cu_seqlens
+    d = q.shape[-1]
+    grp = w.Hq // w.Hkv
+    qv, kvv, vv = val_of(q), val_of(k), val_of(v)
+    q8 = _dequant_tokens(qz.q8, qz.sq8, cu, d, w.Hq)
+    k8 = _dequant_tokens(qz.k8, qz.sk8, cu, d, w.Hkv)
+    q4 = _dequant_tokens(_unpack4(qz.q4), qz.sq4, cu, d, w.Hq) if qz.q4 is not None else None
+    k4 = _dequant_tokens(_unpack4(qz.k4), qz.sk4, cu, d, w.Hkv) if qz.k4 is not None else None
+    out = np.zeros((cu[-1], w.Hq, d))
+    gt0 = 0
+    for b in range(len(cu) - 1):
+        L = cu[b + 1] - cu[b]
+        for h in range(w.Hq):
+            kvh = h // grp
+            for i in range(L):
+                s = []
+                keys = []
+                for j in range(i + 1):
+                    qt, kt = i // 64, j // 64
+                    if w.mode == "boundary":
+                        dist = qt - kt
+                        if dist < w.b1[h]:
+                            sc = q8[cu[b] + i, h] @ k8[cu[b] + j, kvh]
+                        elif dist < w.b2[h]:
+                            sc = q4[cu[b] + i, h] @ k4[cu[b] + j, kvh]
+                        else:
+                            continue
+                    else:
+                        g = kt // w.G
+                        bit = (int(w.bitmask[h, gt0 + qt, g // 32]) >> (g % 32)) & 1
+                        if bit:
+                            sc = qv[cu[b] + i, h] @ kvv[cu[b] + j, kvh]
+                        else:
+                            sc = q8[cu[b] + i, h] @ k8[cu[b] + j, kvh]
+                    s.append(sc / np.sqrt(d))
+                    keys.append(j)
+                s = np.array(s)
+                p = np.exp(s - s.max())
+                p /= p.sum()
+                out[cu[b] + i, h] = p @ vv[cu[b] + np.array(keys), kvh]
+        gt0 += (L + 63) // 64
+    return out
+
+
+def test_prefill_brute_force_tiny_config():
+    """The tiny configuration (1 x 2 heads x 256 tokens, (b1, b2) = (1, 3)), brute force."""
+    w = wl.tiny()
+    q, k, v = _inputs(w)
+    got, qz, _ = _run_oracle_all_rows(w, q, k, v, w.cu_seqlens)
+    ref = _brute_force_prefill(w, q, k, v, qz)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_prefill_brute_force_bitmask_gqa_varlen():
+    w = wl.custom("bm", [190, 70], 4, 2, 64, 12, "bitmask", G=2, p_bf16=0.4)
+    q, k, v = _inputs(w)
+    got, qz, _ = _run_oracle_all_rows(w, q, k, v, w.cu_seqlens)
+    ref = _brute_force_prefill(w, q, k, v, qz)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_prefill_rows_sum_to_one():
+    """With V = 1 everywhere every output equals 1: each probability row sums to 1."""
+    w = wl.custom("ones", [333], 2, 1, 64, 13, "boundary", b1=[1, 2], b2=[2, 4])
+    q, k, _ = _inputs(w)
+    ones = bits_of(np.ones((333, 1, 64), np.float32))
+    got, _, lse = _run_oracle_all_rows(w, q, k, ones, w.cu_seqlens)
+    assert np.max(np.abs(got - 1.0)) < 1e-12
+    assert np.all(np.isfinite(lse))
+
+
+# --------------------------------------------------------------------------- decode
+def test_decode_matches_naive_dense_softmax():
+    lengths = [64 * 6 + 10, 64 * 3]
+    w = wl.custom("dec", lengths, 4, 2, 64, 21, "boundary", b1=[1, 2, 1, 1], b2=[2, 4, 3, 1],
+                  decode_steps=3, tail_cap=4)
+    t = wl.make_inputs(w, "cpu")
+    k, v = wl.bf16_bits(t["k"]), wl.bf16_bits(t["v"])
+    cu = w.cu_seqlens
+    cache = oracle.Quantised(None, k, v, cu)
+    rp, en = oracle.lists_decode(cu, w.Hq, w.Hkv, w.b1, w.b2)
+    qs, kn, vn = (wl.bf16_bits(x) for x in wl.make_decode_inputs(w, "cpu"))
+    B, cap, d = len(lengths), 4, 64
+    kt = np.zeros((B, w.Hkv, cap, d), np.uint16)
+    vt = np.zeros((B, w.Hkv, cap, d), np.uint16)
+    for step in range(3):
+        kt[:, :, step] = kn[step]
+        vt[:, :, step] = vn[step]
+        tl = np.full(B, step + 1, np.int32)
+        got = oracle.decode_step(qs[step], cu, w.Hkv, cache, rp, en, kt, vt, tl)
+        # naive: dequantise every kept token, append the tail, dense softmax
+        for b in range(B):
+            L = lengths[b]
+            nt = (L + 63) // 64
+            for h in range(w.Hq):
+                kvh = h // 2
+                keys, vals = [], []
+                for kt_ in range(nt):
+                    dist = nt - 1 - kt_
+                    hs = (kvh * 2, kvh * 2 + 1)
+                    p8 = any(dist < w.b1[x] for x in hs)
+                    p4 = any(dist < w.b2[x] for x in hs)
+                    if not p4:
+                        continue
+                    gt = sum((x + 63) // 64 for x in lengths[:b]) + kt_
+                    n = min(64, L - kt_ * 64)
+                    if p8:
+                        kk = cache.k8[kvh, gt, :n] * np.float64(cache.sk8[kvh, gt])
+                        vv = cache.v8[kvh, gt, :n] * np.float64(cache.sv8[kvh, gt])
+                    else:
+                        kk = _unpack4(cache.k4[kvh, gt, :n]) * np.float64(cache.sk4[kvh, gt])
+                        vv = _unpack4(cache.v4[kvh, gt, :n]) * np.float64(cache.sv4[kvh, gt])
+                    keys.append(kk)
+                    vals.append(vv)
+                keys.append(val_of(kt[b, kvh, :step + 1]))
+                vals.append(val_of(vt[b, kvh, :step + 1]))
+                K = np.concatenate(keys)
+                V = np.concatenate(vals)
+                s = K @ val_of(qs[step, b, h]) / 8.0
+                p = np.exp(s - s.max())
+                p /= p.sum()
+                assert np.max(np.abs(got[b, h] - p @ V)) < 1e-12
