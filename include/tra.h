@@ -1,0 +1,256 @@
+/*
+ * tra.h -- C ABI of the tile-routed mixed-precision causal attention library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method (from the pages this library implements):
+ *  - "TriAttention: Unified Sparse Mixed-Precision Attention for Long-Context
+ *    LLM Inference", abstract: every query-key (QK) tile goes to skip, 4-bit or
+ *    8-bit score computation; a head's policy is two diagonal-distance
+ *    boundaries; the boundaries generate precision-grouped traversals for one
+ *    fused kernel that skips omitted tiles and combines both QK precisions into
+ *    one normalised attention output; the quantised keys/values prepared during
+ *    prefill are reused as a compressed KV cache for decoding.
+ *  - "TileMix: Tile-Centric Mixed-Precision Attention for LLM Inference
+ *    Acceleration", abstract: hardware-aligned score tiles, routing decisions
+ *    packed into bitmasks with one bit per group of adjacent key tiles, FP16
+ *    (BF16 here) or INT8 score computation, both paths updating one shared
+ *    online-softmax state; grouped-query attention, variable-length batches and
+ *    INT8 key/value caches.
+ *  - "HyQuant Uses Hybrid Precision to Compress LLM Attention", "How HyQuant
+ *    works": decode-time dequantisation fused into the attention kernel.
+ *
+ * Conventions (the pages print no formulas; these are the readings adopted):
+ *  - Tiles are TRA_TILE = 64 tokens.  A sequence of T tokens has
+ *    nt = ceil(T/64) tiles; tile numbering restarts at every sequence start.
+ *    ntiles = sum over sequences of nt (see tra_num_tiles).
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ *  - Q [ntok][Hq][d], K and V [ntok][Hkv][d], token-major, ntok = cu_seqlens[B].
+ *  - Quantised tensors are tile-major per head:
+ *      X8 int8  [H][ntiles][64][d], X4 uint8 [H][ntiles][64][d/2],
+ *      scales float [H][ntiles].
+ *    One symmetric scale per (head, tile) over the tile's valid rows:
+ *      s8 = fl32(amax/127), s4 = fl32(amax/7),
+ *      code = clamp(round_half_even(fl32(x / s)), -qmax, qmax)
+ *    (IEEE fp32 divide); amax == 0 gives s = 0 and codes 0; rows past the end
+ *    of a sequence are code 0.  INT4: two codes per byte, the even channel in
+ *    the low nibble, two's complement.
+ *  - Boundary policy, dist = qt - kt (tiles): dist < b1 -> INT8,
+ *    b1 <= dist < b2 -> INT4, dist >= b2 -> skip; 1 <= b1 <= b2, so the
+ *    diagonal tile is always kept in INT8.  Storage 8*Hq bytes at any length.
+ *  - Bitmask policy: uint32 [Hq][ntiles][W]; bit g of row (h, q-tile) (word
+ *    g/32, bit g%32) covers k-tiles [g*G, g*G+G): 1 -> BF16, 0 -> INT8; no skip.
+ *  - Traversal lists (CSR): prefill rows are (h, global q-tile), h-major;
+ *    decode-cache rows are (b, kv-head), b-major.  entry = (prec << 28) | kt,
+ *    kt local to the sequence, prec = TRA_PREC_*; a row lists its INT4 tiles
+ *    ascending, then INT8 ascending, then BF16 ascending.
+ *  - Softmax scale: any positive float; 1/sqrt(d) is the usual choice.
+ *  - GQA: query head h reads KV head h / (Hq/Hkv).
+ *
+ * Memory and streams: every buffer is caller-owned device memory unless a
+ * parameter says "host".  The library allocates nothing, never synchronises the
+ * device, and enqueues all work on the given stream (a cudaStream_t passed as
+ * void*; NULL = legacy default stream).  Pointers to device buffers must be
+ * 16-byte aligned.  Every call validates its arguments on the host before any
+ * launch and returns a tra_status; tra_last_error() gives a thread-local text.
+ * Errors found on the device (a bounded wait that expired, a full decode tail)
+ * are OR-ed into the caller's int32 status word (TRA_DEV_*), which the caller
+ * zeroes and reads back when it chooses.
+ */
+#ifndef TRA_H
+#define TRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TRA_API __attribute__((visibility("default")))
+#else
+#define TRA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TRA_OK = 0,
+  TRA_ERR_INVALID = 1,     /* bad argument (null pointer, bad size, bad policy) */
+  TRA_ERR_UNSUPPORTED = 2, /* valid but unsupported (e.g. d not 64 or 128) */
+  TRA_ERR_BUFFER = 3,      /* a caller buffer is too small */
+  TRA_ERR_CUDA = 4,        /* a CUDA call or launch failed */
+  TRA_ERR_TIMEOUT = 5      /* reserved for callers that map TRA_DEV_TIMEOUT */
+} tra_status;
+
+#define TRA_TILE 64
+
+#define TRA_PREC_INT4 1
+#define TRA_PREC_INT8 2
+#define TRA_PREC_BF16 3
+
+#define TRA_POLICY_BOUNDARY 0
+#define TRA_POLICY_BITMASK 1
+
+#define TRA_LISTS_PREFILL 0
+#define TRA_LISTS_DECODE_CACHE 1
+
+/* tra_qtiles.formats bits */
+#define TRA_FMT_Q8 0x01u
+#define TRA_FMT_Q4 0x02u
+#define TRA_FMT_K8 0x04u
+#define TRA_FMT_K4 0x08u
+#define TRA_FMT_V8 0x10u
+#define TRA_FMT_V4 0x20u
+
+/* device status word bits */
+#define TRA_DEV_TIMEOUT 0x1      /* a bounded pipeline wait expired */
+#define TRA_DEV_TAIL_FULL 0x2    /* decode: tail_len reached tail_cap */
+
+#define TRA_MAX_HEADS 256        /* Hq limit (policies travel as launch params) */
+#define TRA_MAX_DUMP 64          /* max tiles per integer-accumulator dump */
+#define TRA_MAX_DECODE_SPLITS 64
+
+typedef struct {
+  int32_t B;                        /* sequences */
+  int32_t Hq, Hkv;                  /* query / key-value heads, Hq % Hkv == 0 */
+  int32_t d;                        /* head dim: 64 or 128 */
+  const int32_t* cu_seqlens_dev;    /* device [B+1], cu[0] = 0, non-decreasing */
+  const int32_t* cu_seqlens_host;   /* host copy of the same values */
+} tra_shape;
+
+typedef struct {
+  int32_t mode;                     /* TRA_POLICY_BOUNDARY or TRA_POLICY_BITMASK */
+  const int32_t* b1;                /* host [Hq] (boundary mode) */
+  const int32_t* b2;                /* host [Hq] (boundary mode) */
+  const uint32_t* bitmask_dev;      /* device [Hq][ntiles][W] (bitmask mode) */
+  int32_t G;                        /* k-tiles per bit (bitmask mode), >= 1 */
+  int32_t W;                        /* words per bitmask row, W*32*G >= max nt */
+} tra_policy;
+
+typedef struct {
+  int8_t* q8;  uint8_t* q4;         /* [Hq][ntiles][64][d] / [..][d/2] */
+  int8_t* k8;  uint8_t* k4;         /* [Hkv][ntiles][64][d] / [..][d/2] */
+  int8_t* v8;  uint8_t* v4;
+  float* sq8;  float* sq4;          /* [Hq][ntiles] */
+  float* sk8;  float* sk4;          /* [Hkv][ntiles] */
+  float* sv8;  float* sv4;
+  uint32_t formats;                 /* TRA_FMT_* bits: which fields are present */
+} tra_qtiles;
+
+/* Thread-local description of the last error returned on this thread. */
+TRA_API const char* tra_last_error(void);
+
+/* Library version string. */
+TRA_API const char* tra_version(void);
+
+/* Total tiles over the batch (sum of ceil(T_b/64)), from cu_seqlens_host;
+ * -1 if the shape is invalid. */
+TRA_API int64_t tra_num_tiles(const tra_shape* shape);
+
+/* Bytes of each quantised buffer for `formats` (the sum over present fields,
+ * each rounded up to 256 bytes); 0 on an invalid shape. */
+TRA_API size_t tra_qtiles_bytes(const tra_shape* shape, uint32_t formats);
+
+/*
+ * quantize_qkv_tiles -- per-(head, 64-token tile) symmetric INT8/INT4
+ * quantisation of Q, K and V ("quantized keys and values prepared during
+ * prefill", TriAttention abstract; INT8 tiles, TileMix abstract).
+ * q/k/v: device bf16 [ntok][H][d]; a tensor may be NULL when `out->formats`
+ * requests none of its formats.  Writes the codes and scales selected by
+ * out->formats (layouts above).  Deterministic and bit-exact with the rule in
+ * the header comment.
+ */
+TRA_API tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const uint16_t* k,
+                              const uint16_t* v, const tra_qtiles* out, void* stream);
+
+/*
+ * tra_tile_lists_size -- exact CSR sizes of the traversal lists (host only,
+ * closed form; no device access).  list_kind = TRA_LISTS_PREFILL gives
+ * rows = Hq*ntiles; TRA_LISTS_DECODE_CACHE gives rows = B*Hkv.  *row_ptr_len =
+ * rows + 1.  Fails with TRA_ERR_INVALID on a bad policy and TRA_ERR_UNSUPPORTED
+ * if nnz does not fit in int32.
+ */
+TRA_API tra_status tra_tile_lists_size(const tra_shape* shape, const tra_policy* policy,
+                               int32_t list_kind, int64_t* rows, int64_t* nnz);
+
+/*
+ * build_tile_lists -- precision-grouped traversals ("the selected boundaries
+ * generate precision-grouped traversals", TriAttention abstract; "packs routing
+ * decisions into compact bitmasks ... each routing bit govern multiple adjacent
+ * key tiles", TileMix abstract).
+ * Prefill rows (h, q-tile): boundary mode lists INT4 k-tiles
+ * [max(0,qt-b2+1), qt-b1] then INT8 [max(0,qt-b1+1), qt]; bitmask mode lists
+ * the INT8 k-tiles <= qt then the BF16 ones.  Decode-cache rows (b, kv-head):
+ * a k-tile's precision is the highest any query head of the group gives it at
+ * dist = nt-1-kt (boundary mode), INT8 for all tiles in bitmask mode.
+ * row_ptr: device int32 [row_ptr_len]; entries: device uint32 [entries_cap];
+ * sizes from tra_tile_lists_size, else TRA_ERR_BUFFER.
+ */
+TRA_API tra_status build_tile_lists(const tra_shape* shape, const tra_policy* policy, int32_t list_kind,
+                            int32_t* row_ptr, int64_t row_ptr_len, uint32_t* entries,
+                            int64_t entries_cap, void* stream);
+
+/*
+ * routed_attention_prefill -- fused causal prefill attention over the
+ * precision-grouped traversal: every listed tile's scores come from its
+ * precision (INT8 or INT4 codes multiplied exactly in int32 and rescaled by
+ * sQ*sK, or BF16 with fp32 accumulation); every path updates one online
+ * softmax state per query row; P*V uses bf16 P and the original bf16 V
+ * (TriAttention abstract: "combines contributions from both QK precisions into
+ * one normalized attention output"; TileMix abstract: "both paths update a
+ * shared online-softmax state").
+ * q/k/v: device bf16 as above; tiles: output of quantize_qkv_tiles (Q8/K8
+ * always, Q4/K4 when the policy has INT4 tiles); row_ptr/entries: prefill
+ * lists; out: device bf16 [ntok][Hq][d]; lse: device float [Hq][ntok] natural-
+ * log logsumexp of the scaled scores, or NULL.
+ * Integer-accumulator dump (debug; n_dump = 0 disables): dump_coords device
+ * int32 [n_dump][4] = (b, h, qt, kt); for each listed INT8/INT4 tile the raw
+ * int32 Q-code x K-code^T accumulators go to dump_out [n_dump][64][64]
+ * (row = query within the tile, column = key).  n_dump <= TRA_MAX_DUMP.
+ * status_dev: device int32, receives TRA_DEV_* bits.
+ */
+TRA_API tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* policy,
+                                    const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                    const tra_qtiles* tiles, const int32_t* row_ptr,
+                                    const uint32_t* entries, float softmax_scale, uint16_t* out,
+                                    float* lse, const int32_t* dump_coords, int32_t n_dump,
+                                    int32_t* dump_out, int32_t* status_dev, void* stream);
+
+/* Workspace bytes routed_attention_decode needs (split-K partials); 0 on bad sizes. */
+TRA_API size_t tra_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t d);
+
+/*
+ * routed_attention_decode -- one decode step over the compressed KV cache
+ * ("the quantized keys and values prepared during prefill are then reused in a
+ * compressed key-value (KV) cache for decoding", TriAttention abstract;
+ * "Dequantization is fused with attention computation", HyQuant, "How HyQuant
+ * works").  For each sequence b: the new token's k_new/v_new [b][kvh] is
+ * appended at tail position tail_len[b]; every query head attends to the
+ * cached tiles listed for (b, kv-head) -- K = sK*code and V = sV*code in the
+ * tile's cached format -- plus the bf16 tail tokens [0, tail_len[b]] ; one
+ * softmax per head; then tail_len[b] is incremented.
+ * prefill_shape: the prefill's shape (cu_seqlens give the cached lengths);
+ * policy: the policy the lists were built from (validation only: INT4 cache
+ * formats are required when a boundary policy has b1 < b2);
+ * q: device bf16 [B][Hq][d]; k_new/v_new: device bf16 [B][Hkv][d];
+ * cache: K8/K4/V8/V4 (+scales) from quantize_qkv_tiles;
+ * row_ptr/entries: TRA_LISTS_DECODE_CACHE lists;
+ * k_tail/v_tail: device bf16 [B][Hkv][tail_cap][d]; tail_len_dev: device
+ * int32 [B] (read, then incremented by one); out: device bf16 [B][Hq][d];
+ * workspace: device, >= tra_decode_workspace_bytes(B, Hq, Hkv, d).
+ * A sequence whose tail is full sets TRA_DEV_TAIL_FULL and leaves its output
+ * and tail untouched.
+ */
+TRA_API tra_status routed_attention_decode(const tra_shape* prefill_shape, const tra_policy* policy,
+                                   const uint16_t* q,
+                                   const uint16_t* k_new, const uint16_t* v_new,
+                                   const tra_qtiles* cache, const int32_t* row_ptr,
+                                   const uint32_t* entries, uint16_t* k_tail, uint16_t* v_tail,
+                                   int32_t* tail_len_dev, int32_t tail_cap, float softmax_scale,
+                                   uint16_t* out, void* workspace, size_t workspace_bytes,
+                                   int32_t* status_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRA_H */

@@ -1,0 +1,342 @@
+"""GPU parity: the CUDA library (through the C ABI) against the CPU oracle.
+
+Integer work (codes, scales, traversal lists, integer QK accumulators) must be
+bit-exact.  Floating outputs must satisfy, element by element,
+    max(|o_gpu - o_ref| - ulp_bf16(o_ref) / 2) <= 1e-2   and   mean |o_gpu - o_ref| <= 1e-3,
+i.e. a 1e-2 max / 1e-3 mean budget on top of the unavoidable rounding of the
+bf16 output.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tile_routed_mixed_causal_b200 as tra
+from tile_routed_mixed_causal_b200 import api
+from tile_routed_mixed_causal_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+MAX_TOL, MEAN_TOL = 1e-2, 1e-3
+
+
+def half_ulp_bf16(x):
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8), 0.0)
+
+
+def assert_close(got, ref, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    excess = float(np.max(err - half_ulp_bf16(ref)))
+    mean = float(np.mean(err))
+    assert excess <= MAX_TOL and mean <= MEAN_TOL, \
+        f"{what}: max excess {excess:.3e} (raw max {err.max():.3e}), mean {mean:.3e}"
+    return float(err.max()), mean
+
+
+def to_np_u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+class Case:
+    """A workload materialised on the GPU plus its host copies for the oracle."""
+
+    def __init__(self, w: wl.Workload, gen_device="cpu"):
+        self.w = w
+        t = wl.make_inputs(w, gen_device)
+        self.q, self.k, self.v = (t[n].cuda() for n in ("q", "k", "v"))
+        self.qb, self.kb, self.vb = (wl.bf16_bits(t[n]) for n in ("q", "k", "v"))
+        self.shape = tra.Shape(w.cu_seqlens, w.Hq, w.Hkv, w.d)
+        if w.mode == "boundary":
+            self.policy = tra.Policy.boundary(w.b1, w.b2)
+        else:
+            self.bitmask = torch.from_numpy(w.bitmask.view(np.int32)).cuda()
+            self.policy = tra.Policy.from_bitmask(self.bitmask, w.G)
+
+    def oracle_lists(self):
+        if self.w.mode == "boundary":
+            return oracle.lists_boundary(self.w.cu_seqlens, self.w.b1, self.w.b2)
+        return oracle.lists_bitmask(self.w.cu_seqlens, self.w.bitmask, self.w.G)
+
+
+SMALL = [
+    wl.tiny(),
+    wl.custom("b_d64_gqa_ragged", [130, 64, 1, 200, 577], 4, 2, 64, 31, "boundary"),
+    wl.custom("b_d128_local", [1000], 2, 2, 128, 32, "boundary", b1=[1, 1], b2=[1, 1]),
+    wl.custom("b_d128_all8", [700, 300], 2, 1, 128, 33, "boundary", b1=[12, 3], b2=[12, 9]),
+    wl.custom("b_d128_gqa4", [2049, 640], 8, 2, 128, 34, "boundary",
+              b1=[1, 2, 3, 4, 1, 1, 2, 8], b2=[3, 2, 9, 30, 1, 20, 4, 8]),
+    wl.custom("m_d128_g1", [900, 65, 300], 8, 2, 128, 35, "bitmask", G=1, p_bf16=0.3),
+    wl.custom("m_d64_g3", [1500], 2, 2, 64, 36, "bitmask", G=3, p_bf16=0.5),
+    wl.custom("m_d128_allbf16", [513], 4, 4, 128, 37, "bitmask", G=2, p_bf16=1.0),
+    wl.custom("m_d128_all8", [777], 4, 2, 128, 38, "bitmask", G=4, p_bf16=0.0),
+]
+
+
+def _run_prefill(c: Case, with_lse=True):
+    plan = api.PrefillPlan(c.shape, c.policy)
+    out = torch.zeros_like(c.q)
+    lse = torch.zeros((c.w.Hq, c.w.ntok), dtype=torch.float32, device="cuda") if with_lse else None
+    plan.run(c.q, c.k, c.v, out, lse)
+    torch.cuda.synchronize()
+    assert int(plan.status.item()) == 0
+    return plan, out, lse
+
+
+# ---------------------------------------------------------------- quantiser
+@pytest.mark.parametrize("w", SMALL[:5], ids=lambda w: w.name)
+def test_quantize_bit_exact(w):
+    c = Case(w)
+    qt = tra.QTiles(c.shape, 0x3F)
+    tra.quantize_qkv_tiles(c.shape, c.q, c.k, c.v, qt)
+    torch.cuda.synchronize()
+    for name, bits in (("q", c.qb), ("k", c.kb), ("v", c.vb)):
+        x8, x4, s8, s4 = oracle.quantize(bits, w.cu_seqlens)
+        assert np.array_equal(qt[name + "8"].cpu().numpy(), x8), name + "8"
+        assert np.array_equal(qt[name + "4"].cpu().numpy(), x4), name + "4"
+        assert np.array_equal(qt["s" + name + "8"].cpu().numpy().view(np.uint32), s8.view(np.uint32))
+        assert np.array_equal(qt["s" + name + "4"].cpu().numpy().view(np.uint32), s4.view(np.uint32))
+
+
+def test_quantize_edge_values():
+    """Zero tiles, ties, tiny and huge magnitudes, a partial tile."""
+    w = wl.custom("edge", [64, 70, 3], 2, 2, 128, 40, "boundary")
+    c = Case(w)
+    x = c.q.float()
+    x[0:64, 0] = 0.0                                     # all-zero tile
+    x[64:128, 1] = torch.linspace(-7, 7, 64 * 128, device="cuda").view(64, 128)
+    x[128:134, 0] *= 1e-30                               # denormal-range products
+    x[134:137, 1] *= 3e4
+    q = x.to(torch.bfloat16)
+    qt = tra.QTiles(c.shape, tra.FMT_Q8 | tra.FMT_Q4)
+    tra.quantize_qkv_tiles(c.shape, q, None, None, qt)
+    torch.cuda.synchronize()
+    x8, x4, s8, s4 = oracle.quantize(wl.bf16_bits(q), w.cu_seqlens)
+    assert np.array_equal(qt["q8"].cpu().numpy(), x8)
+    assert np.array_equal(qt["q4"].cpu().numpy(), x4)
+    assert np.array_equal(qt["sq8"].cpu().numpy(), s8)
+    assert np.array_equal(qt["sq4"].cpu().numpy(), s4)
+
+
+# ---------------------------------------------------------------- traversal lists
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_lists_bit_exact(w):
+    c = Case(w)
+    plan = api.PrefillPlan(c.shape, c.policy)
+    plan.lists()
+    torch.cuda.synchronize()
+    rp, en = c.oracle_lists()
+    assert np.array_equal(plan.row_ptr.cpu().numpy(), rp)
+    assert np.array_equal(to_np_u32(plan.entries)[:plan.nnz], en)
+    if w.mode == "boundary":
+        dp = api.DecodePlan(c.shape, c.policy, None, 4)
+        dp.build()
+        torch.cuda.synchronize()
+        rp, en = oracle.lists_decode(w.cu_seqlens, w.Hq, w.Hkv, w.b1, w.b2)
+        assert np.array_equal(dp.row_ptr.cpu().numpy(), rp)
+        assert np.array_equal(to_np_u32(dp.entries)[:dp.nnz], en)
+
+
+# ---------------------------------------------------------------- prefill
+def _oracle_full(c: Case):
+    rp, en = c.oracle_lists()
+    qz = oracle.Quantised(c.qb, c.kb, None, c.w.cu_seqlens)
+    rows = np.arange(len(rp) - 1)
+    out, lse = oracle.prefill_rows(c.qb, c.kb, c.vb, c.w.cu_seqlens, qz, rp, en, rows)
+    return qz, rows, out, lse
+
+
+def _compare_rows(c: Case, rows, ref_out, ref_lse, gpu_out, gpu_lse, what):
+    w = c.w
+    cu = np.asarray(w.cu_seqlens, np.int64)
+    nts = [(int(cu[b + 1] - cu[b]) + 63) // 64 for b in range(w.B)]
+    off = np.concatenate([[0], np.cumsum(nts)])
+    got, ref, gl, rl = [], [], [], []
+    go = gpu_out.float().cpu().numpy()
+    glse = gpu_lse.cpu().numpy() if gpu_lse is not None else None
+    for i, row in enumerate(rows):
+        h, gq = divmod(int(row), int(off[-1]))
+        b = int(np.searchsorted(off, gq, side="right") - 1)
+        qt = gq - off[b]
+        T = int(cu[b + 1] - cu[b])
+        n = min(64, T - qt * 64)
+        toks = cu[b] + qt * 64 + np.arange(n)
+        got.append(go[toks, h])
+        ref.append(ref_out[i, :n])
+        if glse is not None:
+            gl.append(glse[h, toks])
+            rl.append(ref_lse[i, :n])
+    res = assert_close(np.concatenate(got), np.concatenate(ref), what)
+    if glse is not None:
+        assert np.max(np.abs(np.concatenate(gl) - np.concatenate(rl))) < 1e-3, what + " lse"
+    return res
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_prefill_matches_oracle(w):
+    c = Case(w)
+    plan, out, lse = _run_prefill(c)
+    _, rows, ref, ref_lse = _oracle_full(c)
+    _compare_rows(c, rows, ref, ref_lse, out, lse, w.name)
+
+
+def test_prefill_integer_accumulator_dump():
+    """Every INT8/INT4 tile of the tiny configuration: raw int32 Q-code K-code^T, bit-exact."""
+    w = wl.tiny()
+    c = Case(w)
+    plan = api.PrefillPlan(c.shape, c.policy)
+    plan.quantize(c.q, c.k, c.v)
+    plan.lists()
+    rp, en = c.oracle_lists()
+    coords = []
+    for h in range(w.Hq):
+        for qt in range(4):
+            row = h * 4 + qt
+            for e in en[rp[row]:rp[row + 1]]:
+                coords.append((0, h, qt, int(e & 0x0FFFFFFF), int(e >> 28)))
+    dc = torch.tensor([x[:4] for x in coords], dtype=torch.int32, device="cuda")
+    dump = torch.full((len(coords), 64, 64), -7, dtype=torch.int32, device="cuda")
+    out = torch.zeros_like(c.q)
+    plan.attend(c.q, c.k, c.v, out, dump_coords=dc, dump_out=dump)
+    torch.cuda.synchronize()
+    qz = oracle.Quantised(c.qb, c.kb, None, w.cu_seqlens)
+    for i, (_, h, qt, kt, prec) in enumerate(coords):
+        if prec == oracle.INT8:
+            ref = oracle.int_tile(prec, q8t=qz.q8[h, qt], k8t=qz.k8[h, kt])
+        else:
+            ref = oracle.int_tile(prec, q4t=qz.q4[h, qt], k4t=qz.k4[h, kt])
+        assert np.array_equal(dump[i].cpu().numpy(), ref), (h, qt, kt, prec)
+
+
+def _sampled_rows(w, heads, qtiles_per_seq):
+    nts = w.tiles_per_seq
+    off = np.concatenate([[0], np.cumsum(nts)])
+    rows = []
+    for h in heads:
+        for b, nt in enumerate(nts):
+            for qt in qtiles_per_seq(nt):
+                rows.append(h * off[-1] + off[b] + qt)
+    return np.array(rows, np.int64)
+
+
+FULL = {
+    "llama8b_8k": (wl.llama8b_8k, [0, 13, 31], lambda nt: [0, 1, 7, 64, nt - 2, nt - 1]),
+    "bitmask_32k": (wl.bitmask_32k, [0, 17, 31], lambda nt: [0, 3, 255, nt - 1]),
+    "varlen": (wl.varlen_8, [0, 27], lambda nt: [0, nt // 2, nt - 1]),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_prefill_full_size_sampled(name):
+    """Full-size configurations, same launch as the benchmark, sampled rows vs the oracle."""
+    make, heads, qts = FULL[name]
+    w = make()
+    c = Case(w, gen_device="cuda")
+    plan, out, lse = _run_prefill(c)
+    rows = _sampled_rows(w, heads, qts)
+    rp, en = c.oracle_lists()
+    # traversal lists are checked in full at this size too
+    assert np.array_equal(plan.row_ptr.cpu().numpy(), rp)
+    assert np.array_equal(to_np_u32(plan.entries)[:plan.nnz], en)
+    qz = oracle.Quantised(c.qb, c.kb, None, w.cu_seqlens)
+    assert np.array_equal(plan.tiles["q8"].cpu().numpy(), qz.q8)
+    assert np.array_equal(plan.tiles["k8"].cpu().numpy(), qz.k8)
+    ref, ref_lse = oracle.prefill_rows(c.qb, c.kb, c.vb, w.cu_seqlens, qz, rp, en, rows)
+    _compare_rows(c, rows, ref, ref_lse, out, lse, name)
+
+
+# ---------------------------------------------------------------- decode
+def _decode_case(w, gen_device="cpu"):
+    c = Case(w, gen_device)
+    fm = tra.FMT_K8 | tra.FMT_K4 | tra.FMT_V8 | tra.FMT_V4
+    cache = tra.QTiles(c.shape, fm)
+    tra.quantize_qkv_tiles(c.shape, None, c.k, c.v, cache)
+    dp = api.DecodePlan(c.shape, c.policy, cache, w.tail_cap)
+    dp.build()
+    qs, kn, vn = wl.make_decode_inputs(w, gen_device)
+    return c, cache, dp, qs.cuda(), kn.cuda(), vn.cuda()
+
+
+DEC = [
+    wl.custom("dec_small", [64 * 6 + 10, 64 * 3, 1], 4, 2, 64, 50, "boundary",
+              b1=[1, 2, 1, 1], b2=[2, 4, 3, 1], decode_steps=5, tail_cap=8),
+    wl.custom("dec_d128_g4", [64 * 40, 64 * 33 + 17], 8, 2, 128, 51, "boundary",
+              b1=[3, 1, 9, 2, 1, 1, 4, 2], b2=[20, 5, 9, 30, 1, 2, 4, 16], decode_steps=4,
+              tail_cap=70),
+    wl.custom("dec_d128_mha", [64 * 20], 2, 2, 128, 52, "boundary", b1=[1, 2], b2=[1, 2],
+              decode_steps=3, tail_cap=3),
+]
+
+
+@pytest.mark.parametrize("w", DEC, ids=lambda w: w.name)
+def test_decode_matches_oracle(w):
+    c, cache, dp, qs, kn, vn = _decode_case(w)
+    cu = w.cu_seqlens
+    ocache = oracle.Quantised(None, c.kb, c.vb, cu)
+    rp, en = oracle.lists_decode(cu, w.Hq, w.Hkv, w.b1, w.b2)
+    kt = np.zeros((w.B, w.Hkv, w.tail_cap, w.d), np.uint16)
+    vt = np.zeros_like(kt)
+    out = torch.zeros((w.B, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
+    for step in range(w.decode_steps):
+        dp.step(qs[step], kn[step], vn[step], out)
+        torch.cuda.synchronize()
+        kt[:, :, step] = wl.bf16_bits(kn[step])
+        vt[:, :, step] = wl.bf16_bits(vn[step])
+        ref = oracle.decode_step(wl.bf16_bits(qs[step]), cu, w.Hkv, ocache, rp, en, kt, vt,
+                                 np.full(w.B, step + 1, np.int32))
+        assert_close(out.float().cpu().numpy(), ref, f"{w.name} step {step}")
+    assert int(dp.status.item()) == 0
+    assert np.array_equal(dp.tail_len.cpu().numpy(), np.full(w.B, w.decode_steps))
+    assert np.array_equal(wl.bf16_bits(dp.k_tail[:, :, :w.decode_steps]), kt[:, :, :w.decode_steps])
+
+
+def test_decode_tail_full_sets_status():
+    w = wl.custom("dec_full", [128], 2, 1, 64, 53, "boundary", b1=[1, 1], b2=[2, 2],
+                  decode_steps=2, tail_cap=1)
+    c, cache, dp, qs, kn, vn = _decode_case(w)
+    out = torch.zeros((1, 2, 64), dtype=torch.bfloat16, device="cuda")
+    dp.step(qs[0], kn[0], vn[0], out)
+    torch.cuda.synchronize()
+    first = out.clone()
+    assert int(dp.status.item()) == 0 and int(dp.tail_len.item()) == 1
+    dp.step(qs[1], kn[1], vn[1], out)
+    torch.cuda.synchronize()
+    assert int(dp.status.item()) & tra.DEV_TAIL_FULL
+    assert int(dp.tail_len.item()) == 1
+    assert torch.equal(out, first)
+
+
+def test_decode_full_size_sampled():
+    """Batch 16 over a 32K prefix, 64 steps as benchmarked; sampled sequences vs the oracle."""
+    w = wl.decode_32k()
+    c, cache, dp, qs, kn, vn = _decode_case(w, gen_device="cuda")
+    out = torch.zeros((w.B, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
+    check_steps = {0, 31, 63}
+    sample_b = [0, 9, 15]
+    outs = {}
+    for step in range(w.decode_steps):
+        dp.step(qs[step], kn[step], vn[step], out)
+        if step in check_steps:
+            outs[step] = out.float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert int(dp.status.item()) == 0
+    T = w.lengths[0]
+    for b in sample_b:
+        cu1 = np.array([0, T], np.int32)
+        kb = wl.bf16_bits(c.k[b * T:(b + 1) * T])
+        vb = wl.bf16_bits(c.v[b * T:(b + 1) * T])
+        ocache = oracle.Quantised(None, kb, vb, cu1)
+        rp, en = oracle.lists_decode(cu1, w.Hq, w.Hkv, w.b1, w.b2)
+        for step in sorted(check_steps):
+            kt = wl.bf16_bits(kn[:step + 1, b]).transpose(1, 0, 2)[None]
+            vt = wl.bf16_bits(vn[:step + 1, b]).transpose(1, 0, 2)[None]
+            ref = oracle.decode_step(wl.bf16_bits(qs[step, b:b + 1]), cu1, w.Hkv, ocache, rp, en,
+                                     np.ascontiguousarray(kt), np.ascontiguousarray(vt),
+                                     np.array([step + 1], np.int32))
+            assert_close(outs[step][b], ref[0], f"decode b={b} step={step}")

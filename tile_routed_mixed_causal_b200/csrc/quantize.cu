@@ -1,0 +1,128 @@
+// quantize.cu -- per-(head, 64-token tile) symmetric INT8/INT4 quantisation of
+// Q, K and V ("The quantized keys and values prepared during prefill",
+// TriAttention abstract; INT8 tiles and INT8 K/V caches, TileMix abstract).
+//
+// One CTA per (tensor, head, tile): the 64 x d bf16 tile is read once with
+// 16-byte loads into registers, the absolute maximum is reduced with warp
+// shuffles, and the INT8 codes, packed INT4 codes and both scales are written
+// tile-major.  HBM-bound: 2*64*d bytes in, (1 + 1/2)*64*d bytes + 8 out.
+// Arithmetic: s = fl32(amax / qmax) and code = rne(fl32(x / s)) with IEEE
+// division (__fdiv_rn) and round-half-even conversion (__float2int_rn).
+#include "tra_device.cuh"
+#include "tra_launch.h"
+
+namespace tra {
+namespace {
+
+__device__ __forceinline__ int quant_code(float x, float s, int qmax) {
+  if (s == 0.0f) return 0;
+  int c = __float2int_rn(__fdiv_rn(x, s));
+  return c > qmax ? qmax : (c < -qmax ? -qmax : c);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <int D>
+__global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p) {
+  constexpr int kChunks = D / 8;                 // 16-byte chunks per row
+  constexpr int kPasses = kTile * kChunks / 256;  // chunks per thread
+  __shared__ float red[8];
+
+  const long long cta = blockIdx.x;
+  int which = 0;
+  while (which < 2 && cta >= p.cta_begin[which + 1]) ++which;
+  const QuantTensor& t = p.t[which];
+  const long long local = cta - p.cta_begin[which];
+  const int h = (int)(local / p.ntiles);
+  const int gt = (int)(local % p.ntiles);
+
+  // sequence of this tile
+  int b = 0, toff = 0;
+  for (;; ++b) {
+    const int nt = (p.cu[b + 1] - p.cu[b] + kTile - 1) / kTile;
+    if (gt < toff + nt) break;
+    toff += nt;
+  }
+  const int T = p.cu[b + 1] - p.cu[b];
+  const int tt = gt - toff;
+  const int H = t.H;
+
+  uint4 v[kPasses];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kPasses; ++i) {
+    const int f = i * 256 + threadIdx.x;
+    const int r = f / kChunks, c = f % kChunks;
+    const int tok = tt * kTile + r;
+    if (tok < T) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          t.x + ((long long)(p.cu[b] + tok) * H + h) * D + c * 8);
+      v[i] = __ldg(src);
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      amax = fmaxf(amax, fabsf(bf16_lo(w[j])));
+      amax = fmaxf(amax, fabsf(bf16_hi(w[j])));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+
+  const float s8 = __fdiv_rn(amax, 127.0f);
+  const float s4 = __fdiv_rn(amax, 7.0f);
+  const long long tile_base = (long long)h * p.ntiles + gt;
+  if (threadIdx.x == 0) {
+    if (t.s8) t.s8[tile_base] = s8;
+    if (t.s4) t.s4[tile_base] = s4;
+  }
+#pragma unroll
+  for (int i = 0; i < kPasses; ++i) {
+    const int f = i * 256 + threadIdx.x;
+    const int r = f / kChunks, c = f % kChunks;
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    float x[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x[2 * j] = bf16_lo(w[j]);
+      x[2 * j + 1] = bf16_hi(w[j]);
+    }
+    // rows past the sequence end were loaded as 0 and quantise to code 0
+    if (t.x8) {
+      uint32_t o[2] = {0, 0};
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        o[j >> 2] |= (uint32_t)(quant_code(x[j], s8, 127) & 0xFF) << ((j & 3) * 8);
+      *reinterpret_cast<uint2*>(t.x8 + (tile_base * kTile + r) * D + c * 8) = make_uint2(o[0], o[1]);
+    }
+    if (t.x4) {
+      uint32_t o = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o |= (uint32_t)(quant_code(x[j], s4, 7) & 0x0F) << (j * 4);
+      *reinterpret_cast<uint32_t*>(t.x4 + (tile_base * kTile + r) * (D / 2) + c * 4) = o;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const QuantParams& p, cudaStream_t s) {
+  const long long ctas = p.cta_begin[3];
+  if (ctas == 0) return cudaSuccess;
+  if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  if (p.d == 128)
+    quantize_kernel<128><<<(unsigned)ctas, 256, 0, s>>>(p);
+  else
+    quantize_kernel<64><<<(unsigned)ctas, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace tra

@@ -1,0 +1,449 @@
+// tra_api.cu -- host side of the C ABI declared in include/tra.h: argument
+// validation, closed-form sizes, TMA tensor-map construction and the launches.
+// Every check happens before any launch; nothing here allocates device memory
+// or synchronises the device.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/tra.h"
+#include "tra_launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+tra_status fail(tra_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+tra_status ok() {
+  g_last_error.clear();
+  return TRA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_tiles(int64_t T) { return (T + TRA_TILE - 1) / TRA_TILE; }
+
+// Validates a shape; fills ntiles, ntok and the largest per-sequence tile count.
+tra_status check_shape(const tra_shape* s, int64_t* ntiles, int64_t* ntok, int64_t* nt_max) {
+  if (!s) return fail(TRA_ERR_INVALID, "shape is NULL");
+  if (s->B < 1) return fail(TRA_ERR_INVALID, "B must be >= 1 (got %d)", s->B);
+  if (s->Hq < 1 || s->Hkv < 1) return fail(TRA_ERR_INVALID, "Hq and Hkv must be >= 1");
+  if (s->Hq % s->Hkv) return fail(TRA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", s->Hq, s->Hkv);
+  if (s->Hq > TRA_MAX_HEADS) return fail(TRA_ERR_UNSUPPORTED, "Hq > %d", TRA_MAX_HEADS);
+  if (s->d != 64 && s->d != 128) return fail(TRA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", s->d);
+  if (!s->cu_seqlens_host || !s->cu_seqlens_dev) return fail(TRA_ERR_INVALID, "cu_seqlens (host and device) required");
+  if (reinterpret_cast<uintptr_t>(s->cu_seqlens_dev) & 3u) return fail(TRA_ERR_INVALID, "cu_seqlens_dev misaligned");
+  if (s->cu_seqlens_host[0] != 0) return fail(TRA_ERR_INVALID, "cu_seqlens[0] must be 0");
+  int64_t t = 0, m = 0;
+  for (int b = 0; b < s->B; ++b) {
+    const int64_t L = (int64_t)s->cu_seqlens_host[b + 1] - s->cu_seqlens_host[b];
+    if (L < 0) return fail(TRA_ERR_INVALID, "cu_seqlens not non-decreasing at %d", b);
+    t += ceil_tiles(L);
+    if (ceil_tiles(L) > m) m = ceil_tiles(L);
+  }
+  if (t * TRA_TILE * (int64_t)s->Hq > (1ll << 31) * 64) return fail(TRA_ERR_UNSUPPORTED, "problem too large");
+  if (ntiles) *ntiles = t;
+  if (ntok) *ntok = s->cu_seqlens_host[s->B];
+  if (nt_max) *nt_max = m;
+  return TRA_OK;
+}
+
+// sum_{q < n} min(q + 1, c)
+int64_t tri_capped(int64_t n, int64_t c) {
+  if (n <= c) return n * (n + 1) / 2;
+  return c * (c + 1) / 2 + (n - c) * c;
+}
+
+tra_status check_policy(const tra_shape* s, const tra_policy* p, int64_t nt_max) {
+  if (!p) return fail(TRA_ERR_INVALID, "policy is NULL");
+  if (p->mode == TRA_POLICY_BOUNDARY) {
+    if (!p->b1 || !p->b2) return fail(TRA_ERR_INVALID, "boundary policy needs host b1 and b2");
+    for (int h = 0; h < s->Hq; ++h) {
+      if (p->b1[h] < 1) return fail(TRA_ERR_INVALID, "b1[%d] = %d < 1", h, p->b1[h]);
+      if (p->b2[h] < p->b1[h]) return fail(TRA_ERR_INVALID, "b2[%d] = %d < b1 = %d", h, p->b2[h], p->b1[h]);
+    }
+    return TRA_OK;
+  }
+  if (p->mode == TRA_POLICY_BITMASK) {
+    if (p->G < 1) return fail(TRA_ERR_INVALID, "G must be >= 1 (got %d)", p->G);
+    if (p->W < 1) return fail(TRA_ERR_INVALID, "W must be >= 1");
+    const int64_t groups = (nt_max + p->G - 1) / p->G;
+    if ((int64_t)p->W * 32 < groups)
+      return fail(TRA_ERR_INVALID, "W = %d words cannot hold %lld groups", p->W, (long long)groups);
+    return TRA_OK;
+  }
+  return fail(TRA_ERR_INVALID, "unknown policy mode %d", p->mode);
+}
+
+bool policy_has_int4(const tra_shape* s, const tra_policy* p) {
+  if (p->mode != TRA_POLICY_BOUNDARY) return false;
+  for (int h = 0; h < s->Hq; ++h)
+    if (p->b2[h] > p->b1[h]) return true;
+  return false;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// int8 tile-major codes viewed as 2-D: d bytes per row, `rows` rows.
+bool map_i8(CUtensorMap* m, const void* base, int d, int64_t rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d};
+  cuuint32_t box[2] = {(cuuint32_t)d, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [ntok][H][d] viewed as 3-D (d, H, ntok); boxes of 64 channels x 1 head x box_rows tokens.
+bool map_bf16(CUtensorMap* m, const void* base, int d, int H, int64_t ntok, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)ntok};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+tra_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(TRA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tra_last_error(void) { return g_last_error.c_str(); }
+
+const char* tra_version(void) { return "tile_routed_mixed_causal_b200 0.1 (sm_100a)"; }
+
+int64_t tra_num_tiles(const tra_shape* shape) {
+  int64_t nt = 0;
+  if (check_shape(shape, &nt, nullptr, nullptr) != TRA_OK) return -1;
+  return nt;
+}
+
+size_t tra_qtiles_bytes(const tra_shape* shape, uint32_t formats) {
+  int64_t nt = 0;
+  if (check_shape(shape, &nt, nullptr, nullptr) != TRA_OK) return 0;
+  const size_t d = shape->d;
+  size_t total = 0;
+  const struct { uint32_t bit; int H; size_t per_row; } f[6] = {
+      {TRA_FMT_Q8, shape->Hq, d}, {TRA_FMT_Q4, shape->Hq, d / 2}, {TRA_FMT_K8, shape->Hkv, d},
+      {TRA_FMT_K4, shape->Hkv, d / 2}, {TRA_FMT_V8, shape->Hkv, d}, {TRA_FMT_V4, shape->Hkv, d / 2}};
+  for (const auto& x : f)
+    if (formats & x.bit)
+      total += round256((size_t)x.H * nt * TRA_TILE * x.per_row) + round256((size_t)x.H * nt * 4);
+  return total;
+}
+
+tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const uint16_t* k,
+                              const uint16_t* v, const tra_qtiles* out, void* stream) {
+  int64_t nt = 0, ntok = 0;
+  tra_status st = check_shape(shape, &nt, &ntok, nullptr);
+  if (st != TRA_OK) return st;
+  if (!out) return fail(TRA_ERR_INVALID, "out is NULL");
+  const uint32_t f = out->formats;
+  if (f & ~0x3Fu) return fail(TRA_ERR_INVALID, "unknown format bits 0x%x", f);
+  tra::QuantParams p{};
+  const uint16_t* src[3] = {q, k, v};
+  const int H[3] = {shape->Hq, shape->Hkv, shape->Hkv};
+  int8_t* o8[3] = {out->q8, out->k8, out->v8};
+  uint8_t* o4[3] = {out->q4, out->k4, out->v4};
+  float* s8[3] = {out->sq8, out->sk8, out->sv8};
+  float* s4[3] = {out->sq4, out->sk4, out->sv4};
+  const char* nm[3] = {"q", "k", "v"};
+  p.cta_begin[0] = 0;
+  for (int i = 0; i < 3; ++i) {
+    const bool want8 = f & (TRA_FMT_Q8 << (2 * i));
+    const bool want4 = f & (TRA_FMT_Q4 << (2 * i));
+    tra::QuantTensor& t = p.t[i];
+    t = tra::QuantTensor{};
+    if (want8 || want4) {
+      if (!src[i]) return fail(TRA_ERR_INVALID, "%s is NULL but its formats are requested", nm[i]);
+      if (!aligned16(src[i])) return fail(TRA_ERR_INVALID, "%s not 16-byte aligned", nm[i]);
+      if (want8 && (!o8[i] || !s8[i] || !aligned16(o8[i]) || !aligned16(s8[i])))
+        return fail(TRA_ERR_INVALID, "%s8 codes/scales missing or misaligned", nm[i]);
+      if (want4 && (!o4[i] || !s4[i] || !aligned16(o4[i]) || !aligned16(s4[i])))
+        return fail(TRA_ERR_INVALID, "%s4 codes/scales missing or misaligned", nm[i]);
+      t.x = src[i];
+      t.H = H[i];
+      t.x8 = want8 ? o8[i] : nullptr;
+      t.s8 = want8 ? s8[i] : nullptr;
+      t.x4 = want4 ? o4[i] : nullptr;
+      t.s4 = want4 ? s4[i] : nullptr;
+    }
+    p.cta_begin[i + 1] = p.cta_begin[i] + (t.x ? (long long)t.H * nt : 0);
+  }
+  p.cu = shape->cu_seqlens_dev;
+  p.B = shape->B;
+  p.d = shape->d;
+  p.ntiles = (int)nt;
+  if (nt == 0) return ok();
+  cudaError_t e = tra::launch_quantize(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return ok();
+}
+
+tra_status tra_tile_lists_size(const tra_shape* shape, const tra_policy* policy, int32_t list_kind,
+                               int64_t* rows, int64_t* nnz) {
+  int64_t nt = 0, nt_max = 0;
+  tra_status st = check_shape(shape, &nt, nullptr, &nt_max);
+  if (st != TRA_OK) return st;
+  st = check_policy(shape, policy, nt_max);
+  if (st != TRA_OK) return st;
+  if (!rows || !nnz) return fail(TRA_ERR_INVALID, "rows/nnz outputs are NULL");
+  const int32_t* cu = shape->cu_seqlens_host;
+  int64_t total = 0;
+  if (list_kind == TRA_LISTS_PREFILL) {
+    *rows = (int64_t)shape->Hq * nt;
+    for (int h = 0; h < shape->Hq; ++h)
+      for (int b = 0; b < shape->B; ++b) {
+        const int64_t n = ceil_tiles(cu[b + 1] - cu[b]);
+        total += tri_capped(n, policy->mode == TRA_POLICY_BOUNDARY ? policy->b2[h] : (1ll << 40));
+      }
+  } else if (list_kind == TRA_LISTS_DECODE_CACHE) {
+    *rows = (int64_t)shape->B * shape->Hkv;
+    const int grp = shape->Hq / shape->Hkv;
+    for (int b = 0; b < shape->B; ++b) {
+      const int64_t n = ceil_tiles(cu[b + 1] - cu[b]);
+      for (int kvh = 0; kvh < shape->Hkv; ++kvh) {
+        if (policy->mode != TRA_POLICY_BOUNDARY) {
+          total += n;
+          continue;
+        }
+        int64_t m = 0;
+        for (int j = 0; j < grp; ++j) m = std::max<int64_t>(m, policy->b2[kvh * grp + j]);
+        total += std::min(n, m);
+      }
+    }
+  } else {
+    return fail(TRA_ERR_INVALID, "unknown list kind %d", list_kind);
+  }
+  if (total >= (1ll << 31)) return fail(TRA_ERR_UNSUPPORTED, "list has %lld entries (> int32)", (long long)total);
+  *nnz = total;
+  return ok();
+}
+
+tra_status build_tile_lists(const tra_shape* shape, const tra_policy* policy, int32_t list_kind,
+                            int32_t* row_ptr, int64_t row_ptr_len, uint32_t* entries,
+                            int64_t entries_cap, void* stream) {
+  int64_t rows = 0, nnz = 0;
+  tra_status st = tra_tile_lists_size(shape, policy, list_kind, &rows, &nnz);
+  if (st != TRA_OK) return st;
+  if (!row_ptr || (!entries && nnz > 0)) return fail(TRA_ERR_INVALID, "row_ptr/entries NULL");
+  if (!aligned16(row_ptr) || (entries && !aligned16(entries)))
+    return fail(TRA_ERR_INVALID, "row_ptr/entries not 16-byte aligned");
+  if (row_ptr_len < rows + 1) return fail(TRA_ERR_BUFFER, "row_ptr needs %lld entries", (long long)(rows + 1));
+  if (entries_cap < nnz) return fail(TRA_ERR_BUFFER, "entries needs %lld entries", (long long)nnz);
+  if (policy->mode == TRA_POLICY_BITMASK && list_kind == TRA_LISTS_PREFILL) {
+    if (!policy->bitmask_dev || (reinterpret_cast<uintptr_t>(policy->bitmask_dev) & 3u))
+      return fail(TRA_ERR_INVALID, "bitmask_dev NULL or misaligned");
+  }
+  int64_t nt = tra_num_tiles(shape);
+  tra::ListParams p;
+  memset(&p, 0, sizeof p);
+  p.cu = shape->cu_seqlens_dev;
+  p.B = shape->B;
+  p.Hq = shape->Hq;
+  p.Hkv = shape->Hkv;
+  p.ntiles = (int)nt;
+  p.mode = policy->mode;
+  p.kind = list_kind;
+  p.bitmask = policy->bitmask_dev;
+  p.G = policy->G;
+  p.W = policy->W;
+  p.row_ptr = row_ptr;
+  p.entries = entries;
+  p.rows = rows;
+  if (policy->mode == TRA_POLICY_BOUNDARY)
+    for (int h = 0; h < shape->Hq; ++h) {
+      p.b1[h] = policy->b1[h];
+      p.b2[h] = policy->b2[h];
+    }
+  cudaError_t e = tra::launch_lists(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lists launch");
+  return ok();
+}
+
+tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* policy,
+                                    const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                    const tra_qtiles* tiles, const int32_t* row_ptr,
+                                    const uint32_t* entries, float softmax_scale, uint16_t* out,
+                                    float* lse, const int32_t* dump_coords, int32_t n_dump,
+                                    int32_t* dump_out, int32_t* status_dev, void* stream) {
+  int64_t nt = 0, ntok = 0, nt_max = 0;
+  tra_status st = check_shape(shape, &nt, &ntok, &nt_max);
+  if (st != TRA_OK) return st;
+  st = check_policy(shape, policy, nt_max);
+  if (st != TRA_OK) return st;
+  if (!q || !k || !v || !out || !tiles || !row_ptr || !entries || !status_dev)
+    return fail(TRA_ERR_INVALID, "q, k, v, out, tiles, row_ptr, entries and status are required");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned16(lse)))
+    return fail(TRA_ERR_INVALID, "q/k/v/out/lse must be 16-byte aligned");
+  const uint32_t need8 = TRA_FMT_Q8 | TRA_FMT_K8;
+  if ((tiles->formats & need8) != need8 || !tiles->q8 || !tiles->k8 || !tiles->sq8 || !tiles->sk8)
+    return fail(TRA_ERR_INVALID, "prefill needs Q8 and K8 tiles");
+  if (!aligned16(tiles->q8) || !aligned16(tiles->k8)) return fail(TRA_ERR_INVALID, "Q8/K8 misaligned");
+  if (policy_has_int4(shape, policy)) {
+    const uint32_t need4 = TRA_FMT_Q4 | TRA_FMT_K4;
+    if ((tiles->formats & need4) != need4 || !tiles->q4 || !tiles->k4 || !tiles->sq4 || !tiles->sk4)
+      return fail(TRA_ERR_INVALID, "the policy has INT4 tiles: Q4 and K4 tiles are required");
+    if (!aligned16(tiles->q4) || !aligned16(tiles->k4)) return fail(TRA_ERR_INVALID, "Q4/K4 misaligned");
+  }
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
+    return fail(TRA_ERR_INVALID, "softmax_scale must be positive and finite");
+  if (n_dump < 0 || n_dump > TRA_MAX_DUMP) return fail(TRA_ERR_INVALID, "n_dump must be in [0, %d]", TRA_MAX_DUMP);
+  if (n_dump > 0 && (!dump_coords || !dump_out)) return fail(TRA_ERR_INVALID, "dump buffers required");
+  if (ntok == 0 || nt == 0) return ok();
+  tra::PrefillParams p{};
+  p.cu = shape->cu_seqlens_dev;
+  p.B = shape->B;
+  p.Hq = shape->Hq;
+  p.Hkv = shape->Hkv;
+  p.d = shape->d;
+  p.ntiles = (int)nt;
+  p.mode = policy->mode;
+  p.jmax = (int)((nt_max + 1) / 2);
+  p.row_ptr = row_ptr;
+  p.entries = entries;
+  p.q4 = tiles->q4;
+  p.k4 = tiles->k4;
+  p.sq8 = tiles->sq8;
+  p.sq4 = tiles->sq4;
+  p.sk8 = tiles->sk8;
+  p.sk4 = tiles->sk4;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  p.lse = lse;
+  p.dump_coords = dump_coords;
+  p.n_dump = n_dump;
+  p.dump_out = dump_out;
+  p.status = status_dev;
+  tra::PrefillMaps m;
+  memset(&m, 0, sizeof m);
+  const int d = shape->d;
+  bool good = map_i8(&m.q8, tiles->q8, d, (int64_t)shape->Hq * nt * TRA_TILE, 128) &&
+              map_i8(&m.k8, tiles->k8, d, (int64_t)shape->Hkv * nt * TRA_TILE, 64) &&
+              map_bf16(&m.qb, q, d, shape->Hq, ntok, 128) &&
+              map_bf16(&m.kb, k, d, shape->Hkv, ntok, 64) &&
+              map_bf16(&m.vb, v, d, shape->Hkv, ntok, 64);
+  if (!good) return fail(TRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  cudaError_t e = tra::launch_prefill(p, m, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return ok();
+}
+
+size_t tra_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t d) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || d < 1) return 0;
+  const size_t S = (size_t)tra::decode_splits(B, Hkv);
+  return round256((size_t)B * Hq * S * 2 * 4) + round256((size_t)B * Hq * S * d * 4);
+}
+
+tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* policy,
+                                   const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                                   const tra_qtiles* cache, const int32_t* row_ptr,
+                                   const uint32_t* entries, uint16_t* k_tail, uint16_t* v_tail,
+                                   int32_t* tail_len_dev, int32_t tail_cap, float softmax_scale,
+                                   uint16_t* out, void* workspace, size_t workspace_bytes,
+                                   int32_t* status_dev, void* stream) {
+  int64_t nt = 0, ntok = 0, nt_max = 0;
+  tra_status st = check_shape(shape, &nt, &ntok, &nt_max);
+  if (st != TRA_OK) return st;
+  st = check_policy(shape, policy, nt_max);
+  if (st != TRA_OK) return st;
+  if (shape->Hq / shape->Hkv > 8) return fail(TRA_ERR_UNSUPPORTED, "decode supports Hq/Hkv <= 8");
+  if (!q || !k_new || !v_new || !cache || !row_ptr || !entries || !k_tail || !v_tail ||
+      !tail_len_dev || !out || !workspace || !status_dev)
+    return fail(TRA_ERR_INVALID, "a required pointer is NULL");
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_tail) ||
+      !aligned16(v_tail) || !aligned16(out) || !aligned16(workspace))
+    return fail(TRA_ERR_INVALID, "q/k_new/v_new/tails/out/workspace must be 16-byte aligned");
+  if (tail_cap < 1) return fail(TRA_ERR_INVALID, "tail_cap must be >= 1");
+  const uint32_t need8 = TRA_FMT_K8 | TRA_FMT_V8;
+  if ((cache->formats & need8) != need8 || !cache->k8 || !cache->v8 || !cache->sk8 || !cache->sv8)
+    return fail(TRA_ERR_INVALID, "decode needs K8 and V8 cache tiles");
+  if (!aligned16(cache->k8) || !aligned16(cache->v8)) return fail(TRA_ERR_INVALID, "K8/V8 misaligned");
+  if (policy_has_int4(shape, policy)) {
+    const uint32_t need4 = TRA_FMT_K4 | TRA_FMT_V4;
+    if ((cache->formats & need4) != need4 || !cache->k4 || !cache->v4 || !cache->sk4 || !cache->sv4)
+      return fail(TRA_ERR_INVALID, "the policy has INT4 tiles: K4 and V4 cache tiles are required");
+    if (!aligned16(cache->k4) || !aligned16(cache->v4)) return fail(TRA_ERR_INVALID, "K4/V4 misaligned");
+  }
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
+    return fail(TRA_ERR_INVALID, "softmax_scale must be positive and finite");
+  const size_t need = tra_decode_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->d);
+  if (workspace_bytes < need) return fail(TRA_ERR_BUFFER, "workspace needs %zu bytes", need);
+  tra::DecodeParams p{};
+  p.cu = shape->cu_seqlens_dev;
+  p.B = shape->B;
+  p.Hq = shape->Hq;
+  p.Hkv = shape->Hkv;
+  p.d = shape->d;
+  p.ntiles = (int)nt;
+  p.splits = tra::decode_splits(shape->B, shape->Hkv);
+  p.q = q;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k8 = cache->k8;
+  p.k4 = cache->k4;
+  p.v8 = cache->v8;
+  p.v4 = cache->v4;
+  p.sk8 = cache->sk8;
+  p.sk4 = cache->sk4;
+  p.sv8 = cache->sv8;
+  p.sv4 = cache->sv4;
+  p.row_ptr = row_ptr;
+  p.entries = entries;
+  p.k_tail = k_tail;
+  p.v_tail = v_tail;
+  p.tail_len = tail_len_dev;
+  p.tail_cap = tail_cap;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  const size_t S = (size_t)p.splits;
+  p.part_ml = reinterpret_cast<float*>(workspace);
+  p.part_o = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
+                                      round256((size_t)shape->B * shape->Hq * S * 2 * 4));
+  p.status = status_dev;
+  cudaError_t e = tra::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,108 @@
+// tra_launch.h -- internal launch parameter blocks shared by the host ABI
+// (tra_api.cu) and the kernel files.  Not part of the public C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tra.h"
+
+namespace tra {
+
+// ------------------------------------------------------------ quantisation
+struct QuantTensor {
+  const uint16_t* x;   // bf16 [ntok][H][d]
+  int H;
+  int8_t* x8;          // nullable
+  uint8_t* x4;         // nullable
+  float* s8;
+  float* s4;
+};
+
+struct QuantParams {
+  QuantTensor t[3];          // Q, K, V (H = 0 or x = null: skipped)
+  long long cta_begin[4];    // prefix of H*ntiles over the three tensors
+  const int32_t* cu;         // device cu_seqlens
+  int B, d, ntiles;
+};
+
+cudaError_t launch_quantize(const QuantParams& p, cudaStream_t s);
+
+// ------------------------------------------------------------ traversal lists
+struct ListParams {
+  const int32_t* cu;
+  int B, Hq, Hkv, ntiles, mode, kind;
+  const uint32_t* bitmask;
+  int G, W;
+  int32_t* row_ptr;
+  uint32_t* entries;
+  long long rows;
+  int32_t b1[TRA_MAX_HEADS];
+  int32_t b2[TRA_MAX_HEADS];
+};
+
+cudaError_t launch_lists(const ListParams& p, cudaStream_t s);
+
+// ------------------------------------------------------------ prefill
+struct PrefillParams {
+  const int32_t* cu;
+  int B, Hq, Hkv, d, ntiles;
+  int mode;              // TRA_POLICY_*
+  int jmax;              // max over sequences of ceil(nt/2) (q-tile pairs)
+  const int32_t* row_ptr;
+  const uint32_t* entries;
+  const uint8_t* q4;     // packed INT4 codes [Hq][ntiles][64][d/2]
+  const uint8_t* k4;     // [Hkv][ntiles][64][d/2]
+  const float* sq8;
+  const float* sq4;
+  const float* sk8;
+  const float* sk4;
+  float scale_log2;      // softmax_scale * log2(e)
+  uint16_t* out;         // bf16 [ntok][Hq][d]
+  float* lse;            // [Hq][ntok] or null
+  const int32_t* dump_coords;
+  int n_dump;
+  int32_t* dump_out;
+  int32_t* status;
+};
+
+struct PrefillMaps {
+  CUtensorMap q8, k8;    // int8 tiles, 2-D (d bytes x rows)
+  CUtensorMap qb, kb, vb;  // bf16, 3-D (d, H, ntok)
+};
+
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s);
+
+// ------------------------------------------------------------ decode
+struct DecodeParams {
+  const int32_t* cu;
+  int B, Hq, Hkv, d, ntiles, splits;
+  const uint16_t* q;       // [B][Hq][d]
+  const uint16_t* k_new;   // [B][Hkv][d]
+  const uint16_t* v_new;
+  const int8_t* k8;
+  const uint8_t* k4;
+  const int8_t* v8;
+  const uint8_t* v4;
+  const float* sk8;
+  const float* sk4;
+  const float* sv8;
+  const float* sv4;
+  const int32_t* row_ptr;
+  const uint32_t* entries;
+  uint16_t* k_tail;        // [B][Hkv][cap][d]
+  uint16_t* v_tail;
+  int32_t* tail_len;
+  int tail_cap;
+  float scale_log2;
+  uint16_t* out;           // [B][Hq][d]
+  float* part_ml;          // [B][Hq][splits][2]
+  float* part_o;           // [B][Hq][splits][d]
+  int32_t* status;
+};
+
+int decode_splits(int B, int Hkv);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+
+}  // namespace tra
