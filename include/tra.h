@@ -104,6 +104,7 @@ typedef enum {
 /* device status word bits */
 #define TRA_DEV_TIMEOUT 0x1      /* a bounded pipeline wait expired */
 #define TRA_DEV_TAIL_FULL 0x2    /* decode: tail_len reached tail_cap */
+#define TRA_DEV_BAD_LIST 0x4     /* prefill: an INT4 list entry but no INT4 tiles */
 
 #define TRA_MAX_HEADS 256        /* Hq limit (policies travel as launch params) */
 #define TRA_MAX_DUMP 64          /* max tiles per integer-accumulator dump */

@@ -174,7 +174,9 @@ def _compare_rows(c: Case, rows, ref_out, ref_lse, gpu_out, gpu_lse, what):
             rl.append(ref_lse[i, :n])
     res = assert_close(np.concatenate(got), np.concatenate(ref), what)
     if glse is not None:
-        assert np.max(np.abs(np.concatenate(gl) - np.concatenate(rl))) < 1e-3, what + " lse"
+        # l is summed from the bf16-rounded P the MMA consumes (relative error <= 2^-9 per
+        # term), so log(l) may differ from the exact fp64 value by up to about 2^-9.
+        assert np.max(np.abs(np.concatenate(gl) - np.concatenate(rl))) < 2.0 ** -8, what + " lse"
     return res
 
 

@@ -110,6 +110,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kvh = h / grp;
   const int qt0 = 2 * j;
   const bool has_second = qt0 + 1 < nt;
+  // INT4 operands exist only for boundary policies with an INT4 region; a list
+  // entry asking for INT4 without them is reported, never read
+  const bool int4 = MODE == TRA_POLICY_BOUNDARY && p.has_int4;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (base - smem_u32(smem_raw));
@@ -191,6 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = i % NST, use = i / NST;
         const uint32_t prec = val >> 28;
         const int kt = (int)(val & 0x0FFFFFFFu);
+        if (prec == TRA_PREC_INT4 && !int4) {
+          *err = TRA_DEV_BAD_LIST;
+          break;
+        }
         if (prec != TRA_PREC_INT4) {
           if (use > 0 && !mbar_wait(bar_kfree(s), (use - 1) & 1, err)) break;
           const uint32_t dst = sK + s * C::kKBytes;
@@ -218,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdPV = instr_desc(1, 1, 0, 1, D, 128);
       const uint32_t tS = tmem, tO = tmem + 128;
       bool ok = mbar_wait(bar_q, 0, err);
-      if (ok && MODE == TRA_POLICY_BOUNDARY) ok = mbar_wait(bar_q4, 0, err);
+      if (ok && int4) ok = mbar_wait(bar_q4, 0, err);
       tc_fence_after();
       uint32_t kph = 0, k4ph = 0;  // per-slot phase bits of kfull / k4full
       auto issue_pv = [&](int jj) -> bool {
@@ -245,6 +252,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (; c.next(val, mask); ++i) {
           const int s = i % NST, buf = i & 1;
           const uint32_t prec = val >> 28;
+          if (prec == TRA_PREC_INT4 && !int4) {
+            *err = TRA_DEV_BAD_LIST;
+            ok = false;
+            break;
+          }
           if (prec == TRA_PREC_INT4) {
             ok = mbar_wait(bar_k4full(s), (k4ph >> s) & 1, err);
             k4ph ^= 1u << s;
@@ -290,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kPackedRow = D / 2;          // bytes per packed row
     constexpr int kChunksPerRow = kPackedRow / 16;
     bool ok = true;
-    if (MODE == TRA_POLICY_BOUNDARY) {
+    if (int4) {
       // Q: 128 rows (two q-tiles); rows of a missing second q-tile stay zero
       const uint8_t* src = p.q4 + (long long)row0 * kTile * kPackedRow;
       const int rows = has_second ? 128 : 64;
@@ -340,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_valid = half_valid && tq < T;
     const long long qtile = (long long)h * p.ntiles + toff + qt;
     const float sq8 = half_valid ? __ldg(p.sq8 + qtile) : 0.0f;
-    const float sq4 = (half_valid && MODE == TRA_POLICY_BOUNDARY) ? __ldg(p.sq4 + qtile) : 0.0f;
+    const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) : 0.0f;
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     uint8_t* const prow = gbase + C::kOffP + r * 128;
     float m_run = -INFINITY, l_run = 0.0f;
@@ -366,6 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       const uint32_t prec = val >> 28;
       const int kt = (int)(val & 0x0FFFFFFFu);
+      if (prec == TRA_PREC_INT4 && !int4) {
+        *err = TRA_DEV_BAD_LIST;
+        ok = false;
+        break;
+      }
       const bool applies = ((mask >> half) & 1) && row_valid;
       if (p.n_dump > 0 && applies && prec != TRA_PREC_BF16) {
         for (int di = 0; di < p.n_dump; ++di) {

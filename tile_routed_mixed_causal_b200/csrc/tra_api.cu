@@ -339,6 +339,7 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
   p.d = shape->d;
   p.ntiles = (int)nt;
   p.mode = policy->mode;
+  p.has_int4 = policy_has_int4(shape, policy) ? 1 : 0;
   p.jmax = (int)((nt_max + 1) / 2);
   p.row_ptr = row_ptr;
   p.entries = entries;

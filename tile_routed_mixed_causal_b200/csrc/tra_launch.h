@@ -49,6 +49,7 @@ struct PrefillParams {
   const int32_t* cu;
   int B, Hq, Hkv, d, ntiles;
   int mode;              // TRA_POLICY_*
+  int has_int4;          // Q4/K4 tiles present (boundary policies with some b1 < b2)
   int jmax;              // max over sequences of ceil(nt/2) (q-tile pairs)
   const int32_t* row_ptr;
   const uint32_t* entries;
