@@ -250,6 +250,40 @@ TRA_API tra_status routed_attention_decode(const tra_shape* prefill_shape, const
                                    uint16_t* out, void* workspace, size_t workspace_bytes,
                                    int32_t* status_dev, void* stream);
 
+/*
+ * routed_attention_decode_noalloc -- the same decode step as
+ * routed_attention_decode, for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a deployment convenience of this
+ * library.  Some callers only ever receive input and output buffers -- a
+ * custom operator or plugin inside a host framework that owns every device
+ * allocation and hands out no allocator, or a serving loop that reserved all
+ * of its device memory up front and must not allocate while it decodes -- so
+ * they cannot provide the workspace the regular entry point needs.  This entry
+ * point keeps that scratch in a fixed array of TRA_NOALLOC_SCRATCH_BYTES bytes
+ * inside the library instead: every GPU that loads the library holds the
+ * array until the process exits.  It calls no allocator of any kind.
+ * Arguments, layouts, device status bits and validation are those of
+ * routed_attention_decode, minus workspace/workspace_bytes.
+ * Limits and rules:
+ *  - problems needing more than TRA_NOALLOC_SCRATCH_BYTES of scratch
+ *    (tra_decode_workspace_bytes(B, Hq, Hkv, d)) are rejected with
+ *    TRA_ERR_UNSUPPORTED;
+ *  - the first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture;
+ *  - all calls on a device share the one array, which keeps whatever the last
+ *    call left there; calls whose kernels overlap on the GPU (for example on
+ *    two streams at once) race on it and give wrong results, so issue them on
+ *    one stream or otherwise order them.  No part of the array needs to start
+ *    at zero.
+ */
+#define TRA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+TRA_API tra_status routed_attention_decode_noalloc(
+    const tra_shape* prefill_shape, const tra_policy* policy, const uint16_t* q,
+    const uint16_t* k_new, const uint16_t* v_new, const tra_qtiles* cache, const int32_t* row_ptr,
+    const uint32_t* entries, uint16_t* k_tail, uint16_t* v_tail, int32_t* tail_len_dev,
+    int32_t tail_cap, float softmax_scale, uint16_t* out, int32_t* status_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

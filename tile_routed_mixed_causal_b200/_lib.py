@@ -75,6 +75,7 @@ def load():
         "routed_attention_prefill": ([P, P, P, P, P, P, P, P, F, P, P, P, I32, P, P, P], I32),
         "tra_decode_workspace_bytes": ([I32, I32, I32, I32], SZ),
         "routed_attention_decode": ([P, P, P, P, P, P, P, P, P, P, P, I32, F, P, P, SZ, P, P], I32),
+        "routed_attention_decode_noalloc": ([P, P, P, P, P, P, P, P, P, P, P, I32, F, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -240,3 +241,13 @@ def routed_attention_decode(shape: Shape, policy: Policy, q, k_new, v_new, cache
         _ptr(entries), _ptr(k_tail), _ptr(v_tail), _ptr(tail_len), int(k_tail.shape[2]),
         float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(status), _stream(stream)))
+
+
+def routed_attention_decode_noalloc(shape: Shape, policy: Policy, q, k_new, v_new, cache: QTiles,
+                                    row_ptr, entries, k_tail, v_tail, tail_len, softmax_scale, out,
+                                    status, stream=None):
+    """Decode step without a caller workspace (the library's fixed scratch array is used)."""
+    _check(load().routed_attention_decode_noalloc(
+        shape.c, policy.c, _ptr(q), _ptr(k_new), _ptr(v_new), cache.c, _ptr(row_ptr),
+        _ptr(entries), _ptr(k_tail), _ptr(v_tail), _ptr(tail_len), int(k_tail.shape[2]),
+        float(softmax_scale), _ptr(out), _ptr(status), _stream(stream)))

@@ -146,6 +146,10 @@ tra_status cuda_fail(cudaError_t e, const char* what) {
 
 }  // namespace
 
+namespace tra {
+tra_status report_error(tra_status st, const char* msg) { return fail(st, "%s", msg); }
+}  // namespace tra
+
 extern "C" {
 
 const char* tra_last_error(void) { return g_last_error.c_str(); }

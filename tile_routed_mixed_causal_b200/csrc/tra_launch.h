@@ -104,6 +104,9 @@ struct DecodeParams {
 };
 
 int decode_splits(int B, int Hkv);
+
+// Records `msg` as this thread's tra_last_error() text and returns `st`.
+tra_status report_error(tra_status st, const char* msg);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 
 }  // namespace tra
