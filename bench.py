@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one part only (used for profiler captures); prints a reduced line")
     return ap.parse_args()
 
 
@@ -387,7 +389,20 @@ def main():
     device = torch.device("cuda", local if world > 1 else 0)
     bf16_tflops, hbm_gbs, peak_src = load_peaks()
     stream = torch.cuda.Stream(device)
+    if args.only == "decode":
+        if rank == 0:
+            print(json.dumps({"only": "decode", **decode_bench(device, args.decode_passes, stream,
+                                                              hbm_gbs)}), flush=True)
+        return
     S = prefill_setup(device)
+    if args.only == "prefill":
+        total_ms, attn_ms, _ = run_prefill_bench(S, args.steps, args.warmup, stream)
+        if rank == 0:
+            ops = prefill_ops(S)
+            print(json.dumps({"only": "prefill", "ms_per_step": total_ms / args.steps,
+                              "prefill_kernel_ms": sum(attn_ms) / len(attn_ms),
+                              "TOPS": ops / (total_ms / args.steps * 1e-3) / 1e12}), flush=True)
+        return
     ops = prefill_ops(S)
 
     clocks = ClockSampler(local if world > 1 else 0)

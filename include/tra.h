@@ -153,8 +153,8 @@ TRA_API size_t tra_qtiles_bytes(const tra_shape* shape, uint32_t formats);
 
 /*
  * quantize_qkv_tiles -- per-(head, 64-token tile) symmetric INT8/INT4
- * quantisation of Q, K and V ("quantized keys and values prepared during
- * prefill", TriAttention abstract; INT8 tiles, TileMix abstract).
+ * quantisation of Q, K and V (TriAttention abstract: the prefill prepares
+ * quantised keys and values; TileMix abstract: INT8 tiles and K/V caches).
  * q/k/v: device bf16 [ntok][H][d]; a tensor may be NULL when `out->formats`
  * requests none of its formats.  Writes the codes and scales selected by
  * out->formats (layouts above).  Deterministic and bit-exact with the rule in
@@ -174,10 +174,10 @@ TRA_API tra_status tra_tile_lists_size(const tra_shape* shape, const tra_policy*
                                int32_t list_kind, int64_t* rows, int64_t* nnz);
 
 /*
- * build_tile_lists -- precision-grouped traversals ("the selected boundaries
- * generate precision-grouped traversals", TriAttention abstract; "packs routing
- * decisions into compact bitmasks ... each routing bit govern multiple adjacent
- * key tiles", TileMix abstract).
+ * build_tile_lists -- precision-grouped traversals (TriAttention abstract:
+ * each head's two boundaries are turned into traversals grouped by precision;
+ * TileMix abstract: routing decisions are packed into bitmasks in which one
+ * bit governs several adjacent key tiles).
  * Prefill rows (h, q-tile): boundary mode lists INT4 k-tiles
  * [max(0,qt-b2+1), qt-b1] then INT8 [max(0,qt-b1+1), qt]; bitmask mode lists
  * the INT8 k-tiles <= qt then the BF16 ones.  Decode-cache rows (b, kv-head):
@@ -195,10 +195,11 @@ TRA_API tra_status build_tile_lists(const tra_shape* shape, const tra_policy* po
  * precision-grouped traversal: every listed tile's scores come from its
  * precision (INT8 or INT4 codes multiplied exactly in int32 and rescaled by
  * sQ*sK, or BF16 with fp32 accumulation); every path updates one online
- * softmax state per query row; P*V uses bf16 P and the original bf16 V
- * (TriAttention abstract: "combines contributions from both QK precisions into
- * one normalized attention output"; TileMix abstract: "both paths update a
- * shared online-softmax state").
+ * softmax state per query row; P*V uses bf16 P and the original bf16 V.
+ * (TriAttention abstract: one fused kernel skips the omitted tiles and merges
+ * the contributions of both QK precisions into a single normalised output;
+ * TileMix abstract: the high- and low-precision paths share one online-softmax
+ * state.)
  * q/k/v: device bf16 as above; tiles: output of quantize_qkv_tiles (Q8/K8
  * always, Q4/K4 when the policy has INT4 tiles); row_ptr/entries: prefill
  * lists; out: device bf16 [ntok][Hq][d]; lse: device float [Hq][ntok] natural-
@@ -221,10 +222,10 @@ TRA_API size_t tra_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, in
 
 /*
  * routed_attention_decode -- one decode step over the compressed KV cache
- * ("the quantized keys and values prepared during prefill are then reused in a
- * compressed key-value (KV) cache for decoding", TriAttention abstract;
- * "Dequantization is fused with attention computation", HyQuant, "How HyQuant
- * works").  For each sequence b: the new token's k_new/v_new [b][kvh] is
+ * (TriAttention abstract: the K/V quantised during prefill are reused as a
+ * compressed KV cache when decoding, so the prompt is not re-read at full
+ * precision; HyQuant, "How HyQuant works": dequantisation happens inside the
+ * attention kernel).  For each sequence b: the new token's k_new/v_new [b][kvh] is
  * appended at tail position tail_len[b]; every query head attends to the
  * cached tiles listed for (b, kv-head) -- K = sK*code and V = sV*code in the
  * tile's cached format -- plus the bf16 tail tokens [0, tail_len[b]] ; one

@@ -1,8 +1,8 @@
-// decode.cu -- one decode step over the compressed KV cache ("The quantized
-// keys and values prepared during prefill are then reused in a compressed
-// key-value (KV) cache for decoding, reducing repeated reads of prompt data",
-// TriAttention abstract; "Dequantization is fused with attention computation to
-// reduce extra memory traffic", HyQuant, "How HyQuant works").
+// decode.cu -- one decode step over the compressed KV cache (TriAttention
+// abstract: the K/V quantised during prefill become a compressed KV cache for
+// decoding, which cuts the re-reading of the prompt; HyQuant, "How HyQuant
+// works": dequantisation is done inside the attention kernel so it costs no
+// extra memory pass).
 //
 // Split-K over the cached tiles of each (sequence, KV head): CTA (split, kvh, b)
 // streams its share of the kept INT8/INT4 K/V tiles through a 4-deep ring of

@@ -1,7 +1,7 @@
-// lists.cu -- precision-grouped traversal lists ("the selected boundaries
-// generate precision-grouped traversals", TriAttention abstract; "packs routing
-// decisions into compact bitmasks" with one bit per group of adjacent key
-// tiles, TileMix abstract).
+// lists.cu -- precision-grouped traversal lists (TriAttention abstract: the
+// per-head boundaries are expanded into traversals grouped by precision;
+// TileMix abstract: routing bits packed into bitmasks, one bit per group of
+// adjacent key tiles).
 //
 // One warp per CSR row.  Row lengths have closed forms in every mode (boundary
 // rows keep min(qt+1, b2) tiles, bitmask rows keep all qt+1 causal tiles,

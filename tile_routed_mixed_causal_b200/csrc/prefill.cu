@@ -1,9 +1,8 @@
 // prefill.cu -- fused causal prefill attention over precision-grouped tile
-// traversals ("a fused kernel that skips omitted tiles and combines
-// contributions from both QK precisions into one normalized attention output",
-// TriAttention abstract; "dispatches each tile group through FP16 or INT8 score
-// computation while both paths update a shared online-softmax state", TileMix
-// abstract).
+// traversals (TriAttention abstract: one fused kernel skips omitted tiles and
+// merges both QK precisions into a single normalised output; TileMix abstract:
+// each tile group goes through a high-precision or an INT8 score path and both
+// paths update the same online-softmax state).
 //
 // Work unit: one query head h of one sequence b and one pair of q-tiles
 // (2j, 2j+1) = 128 query rows, the M of one tcgen05 MMA.  The two rows' CSR

@@ -1,6 +1,6 @@
 // quantize.cu -- per-(head, 64-token tile) symmetric INT8/INT4 quantisation of
-// Q, K and V ("The quantized keys and values prepared during prefill",
-// TriAttention abstract; INT8 tiles and INT8 K/V caches, TileMix abstract).
+// Q, K and V (TriAttention abstract: the prefill prepares quantised keys and
+// values; TileMix abstract: INT8 score tiles and INT8 K/V caches).
 //
 // One CTA per (tensor, head, tile): the 64 x d bf16 tile is read once with
 // 16-byte loads into registers, the absolute maximum is reduced with warp
