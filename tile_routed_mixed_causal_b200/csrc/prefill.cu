@@ -11,48 +11,58 @@
 // only one q-tile's list (or with a different precision) is computed for all
 // 128 rows and masked to -inf in the other half, so routing stays exact.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer: Q tiles once, then K (INT8 codes or BF16) and V
-//               (BF16) tiles into an NST-deep ring;
+// Two work units share one CTA (384 threads) so that one unit's softmax runs
+// while the tensor core works on the other's tiles:
+//   warp 0      TMA producer: both units' Q tiles once, then K (INT8 codes or
+//               BF16) and V (BF16) tiles into one NST-deep ring, in the
+//               interleaved order of the two units' traversals;
 //   warp 1      TMEM owner and MMA issuer: S = Q K^T with kind::i8 (INT8/INT4,
-//               exact int32) or kind::f16 (BF16, fp32) into a double-buffered S
-//               in TMEM, then O += P V (bf16) into TMEM;
+//               exact int32) or kind::f16 (BF16, fp32) into the unit's S in
+//               TMEM, then O += P V with P read from TMEM (bf16) and V from
+//               shared memory;
 //   warps 2-3   INT4 expanders: packed INT4 codes (Q once, K per INT4 entry)
 //               sign-extended to int8 in the swizzled operand layout (tcgen05
 //               has no integer 4-bit MMA, so INT4 tiles run as int8 MMAs);
-//   warps 4-7   softmax / epilogue: one thread per query row (TMEM lane):
-//               S -> scaled log2 scores -> mask -> online softmax with lazy
-//               rescaling of O -> bf16 P in shared memory; finally O / l.
+//   warps 4-7   softmax / epilogue of unit 0, warps 8-11 of unit 1: one thread
+//               per query row (TMEM lane): S -> log2-domain scores -> mask ->
+//               online softmax with lazy rescaling of O -> bf16 P into TMEM;
+//               finally O / l.
 #include "tra_device.cuh"
 #include "tra_launch.h"
 
 namespace tra {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+constexpr int kUnits = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 2^8 growth
+constexpr int kSmemLimit = 232448;         // max dynamic shared memory per CTA on sm_100
 
 template <int D, int MODE>
 struct Cfg {
-  static constexpr int kStages = 4;
   static constexpr int kQ8Bytes = 128 * D;                                    // int8 Q codes
   static constexpr int kQxBytes = MODE == TRA_POLICY_BITMASK ? 128 * D * 2 : 128 * D;
+  static constexpr int kQUnitBytes = kQ8Bytes + kQxBytes;
   static constexpr int kKBytes = 64 * D * 2;                                  // slot fits bf16
   static constexpr int kVBytes = 64 * D * 2;
-  static constexpr int kPBytes = 128 * 64 * 2;
-  static constexpr int kOffQ8 = 0;
-  static constexpr int kOffQx = kOffQ8 + kQ8Bytes;
-  static constexpr int kOffK = kOffQx + kQxBytes;
+  static constexpr int kFixed = kUnits * kQUnitBytes + 2048;                  // + barriers, slack
+  static constexpr int kStagesFit = (kSmemLimit - kFixed) / (kKBytes + kVBytes);
+  static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
+  static_assert(kStages >= 3, "shared memory too small for the K/V ring");
+  static constexpr int kOffQ = 0;                                             // unit u at u * kQUnitBytes
+  static constexpr int kOffK = kUnits * kQUnitBytes;
   static constexpr int kOffV = kOffK + kStages * kKBytes;
-  static constexpr int kOffP = kOffV + kStages * kVBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;
-  static constexpr int kNumBars = 2 + 5 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kOffBar = kOffV + kStages * kVBytes;
+  static constexpr int kNumBars = 2 + 5 * kStages + 4 * kUnits + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
   // int8 K-major rows of D bytes: 128-byte swizzle for D = 128, 64-byte for D = 64
   static constexpr uint32_t kI8Layout = D == 128 ? kSwz128 : kSwz64;
   static constexpr uint32_t kI8Sbo = D == 128 ? 1024 : 512;
   static constexpr int kSlabs = D / 64;  // bf16 64-element (128-byte) slabs per row
+  // TMEM columns of unit u: S at u*256, P (bf16 pairs) at u*256+64, O at u*256+128
+  static constexpr uint32_t kTmemCols = 512;
 };
 
 // Byte offset of 16-byte chunk `c` of row `r` in a swizzled K-major int8 tile.
@@ -68,6 +78,7 @@ __device__ __forceinline__ uint32_t i8_swz_offset(int r, int c) {
 struct MergeCursor {
   const uint32_t* e;
   int p0, e0, p1, e1;
+  __device__ __forceinline__ bool more() const { return p0 < e0 || p1 < e1; }
   __device__ __forceinline__ bool next(uint32_t& val, int& mask) {
     const uint32_t a = p0 < e0 ? __ldg(e + p0) : 0xFFFFFFFFu;
     const uint32_t b = p1 < e1 ? __ldg(e + p1) : 0xFFFFFFFFu;
@@ -83,10 +94,86 @@ struct MergeCursor {
   }
 };
 
+// Interleaving of the two units' traversals: alternate while both have
+// entries, then drain the other.  Every role that walks the shared ring
+// replays the same sequence.  (Two named cursors, so that nothing is indexed
+// at run time and the state stays in registers.)
+struct Schedule {
+  MergeCursor c0, c1;
+  int turn;
+  __device__ __forceinline__ bool next(int& u, uint32_t& val, int& mask) {
+    if (turn == 0) {
+      if (c0.next(val, mask)) { u = 0; turn = 1; return true; }
+      if (c1.next(val, mask)) { u = 1; return true; }
+    } else {
+      if (c1.next(val, mask)) { u = 1; turn = 0; return true; }
+      if (c0.next(val, mask)) { u = 0; return true; }
+    }
+    return false;
+  }
+  __device__ __forceinline__ bool more(int u) const { return u ? c1.more() : c0.more(); }
+};
+
+// One work unit: query head h of sequence b, q-tiles (2j, 2j+1).
+struct Unit {
+  bool valid, has_second;
+  int h, b, kvh, qt0, nt, T, seq0, toff, row0;
+};
+
+// Unit `id` in launch order: heaviest q-tile pairs (largest j) first, heads fastest.
+__device__ __forceinline__ Unit make_unit(const PrefillParams& p, long long id) {
+  Unit x;
+  const long long total = (long long)p.jmax * p.B * p.Hq;
+  x.h = (int)(id % p.Hq);
+  x.b = (int)((id / p.Hq) % p.B);
+  x.kvh = x.h / (p.Hq / p.Hkv);
+  x.qt0 = 2 * (p.jmax - 1 - (int)(id / ((long long)p.Hq * p.B)));
+  x.valid = false;
+  x.seq0 = x.T = x.nt = x.toff = x.row0 = 0;
+  x.has_second = false;
+  if (id < total) {
+    x.seq0 = __ldg(p.cu + x.b);
+    x.T = __ldg(p.cu + x.b + 1) - x.seq0;
+    x.nt = (x.T + kTile - 1) / kTile;
+    x.valid = x.qt0 < x.nt;
+  }
+  if (x.valid) {
+    x.toff = seq_tile_offset(p.cu, x.b);
+    x.has_second = x.qt0 + 1 < x.nt;
+    x.row0 = x.h * p.ntiles + x.toff + x.qt0;
+  }
+  return x;
+}
+
+__device__ __forceinline__ MergeCursor unit_cursor(const PrefillParams& p, const Unit& x) {
+  MergeCursor c;
+  c.e = p.entries;
+  if (x.valid) {
+    c.p0 = __ldg(p.row_ptr + x.row0);
+    c.e0 = __ldg(p.row_ptr + x.row0 + 1);
+    c.p1 = c.e0;
+    c.e1 = x.has_second ? __ldg(p.row_ptr + x.row0 + 2) : c.e0;
+  } else {
+    c.p0 = c.e0 = c.p1 = c.e1 = 0;
+  }
+  return c;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// O += P V with the 128 x 16 bf16 A operand (P) read from TMEM.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 template <int D, int MODE>
@@ -96,30 +183,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NST = C::kStages;
   extern __shared__ uint8_t smem_raw[];
 
-  // ---- work unit: heaviest q-tile pairs first, heads fastest
-  const int h = blockIdx.x % p.Hq;
-  const int b = (blockIdx.x / p.Hq) % p.B;
-  const int j = p.jmax - 1 - (int)(blockIdx.x / (p.Hq * p.B));
-  const int seq0 = __ldg(p.cu + b);
-  const int T = __ldg(p.cu + b + 1) - seq0;
-  const int nt = (T + kTile - 1) / kTile;
-  if (2 * j >= nt) return;  // uniform exit, before any barrier or TMEM use
-  const int toff = seq_tile_offset(p.cu, b);
-  const int grp = p.Hq / p.Hkv;
-  const int kvh = h / grp;
-  const int qt0 = 2 * j;
-  const bool has_second = qt0 + 1 < nt;
+  // ---- the CTA's two work units
+  const Unit un0 = make_unit(p, (long long)blockIdx.x * kUnits);
+  const Unit un1 = make_unit(p, (long long)blockIdx.x * kUnits + 1);
+  if (!un0.valid && !un1.valid) return;  // uniform exit, before any barrier or TMEM use
   // INT4 operands exist only for boundary policies with an INT4 region; a list
   // entry asking for INT4 without them is reported, never read
   const bool int4 = MODE == TRA_POLICY_BOUNDARY && p.has_int4;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (base - smem_u32(smem_raw));
-  const uint32_t sQ8 = base + C::kOffQ8;
-  const uint32_t sQx = base + C::kOffQx;
+  auto sQ8 = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes; };
+  auto sQx = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes; };
   const uint32_t sK = base + C::kOffK;
   const uint32_t sV = base + C::kOffV;
-  const uint32_t sP = base + C::kOffP;
   const uint32_t bars = base + C::kOffBar;
   const uint32_t bar_q = bars + 0 * 8;
   const uint32_t bar_q4 = bars + 1 * 8;
@@ -128,11 +205,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_kfree = [&](int s) { return bars + (2 + 2 * NST + s) * 8; };
   auto bar_vfull = [&](int s) { return bars + (2 + 3 * NST + s) * 8; };
   auto bar_vfree = [&](int s) { return bars + (2 + 4 * NST + s) * 8; };
-  auto bar_sfull = [&](int s) { return bars + (2 + 5 * NST + s) * 8; };
-  auto bar_sfree = [&](int s) { return bars + (4 + 5 * NST + s) * 8; };
-  const uint32_t bar_pfull = bars + (6 + 5 * NST) * 8;
-  const uint32_t bar_ofull = bars + (7 + 5 * NST) * 8;
-  const uint32_t bar_done = bars + (8 + 5 * NST) * 8;
+  auto bar_sfull = [&](int u) { return bars + (2 + 5 * NST + 4 * u + 0) * 8; };
+  auto bar_sfree = [&](int u) { return bars + (2 + 5 * NST + 4 * u + 1) * 8; };
+  auto bar_pfull = [&](int u) { return bars + (2 + 5 * NST + 4 * u + 2) * 8; };
+  auto bar_ofull = [&](int u) { return bars + (2 + 5 * NST + 4 * u + 3) * 8; };
+  const uint32_t bar_done = bars + (2 + 5 * NST + 4 * kUnits) * 8;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kOffMisc);
   volatile int* const err = reinterpret_cast<volatile int*>(gbase + C::kOffMisc + 16);
 
@@ -149,18 +226,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_vfull(s), 1);
       mbar_init(bar_vfree(s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_sfull(s), 1);
-      mbar_init(bar_sfree(s), 128);
+    for (int u = 0; u < kUnits; ++u) {
+      mbar_init(bar_sfull(u), 1);
+      mbar_init(bar_sfree(u), 128);
+      mbar_init(bar_pfull(u), 128);
+      mbar_init(bar_ofull(u), 1);
     }
-    mbar_init(bar_pfull, 128);
-    mbar_init(bar_ofull, 1);
     mbar_init(bar_done, 1);
     *err = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -168,31 +245,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int row0 = h * p.ntiles + toff + qt0;
-  MergeCursor cur0;
-  cur0.e = p.entries;
-  cur0.p0 = __ldg(p.row_ptr + row0);
-  cur0.e0 = __ldg(p.row_ptr + row0 + 1);
-  cur0.p1 = cur0.e0;
-  cur0.e1 = has_second ? __ldg(p.row_ptr + row0 + 2) : cur0.e0;
+  Schedule sched0;
+  sched0.turn = 0;
+  sched0.c0 = unit_cursor(p, un0);
+  sched0.c1 = unit_cursor(p, un1);
+#define TRA_UNIT_FIELD(u, f) ((u) ? un1.f : un0.f)
 
   if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
-      const uint32_t qbytes = C::kQ8Bytes + (MODE == TRA_POLICY_BITMASK ? 128 * D * 2 : 0);
-      mbar_arrive_expect_tx(bar_q, qbytes);
-      tma_load_2d(sQ8, &m.q8, bar_q, 0, row0 * kTile);
-      if (MODE == TRA_POLICY_BITMASK) {
-        for (int sl = 0; sl < C::kSlabs; ++sl)
-          tma_load_3d(sQx + sl * 128 * 128, &m.qb, bar_q, sl * 64, h, seq0 + qt0 * kTile);
+      constexpr uint32_t kQBytes = C::kQ8Bytes + (MODE == TRA_POLICY_BITMASK ? 128 * D * 2 : 0);
+      mbar_arrive_expect_tx(bar_q, (un0.valid ? kQBytes : 0u) + (un1.valid ? kQBytes : 0u));
+      for (int u = 0; u < kUnits; ++u) {
+        const Unit x = u ? un1 : un0;
+        if (!x.valid) continue;
+        tma_load_2d(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
+        if (MODE == TRA_POLICY_BITMASK) {
+          for (int sl = 0; sl < C::kSlabs; ++sl)
+            tma_load_3d(sQx(u) + sl * 128 * 128, &m.qb, bar_q, sl * 64, x.h,
+                        x.seq0 + x.qt0 * kTile);
+        }
       }
-      MergeCursor c = cur0;
+      Schedule sc = sched0;
       uint32_t val;
-      int mask;
-      for (int i = 0; c.next(val, mask); ++i) {
-        const int s = i % NST, use = i / NST;
+      int mask, u;
+      for (int g = 0; sc.next(u, val, mask); ++g) {
+        const int s = g % NST, use = g / NST;
         const uint32_t prec = val >> 28;
         const int kt = (int)(val & 0x0FFFFFFFu);
+        const int kvh = TRA_UNIT_FIELD(u, kvh), toff = TRA_UNIT_FIELD(u, toff);
+        const int seq0 = TRA_UNIT_FIELD(u, seq0);
         if (prec == TRA_PREC_INT4 && !int4) {
           *err = TRA_DEV_BAD_LIST;
           break;
@@ -206,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             mbar_arrive_expect_tx(bar_kfull(s), 64 * D * 2);
             for (int sl = 0; sl < C::kSlabs; ++sl)
-              tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(s), sl * 64, kvh, seq0 + kt * kTile);
+              tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(s), sl * 64, kvh,
+                          seq0 + kt * kTile);
           }
         }
         if (use > 0 && !mbar_wait(bar_vfree(s), (use - 1) & 1, err)) break;
@@ -222,34 +305,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdI8 = instr_desc(2, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdQK16 = instr_desc(1, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdPV = instr_desc(1, 1, 0, 1, D, 128);
-      const uint32_t tS = tmem, tO = tmem + 128;
       bool ok = mbar_wait(bar_q, 0, err);
       if (ok && int4) ok = mbar_wait(bar_q4, 0, err);
       tc_fence_after();
-      uint32_t kph = 0, k4ph = 0;  // per-slot phase bits of kfull / k4full
-      auto issue_pv = [&](int jj) -> bool {
-        const int s = jj % NST;
-        if (!mbar_wait(bar_pfull, jj & 1, err)) return false;
-        if (!mbar_wait(bar_vfull(s), (jj / NST) & 1, err)) return false;
+      uint32_t kph = 0, k4ph = 0;       // per-slot phase bits of kfull / k4full
+      // per unit: entries whose QK was issued (negative once its last PV is
+      // issued), and the ring slot / schedule step of its pending P V
+      int cnt0 = 0, cnt1 = 0, pslot0 = 0, pslot1 = 0, pg0 = 0, pg1 = 0;
+      // O_u += P_u(idx) V(slot); P from TMEM, V (MN-major) from shared memory
+      auto issue_pv = [&](int u, int idx, int slot, int gg) -> bool {
+        if (!mbar_wait(bar_pfull(u), idx & 1, err)) return false;
+        if (!mbar_wait(bar_vfull(slot), (gg / NST) & 1, err)) return false;
         tc_fence_after();
-        const uint32_t vb = sV + s * C::kVBytes;
+        const uint32_t vb = sV + slot * C::kVBytes;
+        const uint32_t tO = tmem + u * 256 + 128, tP = tmem + u * 256 + 64;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = smem_desc(sP + kk * 32, 16, 1024, kSwz128);
           const uint64_t bd = smem_desc(vb + kk * 2048, 64 * 128, 1024, kSwz128);
-          mma_bf16(tO, a, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tO, tP + kk * 8, bd, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar_ofull);
-        mma_commit(bar_vfree(s));
+        mma_commit(bar_ofull(u));
+        mma_commit(bar_vfree(slot));
         return true;
       };
-      int i = 0;
       if (ok) {
-        MergeCursor c = cur0;
+        Schedule sc = sched0;
         uint32_t val;
-        int mask;
-        for (; c.next(val, mask); ++i) {
-          const int s = i % NST, buf = i & 1;
+        int mask, u;
+        for (int g = 0; sc.next(u, val, mask); ++g) {
+          const int s = g % NST;
           const uint32_t prec = val >> 28;
           if (prec == TRA_PREC_INT4 && !int4) {
             *err = TRA_DEV_BAD_LIST;
@@ -263,21 +347,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait(bar_kfull(s), (kph >> s) & 1, err);
             kph ^= 1u << s;
           }
-          if (ok && i >= 2) ok = mbar_wait(bar_sfree(buf), ((i >> 1) - 1) & 1, err);
+          const int i = u ? cnt1 : cnt0;
+          if (ok && i >= 1) ok = mbar_wait(bar_sfree(u), (i - 1) & 1, err);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kb = sK + s * C::kKBytes;
-          const uint32_t dS = tS + buf * 64;
+          const uint32_t dS = tmem + u * 256;
           if (prec == TRA_PREC_BF16) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const int sl = kk >> 2, off = (kk & 3) * 32;
-              const uint64_t a = smem_desc(sQx + sl * 128 * 128 + off, 16, 1024, kSwz128);
+              const uint64_t a = smem_desc(sQx(u) + sl * 128 * 128 + off, 16, 1024, kSwz128);
               const uint64_t bd = smem_desc(kb + sl * 64 * 128 + off, 16, 1024, kSwz128);
               mma_bf16(dS, a, bd, kIdQK16, kk > 0 ? 1u : 0u);
             }
           } else {
-            const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8 : sQx;
+            const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(u) : sQx(u);
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk) {
               const uint64_t a = smem_desc(qa + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
@@ -285,11 +370,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_i8(dS, a, bd, kIdI8, kk > 0 ? 1u : 0u);
             }
           }
-          mma_commit(bar_sfull(buf));
+          mma_commit(bar_sfull(u));
           mma_commit(bar_kfree(s));
-          if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+          if (i >= 1 && !issue_pv(u, i - 1, u ? pslot1 : pslot0, u ? pg1 : pg0)) { ok = false; break; }
+          int ncnt = i + 1;
+          // a unit with no entries left releases its last V slot now, so the
+          // other unit's loads can keep using the ring
+          if (!sc.more(u)) {
+            if (!issue_pv(u, i, s, g)) { ok = false; break; }
+            ncnt = -1;  // done: the P V of every entry has been issued
+          }
+          if (u) { cnt1 = ncnt; pslot1 = s; pg1 = g; } else { cnt0 = ncnt; pslot0 = s; pg0 = g; }
         }
-        if (ok && i >= 1) issue_pv(i - 1);
+        if (ok && cnt0 > 0 && !issue_pv(0, cnt0 - 1, pslot0, pg0)) ok = false;
+        if (ok && cnt1 > 0 && !issue_pv(1, cnt1 - 1, pslot1, pg1)) ok = false;
       }
       // all MMAs issued by this thread complete before TMEM is released
       mma_commit(bar_done);
@@ -300,32 +394,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = threadIdx.x - 64;  // 0..63
     constexpr int kPackedRow = D / 2;          // bytes per packed row
     constexpr int kChunksPerRow = kPackedRow / 16;
-    bool ok = true;
     if (int4) {
-      // Q: 128 rows (two q-tiles); rows of a missing second q-tile stay zero
-      const uint8_t* src = p.q4 + (long long)row0 * kTile * kPackedRow;
-      const int rows = has_second ? 128 : 64;
-      for (int f = t; f < 128 * kChunksPerRow; f += 64) {
-        const int r = f / kChunksPerRow, c = f % kChunksPerRow;
-        uint4 w = make_uint4(0, 0, 0, 0);
-        if (r < rows) w = __ldg(reinterpret_cast<const uint4*>(src + r * kPackedRow + c * 16));
-        const uint2 e0 = expand_int4x8(w.x), e1 = expand_int4x8(w.y);
-        const uint2 e2 = expand_int4x8(w.z), e3 = expand_int4x8(w.w);
-        uint8_t* dst = gbase + C::kOffQx;
-        *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * c)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
-        *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * c + 1)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+      // Q: 128 rows (two q-tiles) per unit; rows of a missing q-tile stay zero
+      for (int u = 0; u < kUnits; ++u) {
+        const Unit x = u ? un1 : un0;
+        if (!x.valid) continue;
+        const uint8_t* src = p.q4 + (long long)x.row0 * kTile * kPackedRow;
+        const int rows = x.has_second ? 128 : 64;
+        uint8_t* dst = gbase + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes;
+        for (int f = t; f < 128 * kChunksPerRow; f += 64) {
+          const int r = f / kChunksPerRow, c = f % kChunksPerRow;
+          uint4 w = make_uint4(0, 0, 0, 0);
+          if (r < rows) w = __ldg(reinterpret_cast<const uint4*>(src + r * kPackedRow + c * 16));
+          const uint2 e0 = expand_int4x8(w.x), e1 = expand_int4x8(w.y);
+          const uint2 e2 = expand_int4x8(w.z), e3 = expand_int4x8(w.w);
+          *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * c)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+          *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * c + 1)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(bar_q4);
-      MergeCursor c = cur0;
+      Schedule sc = sched0;
       uint32_t val;
-      int mask;
-      for (int i = 0; c.next(val, mask); ++i) {
+      int mask, u;
+      for (int g = 0; sc.next(u, val, mask); ++g) {
         if ((val >> 28) != TRA_PREC_INT4) continue;
-        const int s = i % NST, use = i / NST;
-        if (use > 0 && !mbar_wait(bar_kfree(s), (use - 1) & 1, err)) { ok = false; break; }
+        const int s = g % NST, use = g / NST;
+        if (use > 0 && !mbar_wait(bar_kfree(s), (use - 1) & 1, err)) break;
         const int kt = (int)(val & 0x0FFFFFFFu);
-        const uint8_t* ks = p.k4 + ((long long)(kvh * p.ntiles + toff + kt) * kTile) * kPackedRow;
+        const uint8_t* ks = p.k4 + ((long long)(TRA_UNIT_FIELD(u, kvh) * p.ntiles +
+                                                TRA_UNIT_FIELD(u, toff) + kt) * kTile) * kPackedRow;
         uint8_t* dst = gbase + C::kOffK + s * C::kKBytes;
         for (int f = t; f < 64 * kChunksPerRow; f += 64) {
           const int r = f / kChunksPerRow, cc = f % kChunksPerRow;
@@ -339,42 +437,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar_k4full(s));
       }
     }
-    (void)ok;
   } else {
     // ================================================================ softmax / epilogue
-    const int r = threadIdx.x - 128;       // query row of the unit = TMEM lane
-    const int q4 = warp & 3;               // TMEM lane quarter of this warp
+    const int u = (warp - 4) >> 2;               // unit of this warpgroup
+    const Unit x = make_unit(p, (long long)blockIdx.x * kUnits + u);
+    const int r = (threadIdx.x - 128) & 127;     // query row of the unit = TMEM lane
+    const int q4 = warp & 3;                     // TMEM lane quarter of this warp
     const int half = r >> 6, rr = r & 63;
-    const int qt = qt0 + half;
-    const bool half_valid = qt < nt;
-    const int tq = qt * kTile + rr;        // query position in the sequence
-    const bool row_valid = half_valid && tq < T;
-    const long long qtile = (long long)h * p.ntiles + toff + qt;
+    const int qt = x.qt0 + half;
+    const bool half_valid = x.valid && qt < x.nt;
+    const int tq = qt * kTile + rr;              // query position in the sequence
+    const bool row_valid = half_valid && tq < x.T;
+    const long long qtile = (long long)x.h * p.ntiles + x.toff + qt;
     const float sq8 = half_valid ? __ldg(p.sq8 + qtile) : 0.0f;
     const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) : 0.0f;
-    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-    uint8_t* const prow = gbase + C::kOffP + r * 128;
+    const uint32_t lane_addr = ((uint32_t)(q4 * 32) << 16) + (uint32_t)(u * 256);
+    const uint32_t tS = tmem + lane_addr, tP = tS + 64, tO = tS + 128;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     int i = 0;
-    MergeCursor c = cur0;
+    MergeCursor c = unit_cursor(p, x);
     uint32_t val;
     int mask;
     for (; c.next(val, mask); ++i) {
-      const int buf = i & 1;
-      if (!mbar_wait(bar_sfull(buf), (i >> 1) & 1, err)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[64];
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        tmem_ld32(tmem + lane_addr + buf * 64, lo);
-        tmem_ld32(tmem + lane_addr + buf * 64 + 32, hi);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_sfree(buf));
-
+      if (!mbar_wait(bar_sfull(u), i & 1, err)) { ok = false; break; }
       const uint32_t prec = val >> 28;
       const int kt = (int)(val & 0x0FFFFFFFu);
       if (prec == TRA_PREC_INT4 && !int4) {
@@ -382,116 +468,159 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
-      const bool applies = ((mask >> half) & 1) && row_valid;
-      if (p.n_dump > 0 && applies && prec != TRA_PREC_BF16) {
-        for (int di = 0; di < p.n_dump; ++di) {
-          const int* dc = p.dump_coords + di * 4;
-          if (__ldg(dc) == b && __ldg(dc + 1) == h && __ldg(dc + 2) == qt && __ldg(dc + 3) == kt) {
-            int32_t* dst = p.dump_out + ((long long)di * 64 + rr) * 64;
-            for (int cc = 0; cc < 64; ++cc) dst[cc] = (int32_t)sr[cc];
+      // A half (64 rows = 2 warps) whose q-tile does not list this entry adds
+      // P = 0: its warps skip the TMEM read and every exponential.
+      const bool half_applies = ((mask >> half) & 1) && half_valid;
+      uint32_t pk[32];
+      bool warp_need = false;
+      float alpha = 1.0f;
+      if (!half_applies) {
+        tc_fence_before();
+        mbar_arrive(bar_sfree(u));
+#pragma unroll
+        for (int k = 0; k < 32; ++k) pk[k] = 0u;
+      } else {
+        tc_fence_after();
+        uint32_t sr[64];
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+          tmem_ld32(tS, lo);
+          tmem_ld32(tS + 32, hi);
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_sfree(u));
+        if (p.n_dump > 0 && row_valid && prec != TRA_PREC_BF16) {
+          for (int di = 0; di < p.n_dump; ++di) {
+            const int* dc = p.dump_coords + di * 4;
+            if (__ldg(dc) == x.b && __ldg(dc + 1) == x.h && __ldg(dc + 2) == qt &&
+                __ldg(dc + 3) == kt) {
+              int32_t* dst = p.dump_out + ((long long)di * 64 + rr) * 64;
+              for (int cc = 0; cc < 64; ++cc) dst[cc] = (int32_t)sr[cc];
+            }
           }
         }
-      }
-      const long long ktile = (long long)kvh * p.ntiles + toff + kt;
-      float f = p.scale_log2;
-      if (prec == TRA_PREC_INT8) f *= sq8 * __ldg(p.sk8 + ktile);
-      else if (prec == TRA_PREC_INT4) f *= sq4 * __ldg(p.sk4 + ktile);
-      // number of valid keys of this tile for this row (causal and sequence end)
-      int nvalid = 0;
-      if (applies) nvalid = min(min(tq - kt * kTile + 1, T - kt * kTile), kTile);
-      float s[64];
-      float m_tile = -INFINITY;
+        const long long ktile = (long long)x.kvh * p.ntiles + x.toff + kt;
+        float f = p.scale_log2;  // log2-domain score = raw * f
+        if (prec == TRA_PREC_INT8) f *= sq8 * __ldg(p.sk8 + ktile);
+        else if (prec == TRA_PREC_INT4) f *= sq4 * __ldg(p.sk4 + ktile);
+        // valid keys of this tile for this row (causal and sequence end); only the
+        // diagonal tile and a sequence's last tile have fewer than 64
+        const int nvalid =
+            row_valid ? min(min(tq - kt * kTile + 1, x.T - kt * kTile), kTile) : 0;
+        const bool full = __all_sync(0xffffffffu, nvalid >= kTile);
+        // raw scores as exact floats: BF16 accumulators are fp32 already; int32
+        // accumulators (|S| < 2^22) become floats by adding them to the bit
+        // pattern of 1.5*2^23 and subtracting that value (exact, no I2F)
+        float xs[64];
 #pragma unroll
-      for (int cc = 0; cc < 64; ++cc) {
-        const float raw = prec == TRA_PREC_BF16 ? __uint_as_float(sr[cc]) : (float)(int)sr[cc];
-        s[cc] = cc < nvalid ? raw * f : -INFINITY;
-        m_tile = fmaxf(m_tile, s[cc]);
-      }
-      const float m_new = fmaxf(m_run, m_tile);
-      const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
-      const bool warp_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.0f;
-      if (warp_need && m_new > m_run) {
-        alpha = ex2(m_run - m_new);  // m_run = -inf gives 0
-        m_run = m_new;
-      }
-      float l_tile = 0.0f;
-      uint32_t pk[32];
+        for (int cc = 0; cc < 64; ++cc)
+          xs[cc] = prec == TRA_PREC_BF16 ? __uint_as_float(sr[cc])
+                                         : __uint_as_float(sr[cc] + 0x4B400000u) - 12582912.0f;
+        if (!full) {
 #pragma unroll
-      for (int cc = 0; cc < 64; cc += 2) {
-        const float p0 = cc < nvalid ? ex2(s[cc] - m_run) : 0.0f;
-        const float p1 = cc + 1 < nvalid ? ex2(s[cc + 1] - m_run) : 0.0f;
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        const float2 pr = __bfloat1622float2(pb);
-        l_tile += pr.x + pr.y;
-        pk[cc >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
+          for (int cc = 0; cc < 64; ++cc) xs[cc] = cc < nvalid ? xs[cc] : -INFINITY;
+        }
+        float mx8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = xs[k];
+#pragma unroll
+        for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], xs[cc]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_tile = mx == -INFINITY ? -INFINITY : mx * f;  // f > 0 keeps the argmax
+        const float m_new = fmaxf(m_run, m_tile);
+        const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
+        warp_need = __any_sync(0xffffffffu, need);
+        if (warp_need && m_new > m_run) {
+          alpha = ex2(m_run - m_new);  // m_run = -inf gives 0
+          m_run = m_new;
+        }
+        float ls[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ls[k] = 0.0f;
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 2) {
+          float p0 = ex2(fmaf(xs[cc], f, -m_run));
+          float p1 = ex2(fmaf(xs[cc + 1], f, -m_run));
+          if (!full) {
+            p0 = cc < nvalid ? p0 : 0.0f;
+            p1 = cc + 1 < nvalid ? p1 : 0.0f;
+          }
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(&pb);
+          ls[(cc >> 1) & 7] += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+          pk[cc >> 1] = w;
+        }
+        const float l_tile = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        l_run = l_run * alpha + l_tile;
       }
-      l_run = l_run * alpha + l_tile;
       if (i > 0) {
-        if (!mbar_wait(bar_ofull, (i - 1) & 1, err)) { ok = false; break; }
+        // PV(i-1) must have read the previous P before it is overwritten, and
+        // must be complete before O is rescaled
+        if (!mbar_wait(bar_ofull(u), (i - 1) & 1, err)) { ok = false; break; }
         tc_fence_after();
         if (warp_need) {
 #pragma unroll 1
           for (int col = 0; col < D; col += 32) {
             uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + 128 + col, o);
+            tmem_ld32(tO + col, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tmem + lane_addr + 128 + col, o);
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(tO + col, o);
           }
-          tmem_wait_st();
         }
       }
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-      fence_proxy_async_smem();
+      tmem_st32(tP, pk);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_pfull);
+      mbar_arrive(bar_pfull(u));
     }
     // ---- epilogue: O / l
-    if (ok && i > 0 && mbar_wait(bar_ofull, (i - 1) & 1, err)) {
+    if (ok && i > 0 && mbar_wait(bar_ofull(u), (i - 1) & 1, err)) {
       tc_fence_after();
       const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-      uint16_t* orow = p.out + ((long long)(seq0 + tq) * p.Hq + h) * D;
+      uint16_t* orow = p.out + ((long long)(x.seq0 + tq) * p.Hq + x.h) * D;
 #pragma unroll 1
       for (int col = 0; col < D; col += 32) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_addr + 128 + col, o);
+        tmem_ld32(tO + col, o);
         tmem_wait_ld();
         if (row_valid) {
 #pragma unroll
-          for (int x = 0; x < 32; x += 8) {
+          for (int k = 0; k < 32; k += 8) {
             uint32_t w[4];
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
-              const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(o[x + 2 * y]) * inv,
-                                                              __uint_as_float(o[x + 2 * y + 1]) * inv);
+              const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(o[k + 2 * y]) * inv,
+                                                              __uint_as_float(o[k + 2 * y + 1]) * inv);
               w[y] = *reinterpret_cast<const uint32_t*>(&v2);
             }
-            *reinterpret_cast<uint4*>(orow + col + x) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(orow + col + k) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
       if (row_valid && p.lse)
-        p.lse[(long long)h * __ldg(p.cu + p.B) + seq0 + tq] =
+        p.lse[(long long)x.h * __ldg(p.cu + p.B) + x.seq0 + tq] =
             (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
   }
 
+#undef TRA_UNIT_FIELD
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
   if (threadIdx.x == 0 && *err) atomicOr(p.status, *err);
 }
 
 template <int D, int MODE>
 cudaError_t launch_one(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s) {
   using C = Cfg<D, MODE>;
-  const long long ctas = (long long)p.jmax * p.B * p.Hq;
+  const long long units = (long long)p.jmax * p.B * p.Hq;
+  const long long ctas = (units + kUnits - 1) / kUnits;
   if (ctas == 0) return cudaSuccess;
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, MODE>,
