@@ -11,29 +11,30 @@
 // only one q-tile's list (or with a different precision) is computed for all
 // 128 rows and masked to -inf in the other half, so routing stays exact.
 //
-// Two work units share one CTA (384 threads) so that one unit's softmax runs
+// Two work units share one CTA (416 threads) so that one unit's softmax runs
 // while the tensor core works on the other's tiles:
 //   warp 0      TMA producer: both units' Q tiles once, then K (INT8 codes or
 //               BF16) and V (BF16) tiles into one NST-deep ring, in the
 //               interleaved order of the two units' traversals;
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T with kind::i8 (INT8/INT4,
-//               exact int32) or kind::f16 (BF16, fp32) into the unit's S in
-//               TMEM, then O += P V with P read from TMEM (bf16) and V from
-//               shared memory;
+//   warps 1, 12 MMA issuers, one per unit (warp 1 also owns TMEM): S = Q K^T
+//               with kind::i8 (INT8/INT4, exact int32) or kind::f16 (BF16,
+//               fp32) into the unit's S in TMEM, then O += P V with P read
+//               from TMEM (bf16, double-buffered) and V from shared memory;
 //   warps 2-3   INT4 expanders: packed INT4 codes (Q once, K per INT4 entry)
 //               sign-extended to int8 in the swizzled operand layout (tcgen05
 //               has no integer 4-bit MMA, so INT4 tiles run as int8 MMAs);
 //   warps 4-7   softmax / epilogue of unit 0, warps 8-11 of unit 1: one thread
 //               per query row (TMEM lane): S -> log2-domain scores -> mask ->
 //               online softmax with lazy rescaling of O -> bf16 P into TMEM;
-//               finally O / l.
+//               finally O / l.  P is double-buffered so that P(i+1) can be
+//               written while P V of entry i is still running.
 #include "tra_device.cuh"
 #include "tra_launch.h"
 
 namespace tra {
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 416;
 constexpr int kUnits = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 2^8 growth
 constexpr int kSmemLimit = 232448;         // max dynamic shared memory per CTA on sm_100
@@ -53,7 +54,7 @@ struct Cfg {
   static constexpr int kOffK = kUnits * kQUnitBytes;
   static constexpr int kOffV = kOffK + kStages * kKBytes;
   static constexpr int kOffBar = kOffV + kStages * kVBytes;
-  static constexpr int kNumBars = 2 + 5 * kStages + 4 * kUnits + 1;
+  static constexpr int kNumBars = 2 + 5 * kStages + 6 * kUnits + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
@@ -61,7 +62,8 @@ struct Cfg {
   static constexpr uint32_t kI8Layout = D == 128 ? kSwz128 : kSwz64;
   static constexpr uint32_t kI8Sbo = D == 128 ? 1024 : 512;
   static constexpr int kSlabs = D / 64;  // bf16 64-element (128-byte) slabs per row
-  // TMEM columns of unit u: S at u*256, P (bf16 pairs) at u*256+64, O at u*256+128
+  // TMEM columns of unit u: S at u*256, P buffers (bf16 pairs) at u*256+64 and
+  // u*256+96, O at u*256+128
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -205,11 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_kfree = [&](int s) { return bars + (2 + 2 * NST + s) * 8; };
   auto bar_vfull = [&](int s) { return bars + (2 + 3 * NST + s) * 8; };
   auto bar_vfree = [&](int s) { return bars + (2 + 4 * NST + s) * 8; };
-  auto bar_sfull = [&](int u) { return bars + (2 + 5 * NST + 4 * u + 0) * 8; };
-  auto bar_sfree = [&](int u) { return bars + (2 + 5 * NST + 4 * u + 1) * 8; };
-  auto bar_pfull = [&](int u) { return bars + (2 + 5 * NST + 4 * u + 2) * 8; };
-  auto bar_ofull = [&](int u) { return bars + (2 + 5 * NST + 4 * u + 3) * 8; };
-  const uint32_t bar_done = bars + (2 + 5 * NST + 4 * kUnits) * 8;
+  auto bar_sfull = [&](int u) { return bars + (2 + 5 * NST + 6 * u + 0) * 8; };
+  auto bar_sfree = [&](int u) { return bars + (2 + 5 * NST + 6 * u + 1) * 8; };
+  auto bar_pfull = [&](int u, int pb) { return bars + (2 + 5 * NST + 6 * u + 2 + pb) * 8; };
+  auto bar_ofull = [&](int u, int pb) { return bars + (2 + 5 * NST + 6 * u + 4 + pb) * 8; };
+  const uint32_t bar_done = bars + (2 + 5 * NST + 6 * kUnits) * 8;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kOffMisc);
   volatile int* const err = reinterpret_cast<volatile int*>(gbase + C::kOffMisc + 16);
 
@@ -229,10 +231,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = 0; u < kUnits; ++u) {
       mbar_init(bar_sfull(u), 1);
       mbar_init(bar_sfree(u), 128);
-      mbar_init(bar_pfull(u), 128);
-      mbar_init(bar_ofull(u), 1);
+      for (int pb = 0; pb < 2; ++pb) {
+        mbar_init(bar_pfull(u, pb), 128);
+        mbar_init(bar_ofull(u, pb), 1);
+      }
     }
-    mbar_init(bar_done, 1);
+    mbar_init(bar_done, kUnits);  // one commit per MMA-issuing thread
     *err = 0;
     fence_barrier_init();
   }
@@ -299,36 +303,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                       seq0 + kt * kTile);
       }
     }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
+  } else if (warp == 1 || warp == 12) {
+    // ================================================================ MMA issuers
     if (lane == 0) {
+      const int mu = warp == 1 ? 0 : 1;  // the unit this thread issues for
       constexpr uint32_t kIdI8 = instr_desc(2, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdQK16 = instr_desc(1, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdPV = instr_desc(1, 1, 0, 1, D, 128);
+      const uint32_t tU = tmem + mu * 256;
       bool ok = mbar_wait(bar_q, 0, err);
       if (ok && int4) ok = mbar_wait(bar_q4, 0, err);
       tc_fence_after();
-      uint32_t kph = 0, k4ph = 0;       // per-slot phase bits of kfull / k4full
-      // per unit: entries whose QK was issued (negative once its last PV is
-      // issued), and the ring slot / schedule step of its pending P V
-      int cnt0 = 0, cnt1 = 0, pslot0 = 0, pslot1 = 0, pg0 = 0, pg1 = 0;
-      // O_u += P_u(idx) V(slot); P from TMEM, V (MN-major) from shared memory
-      auto issue_pv = [&](int u, int idx, int slot, int gg) -> bool {
-        if (!mbar_wait(bar_pfull(u), idx & 1, err)) return false;
+      // O += P(idx) V(slot): P from TMEM buffer idx & 1, V (MN-major) from shared memory
+      auto issue_pv = [&](int idx, int slot, int gg) -> bool {
+        const int pb = idx & 1;
+        if (!mbar_wait(bar_pfull(mu, pb), (idx >> 1) & 1, err)) return false;
         if (!mbar_wait(bar_vfull(slot), (gg / NST) & 1, err)) return false;
         tc_fence_after();
         const uint32_t vb = sV + slot * C::kVBytes;
-        const uint32_t tO = tmem + u * 256 + 128, tP = tmem + u * 256 + 64;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = smem_desc(vb + kk * 2048, 64 * 128, 1024, kSwz128);
-          mma_bf16_ts(tO, tP + kk * 8, bd, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tU + 128, tU + 64 + pb * 32 + kk * 8, bd, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar_ofull(u));
+        mma_commit(bar_ofull(mu, pb));
         mma_commit(bar_vfree(slot));
         return true;
       };
       if (ok) {
+        uint32_t kph = 0, k4ph = 0;  // per-slot phase bits of kfull / k4full over every step
+        int i = 0;                    // entries of this unit issued so far
+        int pslot = 0, pg = 0;        // ring slot and step of the entry whose P V is pending
         Schedule sc = sched0;
         uint32_t val;
         int mask, u;
@@ -340,54 +345,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (prec == TRA_PREC_INT4) {
-            ok = mbar_wait(bar_k4full(s), (k4ph >> s) & 1, err);
-            k4ph ^= 1u << s;
-          } else {
-            ok = mbar_wait(bar_kfull(s), (kph >> s) & 1, err);
-            kph ^= 1u << s;
-          }
-          const int i = u ? cnt1 : cnt0;
-          if (ok && i >= 1) ok = mbar_wait(bar_sfree(u), (i - 1) & 1, err);
-          if (!ok) break;
+          const bool is4 = prec == TRA_PREC_INT4;
+          const uint32_t bit = 1u << s;
+          const uint32_t ph = ((is4 ? k4ph : kph) & bit) ? 1u : 0u;
+          if (is4) k4ph ^= bit; else kph ^= bit;
+          if (u != mu) continue;  // the other unit's step: only its slot phase matters here
+          if (!mbar_wait(is4 ? bar_k4full(s) : bar_kfull(s), ph, err)) { ok = false; break; }
+          if (i >= 1 && !mbar_wait(bar_sfree(mu), (i - 1) & 1, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kb = sK + s * C::kKBytes;
-          const uint32_t dS = tmem + u * 256;
           if (prec == TRA_PREC_BF16) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const int sl = kk >> 2, off = (kk & 3) * 32;
-              const uint64_t a = smem_desc(sQx(u) + sl * 128 * 128 + off, 16, 1024, kSwz128);
+              const uint64_t a = smem_desc(sQx(mu) + sl * 128 * 128 + off, 16, 1024, kSwz128);
               const uint64_t bd = smem_desc(kb + sl * 64 * 128 + off, 16, 1024, kSwz128);
-              mma_bf16(dS, a, bd, kIdQK16, kk > 0 ? 1u : 0u);
+              mma_bf16(tU, a, bd, kIdQK16, kk > 0 ? 1u : 0u);
             }
           } else {
-            const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(u) : sQx(u);
+            const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(mu) : sQx(mu);
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk) {
               const uint64_t a = smem_desc(qa + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
               const uint64_t bd = smem_desc(kb + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
-              mma_i8(dS, a, bd, kIdI8, kk > 0 ? 1u : 0u);
+              mma_i8(tU, a, bd, kIdI8, kk > 0 ? 1u : 0u);
             }
           }
-          mma_commit(bar_sfull(u));
+          mma_commit(bar_sfull(mu));
           mma_commit(bar_kfree(s));
-          if (i >= 1 && !issue_pv(u, i - 1, u ? pslot1 : pslot0, u ? pg1 : pg0)) { ok = false; break; }
-          int ncnt = i + 1;
-          // a unit with no entries left releases its last V slot now, so the
-          // other unit's loads can keep using the ring
-          if (!sc.more(u)) {
-            if (!issue_pv(u, i, s, g)) { ok = false; break; }
-            ncnt = -1;  // done: the P V of every entry has been issued
-          }
-          if (u) { cnt1 = ncnt; pslot1 = s; pg1 = g; } else { cnt0 = ncnt; pslot0 = s; pg0 = g; }
+          if (i >= 1 && !issue_pv(i - 1, pslot, pg)) { ok = false; break; }
+          pslot = s;
+          pg = g;
+          ++i;
         }
-        if (ok && cnt0 > 0 && !issue_pv(0, cnt0 - 1, pslot0, pg0)) ok = false;
-        if (ok && cnt1 > 0 && !issue_pv(1, cnt1 - 1, pslot1, pg1)) ok = false;
+        if (ok && i >= 1) issue_pv(i - 1, pslot, pg);
       }
-      // all MMAs issued by this thread complete before TMEM is released
+      // every MMA of this thread completes before TMEM is released
       mma_commit(bar_done);
-      mbar_wait(bar_done, 0, err);
+      mbar_wait_drain(bar_done, 0);
     }
   } else if (warp == 2 || warp == 3) {
     // ================================================================ INT4 expanders
@@ -452,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sq8 = half_valid ? __ldg(p.sq8 + qtile) : 0.0f;
     const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) : 0.0f;
     const uint32_t lane_addr = ((uint32_t)(q4 * 32) << 16) + (uint32_t)(u * 256);
-    const uint32_t tS = tmem + lane_addr, tP = tS + 64, tO = tS + 128;
+    const uint32_t tS = tmem + lane_addr, tO = tS + 128;  // P buffers at tS + 64 + 32 * pb
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     int i = 0;
@@ -461,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int mask;
     for (; c.next(val, mask); ++i) {
       if (!mbar_wait(bar_sfull(u), i & 1, err)) { ok = false; break; }
+      const int pb = i & 1;
       const uint32_t prec = val >> 28;
       const int kt = (int)(val & 0x0FFFFFFFu);
       if (prec == TRA_PREC_INT4 && !int4) {
@@ -556,30 +552,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l_tile = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         l_run = l_run * alpha + l_tile;
       }
-      if (i > 0) {
-        // PV(i-1) must have read the previous P before it is overwritten, and
-        // must be complete before O is rescaled
-        if (!mbar_wait(bar_ofull(u), (i - 1) & 1, err)) { ok = false; break; }
+      if (warp_need && i >= 1) {
+        // rescaling O needs every earlier P V complete: the commit of P V(i-1)
+        // fires after all of that thread's earlier MMAs
+        if (!mbar_wait(bar_ofull(u, (i - 1) & 1), ((i - 1) >> 1) & 1, err)) { ok = false; break; }
         tc_fence_after();
-        if (warp_need) {
 #pragma unroll 1
-          for (int col = 0; col < D; col += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + col, o);
-            tmem_wait_ld();
+        for (int col = 0; col < D; col += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + col, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(tO + col, o);
-          }
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(tO + col, o);
         }
+      } else if (i >= 2) {
+        // P buffer pb was last read by P V(i-2)
+        if (!mbar_wait(bar_ofull(u, pb), ((i - 2) >> 1) & 1, err)) { ok = false; break; }
+        tc_fence_after();
       }
-      tmem_st32(tP, pk);
+      tmem_st32(tS + 64 + pb * 32, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_pfull(u));
+      mbar_arrive(bar_pfull(u, pb));
     }
     // ---- epilogue: O / l
-    if (ok && i > 0 && mbar_wait(bar_ofull(u), (i - 1) & 1, err)) {
+    if (ok && i > 0 && mbar_wait(bar_ofull(u, (i - 1) & 1), ((i - 1) >> 1) & 1, err)) {
       tc_fence_after();
       const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
       uint16_t* orow = p.out + ((long long)(x.seq0 + tq) * p.Hq + x.h) * D;
