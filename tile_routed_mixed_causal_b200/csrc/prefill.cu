@@ -28,6 +28,8 @@
 //               online softmax with lazy rescaling of O -> bf16 P into TMEM;
 //               finally O / l.  P is double-buffered so that P(i+1) can be
 //               written while P V of entry i is still running.
+#include <type_traits>
+
 #include "tra_device.cuh"
 #include "tra_launch.h"
 
@@ -452,9 +454,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int i = 0;
     MergeCursor c = unit_cursor(p, x);
-    uint32_t val;
-    int mask;
-    for (; c.next(val, mask); ++i) {
+    // K-tile scale of an entry (1 for BF16), loaded one entry ahead
+    auto kscale = [&](uint32_t v) -> float {
+      const uint32_t pr = v >> 28;
+      const long long kt_ = (long long)x.kvh * p.ntiles + x.toff + (int)(v & 0x0FFFFFFFu);
+      if (pr == TRA_PREC_INT8) return __ldg(p.sk8 + kt_);
+      if (pr == TRA_PREC_INT4 && int4) return __ldg(p.sk4 + kt_);
+      return 1.0f;
+    };
+    uint32_t nval = 0;
+    int nmask = 0;
+    bool have = c.next(nval, nmask);
+    float nsk = have ? kscale(nval) : 0.0f;
+    for (; have; ++i) {
+      const uint32_t val = nval;
+      const int mask = nmask;
+      const float skt = nsk;
+      have = c.next(nval, nmask);  // look-ahead: list value and scale of the next entry
+      if (have) nsk = kscale(nval);
       if (!mbar_wait(bar_sfull(u), i & 1, err)) { ok = false; break; }
       const int pb = i & 1;
       const uint32_t prec = val >> 28;
@@ -497,60 +514,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        const long long ktile = (long long)x.kvh * p.ntiles + x.toff + kt;
-        float f = p.scale_log2;  // log2-domain score = raw * f
-        if (prec == TRA_PREC_INT8) f *= sq8 * __ldg(p.sk8 + ktile);
-        else if (prec == TRA_PREC_INT4) f *= sq4 * __ldg(p.sk4 + ktile);
+        // log2-domain score = raw * f
+        const float f = p.scale_log2 * skt *
+                        (prec == TRA_PREC_INT8 ? sq8 : (prec == TRA_PREC_INT4 ? sq4 : 1.0f));
         // valid keys of this tile for this row (causal and sequence end); only the
         // diagonal tile and a sequence's last tile have fewer than 64
         const int nvalid =
             row_valid ? min(min(tq - kt * kTile + 1, x.T - kt * kTile), kTile) : 0;
         const bool full = __all_sync(0xffffffffu, nvalid >= kTile);
-        // raw scores as exact floats: BF16 accumulators are fp32 already; int32
-        // accumulators (|S| < 2^22) become floats by adding them to the bit
-        // pattern of 1.5*2^23 and subtracting that value (exact, no I2F)
-        float xs[64];
+        // raw scores as floats: fp32 accumulators as they are, int32 ones
+        // converted (exact: |S| < 2^24)
+        auto softmax_row = [&](auto int_tag) {
+          constexpr bool kInt = decltype(int_tag)::value;
+          float xs[64];
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc)
-          xs[cc] = prec == TRA_PREC_BF16 ? __uint_as_float(sr[cc])
-                                         : __uint_as_float(sr[cc] + 0x4B400000u) - 12582912.0f;
-        if (!full) {
-#pragma unroll
-          for (int cc = 0; cc < 64; ++cc) xs[cc] = cc < nvalid ? xs[cc] : -INFINITY;
-        }
-        float mx8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = xs[k];
-#pragma unroll
-        for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], xs[cc]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float m_tile = mx == -INFINITY ? -INFINITY : mx * f;  // f > 0 keeps the argmax
-        const float m_new = fmaxf(m_run, m_tile);
-        const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
-        warp_need = __any_sync(0xffffffffu, need);
-        if (warp_need && m_new > m_run) {
-          alpha = ex2(m_run - m_new);  // m_run = -inf gives 0
-          m_run = m_new;
-        }
-        float ls[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) ls[k] = 0.0f;
-#pragma unroll
-        for (int cc = 0; cc < 64; cc += 2) {
-          float p0 = ex2(fmaf(xs[cc], f, -m_run));
-          float p1 = ex2(fmaf(xs[cc + 1], f, -m_run));
+          for (int cc = 0; cc < 64; ++cc)
+            xs[cc] = kInt ? (float)(int)sr[cc] : __uint_as_float(sr[cc]);
           if (!full) {
-            p0 = cc < nvalid ? p0 : 0.0f;
-            p1 = cc + 1 < nvalid ? p1 : 0.0f;
+#pragma unroll
+            for (int cc = 0; cc < 64; ++cc) xs[cc] = cc < nvalid ? xs[cc] : -INFINITY;
           }
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(&pb);
-          ls[(cc >> 1) & 7] += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
-          pk[cc >> 1] = w;
-        }
-        const float l_tile = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        l_run = l_run * alpha + l_tile;
+          float mx8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = xs[k];
+#pragma unroll
+          for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], xs[cc]);
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float m_tile = mx == -INFINITY ? -INFINITY : mx * f;  // f > 0 keeps the argmax
+          const float m_new = fmaxf(m_run, m_tile);
+          const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
+          warp_need = __any_sync(0xffffffffu, need);
+          if (warp_need && m_new > m_run) {
+            alpha = ex2(m_run - m_new);  // m_run = -inf gives 0
+            m_run = m_new;
+          }
+          // P in bf16 for the MMA; l sums the same bf16-rounded values, so the
+          // normalisation matches what P V accumulates.  Packed fp32x2 FMA/add.
+          const float2 f2 = make_float2(f, f), nm2 = make_float2(-m_run, -m_run);
+          float2 ls[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) ls[k] = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int cc = 0; cc < 64; cc += 2) {
+            const float2 arg = __ffma2_rn(make_float2(xs[cc], xs[cc + 1]), f2, nm2);
+            float p0 = ex2(arg.x);
+            float p1 = ex2(arg.y);
+            if (!full) {
+              p0 = cc < nvalid ? p0 : 0.0f;
+              p1 = cc + 1 < nvalid ? p1 : 0.0f;
+            }
+            const __nv_bfloat162 pbf = __floats2bfloat162_rn(p0, p1);
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(&pbf);
+            ls[(cc >> 1) & 3] = __fadd2_rn(
+                ls[(cc >> 1) & 3],
+                make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+            pk[cc >> 1] = w;
+          }
+          const float2 l2 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+          l_run = l_run * alpha + (l2.x + l2.y);
+        };
+        if (prec == TRA_PREC_BF16)
+          softmax_row(std::integral_constant<bool, false>{});
+        else
+          softmax_row(std::integral_constant<bool, true>{});
       }
       if (warp_need && i >= 1) {
         // rescaling O needs every earlier P V complete: the commit of P V(i-1)
