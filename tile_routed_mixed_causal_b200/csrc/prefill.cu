@@ -18,16 +18,17 @@
 //               interleaved order of the two units' traversals;
 //   warps 1, 12 MMA issuers, one per unit (warp 1 also owns TMEM): S = Q K^T
 //               with kind::i8 (INT8/INT4, exact int32) or kind::f16 (BF16,
-//               fp32) into the unit's S in TMEM, then O += P V with P read
-//               from TMEM (bf16, double-buffered) and V from shared memory;
+//               fp32) into one of the unit's two S buffers in TMEM, then
+//               O += P V with P read from TMEM (bf16) and V from shared memory;
 //   warps 2-3   INT4 expanders: packed INT4 codes (Q once, K per INT4 entry)
 //               sign-extended to int8 in the swizzled operand layout (tcgen05
 //               has no integer 4-bit MMA, so INT4 tiles run as int8 MMAs);
 //   warps 4-7   softmax / epilogue of unit 0, warps 8-11 of unit 1: one thread
 //               per query row (TMEM lane): S -> log2-domain scores -> mask ->
 //               online softmax with lazy rescaling of O -> bf16 P into TMEM;
-//               finally O / l.  P is double-buffered so that P(i+1) can be
-//               written while P V of entry i is still running.
+//               finally O / l.  P(i) overwrites S(i) in its TMEM buffer; with
+//               two buffers QK(i+1) runs while entry i is in the softmax, and
+//               the softmax never waits for a P V except to rescale O.
 #include <type_traits>
 
 #include "tra_device.cuh"
@@ -64,8 +65,8 @@ struct Cfg {
   static constexpr uint32_t kI8Layout = D == 128 ? kSwz128 : kSwz64;
   static constexpr uint32_t kI8Sbo = D == 128 ? 1024 : 512;
   static constexpr int kSlabs = D / 64;  // bf16 64-element (128-byte) slabs per row
-  // TMEM columns of unit u: S at u*256, P buffers (bf16 pairs) at u*256+64 and
-  // u*256+96, O at u*256+128
+  // TMEM columns of unit u: S/P buffer b at u*256 + 64*b (P, bf16 pairs, in its
+  // first 32 columns), O at u*256+128
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -209,10 +210,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_kfree = [&](int s) { return bars + (2 + 2 * NST + s) * 8; };
   auto bar_vfull = [&](int s) { return bars + (2 + 3 * NST + s) * 8; };
   auto bar_vfree = [&](int s) { return bars + (2 + 4 * NST + s) * 8; };
-  auto bar_sfull = [&](int u) { return bars + (2 + 5 * NST + 6 * u + 0) * 8; };
-  auto bar_sfree = [&](int u) { return bars + (2 + 5 * NST + 6 * u + 1) * 8; };
-  auto bar_pfull = [&](int u, int pb) { return bars + (2 + 5 * NST + 6 * u + 2 + pb) * 8; };
-  auto bar_ofull = [&](int u, int pb) { return bars + (2 + 5 * NST + 6 * u + 4 + pb) * 8; };
+  auto bar_sfull = [&](int u, int sb) { return bars + (2 + 5 * NST + 6 * u + sb) * 8; };
+  auto bar_pfull = [&](int u, int sb) { return bars + (2 + 5 * NST + 6 * u + 2 + sb) * 8; };
+  auto bar_ofull = [&](int u) { return bars + (2 + 5 * NST + 6 * u + 4) * 8; };
+  // completes once every MMA of unit u (its last P V included) is done
+  auto bar_ofinal = [&](int u) { return bars + (2 + 5 * NST + 6 * u + 5) * 8; };
   const uint32_t bar_done = bars + (2 + 5 * NST + 6 * kUnits) * 8;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kOffMisc);
   volatile int* const err = reinterpret_cast<volatile int*>(gbase + C::kOffMisc + 16);
@@ -231,12 +233,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_vfree(s), 1);
     }
     for (int u = 0; u < kUnits; ++u) {
-      mbar_init(bar_sfull(u), 1);
-      mbar_init(bar_sfree(u), 128);
-      for (int pb = 0; pb < 2; ++pb) {
-        mbar_init(bar_pfull(u, pb), 128);
-        mbar_init(bar_ofull(u, pb), 1);
+      for (int sb = 0; sb < 2; ++sb) {
+        mbar_init(bar_sfull(u, sb), 1);
+        mbar_init(bar_pfull(u, sb), 128);
       }
+      mbar_init(bar_ofull(u), 1);
+      mbar_init(bar_ofinal(u), 1);
     }
     mbar_init(bar_done, kUnits);  // one commit per MMA-issuing thread
     *err = 0;
@@ -326,9 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = smem_desc(vb + kk * 2048, 64 * 128, 1024, kSwz128);
-          mma_bf16_ts(tU + 128, tU + 64 + pb * 32 + kk * 8, bd, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tU + 128, tU + pb * 64 + kk * 8, bd, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar_ofull(mu, pb));
+        mma_commit(bar_ofull(mu));
         mma_commit(bar_vfree(slot));
         return true;
       };
@@ -352,9 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = ((is4 ? k4ph : kph) & bit) ? 1u : 0u;
           if (is4) k4ph ^= bit; else kph ^= bit;
           if (u != mu) continue;  // the other unit's step: only its slot phase matters here
+          // S buffer i & 1 last held entry i-2, whose P V this thread has already
+          // issued; MMAs of one thread run in order, so QK(i) cannot overtake it
           if (!mbar_wait(is4 ? bar_k4full(s) : bar_kfull(s), ph, err)) { ok = false; break; }
-          if (i >= 1 && !mbar_wait(bar_sfree(mu), (i - 1) & 1, err)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t tSb = tU + (i & 1) * 64;
           const uint32_t kb = sK + s * C::kKBytes;
           if (prec == TRA_PREC_BF16) {
 #pragma unroll
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int sl = kk >> 2, off = (kk & 3) * 32;
               const uint64_t a = smem_desc(sQx(mu) + sl * 128 * 128 + off, 16, 1024, kSwz128);
               const uint64_t bd = smem_desc(kb + sl * 64 * 128 + off, 16, 1024, kSwz128);
-              mma_bf16(tU, a, bd, kIdQK16, kk > 0 ? 1u : 0u);
+              mma_bf16(tSb, a, bd, kIdQK16, kk > 0 ? 1u : 0u);
             }
           } else {
             const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(mu) : sQx(mu);
@@ -370,17 +374,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < D / 32; ++kk) {
               const uint64_t a = smem_desc(qa + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
               const uint64_t bd = smem_desc(kb + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
-              mma_i8(tU, a, bd, kIdI8, kk > 0 ? 1u : 0u);
+              mma_i8(tSb, a, bd, kIdI8, kk > 0 ? 1u : 0u);
             }
           }
-          mma_commit(bar_sfull(mu));
+          mma_commit(bar_sfull(mu, i & 1));
           mma_commit(bar_kfree(s));
           if (i >= 1 && !issue_pv(i - 1, pslot, pg)) { ok = false; break; }
           pslot = s;
           pg = g;
           ++i;
         }
-        if (ok && i >= 1) issue_pv(i - 1, pslot, pg);
+        if (ok && i >= 1 && issue_pv(i - 1, pslot, pg)) mma_commit(bar_ofinal(mu));
       }
       // every MMA of this thread completes before TMEM is released
       mma_commit(bar_done);
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sq8 = half_valid ? __ldg(p.sq8 + qtile) : 0.0f;
     const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) : 0.0f;
     const uint32_t lane_addr = ((uint32_t)(q4 * 32) << 16) + (uint32_t)(u * 256);
-    const uint32_t tS = tmem + lane_addr, tO = tS + 128;  // P buffers at tS + 64 + 32 * pb
+    const uint32_t tU = tmem + lane_addr, tO = tU + 128;  // S/P buffer b at tU + 64 * b
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     int i = 0;
@@ -472,8 +476,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float skt = nsk;
       have = c.next(nval, nmask);  // look-ahead: list value and scale of the next entry
       if (have) nsk = kscale(nval);
-      if (!mbar_wait(bar_sfull(u), i & 1, err)) { ok = false; break; }
-      const int pb = i & 1;
+      const int sb = i & 1;
+      const uint32_t tS = tU + sb * 64;
+      if (!mbar_wait(bar_sfull(u, sb), (i >> 1) & 1, err)) { ok = false; break; }
       const uint32_t prec = val >> 28;
       const int kt = (int)(val & 0x0FFFFFFFu);
       if (prec == TRA_PREC_INT4 && !int4) {
@@ -488,8 +493,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool warp_need = false;
       float alpha = 1.0f;
       if (!half_applies) {
-        tc_fence_before();
-        mbar_arrive(bar_sfree(u));
 #pragma unroll
         for (int k = 0; k < 32; ++k) pk[k] = 0u;
       } else {
@@ -502,8 +505,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tS + 32, hi);
         }
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar_sfree(u));
         if (p.n_dump > 0 && row_valid && prec != TRA_PREC_BF16) {
           for (int di = 0; di < p.n_dump; ++di) {
             const int* dc = p.dump_coords + di * 4;
@@ -580,9 +581,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           softmax_row(std::integral_constant<bool, true>{});
       }
       if (warp_need && i >= 1) {
-        // rescaling O needs every earlier P V complete: the commit of P V(i-1)
-        // fires after all of that thread's earlier MMAs
-        if (!mbar_wait(bar_ofull(u, (i - 1) & 1), ((i - 1) >> 1) & 1, err)) { ok = false; break; }
+        // rescaling O needs every earlier P V complete.  sfull(i) already implies
+        // P V(<= i-2) complete (they were issued before QK(i)), so ofull is at
+        // phase i-1 or i and the parity wait below is exact.
+        if (!mbar_wait(bar_ofull(u), (i - 1) & 1, err)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
         for (int col = 0; col < D; col += 32) {
@@ -593,18 +595,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
           tmem_st32(tO + col, o);
         }
-      } else if (i >= 2) {
-        // P buffer pb was last read by P V(i-2)
-        if (!mbar_wait(bar_ofull(u, pb), ((i - 2) >> 1) & 1, err)) { ok = false; break; }
-        tc_fence_after();
       }
-      tmem_st32(tS + 64 + pb * 32, pk);
+      tmem_st32(tS, pk);  // P(i) over S(i), which this thread has read
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_pfull(u, pb));
+      mbar_arrive(bar_pfull(u, sb));
     }
     // ---- epilogue: O / l
-    if (ok && i > 0 && mbar_wait(bar_ofull(u, (i - 1) & 1), ((i - 1) >> 1) & 1, err)) {
+    // (a parity wait on ofull could pass one phase early here, so the epilogue
+    // waits for the unit's final commit instead)
+    if (ok && i > 0 && mbar_wait(bar_ofinal(u), 0, err)) {
       tc_fence_after();
       const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
       uint16_t* orow = p.out + ((long long)(x.seq0 + tq) * p.Hq + x.h) * D;
