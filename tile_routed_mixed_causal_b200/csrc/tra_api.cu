@@ -113,18 +113,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// int8 tile-major codes viewed as 2-D: d bytes per row, `rows` rows.
-bool map_i8(CUtensorMap* m, const void* base, int d, int64_t rows, int box_rows) {
+// Tile-major codes viewed as 2-D: row_bytes per row (a row of a tile), `rows`
+// rows; the swizzle span equals the row (128, 64 or 32 bytes).
+bool map_i8(CUtensorMap* m, const void* base, int row_bytes, int64_t rows, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d};
-  cuuint32_t box[2] = {(cuuint32_t)d, (cuuint32_t)box_rows};
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw = row_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE,
-            d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bf16 [ntok][H][d] viewed as 3-D (d, H, ntok); boxes of 64 channels x 1 head x box_rows tokens.
@@ -377,7 +380,8 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
 size_t tra_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t d) {
   if (B < 1 || Hq < 1 || Hkv < 1 || d < 1) return 0;
   const size_t S = (size_t)tra::decode_splits(B, Hkv);
-  return round256((size_t)B * Hq * S * 2 * 4) + round256((size_t)B * Hq * S * d * 4);
+  return round256((size_t)B * Hq * S * 2 * 4) + round256((size_t)B * Hq * S * d * 4) +
+         round256((size_t)B * 4);
 }
 
 tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* policy,
@@ -425,10 +429,6 @@ tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* pol
   p.q = q;
   p.k_new = k_new;
   p.v_new = v_new;
-  p.k8 = cache->k8;
-  p.k4 = cache->k4;
-  p.v8 = cache->v8;
-  p.v4 = cache->v4;
   p.sk8 = cache->sk8;
   p.sk4 = cache->sk4;
   p.sv8 = cache->sv8;
@@ -445,8 +445,20 @@ tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* pol
   p.part_ml = reinterpret_cast<float*>(workspace);
   p.part_o = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
                                       round256((size_t)shape->B * shape->Hq * S * 2 * 4));
+  p.skip = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(workspace) +
+                                      round256((size_t)shape->B * shape->Hq * S * 2 * 4) +
+                                      round256((size_t)shape->B * shape->Hq * S * shape->d * 4));
   p.status = status_dev;
-  cudaError_t e = tra::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+  tra::DecodeMaps m;
+  memset(&m, 0, sizeof m);
+  const int64_t rows = (int64_t)shape->Hkv * nt * TRA_TILE;
+  const bool has4 = cache->k4 && cache->v4;  // INT4 maps unused (never loaded) without INT4 tiles
+  bool good = map_i8(&m.k8, cache->k8, shape->d, rows, 64) &&
+              map_i8(&m.v8, cache->v8, shape->d, rows, 64) &&
+              map_i8(&m.k4, has4 ? (const void*)cache->k4 : cache->k8, shape->d / 2, rows, 64) &&
+              map_i8(&m.v4, has4 ? (const void*)cache->v4 : cache->v8, shape->d / 2, rows, 64);
+  if (!good) return fail(TRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  cudaError_t e = tra::launch_decode(p, m, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
 }

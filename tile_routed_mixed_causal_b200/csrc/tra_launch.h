@@ -82,10 +82,6 @@ struct DecodeParams {
   const uint16_t* q;       // [B][Hq][d]
   const uint16_t* k_new;   // [B][Hkv][d]
   const uint16_t* v_new;
-  const int8_t* k8;
-  const uint8_t* k4;
-  const int8_t* v8;
-  const uint8_t* v4;
   const float* sk8;
   const float* sk4;
   const float* sv8;
@@ -100,13 +96,19 @@ struct DecodeParams {
   uint16_t* out;           // [B][Hq][d]
   float* part_ml;          // [B][Hq][splits][2]
   float* part_o;           // [B][Hq][splits][d]
+  int32_t* skip;           // [B]: 1 when the sequence's tail is full this step
   int32_t* status;
 };
 
+struct DecodeMaps {
+  CUtensorMap k8, v8;      // int8 codes, 2-D (d bytes x rows), box 64 rows
+  CUtensorMap k4, v4;      // packed INT4 codes (d/2 bytes x rows)
+};
+
 int decode_splits(int B, int Hkv);
+cudaError_t launch_decode(const DecodeParams& p, const DecodeMaps& m, cudaStream_t s);
 
 // Records `msg` as this thread's tra_last_error() text and returns `st`.
 tra_status report_error(tra_status st, const char* msg);
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 
 }  // namespace tra
