@@ -11,12 +11,11 @@
 // bank-conflict free.  Each consumer warp takes every fourth tile and keeps its
 // own online-softmax state for all query heads of the GQA group, so the loop has
 // no block barrier and every cached byte is read once per group:
-//   scores: lane j owns keys j and j+32; codes become exact floats (byte
-//           permute into the mantissa of 2^23, then one packed subtraction) and
-//           meet q (fp32, broadcast from shared memory) in packed fp32x2 FMAs;
-//   softmax: warp max / sum per head, K scale and 1/sqrt(d) folded into the
-//           exponent, V scale folded into P;
-//   P V:    lane l owns D/32 consecutive channels and accumulates o for every head.
+//   scores: S^T = K Q^T on the tensor cores (mma.sync m16n8k16, f16 codes exact,
+//           fp32 accumulation), K tiles fed by ldmatrix;
+//   softmax: per head over the warp's fragment lanes, K scale and 1/sqrt(d)
+//           folded into the exponent, V scale folded into P (f16, staged per warp);
+//   P V:    O^T += V^T P^T on the tensor cores, V fed by ldmatrix.trans.
 // The last split also covers the bf16 tail (earlier decode tokens + the new
 // one).  The four warps' states are merged per CTA, and a small combine kernel
 // merges the splits and advances tail_len.
@@ -63,21 +62,76 @@ __device__ __forceinline__ void i4x8_to_f2(uint32_t w, float2 (&f)[4]) {
   i8x4_to_f2(e.y, f[2], f[3]);
 }
 
+// ---------------------------------------------------------------- mma.sync helpers
+// The GQA group's contractions run on the tensor cores as m16n8k16 MMAs (f16
+// inputs, fp32 accumulation): scores S^T = K Q^T (M = 16 keys, N = 8 heads) and
+// O^T += V^T P^T (M = 16 channels, N = 8 heads).  Codes reach f16 exactly: each
+// biased byte / nibble becomes the low mantissa byte of 1024.0h, and one packed
+// subtraction removes the bias.  ldmatrix on the int8 tiles, viewed as 16-bit
+// pairs, hands every thread four consecutive codes; the k (channel or key)
+// order inside an MMA is a permutation applied identically to both operands.
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Two biased bytes (selected by `sel` from x) -> f16x2 of (byte - bias).
+__device__ __forceinline__ uint32_t h2_from_bytes(uint32_t x, uint32_t sel, uint32_t bias2) {
+  uint32_t h = __byte_perm(x, 0x6464u, sel);
+  asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(h) : "r"(bias2));
+  return h;
+}
+constexpr uint32_t kSel01 = 0x5140, kSel23 = 0x5342, kSel02 = 0x5240, kSel13 = 0x5341;
+constexpr uint32_t kBias8 = 0x64806480u;  // f16x2 (1152, 1152) = 1024 + 128
+constexpr uint32_t kBias4 = 0x64086408u;  // f16x2 (1032, 1032) = 1024 + 8
+
+// Named barrier over the whole CTA, usable from different code locations.
+__device__ __forceinline__ void named_sync(int id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kDecThreads) : "memory");
+}
+
+__device__ __forceinline__ uint32_t f16x2_from(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 template <int D, int GRP>
 struct DecCfg {
   static constexpr int kRow8 = D;                // INT8 row bytes
   static constexpr int kRow4 = D / 2;            // INT4 row bytes
   static constexpr int kTileBytes = kTile * D;   // INT8 codes of one K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kPStride = 72;            // f16 per head row of P (bank-conflict free)
   static constexpr int kOffQ = kDecStages * kStageBytes;  // q: [D/2 pairs][GRP] float2
   static constexpr int kQBytes = (D / 2) * GRP * 8;
-  static constexpr int kOffP = kOffQ + kQBytes;            // p: [warp][64 keys][GRP] float
-  static constexpr int kPBytes = kConsumers * kTile * GRP * 4;
-  static constexpr int kOffRed = kOffP + kPBytes;          // merge: [warp][GRP][D + 2] float
-  static constexpr int kRedBytes = kConsumers * GRP * (D + 2) * 4;
-  static constexpr int kOffBar = kOffRed + kRedBytes;
+  static constexpr int kOffP = kOffQ + kQBytes;            // P: [warp][8 heads][kPStride] f16
+  static constexpr int kPBytes = kConsumers * 8 * kPStride * 2;
+  static constexpr int kOffT = kOffP + kPBytes;            // tail p: [64 keys][GRP] float
+  static constexpr int kTBytes = kTile * GRP * 4;
+  static constexpr int kStates = kConsumers + 1;           // four warps + the bf16 tail
+  // merge area [state][GRP][D + 2] floats, aliasing the drained ring
+  static constexpr int kOffRed = 0;
+  static constexpr int kRedBytes = kStates * GRP * (D + 2) * 4;
+  static_assert(kRedBytes <= kDecStages * kStageBytes, "merge area must fit in the ring");
+  static constexpr int kOffBar = kOffT + kTBytes;
   static constexpr int kSmem = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
-  static constexpr int kCh = D / 32;             // P V channels per lane
+  static constexpr int kCh = D / 32;             // tail P V channels per lane
+  static constexpr int kB8 = D / 16;             // 16-channel blocks (INT8 fragments)
+  static constexpr int kB4 = D / 32;             // 32-channel blocks (INT4 fragments)
 };
 
 template <int D, int GRP>
@@ -88,7 +142,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   const uint32_t base = (smem_u32(dsm_raw) + 1023u) & ~1023u;
   uint8_t* const sm = dsm_raw + (base - smem_u32(dsm_raw));
   float2* const q2 = reinterpret_cast<float2*>(sm + C::kOffQ);
-  float* const p_sm = reinterpret_cast<float*>(sm + C::kOffP);
   float* const red = reinterpret_cast<float*>(sm + C::kOffRed);
   const uint32_t bar_full = base + C::kOffBar;
   const uint32_t bar_empty = bar_full + kDecStages * 8;
@@ -126,7 +179,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       p.v_tail[dst + c] = p.v_new[src + c];
     }
   }
-  // q of the group's heads as fp32 channel pairs: q2[pair][g]
+  // q of the group's heads as fp32 channel pairs q2[pair][g] (tail path and fragments)
   for (int x = t; x < (D / 2) * GRP; x += kDecThreads) {
     const int cp = x / GRP, g = x % GRP;
     float2 v = make_float2(0.0f, 0.0f);
@@ -136,6 +189,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       v = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
     }
     q2[cp * GRP + g] = v;
+  }
+  // zero the P rows of padded heads (never written; N = 8 heads per MMA)
+  {
+    __half* pz = reinterpret_cast<__half*>(sm + C::kOffP);
+    for (int x = t; x < kConsumers * 8 * C::kPStride; x += kDecThreads) pz[x] = __float2half(0.0f);
   }
   if (t == 0) {
     for (int s = 0; s < kDecStages; ++s) {
@@ -168,73 +226,138 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         }
       }
     }
+    named_sync(1);  // ring drained
+    named_sync(2);  // merge area written
   } else {
     // ------------------------------------------------------------ consumers
-    float m_run[GRP], l_run[GRP];
-    float2 o2[GRP][C::kCh / 2];  // this lane's channels lane*kCh .. for every head
-#pragma unroll
-    for (int g = 0; g < GRP; ++g) {
-      m_run[g] = -INFINITY;
-      l_run[g] = 0.0f;
-#pragma unroll
-      for (int k = 0; k < C::kCh / 2; ++k) o2[g][k] = make_float2(0.0f, 0.0f);
+    const int g = lane >> 2, tq = lane & 3;  // fragment group / thread in group
+    // Power-of-two scale keeping q inside the f16 range (exact: only the exponent moves)
+    float qmax = 0.0f;
+    for (int x = lane; x < (D / 2) * GRP; x += 32) {
+      const float2 v = q2[x];
+      qmax = fmaxf(qmax, fmaxf(fabsf(v.x), fabsf(v.y)));
     }
-    float* const pw = p_sm + warp * kTile * GRP;
-
-    // online-softmax update with this block's scores s[k][g] (lane keys j, j+32),
-    // then P V with p * vscale staged in shared memory; vload(key, v) gives this
-    // lane's channels of V row `key` as floats
-    auto softmax_pv = [&](float (&s)[2][GRP], float vscale, auto vload) {
-      float alpha[GRP];
 #pragma unroll
-      for (int g = 0; g < GRP; ++g) {
-        float mt = fmaxf(s[0][g], s[1][g]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
-        const float m_new = fmaxf(m_run[g], mt);
-        const float mb = m_new == -INFINITY ? 0.0f : m_new;
-        const float p0 = ex2(s[0][g] - mb), p1 = ex2(s[1][g] - mb);  // ex2(-inf) = 0
-        float ps = p0 + p1;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-        alpha[g] = ex2(m_run[g] - mb);
-        l_run[g] = l_run[g] * alpha[g] + ps;
-        m_run[g] = m_new;
-        pw[lane * GRP + g] = p0 * vscale;
-        pw[(lane + 32) * GRP + g] = p1 * vscale;
-      }
-      __syncwarp();
-#pragma unroll
-      for (int g = 0; g < GRP; ++g)
-#pragma unroll
-        for (int k = 0; k < C::kCh / 2; ++k)
-          o2[g][k] = __fmul2_rn(o2[g][k], make_float2(alpha[g], alpha[g]));
-#pragma unroll 4
-      for (int key = 0; key < kTile; ++key) {
-        float2 v[C::kCh / 2];
-        vload(key, v);
-        float pp[GRP];
-        if constexpr (GRP % 4 == 0) {
-#pragma unroll
-          for (int g = 0; g < GRP; g += 4) {
-            const float4 q4 = *reinterpret_cast<const float4*>(pw + key * GRP + g);
-            pp[g] = q4.x;
-            pp[g + 1] = q4.y;
-            pp[g + 2] = q4.z;
-            pp[g + 3] = q4.w;
-          }
-        } else {
-#pragma unroll
-          for (int g = 0; g < GRP; ++g) pp[g] = pw[key * GRP + g];
-        }
-#pragma unroll
-        for (int g = 0; g < GRP; ++g)
-#pragma unroll
-          for (int k = 0; k < C::kCh / 2; ++k)
-            o2[g][k] = __ffma2_rn(v[k], make_float2(pp[g], pp[g]), o2[g][k]);
-      }
-      __syncwarp();
+    for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+    int qexp = 0;
+    if (qmax > 16384.0f) frexpf(qmax / 16384.0f, &qexp);
+    const float qs = ldexpf(1.0f, -qexp), q_unscale = ldexpf(1.0f, qexp);
+    // B fragments of q for head g (zero for padded heads), in the channel order
+    // the K codes arrive in:
+    //   INT8, 16-channel block j: (16j+4t, +1) and (16j+4t+2, +3)
+    //   INT4, 32-channel block j, half ab: (32j+8t+4ab, +1) and (32j+8t+4ab+2, +3)
+    auto qv = [&](int c) -> float {
+      if (g >= grp) return 0.0f;
+      const float2 v = q2[(c >> 1) * GRP + g];
+      return (c & 1 ? v.y : v.x) * qs;
     };
+    uint32_t qb8[C::kB8][2], qb4[C::kB4][2][2];
+#pragma unroll
+    for (int j = 0; j < C::kB8; ++j) {
+      const int c = 16 * j + 4 * tq;
+      qb8[j][0] = f16x2_from(qv(c), qv(c + 1));
+      qb8[j][1] = f16x2_from(qv(c + 2), qv(c + 3));
+    }
+#pragma unroll
+    for (int j = 0; j < C::kB4; ++j)
+#pragma unroll
+      for (int ab = 0; ab < 2; ++ab) {
+        const int c = 32 * j + 8 * tq + 4 * ab;
+        qb4[j][ab][0] = f16x2_from(qv(c), qv(c + 1));
+        qb4[j][ab][1] = f16x2_from(qv(c + 2), qv(c + 3));
+      }
+
+    // this lane's state for heads 2tq, 2tq+1; O^T fragments: INT8 tiles accumulate in
+    // o8 (channels 16j + 2g, +1), INT4 tiles in o4 (channels 32j + 4g + 2ab, +1)
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+    float o8[C::kB8][4], o4[C::kB4][2][4];
+#pragma unroll
+    for (int j = 0; j < C::kB8; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o8[j][k] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < C::kB4; ++j)
+#pragma unroll
+      for (int ab = 0; ab < 2; ++ab)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o4[j][ab][k] = 0.0f;
+    __half* const pw = reinterpret_cast<__half*>(sm + C::kOffP) + warp * 8 * C::kPStride;
+    const uint32_t pw_addr = smem_u32(pw);
+    const int mrow = lane & 7, mj = lane >> 3;  // ldmatrix: this lane's row / matrix
+
+    // bf16 tail (last split, warp 0): tokens [0, tl) of the tail buffer and the new
+    // token at tl, CUDA-core fp32 math with its own softmax state
+    auto tail_pass = [&](float (&tm)[GRP], float (&tlsum)[GRP], float2 (&to)[GRP][C::kCh / 2]) {
+        float* tp = reinterpret_cast<float*>(sm + C::kOffT);
+        const long long tbase = ((long long)b * p.Hkv + kvh) * p.tail_cap;
+        const long long nbase = ((long long)b * p.Hkv + kvh) * D;
+        for (int t0 = 0; t0 <= tl; t0 += kTile) {
+          float sc[2][GRP];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int pos = t0 + lane + 32 * k;
+            float2 acc[GRP];
+#pragma unroll
+            for (int gg = 0; gg < GRP; ++gg) acc[gg] = make_float2(0.0f, 0.0f);
+            if (pos <= tl) {
+              const uint16_t* kr = pos == tl ? p.k_new + nbase : p.k_tail + (tbase + pos) * D;
+              for (int c = 0; c < D / 8; ++c) {
+                const uint4 w = *reinterpret_cast<const uint4*>(kr + c * 8);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                  const float2 kk = make_float2(__uint_as_float(ww[x] << 16),
+                                                __uint_as_float(ww[x] & 0xFFFF0000u));
+#pragma unroll
+                  for (int gg = 0; gg < GRP; ++gg)
+                    acc[gg] = __ffma2_rn(kk, q2[(c * 4 + x) * GRP + gg], acc[gg]);
+                }
+              }
+            }
+#pragma unroll
+            for (int gg = 0; gg < GRP; ++gg)
+              sc[k][gg] = pos <= tl ? (acc[gg].x + acc[gg].y) * p.scale_log2 : -INFINITY;
+          }
+          float al[GRP];
+#pragma unroll
+          for (int gg = 0; gg < GRP; ++gg) {
+            float mx = fmaxf(sc[0][gg], sc[1][gg]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float m_new = fmaxf(tm[gg], mx);
+            const float mb = m_new == -INFINITY ? 0.0f : m_new;
+            const float p0 = ex2(sc[0][gg] - mb), p1 = ex2(sc[1][gg] - mb);
+            float ps = p0 + p1;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+            al[gg] = ex2(tm[gg] - mb);
+            tlsum[gg] = tlsum[gg] * al[gg] + ps;
+            tm[gg] = m_new;
+            tp[lane * GRP + gg] = p0;
+            tp[(lane + 32) * GRP + gg] = p1;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int gg = 0; gg < GRP; ++gg)
+#pragma unroll
+            for (int k = 0; k < C::kCh / 2; ++k)
+              to[gg][k] = __fmul2_rn(to[gg][k], make_float2(al[gg], al[gg]));
+          for (int key = 0; key < kTile; ++key) {
+            const int pos = t0 + key;
+            if (pos > tl) break;
+            const uint16_t* vr = pos == tl ? p.v_new + nbase : p.v_tail + (tbase + pos) * D;
+#pragma unroll
+            for (int k = 0; k < C::kCh / 2; ++k) {
+              const uint32_t w = *reinterpret_cast<const uint32_t*>(vr + lane * C::kCh + 2 * k);
+              const float2 vv = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+#pragma unroll
+              for (int gg = 0; gg < GRP; ++gg)
+                to[gg][k] = __ffma2_rn(vv, make_float2(tp[key * GRP + gg], tp[key * GRP + gg]), to[gg][k]);
+            }
+          }
+          __syncwarp();
+        }
+          };
 
     bool ok = true;
     for (int i = warp; i < ntile; i += kConsumers) {
@@ -244,186 +367,255 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       const int kt = (int)(e & 0x0FFFFFFFu);
       const long long tile = (long long)kvh * p.ntiles + toff + kt;
       const int nvalid = min(kTile, T - kt * kTile);
-      const uint8_t* kb = sm + s * C::kStageBytes;
-      const uint8_t* vb = kb + C::kTileBytes;
-      float sc[2][GRP];
-      float2 acc[2][GRP];
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int g = 0; g < GRP; ++g) acc[k][g] = make_float2(0.0f, 0.0f);
+      const uint32_t kb = base + s * C::kStageBytes;
+      const uint32_t vb = kb + C::kTileBytes;
       const bool is8 = (e >> 28) == TRA_PREC_INT8;
+
+      // ---- scores: sacc[kb] = S^T fragment of keys 16kb + (g, g+8), heads (2tq, 2tq+1)
+      float sacc[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) sacc[k][x] = 0.0f;
       if (is8) {
-        // 16 codes (one swizzled chunk) per key per step
-#pragma unroll 2
-        for (int c = 0; c < C::kRow8 / 16; ++c) {
-          const uint4 w0 = *reinterpret_cast<const uint4*>(kb + swz<C::kRow8>(lane, c));
-          const uint4 w1 = *reinterpret_cast<const uint4*>(kb + swz<C::kRow8>(lane + 32, c));
-          const uint32_t a0[4] = {w0.x, w0.y, w0.z, w0.w}, a1[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-          for (int wd = 0; wd < 4; ++wd) {
-            float2 k0[2], k1[2];
-            i8x4_to_f2(a0[wd], k0[0], k0[1]);
-            i8x4_to_f2(a1[wd], k1[0], k1[1]);
+        for (int cb = 0; cb < D / 32; ++cb)
 #pragma unroll
-            for (int hp = 0; hp < 2; ++hp) {
-              const int cp = c * 8 + wd * 2 + hp;  // channel pair
+          for (int k = 0; k < 4; ++k) {
+            uint32_t r[4];
+            ldsm_x4(kb + swz<C::kRow8>(16 * k + mrow + 8 * (mj & 1), 2 * cb + (mj >> 1)), r);
 #pragma unroll
-              for (int g = 0; g < GRP; ++g) {
-                const float2 qq = q2[cp * GRP + g];
-                acc[0][g] = __ffma2_rn(k0[hp], qq, acc[0][g]);
-                acc[1][g] = __ffma2_rn(k1[hp], qq, acc[1][g]);
-              }
+            for (int h = 0; h < 2; ++h) {  // channels 32cb + 16h ..
+              const uint32_t u0 = r[2 * h] ^ 0x80808080u, u1 = r[2 * h + 1] ^ 0x80808080u;
+              const uint32_t a[4] = {h2_from_bytes(u0, kSel01, kBias8), h2_from_bytes(u1, kSel01, kBias8),
+                                     h2_from_bytes(u0, kSel23, kBias8), h2_from_bytes(u1, kSel23, kBias8)};
+              mma16816(sacc[k], a, qb8[2 * cb + h][0], qb8[2 * cb + h][1]);
             }
           }
-        }
       } else {
-        // 32 codes (one swizzled chunk of packed INT4) per key per step
-#pragma unroll 1
-        for (int c = 0; c < C::kRow4 / 16; ++c) {
-          const uint4 w0 = *reinterpret_cast<const uint4*>(kb + swz<C::kRow4>(lane, c));
-          const uint4 w1 = *reinterpret_cast<const uint4*>(kb + swz<C::kRow4>(lane + 32, c));
-          const uint32_t a0[4] = {w0.x, w0.y, w0.z, w0.w}, a1[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-          for (int wd = 0; wd < 4; ++wd) {
-            float2 k0[4], k1[4];
-            i4x8_to_f2(a0[wd], k0);
-            i4x8_to_f2(a1[wd], k1);
+        for (int cb = 0; cb < D / 64; ++cb)
 #pragma unroll
-            for (int hp = 0; hp < 4; ++hp) {
-              const int cp = c * 16 + wd * 4 + hp;
+          for (int k = 0; k < 4; ++k) {
+            uint32_t r[4];
+            ldsm_x4(kb + swz<C::kRow4>(16 * k + mrow + 8 * (mj & 1), 2 * cb + (mj >> 1)), r);
 #pragma unroll
-              for (int g = 0; g < GRP; ++g) {
-                const float2 qq = q2[cp * GRP + g];
-                acc[0][g] = __ffma2_rn(k0[hp], qq, acc[0][g]);
-                acc[1][g] = __ffma2_rn(k1[hp], qq, acc[1][g]);
+            for (int h = 0; h < 2; ++h) {  // packed bytes 16h.. = channels 64cb + 32h ..
+              // codes of keys g / g+8 at channels 8tq .. 8tq+7, in channel order as bytes
+              uint32_t c0[2], c1[2];
+              {
+                const uint32_t x0 = r[2 * h] ^ 0x88888888u, x1 = r[2 * h + 1] ^ 0x88888888u;
+                const uint32_t lo0 = x0 & 0x0F0F0F0Fu, hi0 = (x0 >> 4) & 0x0F0F0F0Fu;
+                const uint32_t lo1 = x1 & 0x0F0F0F0Fu, hi1 = (x1 >> 4) & 0x0F0F0F0Fu;
+                c0[0] = __byte_perm(lo0, hi0, 0x5140);
+                c0[1] = __byte_perm(lo0, hi0, 0x7362);
+                c1[0] = __byte_perm(lo1, hi1, 0x5140);
+                c1[1] = __byte_perm(lo1, hi1, 0x7362);
+              }
+#pragma unroll
+              for (int ab = 0; ab < 2; ++ab) {
+                const uint32_t a[4] = {h2_from_bytes(c0[ab], kSel01, kBias4),
+                                       h2_from_bytes(c1[ab], kSel01, kBias4),
+                                       h2_from_bytes(c0[ab], kSel23, kBias4),
+                                       h2_from_bytes(c1[ab], kSel23, kBias4)};
+                mma16816(sacc[k], a, qb4[2 * cb + h][ab][0], qb4[2 * cb + h][ab][1]);
               }
             }
           }
-        }
       }
-      const float ks = (is8 ? __ldg(p.sk8 + tile) : __ldg(p.sk4 + tile)) * p.scale_log2;
+      // ---- online softmax for heads 2tq, 2tq+1 over keys 16k + g (+8)
+      const float ks = (is8 ? __ldg(p.sk8 + tile) : __ldg(p.sk4 + tile)) * p.scale_log2 * q_unscale;
       const float vs = is8 ? __ldg(p.sv8 + tile) : __ldg(p.sv4 + tile);
+      float sv[2][8];  // [head][key slot: 2k + (g / g+8)]
 #pragma unroll
-      for (int g = 0; g < GRP; ++g) {
-        sc[0][g] = lane < nvalid ? (acc[0][g].x + acc[0][g].y) * ks : -INFINITY;
-        sc[1][g] = lane + 32 < nvalid ? (acc[1][g].x + acc[1][g].y) * ks : -INFINITY;
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int key0 = 16 * k + g, key1 = key0 + 8;
+          sv[hh][2 * k] = key0 < nvalid ? sacc[k][hh] * ks : -INFINITY;
+          sv[hh][2 * k + 1] = key1 < nvalid ? sacc[k][2 + hh] * ks : -INFINITY;
+        }
+      float mt[2], alpha[2] = {1.0f, 1.0f};
+      bool need = false;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float x = sv[hh][0];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) x = fmaxf(x, sv[hh][k]);
+        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+        mt[hh] = x;
+        need |= fmaxf(m_run[hh], x) > m_run[hh] + 8.0f;  // true for the first finite max
       }
-      if (is8) {
-        softmax_pv(sc, vs, [&](int key, float2 (&v)[C::kCh / 2]) {
-          if constexpr (D == 128) {  // channels 4*lane .. 4*lane+3
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(
-                vb + swz<C::kRow8>(key, lane >> 2) + (lane & 3) * 4);
-            i8x4_to_f2(w, v[0], v[1]);
-          } else {  // D = 64: channels 2*lane, 2*lane+1
-            const uint32_t w = *reinterpret_cast<const uint16_t*>(
-                vb + swz<C::kRow8>(key, lane >> 3) + (lane & 7) * 2);
-            float2 a, bb;
-            i8x4_to_f2(w, a, bb);
-            v[0] = a;
+      // lazy rescaling: the reference max moves only when it grew by more than 2^8
+      const bool warp_need = __any_sync(0xffffffffu, need);
+      if (warp_need) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const float m_new = fmaxf(m_run[hh], mt[hh]);
+          if (m_new > m_run[hh]) {
+            alpha[hh] = ex2(m_run[hh] - m_new);  // -inf -> 0
+            m_run[hh] = m_new;
           }
-        });
-      } else {
-        softmax_pv(sc, vs, [&](int key, float2 (&v)[C::kCh / 2]) {
-          if constexpr (D == 128) {  // channels 4*lane .. 4*lane+3 = two packed bytes
-            const uint32_t w = *reinterpret_cast<const uint16_t*>(
-                vb + swz<C::kRow4>(key, lane >> 3) + (lane & 7) * 2);
-            float2 f[4];
-            i4x8_to_f2(w, f);
-            v[0] = f[0];
-            v[1] = f[1];
-          } else {  // D = 64: channels 2*lane, 2*lane+1 = one packed byte
-            const uint32_t w = *reinterpret_cast<const uint8_t*>(
-                vb + swz<C::kRow4>(key, lane >> 4) + (lane & 15));
-            float2 f[4];
-            i4x8_to_f2(w, f);
-            v[0] = f[0];
-          }
-        });
+        }
       }
-      // stage s may be refilled once every lane of this warp is done with it
+      const bool real0 = 2 * tq < grp, real1 = 2 * tq + 1 < grp;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const float mb = m_run[hh] == -INFINITY ? 0.0f : m_run[hh];
+        const bool real = hh == 0 ? real0 : real1;
+        float ps = 0.0f;
+        __half* prow = pw + (2 * tq + hh) * C::kPStride;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float p0 = real ? ex2(sv[hh][2 * k] - mb) : 0.0f;
+          const float p1 = real ? ex2(sv[hh][2 * k + 1] - mb) : 0.0f;
+          ps += p0 + p1;
+          prow[16 * k + g] = __float2half_rn(p0 * vs);
+          prow[16 * k + g + 8] = __float2half_rn(p1 * vs);
+        }
+        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+        l_run[hh] = l_run[hh] * alpha[hh] + ps;
+      }
+      if (warp_need) {
+#pragma unroll
+        for (int j = 0; j < C::kB8; ++j) {
+          o8[j][0] *= alpha[0]; o8[j][1] *= alpha[1];
+          o8[j][2] *= alpha[0]; o8[j][3] *= alpha[1];
+        }
+#pragma unroll
+        for (int j = 0; j < C::kB4; ++j)
+#pragma unroll
+          for (int ab = 0; ab < 2; ++ab) {
+            o4[j][ab][0] *= alpha[0]; o4[j][ab][1] *= alpha[1];
+            o4[j][ab][2] *= alpha[0]; o4[j][ab][3] *= alpha[1];
+          }
+      }
+      __syncwarp();
+      // ---- O^T += V^T P^T: B fragment = P[head g][keys 16k + 2tq (+1), +8 (+9)]
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t pb0, pb1;
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(pb0) : "r"(pw_addr + (g * C::kPStride + 16 * k + 2 * tq) * 2));
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(pb1) : "r"(pw_addr + (g * C::kPStride + 16 * k + 2 * tq + 8) * 2));
+        if (is8) {
+#pragma unroll
+          for (int cp = 0; cp < D / 32; ++cp) {
+            uint32_t r[4];
+            ldsm_x4_t(vb + swz<C::kRow8>(16 * k + mrow + 8 * (mj & 1), 2 * cp + (mj >> 1)), r);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // channels 32cp + 16h + (2g, 2g+1)
+              const uint32_t u0 = r[2 * h] ^ 0x80808080u, u1 = r[2 * h + 1] ^ 0x80808080u;
+              const uint32_t a[4] = {h2_from_bytes(u0, kSel02, kBias8), h2_from_bytes(u0, kSel13, kBias8),
+                                     h2_from_bytes(u1, kSel02, kBias8), h2_from_bytes(u1, kSel13, kBias8)};
+              mma16816(o8[2 * cp + h], a, pb0, pb1);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int cp = 0; cp < D / 64; ++cp) {
+            uint32_t r[4];
+            ldsm_x4_t(vb + swz<C::kRow4>(16 * k + mrow + 8 * (mj & 1), 2 * cp + (mj >> 1)), r);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // 32 channels 64cp + 32h .. (4g .. 4g+3)
+              const uint32_t x0 = r[2 * h] ^ 0x88888888u, x1 = r[2 * h + 1] ^ 0x88888888u;
+              const uint32_t lo0 = x0 & 0x0F0F0F0Fu, hi0 = (x0 >> 4) & 0x0F0F0F0Fu;
+              const uint32_t lo1 = x1 & 0x0F0F0F0Fu, hi1 = (x1 >> 4) & 0x0F0F0F0Fu;
+              const uint32_t aA[4] = {h2_from_bytes(lo0, kSel02, kBias4), h2_from_bytes(hi0, kSel02, kBias4),
+                                      h2_from_bytes(lo1, kSel02, kBias4), h2_from_bytes(hi1, kSel02, kBias4)};
+              mma16816(o4[2 * cp + h][0], aA, pb0, pb1);
+              const uint32_t aB[4] = {h2_from_bytes(lo0, kSel13, kBias4), h2_from_bytes(hi0, kSel13, kBias4),
+                                      h2_from_bytes(lo1, kSel13, kBias4), h2_from_bytes(hi1, kSel13, kBias4)};
+              mma16816(o4[2 * cp + h][1], aB, pb0, pb1);
+            }
+          }
+        }
+      }
+      // stage s and this warp's P rows may be reused once every lane is done
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty + s * 8);
     }
 
-    // ---- bf16 tail on the last split: tokens [0, tl) from the tail buffer, tl = new token
-    if (ok && last && warp == 0) {
-      const long long tbase = ((long long)b * p.Hkv + kvh) * p.tail_cap;
-      const long long nbase = ((long long)b * p.Hkv + kvh) * D;
-      for (int t0 = 0; t0 <= tl; t0 += kTile) {
-        float sc[2][GRP];
+    // ---- bf16 tail (computed below by warp 0) and the shared-memory merge; the
+    // merge area aliases the ring, so every warp must be done with the ring first
+    float tm[GRP], tlsum[GRP];
+    float2 to[GRP][C::kCh / 2];
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int pos = t0 + lane + 32 * k;
-          float2 acc[GRP];
+    for (int gg = 0; gg < GRP; ++gg) {
+      tm[gg] = -INFINITY;
+      tlsum[gg] = 0.0f;
 #pragma unroll
-          for (int g = 0; g < GRP; ++g) acc[g] = make_float2(0.0f, 0.0f);
-          if (pos <= tl) {
-            const uint16_t* kr = pos == tl ? p.k_new + nbase : p.k_tail + (tbase + pos) * D;
-            for (int c = 0; c < D / 8; ++c) {
-              const uint4 w = *reinterpret_cast<const uint4*>(kr + c * 8);
-              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      for (int k = 0; k < C::kCh / 2; ++k) to[gg][k] = make_float2(0.0f, 0.0f);
+    }
+    if (warp == 0 && ok && last) tail_pass(tm, tlsum, to);
+    named_sync(1);
+    float* rw = red + warp * GRP * (D + 2);
+    for (int x = lane; x < GRP * (D + 2); x += 32) rw[x] = 0.0f;
+    __syncwarp();
 #pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                const float2 kk = make_float2(__uint_as_float(ww[x] << 16),
-                                              __uint_as_float(ww[x] & 0xFFFF0000u));
+    for (int hh = 0; hh < 2; ++hh) {
+      const int hd = 2 * tq + hh;
+      if (hd < GRP) {
 #pragma unroll
-                for (int g = 0; g < GRP; ++g)
-                  acc[g] = __ffma2_rn(kk, q2[(c * 4 + x) * GRP + g], acc[g]);
-              }
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < GRP; ++g)
-            sc[k][g] = pos <= tl ? (acc[g].x + acc[g].y) * p.scale_log2 : -INFINITY;
+        for (int j = 0; j < C::kB8; ++j) {
+          rw[hd * (D + 2) + 16 * j + 2 * g] = o8[j][hh];
+          rw[hd * (D + 2) + 16 * j + 2 * g + 1] = o8[j][2 + hh];
         }
-        softmax_pv(sc, 1.0f, [&](int key, float2 (&v)[C::kCh / 2]) {
-          const int pos = t0 + key;
-          if (pos > tl) {
+        if (g == 0) {
+          rw[hd * (D + 2) + D] = m_run[hh];
+          rw[hd * (D + 2) + D + 1] = l_run[hh];
+        }
+      }
+    }
+    __syncwarp();
 #pragma unroll
-            for (int k = 0; k < C::kCh / 2; ++k) v[k] = make_float2(0.0f, 0.0f);
-            return;
-          }
-          const uint16_t* vr = pos == tl ? p.v_new + nbase : p.v_tail + (tbase + pos) * D;
+    for (int hh = 0; hh < 2; ++hh) {
+      const int hd = 2 * tq + hh;
+      if (hd < GRP) {
 #pragma unroll
-          for (int k = 0; k < C::kCh / 2; ++k) {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(vr + lane * C::kCh + 2 * k);
-            v[k] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+        for (int j = 0; j < C::kB4; ++j)
+#pragma unroll
+          for (int ab = 0; ab < 2; ++ab) {
+            rw[hd * (D + 2) + 32 * j + 4 * g + 2 * ab] += o4[j][ab][hh];
+            rw[hd * (D + 2) + 32 * j + 4 * g + 2 * ab + 1] += o4[j][ab][2 + hh];
           }
-        });
       }
     }
 
-    // ---- this warp's state into shared memory for the CTA merge
-    float* rw = red + warp * GRP * (D + 2);
+    if (warp == 0) {
+      float* rt = red + kConsumers * GRP * (D + 2);
 #pragma unroll
-    for (int g = 0; g < GRP; ++g) {
+      for (int gg = 0; gg < GRP; ++gg) {
 #pragma unroll
-      for (int k = 0; k < C::kCh / 2; ++k)
-        *reinterpret_cast<float2*>(rw + g * (D + 2) + lane * C::kCh + 2 * k) = o2[g][k];
-      if (lane == 0) {
-        rw[g * (D + 2) + D] = m_run[g];
-        rw[g * (D + 2) + D + 1] = l_run[g];
+        for (int k = 0; k < C::kCh / 2; ++k)
+          *reinterpret_cast<float2*>(rt + gg * (D + 2) + lane * C::kCh + 2 * k) = to[gg][k];
+        if (lane == 0) {
+          rt[gg * (D + 2) + D] = tm[gg];
+          rt[gg * (D + 2) + D + 1] = tlsum[gg];
+        }
       }
     }
+    named_sync(2);
   }
-  __syncthreads();
-  // merge the consumer warps into this split's partial (m, l, o)
+  // merge the consumer warps and the tail into this split's partial (m, l, o)
   for (int x = t; x < GRP * D; x += kDecThreads) {
-    const int g = x / D, c = x % D;
-    if (g >= grp) continue;
+    const int gg = x / D, c = x % D;
+    if (gg >= grp) continue;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, red[(w * GRP + g) * (D + 2) + D]);
+    for (int w = 0; w < C::kStates; ++w) M = fmaxf(M, red[(w * GRP + gg) * (D + 2) + D]);
     float L = 0.0f, o = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kConsumers; ++w) {
-      const float* r = red + (w * GRP + g) * (D + 2);
+    for (int w = 0; w < C::kStates; ++w) {
+      const float* r = red + (w * GRP + gg) * (D + 2);
       const float wt = r[D] == -INFINITY ? 0.0f : ex2(r[D] - M);
       L += r[D + 1] * wt;
       o += r[c] * wt;
     }
-    const long long pi = ((long long)b * p.Hq + kvh * grp + g) * p.splits + split;
+    const long long pi = ((long long)b * p.Hq + kvh * grp + gg) * p.splits + split;
     p.part_o[pi * D + c] = o;
     if (c == 0) {
       p.part_ml[pi * 2] = M;
