@@ -14,7 +14,8 @@
 // Two work units share one CTA (416 threads) so that one unit's softmax runs
 // while the tensor core works on the other's tiles:
 //   warp 0      TMA producer: both units' Q tiles once, then K (INT8 codes or
-//               BF16) and V (BF16) tiles into one NST-deep ring, in the
+//               BF16) into a K ring and V (BF16) into a deeper V ring (K slots
+//               free up right after QK, V slots only after P V), in the
 //               interleaved order of the two units' traversals;
 //   warps 1, 12 MMA issuers, one per unit (warp 1 also owns TMEM): S = Q K^T
 //               with kind::i8 (INT8/INT4, exact int32) or kind::f16 (BF16,
@@ -22,7 +23,10 @@
 //               O += P V with P read from TMEM (bf16) and V from shared memory;
 //   warps 2-3   INT4 expanders: packed INT4 codes (Q once, K per INT4 entry)
 //               sign-extended to int8 in the swizzled operand layout (tcgen05
-//               has no integer 4-bit MMA, so INT4 tiles run as int8 MMAs);
+//               has no integer 4-bit MMA, so INT4 tiles run as int8 MMAs), into
+//               a K4 ring of their own.  Each ring has exactly one filler that
+//               takes its slots in order, so a parity wait on a slot's free
+//               barrier never aliases a phase two uses back;
 //   warps 4-7   softmax / epilogue of unit 0, warps 8-11 of unit 1: one thread
 //               per query row (TMEM lane): S -> log2-domain scores -> mask ->
 //               online softmax with lazy rescaling of O -> bf16 P into TMEM;
@@ -47,17 +51,23 @@ struct Cfg {
   static constexpr int kQ8Bytes = 128 * D;                                    // int8 Q codes
   static constexpr int kQxBytes = MODE == TRA_POLICY_BITMASK ? 128 * D * 2 : 128 * D;
   static constexpr int kQUnitBytes = kQ8Bytes + kQxBytes;
-  static constexpr int kKBytes = 64 * D * 2;                                  // slot fits bf16
+  // K slot: BF16 or INT8 codes under a bitmask policy, INT8 codes only under boundaries
+  static constexpr int kKBytes = MODE == TRA_POLICY_BITMASK ? 64 * D * 2 : 64 * D;
+  static constexpr int kK4Bytes = 64 * D;                                     // expanded INT4 K
   static constexpr int kVBytes = 64 * D * 2;
-  static constexpr int kFixed = kUnits * kQUnitBytes + 2048;                  // + barriers, slack
-  static constexpr int kStagesFit = (kSmemLimit - kFixed) / (kKBytes + kVBytes);
-  static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
-  static_assert(kStages >= 3, "shared memory too small for the K/V ring");
+  static constexpr int kStagesK = 3;
+  static constexpr int kStagesK4 = MODE == TRA_POLICY_BOUNDARY ? 2 : 0;
+  static constexpr int kFixed = kUnits * kQUnitBytes + kStagesK * kKBytes + kStagesK4 * kK4Bytes +
+                                2048;                                         // + barriers, slack
+  static constexpr int kStagesVFit = (kSmemLimit - kFixed) / kVBytes;
+  static constexpr int kStagesV = kStagesVFit > 6 ? 6 : kStagesVFit;
+  static_assert(kStagesV >= 3, "shared memory too small for the V ring");
   static constexpr int kOffQ = 0;                                             // unit u at u * kQUnitBytes
   static constexpr int kOffK = kUnits * kQUnitBytes;
-  static constexpr int kOffV = kOffK + kStages * kKBytes;
-  static constexpr int kOffBar = kOffV + kStages * kVBytes;
-  static constexpr int kNumBars = 2 + 5 * kStages + 6 * kUnits + 1;
+  static constexpr int kOffK4 = kOffK + kStagesK * kKBytes;
+  static constexpr int kOffV = kOffK4 + kStagesK4 * kK4Bytes;
+  static constexpr int kOffBar = kOffV + kStagesV * kVBytes;
+  static constexpr int kNumBars = 2 + 2 * kStagesK + 2 * kStagesK4 + 2 * kStagesV + 6 * kUnits + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
@@ -185,7 +195,8 @@ template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps m) {
   using C = Cfg<D, MODE>;
-  constexpr int NST = C::kStages;
+  constexpr int NSK = C::kStagesK, NSV = C::kStagesV;
+  constexpr int NS4 = C::kStagesK4 > 0 ? C::kStagesK4 : 1;  // (no K4 ring without INT4)
   extern __shared__ uint8_t smem_raw[];
 
   // ---- the CTA's two work units
@@ -201,21 +212,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sQ8 = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes; };
   auto sQx = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes; };
   const uint32_t sK = base + C::kOffK;
+  const uint32_t sK4 = base + C::kOffK4;
   const uint32_t sV = base + C::kOffV;
   const uint32_t bars = base + C::kOffBar;
   const uint32_t bar_q = bars + 0 * 8;
   const uint32_t bar_q4 = bars + 1 * 8;
   auto bar_kfull = [&](int s) { return bars + (2 + s) * 8; };
-  auto bar_k4full = [&](int s) { return bars + (2 + NST + s) * 8; };
-  auto bar_kfree = [&](int s) { return bars + (2 + 2 * NST + s) * 8; };
-  auto bar_vfull = [&](int s) { return bars + (2 + 3 * NST + s) * 8; };
-  auto bar_vfree = [&](int s) { return bars + (2 + 4 * NST + s) * 8; };
-  auto bar_sfull = [&](int u, int sb) { return bars + (2 + 5 * NST + 6 * u + sb) * 8; };
-  auto bar_pfull = [&](int u, int sb) { return bars + (2 + 5 * NST + 6 * u + 2 + sb) * 8; };
-  auto bar_ofull = [&](int u) { return bars + (2 + 5 * NST + 6 * u + 4) * 8; };
+  auto bar_kfree = [&](int s) { return bars + (2 + NSK + s) * 8; };
+  auto bar_k4full = [&](int s) { return bars + (2 + 2 * NSK + s) * 8; };
+  auto bar_k4free = [&](int s) { return bars + (2 + 2 * NSK + NS4 + s) * 8; };
+  constexpr int kVB = 2 + 2 * NSK + 2 * C::kStagesK4;  // first V ring barrier
+  auto bar_vfull = [&](int s) { return bars + (kVB + s) * 8; };
+  auto bar_vfree = [&](int s) { return bars + (kVB + NSV + s) * 8; };
+  constexpr int kUB = kVB + 2 * NSV;                    // first per-unit barrier
+  auto bar_sfull = [&](int u, int sb) { return bars + (kUB + 6 * u + sb) * 8; };
+  auto bar_pfull = [&](int u, int sb) { return bars + (kUB + 6 * u + 2 + sb) * 8; };
+  auto bar_ofull = [&](int u) { return bars + (kUB + 6 * u + 4) * 8; };
   // completes once every MMA of unit u (its last P V included) is done
-  auto bar_ofinal = [&](int u) { return bars + (2 + 5 * NST + 6 * u + 5) * 8; };
-  const uint32_t bar_done = bars + (2 + 5 * NST + 6 * kUnits) * 8;
+  auto bar_ofinal = [&](int u) { return bars + (kUB + 6 * u + 5) * 8; };
+  const uint32_t bar_done = bars + (kUB + 6 * kUnits) * 8;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kOffMisc);
   volatile int* const err = reinterpret_cast<volatile int*>(gbase + C::kOffMisc + 16);
 
@@ -225,10 +240,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     mbar_init(bar_q4, 64);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(bar_kfull(s), 1);
-      mbar_init(bar_k4full(s), 64);
       mbar_init(bar_kfree(s), 1);
+    }
+    for (int s = 0; s < C::kStagesK4; ++s) {
+      mbar_init(bar_k4full(s), 64);
+      mbar_init(bar_k4free(s), 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
       mbar_init(bar_vfull(s), 1);
       mbar_init(bar_vfree(s), 1);
     }
@@ -277,8 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       Schedule sc = sched0;
       uint32_t val;
       int mask, u;
+      int nk = 0;  // K ring fills so far (every entry but INT4 ones)
       for (int g = 0; sc.next(u, val, mask); ++g) {
-        const int s = g % NST, use = g / NST;
+        const int sv = g % NSV, usev = g / NSV;  // V ring slot
         const uint32_t prec = val >> 28;
         const int kt = (int)(val & 0x0FFFFFFFu);
         const int kvh = TRA_UNIT_FIELD(u, kvh), toff = TRA_UNIT_FIELD(u, toff);
@@ -288,6 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (prec != TRA_PREC_INT4) {
+          const int s = nk % NSK, use = nk / NSK;  // K ring slot
+          ++nk;
           if (use > 0 && !mbar_wait(bar_kfree(s), (use - 1) & 1, err)) break;
           const uint32_t dst = sK + s * C::kKBytes;
           if (prec == TRA_PREC_INT8) {
@@ -300,10 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                           seq0 + kt * kTile);
           }
         }
-        if (use > 0 && !mbar_wait(bar_vfree(s), (use - 1) & 1, err)) break;
-        mbar_arrive_expect_tx(bar_vfull(s), 64 * D * 2);
+        if (usev > 0 && !mbar_wait(bar_vfree(sv), (usev - 1) & 1, err)) break;
+        mbar_arrive_expect_tx(bar_vfull(sv), 64 * D * 2);
         for (int sl = 0; sl < C::kSlabs; ++sl)
-          tma_load_3d(sV + s * C::kVBytes + sl * 64 * 128, &m.vb, bar_vfull(s), sl * 64, kvh,
+          tma_load_3d(sV + sv * C::kVBytes + sl * 64 * 128, &m.vb, bar_vfull(sv), sl * 64, kvh,
                       seq0 + kt * kTile);
       }
     }
@@ -322,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int idx, int slot, int gg) -> bool {
         const int pb = idx & 1;
         if (!mbar_wait(bar_pfull(mu, pb), (idx >> 1) & 1, err)) return false;
-        if (!mbar_wait(bar_vfull(slot), (gg / NST) & 1, err)) return false;
+        if (!mbar_wait(bar_vfull(slot), (gg / NSV) & 1, err)) return false;
         tc_fence_after();
         const uint32_t vb = sV + slot * C::kVBytes;
 #pragma unroll
@@ -335,14 +358,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       if (ok) {
-        uint32_t kph = 0, k4ph = 0;  // per-slot phase bits of kfull / k4full over every step
+        int nk = 0, n4 = 0;           // K / K4 ring steps so far, both units
         int i = 0;                    // entries of this unit issued so far
-        int pslot = 0, pg = 0;        // ring slot and step of the entry whose P V is pending
+        int pslot = 0, pg = 0;        // V slot and step of the entry whose P V is pending
         Schedule sc = sched0;
         uint32_t val;
         int mask, u;
         for (int g = 0; sc.next(u, val, mask); ++g) {
-          const int s = g % NST;
           const uint32_t prec = val >> 28;
           if (prec == TRA_PREC_INT4 && !int4) {
             *err = TRA_DEV_BAD_LIST;
@@ -350,16 +372,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const bool is4 = prec == TRA_PREC_INT4;
-          const uint32_t bit = 1u << s;
-          const uint32_t ph = ((is4 ? k4ph : kph) & bit) ? 1u : 0u;
-          if (is4) k4ph ^= bit; else kph ^= bit;
-          if (u != mu) continue;  // the other unit's step: only its slot phase matters here
+          const int s = is4 ? n4 % NS4 : nk % NSK;
+          const uint32_t ph = (uint32_t)((is4 ? n4 / NS4 : nk / NSK) & 1);
+          if (is4) ++n4; else ++nk;
+          if (u != mu) continue;  // the other unit's step: only the ring positions matter here
           // S buffer i & 1 last held entry i-2, whose P V this thread has already
           // issued; MMAs of one thread run in order, so QK(i) cannot overtake it
           if (!mbar_wait(is4 ? bar_k4full(s) : bar_kfull(s), ph, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t tSb = tU + (i & 1) * 64;
-          const uint32_t kb = sK + s * C::kKBytes;
+          const uint32_t kb = is4 ? sK4 + s * C::kK4Bytes : sK + s * C::kKBytes;
           if (prec == TRA_PREC_BF16) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -378,9 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           mma_commit(bar_sfull(mu, i & 1));
-          mma_commit(bar_kfree(s));
+          mma_commit(is4 ? bar_k4free(s) : bar_kfree(s));
           if (i >= 1 && !issue_pv(i - 1, pslot, pg)) { ok = false; break; }
-          pslot = s;
+          pslot = g % NSV;
           pg = g;
           ++i;
         }
@@ -418,14 +440,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       Schedule sc = sched0;
       uint32_t val;
       int mask, u;
-      for (int g = 0; sc.next(u, val, mask); ++g) {
+      for (int n4 = 0; sc.next(u, val, mask);) {
         if ((val >> 28) != TRA_PREC_INT4) continue;
-        const int s = g % NST, use = g / NST;
-        if (use > 0 && !mbar_wait(bar_kfree(s), (use - 1) & 1, err)) break;
+        const int s = n4 % NS4, use = n4 / NS4;  // K4 ring slot
+        ++n4;
+        if (use > 0 && !mbar_wait(bar_k4free(s), (use - 1) & 1, err)) break;
         const int kt = (int)(val & 0x0FFFFFFFu);
         const uint8_t* ks = p.k4 + ((long long)(TRA_UNIT_FIELD(u, kvh) * p.ntiles +
                                                 TRA_UNIT_FIELD(u, toff) + kt) * kTile) * kPackedRow;
-        uint8_t* dst = gbase + C::kOffK + s * C::kKBytes;
+        uint8_t* dst = gbase + C::kOffK4 + s * C::kK4Bytes;
         for (int f = t; f < 64 * kChunksPerRow; f += 64) {
           const int r = f / kChunksPerRow, cc = f % kChunksPerRow;
           const uint4 w = __ldg(reinterpret_cast<const uint4*>(ks + r * kPackedRow + cc * 16));
@@ -523,25 +546,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nvalid =
             row_valid ? min(min(tq - kt * kTile + 1, x.T - kt * kTile), kTile) : 0;
         const bool full = __all_sync(0xffffffffu, nvalid >= kTile);
-        // raw scores as floats: fp32 accumulators as they are, int32 ones
-        // converted (exact: |S| < 2^24)
-        auto softmax_row = [&](auto int_tag) {
+        // One row of the tile -> bf16 P and the online-softmax update.  Full
+        // tiles (every key valid) take a copy with no per-column test; only
+        // the diagonal tile and a sequence's last tile take the masked copy.
+        // Raw scores as floats: fp32 accumulators as they are, int32 ones
+        // converted (exact: |S| < 2^24).
+        auto softmax_row = [&](auto int_tag, auto full_tag) {
           constexpr bool kInt = decltype(int_tag)::value;
+          constexpr bool kFull = decltype(full_tag)::value;
           float xs[64];
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc)
+          for (int cc = 0; cc < 64; ++cc) {
             xs[cc] = kInt ? (float)(int)sr[cc] : __uint_as_float(sr[cc]);
-          if (!full) {
-#pragma unroll
-            for (int cc = 0; cc < 64; ++cc) xs[cc] = cc < nvalid ? xs[cc] : -INFINITY;
+            if (!kFull) xs[cc] = cc < nvalid ? xs[cc] : -INFINITY;
           }
-          float mx8[8];
+          float mx4[4];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mx8[k] = xs[k];
+          for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(xs[k], xs[k + 4]);
 #pragma unroll
-          for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], xs[cc]);
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          for (int cc = 8; cc < 64; cc += 8) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(mx4[k], fmaxf(xs[cc + k], xs[cc + k + 4]));
+          }
+          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
           const float m_tile = mx == -INFINITY ? -INFINITY : mx * f;  // f > 0 keeps the argmax
           const float m_new = fmaxf(m_run, m_tile);
           const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
@@ -561,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 arg = __ffma2_rn(make_float2(xs[cc], xs[cc + 1]), f2, nm2);
             float p0 = ex2(arg.x);
             float p1 = ex2(arg.y);
-            if (!full) {
+            if (!kFull) {  // masked columns of a row whose max is still -inf
               p0 = cc < nvalid ? p0 : 0.0f;
               p1 = cc + 1 < nvalid ? p1 : 0.0f;
             }
@@ -575,10 +602,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 l2 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
           l_run = l_run * alpha + (l2.x + l2.y);
         };
-        if (prec == TRA_PREC_BF16)
-          softmax_row(std::integral_constant<bool, false>{});
-        else
-          softmax_row(std::integral_constant<bool, true>{});
+        using T_ = std::true_type;
+        using F_ = std::false_type;
+        if (prec == TRA_PREC_BF16) {
+          if (full) softmax_row(F_{}, T_{}); else softmax_row(F_{}, F_{});
+        } else {
+          if (full) softmax_row(T_{}, T_{}); else softmax_row(T_{}, F_{});
+        }
       }
       if (warp_need && i >= 1) {
         // rescaling O needs every earlier P V complete.  sfull(i) already implies
