@@ -43,7 +43,12 @@ namespace {
 
 constexpr int kThreads = 416;
 constexpr int kUnits = 2;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 2^8 growth
+// log2 units: O and l are rescaled only once the running max has grown by more
+// than 2^16.  Until then P (bf16, exponent range of fp32) may reach 2^16, and
+// with fewer than 2^31 keys per row l < 2^47 and |O| < 2^47 * max|V| stay far
+// inside fp32; rarer rescales matter because each one waits for the previous
+// P V to complete.
+constexpr float kRescaleThreshold = 16.0f;
 constexpr int kSmemLimit = 232448;         // max dynamic shared memory per CTA on sm_100
 
 template <int D, int MODE>
@@ -93,7 +98,6 @@ __device__ __forceinline__ uint32_t i8_swz_offset(int r, int c) {
 struct MergeCursor {
   const uint32_t* e;
   int p0, e0, p1, e1;
-  __device__ __forceinline__ bool more() const { return p0 < e0 || p1 < e1; }
   __device__ __forceinline__ bool next(uint32_t& val, int& mask) {
     const uint32_t a = p0 < e0 ? __ldg(e + p0) : 0xFFFFFFFFu;
     const uint32_t b = p1 < e1 ? __ldg(e + p1) : 0xFFFFFFFFu;
@@ -126,7 +130,6 @@ struct Schedule {
     }
     return false;
   }
-  __device__ __forceinline__ bool more(int u) const { return u ? c1.more() : c0.more(); }
 };
 
 // One work unit: query head h of sequence b, q-tiles (2j, 2j+1).
@@ -513,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = 0: its warps skip the TMEM read and every exponential.
       const bool half_applies = ((mask >> half) & 1) && half_valid;
       uint32_t pk[32];
-      bool warp_need = false;
+      bool warp_need = false, warp_rescale_o = false;
       float alpha = 1.0f;
       if (!half_applies) {
 #pragma unroll
@@ -560,19 +563,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             xs[cc] = kInt ? (float)(int)sr[cc] : __uint_as_float(sr[cc]);
             if (!kFull) xs[cc] = cc < nvalid ? xs[cc] : -INFINITY;
           }
-          float mx4[4];
+          float mx;
+          if (kInt && kFull) {
+            // integer row max on the raw accumulators, independent of the conversions
+            int mi4[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(xs[k], xs[k + 4]);
+            for (int k = 0; k < 4; ++k) mi4[k] = max((int)sr[k], (int)sr[k + 4]);
 #pragma unroll
-          for (int cc = 8; cc < 64; cc += 8) {
+            for (int cc = 8; cc < 64; cc += 8) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(mx4[k], fmaxf(xs[cc + k], xs[cc + k + 4]));
+              for (int k = 0; k < 4; ++k)
+                mi4[k] = __vimax3_s32(mi4[k], (int)sr[cc + k], (int)sr[cc + k + 4]);
+            }
+            mx = (float)max(max(mi4[0], mi4[1]), max(mi4[2], mi4[3]));
+          } else {
+            float mx4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(xs[k], xs[k + 4]);
+#pragma unroll
+            for (int cc = 8; cc < 64; cc += 8) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(mx4[k], fmaxf(xs[cc + k], xs[cc + k + 4]));
+            }
+            mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
           }
-          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
           const float m_tile = mx == -INFINITY ? -INFINITY : mx * f;  // f > 0 keeps the argmax
           const float m_new = fmaxf(m_run, m_tile);
           const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
           warp_need = __any_sync(0xffffffffu, need);
+          // O rows that have seen no key yet are exactly zero: no rescale
+          warp_rescale_o = __any_sync(0xffffffffu, need && m_run != -INFINITY);
           if (warp_need && m_new > m_run) {
             alpha = ex2(m_run - m_new);  // m_run = -inf gives 0
             m_run = m_new;
@@ -610,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (full) softmax_row(T_{}, T_{}); else softmax_row(T_{}, F_{});
         }
       }
-      if (warp_need && i >= 1) {
+      if (warp_rescale_o && i >= 1) {
         // rescaling O needs every earlier P V complete.  sfull(i) already implies
         // P V(<= i-2) complete (they were issued before QK(i)), so ofull is at
         // phase i-1 or i and the parity wait below is exact.
