@@ -59,6 +59,29 @@ def parse():
     return ap.parse_args()
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
+# each dominant kernel, keyed by the SHA-256 prefix of the kernel source that was captured; a
+# source that has changed since reports null.  Captures: profiles/prefill_kernel_bitmask_32k.md
+# and profiles/decode_split_kernel_b16_32k.md.
+PROFILED_TRAFFIC = {
+    "prefill.cu": ("3967798f436d8325", 3_419_179_216),
+    "decode.cu": ("4ad208c3ea7b8b98", 667_361_024),
+}
+
+
+def profiled_traffic(src):
+    import hashlib
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "tile_routed_mixed_causal_b200",
+                        "csrc", src)
+    want, nbytes = PROFILED_TRAFFIC[src]
+    try:
+        with open(path, "rb") as f:
+            have = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return nbytes if have == want else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -264,7 +287,7 @@ def decode_bench(device, passes, stream, hbm_gbs):
         "ms_per_token_step": round(ms / steps, 4),
         "bytes_per_step": int(pass_bytes / steps),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
-                     "frac": round(gbs / hbm_gbs, 4), "traffic": None,
+                     "frac": round(gbs / hbm_gbs, 4), "traffic": profiled_traffic("decode.cu"),
                      "kernel": "decode_split_kernel + decode_combine_kernel (one ABI call)"},
         "gpu_launches_per_step": 2,
     }
@@ -463,7 +486,8 @@ def main():
             },
             "roofline": {
                 "bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak_eff, 2),
-                "unit": "TFLOP/s", "frac": round(achieved / peak_eff, 4), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(achieved / peak_eff, 4),
+                "traffic": profiled_traffic("prefill.cu"),
                 "kernel": "prefill_kernel<128, bitmask>",
                 "peak_basis": f"tile-mix weighted: bf16 {bf16_tflops} TF/s ({peak_src}, burst), "
                               f"int8 = 2x bf16 (nominal ratio)",
