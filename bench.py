@@ -56,6 +56,10 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part only (used for profiler captures); prints a reduced line")
+    ap.add_argument("--workload", choices=["bitmask_32k", "llama8b_8k", "varlen_8"],
+                    default="bitmask_32k",
+                    help="prefill workload for --only prefill (the full bench line always uses "
+                         "bitmask_32k)")
     return ap.parse_args()
 
 
@@ -139,17 +143,21 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- prefill
-def prefill_setup(device):
+def prefill_setup(device, workload="bitmask_32k"):
     import tile_routed_mixed_causal_b200 as tra
     from tile_routed_mixed_causal_b200 import api
     from tile_routed_mixed_causal_b200 import workloads as wl
 
-    w = wl.bitmask_32k()
+    w = getattr(wl, workload)()
     t = wl.make_inputs(w, device)
     q, k, v = t["q"], t["k"], t["v"]
     shape = tra.Shape(w.cu_seqlens, w.Hq, w.Hkv, w.d, device=device)
-    bitmask = torch.from_numpy(w.bitmask.view(np.int32)).to(device)
-    pol = tra.Policy.from_bitmask(bitmask, w.G)
+    if w.mode == "bitmask":
+        bitmask = torch.from_numpy(w.bitmask.view(np.int32)).to(device)
+        pol = tra.Policy.from_bitmask(bitmask, w.G)
+    else:
+        bitmask = torch.zeros(1, dtype=torch.int32, device=device)
+        pol = tra.Policy.boundary(w.b1, w.b2)
     plan = api.PrefillPlan(shape, pol, device=device)
     out = torch.empty_like(q)
     plan.lists()
@@ -317,13 +325,15 @@ def oracle_sample(w, q, k, v, qtiles, head=0):
     return 2 * tiles * TILE_OPS_PER_GEMM * w.d, dt, tiles
 
 
-def cpu_baseline(S, budget_s=15.0):
+def cpu_baseline(S, budget_s=12.0):
     w = S["w"]
     nt = w.ntiles
     rows = []
     ops = secs = tiles = 0
-    # late q-tiles first (the heaviest rows), until the time budget is used
-    for qt in [nt - 1, 3 * nt // 4, nt // 2, nt // 4, nt - 2, 3 * nt // 4 + 1, nt // 2 + 1]:
+    # q-tiles spread over the sequence (heavy late rows first), until the time budget is used
+    order = [nt - 1, 3 * nt // 4, nt // 2, nt // 4]
+    order += [int(x) for x in np.random.default_rng(7).permutation(nt) if int(x) not in order]
+    for qt in order:
         o, s, t = oracle_sample(w, S["q"], S["k"], S["v"], [qt])
         rows.append(qt)
         ops += o
@@ -332,7 +342,8 @@ def cpu_baseline(S, budget_s=15.0):
         if secs > budget_s:
             break
     return {"value": round(ops / secs / 1e12, 8), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"head 0, q-tiles {rows} of the 32K bitmask workload ({tiles} kept tiles, "
+            "sample": f"head 0, {len(rows)} q-tile rows (first {rows[:6]}, then a seeded "
+                      f"permutation) of the 32K bitmask workload ({tiles} kept tiles, "
                       f"quantisation + traversal + fp64 attention), {secs:.1f} s single-threaded"}
 
 
@@ -417,15 +428,22 @@ def main():
             print(json.dumps({"only": "decode", **decode_bench(device, args.decode_passes, stream,
                                                               hbm_gbs)}), flush=True)
         return
-    S = prefill_setup(device)
     if args.only == "prefill":
+        S = prefill_setup(device, args.workload)
         total_ms, attn_ms, _ = run_prefill_bench(S, args.steps, args.warmup, stream)
         if rank == 0:
             ops = prefill_ops(S)
-            print(json.dumps({"only": "prefill", "ms_per_step": total_ms / args.steps,
-                              "prefill_kernel_ms": sum(attn_ms) / len(attn_ms),
-                              "TOPS": ops / (total_ms / args.steps * 1e-3) / 1e12}), flush=True)
+            kern = sum(attn_ms) / len(attn_ms)
+            t_roof = roofline_time(S, bf16_tflops)
+            print(json.dumps({"only": "prefill", "workload": S["w"].name,
+                              "ms_per_step": total_ms / args.steps, "prefill_kernel_ms": kern,
+                              "TOPS": ops / (total_ms / args.steps * 1e-3) / 1e12,
+                              "kernel_TOPS": ops / (kern * 1e-3) / 1e12,
+                              "roofline_frac": t_roof / (kern * 1e-3),
+                              "tiles": S["tiles"], "bf16_tiles": S["n16"], "int8_tiles": S["n8"],
+                              "int4_tiles": S["n4"]}), flush=True)
         return
+    S = prefill_setup(device)
     ops = prefill_ops(S)
 
     clocks = ClockSampler(local if world > 1 else 0)

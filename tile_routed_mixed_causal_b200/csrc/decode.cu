@@ -16,9 +16,10 @@
 //   softmax: per head over the warp's fragment lanes, K scale and 1/sqrt(d)
 //           folded into the exponent, V scale folded into P (f16, staged per warp);
 //   P V:    O^T += V^T P^T on the tensor cores, V fed by ldmatrix.trans.
-// The last split also covers the bf16 tail (earlier decode tokens + the new
-// one).  The four warps' states are merged per CTA, and a small combine kernel
-// merges the splits and advances tail_len.
+// The bf16 tail (earlier decode tokens + the new one) is a split of its own:
+// CTA x = 0 of every (sequence, KV head), scheduled first, whose four warps
+// share the tail keys on the CUDA cores.  The four warps' states are merged per
+// CTA, and a small combine kernel merges the splits and advances tail_len.
 #include "tra_device.cuh"
 #include "tra_launch.h"
 
@@ -40,26 +41,6 @@ __device__ __forceinline__ float ex2(float x) {
 template <int R>
 __device__ __forceinline__ uint32_t swz(int r, int c) {
   return r * R + ((c ^ ((r * R >> 7) & (R / 16 - 1))) << 4);
-}
-
-// Four signed INT8 codes of a word -> two float2 (exact): each byte, offset by
-// 128, is placed in the low mantissa byte of 2^23 and 2^23 + 128 is subtracted.
-__device__ __forceinline__ void i8x4_to_f2(uint32_t w, float2& a, float2& b) {
-  const uint32_t u = w ^ 0x80808080u;
-  const float2 off = make_float2(-8388736.0f, -8388736.0f);
-  a = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)),
-                             __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651))),
-                 off);
-  b = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)),
-                             __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653))),
-                 off);
-}
-
-// Eight INT4 codes of a word (even channel in the low nibble) -> four float2.
-__device__ __forceinline__ void i4x8_to_f2(uint32_t w, float2 (&f)[4]) {
-  const uint2 e = expand_int4x8(w);  // eight int8 codes in channel order
-  i8x4_to_f2(e.x, f[0], f[1]);
-  i8x4_to_f2(e.y, f[2], f[3]);
 }
 
 // ---------------------------------------------------------------- mma.sync helpers
@@ -122,7 +103,7 @@ struct DecCfg {
   static constexpr int kPBytes = kConsumers * 8 * kPStride * 2;
   static constexpr int kOffT = kOffP + kPBytes;            // tail p: [64 keys][GRP] float
   static constexpr int kTBytes = kTile * GRP * 4;
-  static constexpr int kStates = kConsumers + 1;           // four warps + the bf16 tail
+  static constexpr int kStates = kConsumers;               // one state per consumer warp
   // merge area [state][GRP][D + 2] floats, aliasing the drained ring
   static constexpr int kOffRed = 0;
   static constexpr int kRedBytes = kStates * GRP * (D + 2) * 4;
@@ -148,7 +129,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   volatile int* const err =
       reinterpret_cast<volatile int*>(sm + C::kOffBar + 2 * kDecStages * 8);
 
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  // x = 0: the bf16 tail of (b, kvh); x = 1 .. splits-1: data split x - 1
+  const int kvh = blockIdx.y, b = blockIdx.z;
+  const bool tail_cta = blockIdx.x == 0;
+  const int nsplit = p.splits - 1, split = (int)blockIdx.x - 1;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int grp = p.Hq / p.Hkv;
   const int seq0 = __ldg(p.cu + b);
@@ -156,45 +140,22 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   const int toff = seq_tile_offset(p.cu, b);
   const int tl = __ldg(p.tail_len + b);
   if (tl >= p.tail_cap) {
-    if (split == 0 && kvh == 0 && t == 0) {
+    if (tail_cta && kvh == 0 && t == 0) {
       atomicOr(p.status, TRA_DEV_TAIL_FULL);
       p.skip[b] = 1;
     }
     return;
   }
-  if (split == 0 && kvh == 0 && t == 0) p.skip[b] = 0;
-  const long long row = (long long)b * p.Hkv + kvh;
-  const int rs = __ldg(p.row_ptr + row), re = __ldg(p.row_ptr + row + 1);
-  const int n = re - rs;
-  const int my0 = rs + (int)((long long)n * split / p.splits);
-  const int ntile = rs + (int)((long long)n * (split + 1) / p.splits) - my0;
-  const bool last = split == p.splits - 1;
-
-  // append the new token to the tail (split 0; the tail slot tl is read by nobody)
-  if (split == 0) {
-    const long long src = ((long long)b * p.Hkv + kvh) * D;
-    const long long dst = (((long long)b * p.Hkv + kvh) * p.tail_cap + tl) * D;
-    for (int c = t; c < D; c += kDecThreads) {
-      p.k_tail[dst + c] = p.k_new[src + c];
-      p.v_tail[dst + c] = p.v_new[src + c];
-    }
+  if (tail_cta && kvh == 0 && t == 0) p.skip[b] = 0;
+  int my0 = 0, ntile = 0;
+  if (!tail_cta) {
+    const long long row = (long long)b * p.Hkv + kvh;
+    const int rs = __ldg(p.row_ptr + row), re = __ldg(p.row_ptr + row + 1);
+    const int n = re - rs;
+    my0 = rs + (int)((long long)n * split / nsplit);
+    ntile = rs + (int)((long long)n * (split + 1) / nsplit) - my0;
   }
-  // q of the group's heads as fp32 channel pairs q2[pair][g] (tail path and fragments)
-  for (int x = t; x < (D / 2) * GRP; x += kDecThreads) {
-    const int cp = x / GRP, g = x % GRP;
-    float2 v = make_float2(0.0f, 0.0f);
-    if (g < grp) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(
-          p.q + ((long long)b * p.Hq + kvh * grp + g) * D + 2 * cp);
-      v = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-    }
-    q2[cp * GRP + g] = v;
-  }
-  // zero the P rows of padded heads (never written; N = 8 heads per MMA)
-  {
-    __half* pz = reinterpret_cast<__half*>(sm + C::kOffP);
-    for (int x = t; x < kConsumers * 8 * C::kPStride; x += kDecThreads) pz[x] = __float2half(0.0f);
-  }
+  // barriers first, so that the producer's first copies overlap the consumers' set-up
   if (t == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(bar_full + s * 8, 1);
@@ -230,6 +191,32 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     named_sync(2);  // merge area written
   } else {
     // ------------------------------------------------------------ consumers
+    // append the new token to the tail (tail CTA; the tail slot tl is read by nobody)
+    if (tail_cta) {
+      const long long src = ((long long)b * p.Hkv + kvh) * D;
+      const long long dst = (((long long)b * p.Hkv + kvh) * p.tail_cap + tl) * D;
+      for (int c = t; c < D; c += 32 * kConsumers) {
+        p.k_tail[dst + c] = p.k_new[src + c];
+        p.v_tail[dst + c] = p.v_new[src + c];
+      }
+    }
+    // q of the group's heads as fp32 channel pairs q2[pair][g] (tail path and fragments)
+    for (int x = t; x < (D / 2) * GRP; x += 32 * kConsumers) {
+      const int cp = x / GRP, gq = x % GRP;
+      float2 v = make_float2(0.0f, 0.0f);
+      if (gq < grp) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(
+            p.q + ((long long)b * p.Hq + kvh * grp + gq) * D + 2 * cp);
+        v = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+      }
+      q2[cp * GRP + gq] = v;
+    }
+    // zero the P rows of padded heads (never written; N = 8 heads per MMA)
+    {
+      __half* pz = reinterpret_cast<__half*>(sm + C::kOffP);
+      for (int x = t; x < kConsumers * 8 * C::kPStride; x += 32 * kConsumers) pz[x] = __float2half(0.0f);
+    }
+    asm volatile("bar.sync 3, %0;" ::"n"(32 * kConsumers) : "memory");  // consumers only
     const int g = lane >> 2, tq = lane & 3;  // fragment group / thread in group
     // Power-of-two scale keeping q inside the f16 range (exact: only the exponent moves)
     float qmax = 0.0f;
@@ -285,79 +272,80 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     const uint32_t pw_addr = smem_u32(pw);
     const int mrow = lane & 7, mj = lane >> 3;  // ldmatrix: this lane's row / matrix
 
-    // bf16 tail (last split, warp 0): tokens [0, tl) of the tail buffer and the new
-    // token at tl, CUDA-core fp32 math with its own softmax state
+    // bf16 tail (tail CTA): tokens [0, tl) of the tail buffer and the new token at
+    // tl; warp w takes tokens w, w + 4, ..., one per lane, with CUDA-core fp32 math
+    // and its own softmax state.  All of a lane's loads are issued before use.
     auto tail_pass = [&](float (&tm)[GRP], float (&tlsum)[GRP], float2 (&to)[GRP][C::kCh / 2]) {
-        float* tp = reinterpret_cast<float*>(sm + C::kOffT);
-        const long long tbase = ((long long)b * p.Hkv + kvh) * p.tail_cap;
-        const long long nbase = ((long long)b * p.Hkv + kvh) * D;
-        for (int t0 = 0; t0 <= tl; t0 += kTile) {
-          float sc[2][GRP];
+      const long long tbase = ((long long)b * p.Hkv + kvh) * p.tail_cap;
+      const long long nbase = ((long long)b * p.Hkv + kvh) * D;
+      for (int c0 = 0; warp + 4 * c0 <= tl; c0 += 32) {  // this warp's next 32 tokens
+        const int pos = warp + 4 * (c0 + lane);
+        const bool valid = pos <= tl;
+        float2 acc[GRP];
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int pos = t0 + lane + 32 * k;
-            float2 acc[GRP];
+        for (int gg = 0; gg < GRP; ++gg) acc[gg] = make_float2(0.0f, 0.0f);
+        if (valid) {
+          const uint16_t* kr = pos == tl ? p.k_new + nbase : p.k_tail + (tbase + pos) * D;
+          uint4 kw[D / 8];
 #pragma unroll
-            for (int gg = 0; gg < GRP; ++gg) acc[gg] = make_float2(0.0f, 0.0f);
-            if (pos <= tl) {
-              const uint16_t* kr = pos == tl ? p.k_new + nbase : p.k_tail + (tbase + pos) * D;
-              for (int c = 0; c < D / 8; ++c) {
-                const uint4 w = *reinterpret_cast<const uint4*>(kr + c * 8);
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          for (int c = 0; c < D / 8; ++c) kw[c] = *reinterpret_cast<const uint4*>(kr + c * 8);
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                  const float2 kk = make_float2(__uint_as_float(ww[x] << 16),
-                                                __uint_as_float(ww[x] & 0xFFFF0000u));
+          for (int c = 0; c < D / 8; ++c) {
+            const uint32_t ww[4] = {kw[c].x, kw[c].y, kw[c].z, kw[c].w};
 #pragma unroll
-                  for (int gg = 0; gg < GRP; ++gg)
-                    acc[gg] = __ffma2_rn(kk, q2[(c * 4 + x) * GRP + gg], acc[gg]);
-                }
-              }
-            }
-#pragma unroll
-            for (int gg = 0; gg < GRP; ++gg)
-              sc[k][gg] = pos <= tl ? (acc[gg].x + acc[gg].y) * p.scale_log2 : -INFINITY;
-          }
-          float al[GRP];
-#pragma unroll
-          for (int gg = 0; gg < GRP; ++gg) {
-            float mx = fmaxf(sc[0][gg], sc[1][gg]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            const float m_new = fmaxf(tm[gg], mx);
-            const float mb = m_new == -INFINITY ? 0.0f : m_new;
-            const float p0 = ex2(sc[0][gg] - mb), p1 = ex2(sc[1][gg] - mb);
-            float ps = p0 + p1;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-            al[gg] = ex2(tm[gg] - mb);
-            tlsum[gg] = tlsum[gg] * al[gg] + ps;
-            tm[gg] = m_new;
-            tp[lane * GRP + gg] = p0;
-            tp[(lane + 32) * GRP + gg] = p1;
-          }
-          __syncwarp();
-#pragma unroll
-          for (int gg = 0; gg < GRP; ++gg)
-#pragma unroll
-            for (int k = 0; k < C::kCh / 2; ++k)
-              to[gg][k] = __fmul2_rn(to[gg][k], make_float2(al[gg], al[gg]));
-          for (int key = 0; key < kTile; ++key) {
-            const int pos = t0 + key;
-            if (pos > tl) break;
-            const uint16_t* vr = pos == tl ? p.v_new + nbase : p.v_tail + (tbase + pos) * D;
-#pragma unroll
-            for (int k = 0; k < C::kCh / 2; ++k) {
-              const uint32_t w = *reinterpret_cast<const uint32_t*>(vr + lane * C::kCh + 2 * k);
-              const float2 vv = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+            for (int x = 0; x < 4; ++x) {
+              const float2 kk = make_float2(__uint_as_float(ww[x] << 16),
+                                            __uint_as_float(ww[x] & 0xFFFF0000u));
 #pragma unroll
               for (int gg = 0; gg < GRP; ++gg)
-                to[gg][k] = __ffma2_rn(vv, make_float2(tp[key * GRP + gg], tp[key * GRP + gg]), to[gg][k]);
+                acc[gg] = __ffma2_rn(kk, q2[(c * 4 + x) * GRP + gg], acc[gg]);
             }
           }
-          __syncwarp();
         }
-          };
+        float pk[GRP], al[GRP];
+#pragma unroll
+        for (int gg = 0; gg < GRP; ++gg) {
+          const float sc = valid ? (acc[gg].x + acc[gg].y) * p.scale_log2 : -INFINITY;
+          float mx = sc;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float m_new = fmaxf(tm[gg], mx);
+          const float mb = m_new == -INFINITY ? 0.0f : m_new;
+          pk[gg] = valid ? ex2(sc - mb) : 0.0f;
+          float ps = pk[gg];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+          al[gg] = ex2(tm[gg] - mb);  // -inf -> 0
+          tlsum[gg] = tlsum[gg] * al[gg] + ps;
+          tm[gg] = m_new;
+        }
+#pragma unroll
+        for (int gg = 0; gg < GRP; ++gg)
+#pragma unroll
+          for (int k = 0; k < C::kCh / 2; ++k)
+            to[gg][k] = __fmul2_rn(to[gg][k], make_float2(al[gg], al[gg]));
+        // P V: this lane's channels lane * kCh .. + kCh, tokens of the chunk in order
+        const int nk = min(32, (tl - warp) / 4 - c0 + 1);
+#pragma unroll 4
+        for (int j = 0; j < nk; ++j) {
+          const int pj = warp + 4 * (c0 + j);
+          const uint16_t* vr = pj == tl ? p.v_new + nbase : p.v_tail + (tbase + pj) * D;
+          uint32_t vw[C::kCh / 2];
+#pragma unroll
+          for (int k = 0; k < C::kCh / 2; ++k)
+            vw[k] = *reinterpret_cast<const uint32_t*>(vr + lane * C::kCh + 2 * k);
+#pragma unroll
+          for (int gg = 0; gg < GRP; ++gg) {
+            const float pv = __shfl_sync(0xffffffffu, pk[gg], j);
+#pragma unroll
+            for (int k = 0; k < C::kCh / 2; ++k)
+              to[gg][k] = __ffma2_rn(make_float2(__uint_as_float(vw[k] << 16),
+                                                 __uint_as_float(vw[k] & 0xFFFF0000u)),
+                                     make_float2(pv, pv), to[gg][k]);
+          }
+        }
+      }
+    };
 
     bool ok = true;
     for (int i = warp; i < ntile; i += kConsumers) {
@@ -380,7 +368,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       if (is8) {
 #pragma unroll
         for (int cb = 0; cb < D / 32; ++cb)
-#pragma unroll
+#pragma unroll 1
           for (int k = 0; k < 4; ++k) {
             uint32_t r[4];
             ldsm_x4(kb + swz<C::kRow8>(16 * k + mrow + 8 * (mj & 1), 2 * cb + (mj >> 1)), r);
@@ -395,7 +383,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       } else {
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb)
-#pragma unroll
+#pragma unroll 1
           for (int k = 0; k < 4; ++k) {
             uint32_t r[4];
             ldsm_x4(kb + swz<C::kRow4>(16 * k + mrow + 8 * (mj & 1), 2 * cb + (mj >> 1)), r);
@@ -496,7 +484,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       }
       __syncwarp();
       // ---- O^T += V^T P^T: B fragment = P[head g][keys 16k + 2tq (+1), +8 (+9)]
-#pragma unroll
+#pragma unroll 1
       for (int k = 0; k < 4; ++k) {
         uint32_t pb0, pb1;
         asm volatile("ld.shared.b32 %0, [%1];" : "=r"(pb0) : "r"(pw_addr + (g * C::kPStride + 16 * k + 2 * tq) * 2));
@@ -539,68 +527,68 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       if (lane == 0) mbar_arrive(bar_empty + s * 8);
     }
 
-    // ---- bf16 tail (computed below by warp 0) and the shared-memory merge; the
-    // merge area aliases the ring, so every warp must be done with the ring first
-    float tm[GRP], tlsum[GRP];
-    float2 to[GRP][C::kCh / 2];
-#pragma unroll
-    for (int gg = 0; gg < GRP; ++gg) {
-      tm[gg] = -INFINITY;
-      tlsum[gg] = 0.0f;
-#pragma unroll
-      for (int k = 0; k < C::kCh / 2; ++k) to[gg][k] = make_float2(0.0f, 0.0f);
-    }
-    if (warp == 0 && ok && last) tail_pass(tm, tlsum, to);
-    named_sync(1);
+    // ---- the shared-memory merge; the merge area aliases the ring, so every warp
+    // must be done with the ring first.  Tail CTAs fill the slots from the tail pass.
     float* rw = red + warp * GRP * (D + 2);
-    for (int x = lane; x < GRP * (D + 2); x += 32) rw[x] = 0.0f;
-    __syncwarp();
+    if (tail_cta) {
+      float tm[GRP], tlsum[GRP];
+      float2 to[GRP][C::kCh / 2];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int hd = 2 * tq + hh;
-      if (hd < GRP) {
+      for (int gg = 0; gg < GRP; ++gg) {
+        tm[gg] = -INFINITY;
+        tlsum[gg] = 0.0f;
 #pragma unroll
-        for (int j = 0; j < C::kB8; ++j) {
-          rw[hd * (D + 2) + 16 * j + 2 * g] = o8[j][hh];
-          rw[hd * (D + 2) + 16 * j + 2 * g + 1] = o8[j][2 + hh];
-        }
-        if (g == 0) {
-          rw[hd * (D + 2) + D] = m_run[hh];
-          rw[hd * (D + 2) + D + 1] = l_run[hh];
-        }
+        for (int k = 0; k < C::kCh / 2; ++k) to[gg][k] = make_float2(0.0f, 0.0f);
       }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int hd = 2 * tq + hh;
-      if (hd < GRP) {
-#pragma unroll
-        for (int j = 0; j < C::kB4; ++j)
-#pragma unroll
-          for (int ab = 0; ab < 2; ++ab) {
-            rw[hd * (D + 2) + 32 * j + 4 * g + 2 * ab] += o4[j][ab][hh];
-            rw[hd * (D + 2) + 32 * j + 4 * g + 2 * ab + 1] += o4[j][ab][2 + hh];
-          }
-      }
-    }
-
-    if (warp == 0) {
-      float* rt = red + kConsumers * GRP * (D + 2);
+      tail_pass(tm, tlsum, to);
+      named_sync(1);
 #pragma unroll
       for (int gg = 0; gg < GRP; ++gg) {
 #pragma unroll
         for (int k = 0; k < C::kCh / 2; ++k)
-          *reinterpret_cast<float2*>(rt + gg * (D + 2) + lane * C::kCh + 2 * k) = to[gg][k];
+          *reinterpret_cast<float2*>(rw + gg * (D + 2) + lane * C::kCh + 2 * k) = to[gg][k];
         if (lane == 0) {
-          rt[gg * (D + 2) + D] = tm[gg];
-          rt[gg * (D + 2) + D + 1] = tlsum[gg];
+          rw[gg * (D + 2) + D] = tm[gg];
+          rw[gg * (D + 2) + D + 1] = tlsum[gg];
+        }
+      }
+    } else {
+      named_sync(1);
+      for (int x = lane; x < GRP * (D + 2); x += 32) rw[x] = 0.0f;
+      __syncwarp();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int hd = 2 * tq + hh;
+        if (hd < GRP) {
+#pragma unroll
+          for (int j = 0; j < C::kB8; ++j) {
+            rw[hd * (D + 2) + 16 * j + 2 * g] = o8[j][hh];
+            rw[hd * (D + 2) + 16 * j + 2 * g + 1] = o8[j][2 + hh];
+          }
+          if (g == 0) {
+            rw[hd * (D + 2) + D] = m_run[hh];
+            rw[hd * (D + 2) + D + 1] = l_run[hh];
+          }
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int hd = 2 * tq + hh;
+        if (hd < GRP) {
+#pragma unroll
+          for (int j = 0; j < C::kB4; ++j)
+#pragma unroll
+            for (int ab = 0; ab < 2; ++ab) {
+              rw[hd * (D + 2) + 32 * j + 4 * g + 2 * ab] += o4[j][ab][hh];
+              rw[hd * (D + 2) + 32 * j + 4 * g + 2 * ab + 1] += o4[j][ab][2 + hh];
+            }
         }
       }
     }
     named_sync(2);
   }
-  // merge the consumer warps and the tail into this split's partial (m, l, o)
+  // merge the consumer warps into this split's partial (m, l, o)
   for (int x = t; x < GRP * D; x += kDecThreads) {
     const int gg = x / D, c = x % D;
     if (gg >= grp) continue;
@@ -615,7 +603,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       L += r[D + 1] * wt;
       o += r[c] * wt;
     }
-    const long long pi = ((long long)b * p.Hq + kvh * grp + gg) * p.splits + split;
+    const long long pi = ((long long)b * p.Hq + kvh * grp + gg) * p.splits + blockIdx.x;
     p.part_o[pi * D + c] = o;
     if (c == 0) {
       p.part_ml[pi * 2] = M;
@@ -677,13 +665,14 @@ cudaError_t launch_dec_d(const DecodeParams& p, const DecodeMaps& m, cudaStream_
 
 }  // namespace
 
+// Partials per (sequence, KV head): the data splits plus the bf16-tail split.
 int decode_splits(int B, int Hkv) {
-  const int target = 2048;  // about seven waves of two CTAs per SM: a small tail
+  const int target = 1024;  // about 3.5 waves of two CTAs per SM: long CTAs, a small tail
   const int rows = B * Hkv;
   int s = (target + rows - 1) / rows;
   if (s < 1) s = 1;
-  if (s > TRA_MAX_DECODE_SPLITS) s = TRA_MAX_DECODE_SPLITS;
-  return s;
+  if (s > TRA_MAX_DECODE_SPLITS - 1) s = TRA_MAX_DECODE_SPLITS - 1;
+  return s + 1;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodeMaps& m, cudaStream_t s) {
