@@ -76,9 +76,32 @@ __device__ __forceinline__ uint32_t h2_from_bytes(uint32_t x, uint32_t sel, uint
   asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(h) : "r"(bias2));
   return h;
 }
+// Eight signed INT4 codes of a word (channel i in bits 4i .. 4i+3) -> four exact
+// f16x2: channels (0, 4), (1, 5), (2, 6), (3, 7).  One lop3 per pair computes
+// (x & mask) ^ magic, which flips the nibble's sign bit (code + 8) and places it
+// in the low mantissa bits of 1024.0h (even nibbles) or, scaled by 16, of the
+// same (odd nibbles); a packed subtract / fma removes the offset exactly.
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));  // (a & b) ^ c
+  return d;
+}
+__device__ __forceinline__ void i4x8_to_h2(uint32_t x, uint32_t (&h)[4]) {
+  const uint32_t y = x >> 8;
+  h[0] = and_xor(x, 0x000F000Fu, 0x64086408u);
+  h[1] = and_xor(x, 0x00F000F0u, 0x64806480u);
+  h[2] = and_xor(y, 0x000F000Fu, 0x64086408u);
+  h[3] = and_xor(y, 0x00F000F0u, 0x64806480u);
+  const uint32_t bias = 0x64086408u;      // (1032, 1032) = 1024 + 8
+  const uint32_t sixteenth = 0x2C002C00u;  // (1/16, 1/16)
+  const uint32_t m72 = 0xD480D480u;        // (-72, -72) = -(1024 + 128) / 16
+  asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(h[0]) : "r"(bias));
+  asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(h[2]) : "r"(bias));
+  asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h[1]) : "r"(sixteenth), "r"(m72));
+  asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h[3]) : "r"(sixteenth), "r"(m72));
+}
 constexpr uint32_t kSel01 = 0x5140, kSel23 = 0x5342, kSel02 = 0x5240, kSel13 = 0x5341;
 constexpr uint32_t kBias8 = 0x64806480u;  // f16x2 (1152, 1152) = 1024 + 128
-constexpr uint32_t kBias4 = 0x64086408u;  // f16x2 (1032, 1032) = 1024 + 8
 
 // Named barrier over the whole CTA, usable from different code locations.
 __device__ __forceinline__ void named_sync(int id) {
@@ -232,7 +255,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     // B fragments of q for head g (zero for padded heads), in the channel order
     // the K codes arrive in:
     //   INT8, 16-channel block j: (16j+4t, +1) and (16j+4t+2, +3)
-    //   INT4, 32-channel block j, half ab: (32j+8t+4ab, +1) and (32j+8t+4ab+2, +3)
+    //   INT4, 32-channel block j, half ab: (32j+8t+2ab, +4) and (32j+8t+2ab+1, +5)
     auto qv = [&](int c) -> float {
       if (g >= grp) return 0.0f;
       const float2 v = q2[(c >> 1) * GRP + g];
@@ -249,9 +272,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     for (int j = 0; j < C::kB4; ++j)
 #pragma unroll
       for (int ab = 0; ab < 2; ++ab) {
-        const int c = 32 * j + 8 * tq + 4 * ab;
-        qb4[j][ab][0] = f16x2_from(qv(c), qv(c + 1));
-        qb4[j][ab][1] = f16x2_from(qv(c + 2), qv(c + 3));
+        const int c = 32 * j + 8 * tq + 2 * ab;
+        qb4[j][ab][0] = f16x2_from(qv(c), qv(c + 4));
+        qb4[j][ab][1] = f16x2_from(qv(c + 1), qv(c + 5));
       }
 
     // this lane's state for heads 2tq, 2tq+1; O^T fragments: INT8 tiles accumulate in
@@ -389,23 +412,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             ldsm_x4(kb + swz<C::kRow4>(16 * k + mrow + 8 * (mj & 1), 2 * cb + (mj >> 1)), r);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // packed bytes 16h.. = channels 64cb + 32h ..
-              // codes of keys g / g+8 at channels 8tq .. 8tq+7, in channel order as bytes
-              uint32_t c0[2], c1[2];
-              {
-                const uint32_t x0 = r[2 * h] ^ 0x88888888u, x1 = r[2 * h + 1] ^ 0x88888888u;
-                const uint32_t lo0 = x0 & 0x0F0F0F0Fu, hi0 = (x0 >> 4) & 0x0F0F0F0Fu;
-                const uint32_t lo1 = x1 & 0x0F0F0F0Fu, hi1 = (x1 >> 4) & 0x0F0F0F0Fu;
-                c0[0] = __byte_perm(lo0, hi0, 0x5140);
-                c0[1] = __byte_perm(lo0, hi0, 0x7362);
-                c1[0] = __byte_perm(lo1, hi1, 0x5140);
-                c1[1] = __byte_perm(lo1, hi1, 0x7362);
-              }
+              // codes of keys g / g+8 at channels 8tq .. 8tq+7 as channel pairs (c, c+4)
+              uint32_t c0[4], c1[4];
+              i4x8_to_h2(r[2 * h], c0);
+              i4x8_to_h2(r[2 * h + 1], c1);
 #pragma unroll
               for (int ab = 0; ab < 2; ++ab) {
-                const uint32_t a[4] = {h2_from_bytes(c0[ab], kSel01, kBias4),
-                                       h2_from_bytes(c1[ab], kSel01, kBias4),
-                                       h2_from_bytes(c0[ab], kSel23, kBias4),
-                                       h2_from_bytes(c1[ab], kSel23, kBias4)};
+                const uint32_t a[4] = {c0[2 * ab], c1[2 * ab], c0[2 * ab + 1], c1[2 * ab + 1]};
                 mma16816(sacc[k], a, qb4[2 * cb + h][ab][0], qb4[2 * cb + h][ab][1]);
               }
             }
@@ -509,14 +522,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             ldsm_x4_t(vb + swz<C::kRow4>(16 * k + mrow + 8 * (mj & 1), 2 * cp + (mj >> 1)), r);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // 32 channels 64cp + 32h .. (4g .. 4g+3)
-              const uint32_t x0 = r[2 * h] ^ 0x88888888u, x1 = r[2 * h + 1] ^ 0x88888888u;
-              const uint32_t lo0 = x0 & 0x0F0F0F0Fu, hi0 = (x0 >> 4) & 0x0F0F0F0Fu;
-              const uint32_t lo1 = x1 & 0x0F0F0F0Fu, hi1 = (x1 >> 4) & 0x0F0F0F0Fu;
-              const uint32_t aA[4] = {h2_from_bytes(lo0, kSel02, kBias4), h2_from_bytes(hi0, kSel02, kBias4),
-                                      h2_from_bytes(lo1, kSel02, kBias4), h2_from_bytes(hi1, kSel02, kBias4)};
+              // words: keys (2tq, 2tq+1) / (2tq+8, 2tq+9), channels 4g .. 4g+3; the
+              // conversion yields one key pair per channel 4g + 0 .. 3
+              uint32_t v0[4], v1[4];
+              i4x8_to_h2(r[2 * h], v0);
+              i4x8_to_h2(r[2 * h + 1], v1);
+              const uint32_t aA[4] = {v0[0], v0[1], v1[0], v1[1]};
               mma16816(o4[2 * cp + h][0], aA, pb0, pb1);
-              const uint32_t aB[4] = {h2_from_bytes(lo0, kSel13, kBias4), h2_from_bytes(hi0, kSel13, kBias4),
-                                      h2_from_bytes(lo1, kSel13, kBias4), h2_from_bytes(hi1, kSel13, kBias4)};
+              const uint32_t aB[4] = {v0[2], v0[3], v1[2], v1[3]};
               mma16816(o4[2 * cp + h][1], aB, pb0, pb1);
             }
           }
