@@ -294,6 +294,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     __half* const pw = reinterpret_cast<__half*>(sm + C::kOffP) + warp * 8 * C::kPStride;
     const uint32_t pw_addr = smem_u32(pw);
     const int mrow = lane & 7, mj = lane >> 3;  // ldmatrix: this lane's row / matrix
+    // ldmatrix addresses: this lane's row of key block k is 16k + mrow + 8 (mj & 1),
+    // its 16-byte chunk 2 cb + (mj >> 1).  Key blocks are 8-row aligned, so the TMA
+    // swizzle term of the row is the same for every k: per-lane offsets per channel
+    // block, plus 16 k rows.
+    uint32_t off8[D / 32], off4[D / 64];
+#pragma unroll
+    for (int cb = 0; cb < D / 32; ++cb)
+      off8[cb] = swz<C::kRow8>(mrow + 8 * (mj & 1), 2 * cb + (mj >> 1));
+#pragma unroll
+    for (int cb = 0; cb < D / 64; ++cb)
+      off4[cb] = swz<C::kRow4>(mrow + 8 * (mj & 1), 2 * cb + (mj >> 1));
 
     // bf16 tail (tail CTA): tokens [0, tl) of the tail buffer and the new token at
     // tl; warp w takes tokens w, w + 4, ..., one per lane, with CUDA-core fp32 math
@@ -391,10 +402,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       if (is8) {
 #pragma unroll
         for (int cb = 0; cb < D / 32; ++cb)
-#pragma unroll 1
+#pragma unroll
           for (int k = 0; k < 4; ++k) {
             uint32_t r[4];
-            ldsm_x4(kb + swz<C::kRow8>(16 * k + mrow + 8 * (mj & 1), 2 * cb + (mj >> 1)), r);
+            ldsm_x4(kb + 16 * C::kRow8 * k + off8[cb], r);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // channels 32cb + 16h ..
               const uint32_t u0 = r[2 * h] ^ 0x80808080u, u1 = r[2 * h + 1] ^ 0x80808080u;
@@ -406,10 +417,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       } else {
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb)
-#pragma unroll 1
+#pragma unroll
           for (int k = 0; k < 4; ++k) {
             uint32_t r[4];
-            ldsm_x4(kb + swz<C::kRow4>(16 * k + mrow + 8 * (mj & 1), 2 * cb + (mj >> 1)), r);
+            ldsm_x4(kb + 16 * C::kRow4 * k + off4[cb], r);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // packed bytes 16h.. = channels 64cb + 32h ..
               // codes of keys g / g+8 at channels 8tq .. 8tq+7 as channel pairs (c, c+4)
@@ -432,10 +443,18 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       for (int k = 0; k < 4; ++k)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int key0 = 16 * k + g, key1 = key0 + 8;
-          sv[hh][2 * k] = key0 < nvalid ? sacc[k][hh] * ks : -INFINITY;
-          sv[hh][2 * k + 1] = key1 < nvalid ? sacc[k][2 + hh] * ks : -INFINITY;
+          sv[hh][2 * k] = sacc[k][hh] * ks;
+          sv[hh][2 * k + 1] = sacc[k][2 + hh] * ks;
         }
+      if (nvalid < kTile) {  // a sequence's last tile: keys past its end are masked
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            if (16 * k + g >= nvalid) sv[hh][2 * k] = -INFINITY;
+            if (16 * k + g + 8 >= nvalid) sv[hh][2 * k + 1] = -INFINITY;
+          }
+      }
       float mt[2], alpha[2] = {1.0f, 1.0f};
       bool need = false;
 #pragma unroll
@@ -497,7 +516,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       }
       __syncwarp();
       // ---- O^T += V^T P^T: B fragment = P[head g][keys 16k + 2tq (+1), +8 (+9)]
-#pragma unroll 1
+#pragma unroll
       for (int k = 0; k < 4; ++k) {
         uint32_t pb0, pb1;
         asm volatile("ld.shared.b32 %0, [%1];" : "=r"(pb0) : "r"(pw_addr + (g * C::kPStride + 16 * k + 2 * tq) * 2));
@@ -506,7 +525,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 #pragma unroll
           for (int cp = 0; cp < D / 32; ++cp) {
             uint32_t r[4];
-            ldsm_x4_t(vb + swz<C::kRow8>(16 * k + mrow + 8 * (mj & 1), 2 * cp + (mj >> 1)), r);
+            ldsm_x4_t(vb + 16 * C::kRow8 * k + off8[cp], r);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // channels 32cp + 16h + (2g, 2g+1)
               const uint32_t u0 = r[2 * h] ^ 0x80808080u, u1 = r[2 * h + 1] ^ 0x80808080u;
@@ -519,7 +538,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 #pragma unroll
           for (int cp = 0; cp < D / 64; ++cp) {
             uint32_t r[4];
-            ldsm_x4_t(vb + swz<C::kRow4>(16 * k + mrow + 8 * (mj & 1), 2 * cp + (mj >> 1)), r);
+            ldsm_x4_t(vb + 16 * C::kRow4 * k + off4[cp], r);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // 32 channels 64cp + 32h .. (4g .. 4g+3)
               // words: keys (2tq, 2tq+1) / (2tq+8, 2tq+9), channels 4g .. 4g+3; the
@@ -680,7 +699,7 @@ cudaError_t launch_dec_d(const DecodeParams& p, const DecodeMaps& m, cudaStream_
 
 // Partials per (sequence, KV head): the data splits plus the bf16-tail split.
 int decode_splits(int B, int Hkv) {
-  const int target = 1024;  // about 3.5 waves of two CTAs per SM: long CTAs, a small tail
+  const int target = 512;  // under two waves of two CTAs per SM: long CTAs, little set-up
   const int rows = B * Hkv;
   int s = (target + rows - 1) / rows;
   if (s < 1) s = 1;
