@@ -13,10 +13,10 @@
 //
 // Two work units share one CTA (416 threads) so that one unit's softmax runs
 // while the tensor core works on the other's tiles:
-//   warp 0      TMA producer: both units' Q tiles once, then K (INT8 codes or
-//               BF16) into a K ring and V (BF16) into a deeper V ring (K slots
-//               free up right after QK, V slots only after P V), in the
-//               interleaved order of the two units' traversals;
+//   warp 0      TMA producer: both units' Q tiles once, then, in the
+//               interleaved order of the two units' traversals, K (INT8 codes
+//               or BF16) into the unit's K ring and V (BF16) into its V ring
+//               (K slots free up right after QK, V slots only after P V);
 //   warps 1, 12 MMA issuers, one per unit (warp 1 also owns TMEM): S = Q K^T
 //               with kind::i8 (INT8/INT4, exact int32) or kind::f16 (BF16,
 //               fp32) into one of the unit's two S buffers in TMEM, then
@@ -24,9 +24,10 @@
 //   warps 2-3   INT4 expanders: packed INT4 codes (Q once, K per INT4 entry)
 //               sign-extended to int8 in the swizzled operand layout (tcgen05
 //               has no integer 4-bit MMA, so INT4 tiles run as int8 MMAs), into
-//               a K4 ring of their own.  Each ring has exactly one filler that
-//               takes its slots in order, so a parity wait on a slot's free
-//               barrier never aliases a phase two uses back;
+//               the unit's K4 ring.  Every ring belongs to one unit: one filler
+//               and one consumer (the unit's MMA issuer), both taking its slots
+//               in order, so no parity wait on a full or free barrier can
+//               alias a phase two uses away;
 //   warps 4-7   softmax / epilogue of unit 0, warps 8-11 of unit 1: one thread
 //               per query row (TMEM lane): S -> log2-domain scores -> mask ->
 //               online softmax with lazy rescaling of O -> bf16 P into TMEM;
@@ -60,19 +61,21 @@ struct Cfg {
   static constexpr int kKBytes = MODE == TRA_POLICY_BITMASK ? 64 * D * 2 : 64 * D;
   static constexpr int kK4Bytes = 64 * D;                                     // expanded INT4 K
   static constexpr int kVBytes = 64 * D * 2;
-  static constexpr int kStagesK = 3;
+  // ring depths per unit (every ring belongs to one unit)
+  static constexpr int kStagesK = 2;
   static constexpr int kStagesK4 = MODE == TRA_POLICY_BOUNDARY ? 2 : 0;
-  static constexpr int kFixed = kUnits * kQUnitBytes + kStagesK * kKBytes + kStagesK4 * kK4Bytes +
+  static constexpr int kFixed = kUnits * (kQUnitBytes + kStagesK * kKBytes + kStagesK4 * kK4Bytes) +
                                 2048;                                         // + barriers, slack
-  static constexpr int kStagesVFit = (kSmemLimit - kFixed) / kVBytes;
-  static constexpr int kStagesV = kStagesVFit > 6 ? 6 : kStagesVFit;
-  static_assert(kStagesV >= 3, "shared memory too small for the V ring");
+  static constexpr int kStagesVFit = (kSmemLimit - kFixed) / (kUnits * kVBytes);
+  static constexpr int kStagesV = kStagesVFit > 4 ? 4 : kStagesVFit;
+  static_assert(kStagesV >= 2, "shared memory too small for the V rings");
   static constexpr int kOffQ = 0;                                             // unit u at u * kQUnitBytes
-  static constexpr int kOffK = kUnits * kQUnitBytes;
-  static constexpr int kOffK4 = kOffK + kStagesK * kKBytes;
-  static constexpr int kOffV = kOffK4 + kStagesK4 * kK4Bytes;
-  static constexpr int kOffBar = kOffV + kStagesV * kVBytes;
-  static constexpr int kNumBars = 2 + 2 * kStagesK + 2 * kStagesK4 + 2 * kStagesV + 6 * kUnits + 1;
+  static constexpr int kOffK = kUnits * kQUnitBytes;                          // [unit][slot]
+  static constexpr int kOffK4 = kOffK + kUnits * kStagesK * kKBytes;
+  static constexpr int kOffV = kOffK4 + kUnits * kStagesK4 * kK4Bytes;
+  static constexpr int kOffBar = kOffV + kUnits * kStagesV * kVBytes;
+  static constexpr int kUnitBars = 2 * kStagesK + 2 * kStagesK4 + 2 * kStagesV + 6;
+  static constexpr int kNumBars = 2 + kUnits * kUnitBars + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
@@ -198,8 +201,8 @@ template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps m) {
   using C = Cfg<D, MODE>;
-  constexpr int NSK = C::kStagesK, NSV = C::kStagesV;
-  constexpr int NS4 = C::kStagesK4 > 0 ? C::kStagesK4 : 1;  // (no K4 ring without INT4)
+  constexpr int NSK = C::kStagesK, NSV = C::kStagesV, NS4R = C::kStagesK4;
+  constexpr int NS4 = NS4R > 0 ? NS4R : 1;  // (no K4 ring without INT4)
   extern __shared__ uint8_t smem_raw[];
 
   // ---- the CTA's two work units
@@ -214,26 +217,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* const gbase = smem_raw + (base - smem_u32(smem_raw));
   auto sQ8 = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes; };
   auto sQx = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes; };
-  const uint32_t sK = base + C::kOffK;
-  const uint32_t sK4 = base + C::kOffK4;
-  const uint32_t sV = base + C::kOffV;
+  auto sK = [&](int u, int s) { return base + C::kOffK + (u * NSK + s) * C::kKBytes; };
+  auto sK4 = [&](int u, int s) { return base + C::kOffK4 + (u * NS4 + s) * C::kK4Bytes; };
+  auto sV = [&](int u, int s) { return base + C::kOffV + (u * NSV + s) * C::kVBytes; };
   const uint32_t bars = base + C::kOffBar;
   const uint32_t bar_q = bars + 0 * 8;
   const uint32_t bar_q4 = bars + 1 * 8;
-  auto bar_kfull = [&](int s) { return bars + (2 + s) * 8; };
-  auto bar_kfree = [&](int s) { return bars + (2 + NSK + s) * 8; };
-  auto bar_k4full = [&](int s) { return bars + (2 + 2 * NSK + s) * 8; };
-  auto bar_k4free = [&](int s) { return bars + (2 + 2 * NSK + NS4 + s) * 8; };
-  constexpr int kVB = 2 + 2 * NSK + 2 * C::kStagesK4;  // first V ring barrier
-  auto bar_vfull = [&](int s) { return bars + (kVB + s) * 8; };
-  auto bar_vfree = [&](int s) { return bars + (kVB + NSV + s) * 8; };
-  constexpr int kUB = kVB + 2 * NSV;                    // first per-unit barrier
-  auto bar_sfull = [&](int u, int sb) { return bars + (kUB + 6 * u + sb) * 8; };
-  auto bar_pfull = [&](int u, int sb) { return bars + (kUB + 6 * u + 2 + sb) * 8; };
-  auto bar_ofull = [&](int u) { return bars + (kUB + 6 * u + 4) * 8; };
+  // barriers of unit u: K ring full/free, K4 ring full/free, V ring full/free, then
+  // S full (2), P full (2), O full, O final
+  auto ubar = [&](int u, int k) { return bars + (2 + u * C::kUnitBars + k) * 8; };
+  auto bar_kfull = [&](int u, int s) { return ubar(u, s); };
+  auto bar_kfree = [&](int u, int s) { return ubar(u, NSK + s); };
+  auto bar_k4full = [&](int u, int s) { return ubar(u, 2 * NSK + s); };
+  auto bar_k4free = [&](int u, int s) { return ubar(u, 2 * NSK + NS4R + s); };
+  constexpr int kVB = 2 * NSK + 2 * NS4R;  // first V ring barrier of a unit
+  auto bar_vfull = [&](int u, int s) { return ubar(u, kVB + s); };
+  auto bar_vfree = [&](int u, int s) { return ubar(u, kVB + NSV + s); };
+  constexpr int kSB = kVB + 2 * NSV;       // first S/P/O barrier of a unit
+  auto bar_sfull = [&](int u, int sb) { return ubar(u, kSB + sb); };
+  auto bar_pfull = [&](int u, int sb) { return ubar(u, kSB + 2 + sb); };
+  auto bar_ofull = [&](int u) { return ubar(u, kSB + 4); };
   // completes once every MMA of unit u (its last P V included) is done
-  auto bar_ofinal = [&](int u) { return bars + (kUB + 6 * u + 5) * 8; };
-  const uint32_t bar_done = bars + (kUB + 6 * kUnits) * 8;
+  auto bar_ofinal = [&](int u) { return ubar(u, kSB + 5); };
+  const uint32_t bar_done = bars + (2 + kUnits * C::kUnitBars) * 8;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kOffMisc);
   volatile int* const err = reinterpret_cast<volatile int*>(gbase + C::kOffMisc + 16);
 
@@ -243,19 +249,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     mbar_init(bar_q4, 64);
-    for (int s = 0; s < NSK; ++s) {
-      mbar_init(bar_kfull(s), 1);
-      mbar_init(bar_kfree(s), 1);
-    }
-    for (int s = 0; s < C::kStagesK4; ++s) {
-      mbar_init(bar_k4full(s), 64);
-      mbar_init(bar_k4free(s), 1);
-    }
-    for (int s = 0; s < NSV; ++s) {
-      mbar_init(bar_vfull(s), 1);
-      mbar_init(bar_vfree(s), 1);
-    }
     for (int u = 0; u < kUnits; ++u) {
+      for (int s = 0; s < NSK; ++s) {
+        mbar_init(bar_kfull(u, s), 1);
+        mbar_init(bar_kfree(u, s), 1);
+      }
+      for (int s = 0; s < NS4R; ++s) {
+        mbar_init(bar_k4full(u, s), 64);
+        mbar_init(bar_k4free(u, s), 1);
+      }
+      for (int s = 0; s < NSV; ++s) {
+        mbar_init(bar_vfull(u, s), 1);
+        mbar_init(bar_vfree(u, s), 1);
+      }
       for (int sb = 0; sb < 2; ++sb) {
         mbar_init(bar_sfull(u, sb), 1);
         mbar_init(bar_pfull(u, sb), 128);
@@ -300,9 +306,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       Schedule sc = sched0;
       uint32_t val;
       int mask, u;
-      int nk = 0;  // K ring fills so far (every entry but INT4 ones)
-      for (int g = 0; sc.next(u, val, mask); ++g) {
-        const int sv = g % NSV, usev = g / NSV;  // V ring slot
+      int nk0 = 0, nk1 = 0, nv0 = 0, nv1 = 0;  // fills so far of each unit's K and V rings
+      while (sc.next(u, val, mask)) {
+        const int nv = u ? nv1 : nv0;
+        const int sv = nv % NSV, usev = nv / NSV;  // the unit's V ring slot
         const uint32_t prec = val >> 28;
         const int kt = (int)(val & 0x0FFFFFFFu);
         const int kvh = TRA_UNIT_FIELD(u, kvh), toff = TRA_UNIT_FIELD(u, toff);
@@ -312,24 +319,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (prec != TRA_PREC_INT4) {
-          const int s = nk % NSK, use = nk / NSK;  // K ring slot
-          ++nk;
-          if (use > 0 && !mbar_wait(bar_kfree(s), (use - 1) & 1, err)) break;
-          const uint32_t dst = sK + s * C::kKBytes;
+          const int nk = u ? nk1 : nk0;
+          const int s = nk % NSK, use = nk / NSK;  // the unit's K ring slot
+          if (u) ++nk1; else ++nk0;
+          if (use > 0 && !mbar_wait(bar_kfree(u, s), (use - 1) & 1, err)) break;
+          const uint32_t dst = sK(u, s);
           if (prec == TRA_PREC_INT8) {
-            mbar_arrive_expect_tx(bar_kfull(s), 64 * D);
-            tma_load_2d(dst, &m.k8, bar_kfull(s), 0, (kvh * p.ntiles + toff + kt) * kTile);
+            mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D);
+            tma_load_2d(dst, &m.k8, bar_kfull(u, s), 0, (kvh * p.ntiles + toff + kt) * kTile);
           } else {
-            mbar_arrive_expect_tx(bar_kfull(s), 64 * D * 2);
+            mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D * 2);
             for (int sl = 0; sl < C::kSlabs; ++sl)
-              tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(s), sl * 64, kvh,
+              tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(u, s), sl * 64, kvh,
                           seq0 + kt * kTile);
           }
         }
-        if (usev > 0 && !mbar_wait(bar_vfree(sv), (usev - 1) & 1, err)) break;
-        mbar_arrive_expect_tx(bar_vfull(sv), 64 * D * 2);
+        if (u) ++nv1; else ++nv0;
+        if (usev > 0 && !mbar_wait(bar_vfree(u, sv), (usev - 1) & 1, err)) break;
+        mbar_arrive_expect_tx(bar_vfull(u, sv), 64 * D * 2);
         for (int sl = 0; sl < C::kSlabs; ++sl)
-          tma_load_3d(sV + sv * C::kVBytes + sl * 64 * 128, &m.vb, bar_vfull(sv), sl * 64, kvh,
+          tma_load_3d(sV(u, sv) + sl * 64 * 128, &m.vb, bar_vfull(u, sv), sl * 64, kvh,
                       seq0 + kt * kTile);
       }
     }
@@ -344,30 +353,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(bar_q, 0, err);
       if (ok && int4) ok = mbar_wait(bar_q4, 0, err);
       tc_fence_after();
-      // O += P(idx) V(slot): P from TMEM buffer idx & 1, V (MN-major) from shared memory
-      auto issue_pv = [&](int idx, int slot, int gg) -> bool {
-        const int pb = idx & 1;
+      // O += P(idx) V(idx): P from TMEM buffer idx & 1, V (MN-major) from the unit's
+      // V ring, which holds one tile per entry of the unit, in order
+      auto issue_pv = [&](int idx) -> bool {
+        const int pb = idx & 1, slot = idx % NSV;
         if (!mbar_wait(bar_pfull(mu, pb), (idx >> 1) & 1, err)) return false;
-        if (!mbar_wait(bar_vfull(slot), (gg / NSV) & 1, err)) return false;
+        if (!mbar_wait(bar_vfull(mu, slot), (idx / NSV) & 1, err)) return false;
         tc_fence_after();
-        const uint32_t vb = sV + slot * C::kVBytes;
+        const uint32_t vb = sV(mu, slot);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = smem_desc(vb + kk * 2048, 64 * 128, 1024, kSwz128);
           mma_bf16_ts(tU + 128, tU + pb * 64 + kk * 8, bd, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar_ofull(mu));
-        mma_commit(bar_vfree(slot));
+        mma_commit(bar_vfree(mu, slot));
         return true;
       };
       if (ok) {
-        int nk = 0, n4 = 0;           // K / K4 ring steps so far, both units
+        int nk = 0, n4 = 0;           // this unit's K / K4 ring fills consumed so far
         int i = 0;                    // entries of this unit issued so far
-        int pslot = 0, pg = 0;        // V slot and step of the entry whose P V is pending
-        Schedule sc = sched0;
+        MergeCursor c = unit_cursor(p, mu ? un1 : un0);
         uint32_t val;
-        int mask, u;
-        for (int g = 0; sc.next(u, val, mask); ++g) {
+        int mask;
+        while (c.next(val, mask)) {
           const uint32_t prec = val >> 28;
           if (prec == TRA_PREC_INT4 && !int4) {
             *err = TRA_DEV_BAD_LIST;
@@ -378,13 +387,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = is4 ? n4 % NS4 : nk % NSK;
           const uint32_t ph = (uint32_t)((is4 ? n4 / NS4 : nk / NSK) & 1);
           if (is4) ++n4; else ++nk;
-          if (u != mu) continue;  // the other unit's step: only the ring positions matter here
           // S buffer i & 1 last held entry i-2, whose P V this thread has already
           // issued; MMAs of one thread run in order, so QK(i) cannot overtake it
-          if (!mbar_wait(is4 ? bar_k4full(s) : bar_kfull(s), ph, err)) { ok = false; break; }
+          if (!mbar_wait(is4 ? bar_k4full(mu, s) : bar_kfull(mu, s), ph, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t tSb = tU + (i & 1) * 64;
-          const uint32_t kb = is4 ? sK4 + s * C::kK4Bytes : sK + s * C::kKBytes;
+          const uint32_t kb = is4 ? sK4(mu, s) : sK(mu, s);
           if (prec == TRA_PREC_BF16) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -403,13 +411,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           mma_commit(bar_sfull(mu, i & 1));
-          mma_commit(is4 ? bar_k4free(s) : bar_kfree(s));
-          if (i >= 1 && !issue_pv(i - 1, pslot, pg)) { ok = false; break; }
-          pslot = g % NSV;
-          pg = g;
+          mma_commit(is4 ? bar_k4free(mu, s) : bar_kfree(mu, s));
+          if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
           ++i;
         }
-        if (ok && i >= 1 && issue_pv(i - 1, pslot, pg)) mma_commit(bar_ofinal(mu));
+        if (ok && i >= 1 && issue_pv(i - 1)) mma_commit(bar_ofinal(mu));
       }
       // every MMA of this thread completes before TMEM is released
       mma_commit(bar_done);
@@ -443,15 +449,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       Schedule sc = sched0;
       uint32_t val;
       int mask, u;
-      for (int n4 = 0; sc.next(u, val, mask);) {
+      int n40 = 0, n41 = 0;  // fills so far of each unit's K4 ring
+      while (sc.next(u, val, mask)) {
         if ((val >> 28) != TRA_PREC_INT4) continue;
-        const int s = n4 % NS4, use = n4 / NS4;  // K4 ring slot
-        ++n4;
-        if (use > 0 && !mbar_wait(bar_k4free(s), (use - 1) & 1, err)) break;
+        const int n4 = u ? n41 : n40;
+        const int s = n4 % NS4, use = n4 / NS4;  // the unit's K4 ring slot
+        if (u) ++n41; else ++n40;
+        if (use > 0 && !mbar_wait(bar_k4free(u, s), (use - 1) & 1, err)) break;
         const int kt = (int)(val & 0x0FFFFFFFu);
         const uint8_t* ks = p.k4 + ((long long)(TRA_UNIT_FIELD(u, kvh) * p.ntiles +
                                                 TRA_UNIT_FIELD(u, toff) + kt) * kTile) * kPackedRow;
-        uint8_t* dst = gbase + C::kOffK4 + s * C::kK4Bytes;
+        uint8_t* dst = gbase + C::kOffK4 + (u * NS4 + s) * C::kK4Bytes;
         for (int f = t; f < 64 * kChunksPerRow; f += 64) {
           const int r = f / kChunksPerRow, cc = f % kChunksPerRow;
           const uint4 w = __ldg(reinterpret_cast<const uint4*>(ks + r * kPackedRow + cc * 16));
@@ -461,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * cc + 1)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
         }
         fence_proxy_async_smem();
-        mbar_arrive(bar_k4full(s));
+        mbar_arrive(bar_k4full(u, s));
       }
     }
   } else {
