@@ -68,8 +68,8 @@ def parse():
 # source that has changed since reports null.  Captures: profiles/prefill_kernel_bitmask_32k.md
 # and profiles/decode_split_kernel_b16_32k.md.
 PROFILED_TRAFFIC = {
-    "prefill.cu": ("3967798f436d8325", 3_419_179_216),
-    "decode.cu": ("4ad208c3ea7b8b98", 667_361_024),
+    "prefill.cu": ("006591d5deb101dc", 3_384_843_776),
+    "decode.cu": ("fbb72974b738b53e", 663_281_408),
 }
 
 
