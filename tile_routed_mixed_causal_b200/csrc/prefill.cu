@@ -11,17 +11,18 @@
 // only one q-tile's list (or with a different precision) is computed for all
 // 128 rows and masked to -inf in the other half, so routing stays exact.
 //
-// Two work units share one CTA (416 threads) so that one unit's softmax runs
+// Two work units share one CTA (448 threads) so that one unit's softmax runs
 // while the tensor core works on the other's tiles:
-//   warp 0      TMA producer: both units' Q tiles once, then, in the
-//               interleaved order of the two units' traversals, K (INT8 codes
-//               or BF16) into the unit's K ring and V (BF16) into its V ring
-//               (K slots free up right after QK, V slots only after P V);
+//   warps 0, 13 TMA producers, one per unit: the unit's Q tiles once, then in
+//               traversal order K (INT8 codes or BF16) into the unit's K ring
+//               and V (BF16) into its V ring (K slots free up right after QK,
+//               V slots only after P V);
 //   warps 1, 12 MMA issuers, one per unit (warp 1 also owns TMEM): S = Q K^T
 //               with kind::i8 (INT8/INT4, exact int32) or kind::f16 (BF16,
 //               fp32) into one of the unit's two S buffers in TMEM, then
 //               O += P V with P read from TMEM (bf16) and V from shared memory;
-//   warps 2-3   INT4 expanders: packed INT4 codes (Q once, K per INT4 entry)
+//   warps 2, 3  INT4 expanders of units 0, 1: packed INT4 codes (Q once, K per
+//               INT4 entry)
 //               sign-extended to int8 in the swizzled operand layout (tcgen05
 //               has no integer 4-bit MMA, so INT4 tiles run as int8 MMAs), into
 //               the unit's K4 ring.  Every ring belongs to one unit: one filler
@@ -42,7 +43,8 @@
 namespace tra {
 namespace {
 
-constexpr int kThreads = 416;
+constexpr int kThreads = 448;
+constexpr int kProdWarp1 = 13;  // TMA producer of unit 1 (warp 0: unit 0)
 constexpr int kUnits = 2;
 // log2 units: O and l are rescaled only once the running max has grown by more
 // than 2^16.  Until then P (bf16, exponent range of fp32) may reach 2^16, and
@@ -113,25 +115,6 @@ struct MergeCursor {
       val = a; mask = 3; ++p0; ++p1;
     }
     return true;
-  }
-};
-
-// Interleaving of the two units' traversals: alternate while both have
-// entries, then drain the other.  Every role that walks the shared ring
-// replays the same sequence.  (Two named cursors, so that nothing is indexed
-// at run time and the state stays in registers.)
-struct Schedule {
-  MergeCursor c0, c1;
-  int turn;
-  __device__ __forceinline__ bool next(int& u, uint32_t& val, int& mask) {
-    if (turn == 0) {
-      if (c0.next(val, mask)) { u = 0; turn = 1; return true; }
-      if (c1.next(val, mask)) { u = 1; return true; }
-    } else {
-      if (c1.next(val, mask)) { u = 1; turn = 0; return true; }
-      if (c0.next(val, mask)) { u = 0; return true; }
-    }
-    return false;
   }
 };
 
@@ -247,15 +230,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
-    mbar_init(bar_q4, 64);
+    mbar_init(bar_q, kUnits);  // one arrival (with its byte count) per producer
+    mbar_init(bar_q4, 64);  // both expander warps, each after its unit's Q
     for (int u = 0; u < kUnits; ++u) {
       for (int s = 0; s < NSK; ++s) {
         mbar_init(bar_kfull(u, s), 1);
         mbar_init(bar_kfree(u, s), 1);
       }
       for (int s = 0; s < NS4R; ++s) {
-        mbar_init(bar_k4full(u, s), 64);
+        mbar_init(bar_k4full(u, s), 32);  // the unit's expander warp
         mbar_init(bar_k4free(u, s), 1);
       }
       for (int s = 0; s < NSV; ++s) {
@@ -282,20 +265,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  Schedule sched0;
-  sched0.turn = 0;
-  sched0.c0 = unit_cursor(p, un0);
-  sched0.c1 = unit_cursor(p, un1);
-#define TRA_UNIT_FIELD(u, f) ((u) ? un1.f : un0.f)
 
-  if (warp == 0) {
-    // ================================================================ TMA producer
+  if (warp == 0 || warp == kProdWarp1) {
+    // ================================================================ TMA producers
+    // one per unit, each walking its own unit's traversal into its own rings
     if (lane == 0) {
+      const int u = warp == 0 ? 0 : 1;
+      const Unit x = u ? un1 : un0;
       constexpr uint32_t kQBytes = C::kQ8Bytes + (MODE == TRA_POLICY_BITMASK ? 128 * D * 2 : 0);
-      mbar_arrive_expect_tx(bar_q, (un0.valid ? kQBytes : 0u) + (un1.valid ? kQBytes : 0u));
-      for (int u = 0; u < kUnits; ++u) {
-        const Unit x = u ? un1 : un0;
-        if (!x.valid) continue;
+      mbar_arrive_expect_tx(bar_q, x.valid ? kQBytes : 0u);
+      if (x.valid) {
         tma_load_2d(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
         if (MODE == TRA_POLICY_BITMASK) {
           for (int sl = 0; sl < C::kSlabs; ++sl)
@@ -303,43 +282,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                         x.seq0 + x.qt0 * kTile);
         }
       }
-      Schedule sc = sched0;
+      MergeCursor c = unit_cursor(p, x);
       uint32_t val;
-      int mask, u;
-      int nk0 = 0, nk1 = 0, nv0 = 0, nv1 = 0;  // fills so far of each unit's K and V rings
-      while (sc.next(u, val, mask)) {
-        const int nv = u ? nv1 : nv0;
+      int mask;
+      int nk = 0, nv = 0;  // fills so far of this unit's K and V rings
+      while (c.next(val, mask)) {
         const int sv = nv % NSV, usev = nv / NSV;  // the unit's V ring slot
         const uint32_t prec = val >> 28;
         const int kt = (int)(val & 0x0FFFFFFFu);
-        const int kvh = TRA_UNIT_FIELD(u, kvh), toff = TRA_UNIT_FIELD(u, toff);
-        const int seq0 = TRA_UNIT_FIELD(u, seq0);
         if (prec == TRA_PREC_INT4 && !int4) {
           *err = TRA_DEV_BAD_LIST;
           break;
         }
         if (prec != TRA_PREC_INT4) {
-          const int nk = u ? nk1 : nk0;
           const int s = nk % NSK, use = nk / NSK;  // the unit's K ring slot
-          if (u) ++nk1; else ++nk0;
+          ++nk;
           if (use > 0 && !mbar_wait(bar_kfree(u, s), (use - 1) & 1, err)) break;
           const uint32_t dst = sK(u, s);
           if (prec == TRA_PREC_INT8) {
             mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D);
-            tma_load_2d(dst, &m.k8, bar_kfull(u, s), 0, (kvh * p.ntiles + toff + kt) * kTile);
+            tma_load_2d(dst, &m.k8, bar_kfull(u, s), 0, (x.kvh * p.ntiles + x.toff + kt) * kTile);
           } else {
             mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D * 2);
             for (int sl = 0; sl < C::kSlabs; ++sl)
-              tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(u, s), sl * 64, kvh,
-                          seq0 + kt * kTile);
+              tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(u, s), sl * 64, x.kvh,
+                          x.seq0 + kt * kTile);
           }
         }
-        if (u) ++nv1; else ++nv0;
+        ++nv;
         if (usev > 0 && !mbar_wait(bar_vfree(u, sv), (usev - 1) & 1, err)) break;
         mbar_arrive_expect_tx(bar_vfull(u, sv), 64 * D * 2);
         for (int sl = 0; sl < C::kSlabs; ++sl)
-          tma_load_3d(sV(u, sv) + sl * 64 * 128, &m.vb, bar_vfull(u, sv), sl * 64, kvh,
-                      seq0 + kt * kTile);
+          tma_load_3d(sV(u, sv) + sl * 64 * 128, &m.vb, bar_vfull(u, sv), sl * 64, x.kvh,
+                      x.seq0 + kt * kTile);
       }
     }
   } else if (warp == 1 || warp == 12) {
@@ -423,18 +398,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2 || warp == 3) {
     // ================================================================ INT4 expanders
-    const int t = threadIdx.x - 64;  // 0..63
+    // warp 2 for unit 0, warp 3 for unit 1, each walking its own unit's traversal
+    const int u = warp - 2;
+    const int t = lane;
+    const Unit x = u ? un1 : un0;
     constexpr int kPackedRow = D / 2;          // bytes per packed row
     constexpr int kChunksPerRow = kPackedRow / 16;
     if (int4) {
-      // Q: 128 rows (two q-tiles) per unit; rows of a missing q-tile stay zero
-      for (int u = 0; u < kUnits; ++u) {
-        const Unit x = u ? un1 : un0;
-        if (!x.valid) continue;
+      // Q: 128 rows (two q-tiles); rows of a missing q-tile stay zero
+      if (x.valid) {
         const uint8_t* src = p.q4 + (long long)x.row0 * kTile * kPackedRow;
         const int rows = x.has_second ? 128 : 64;
         uint8_t* dst = gbase + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes;
-        for (int f = t; f < 128 * kChunksPerRow; f += 64) {
+        for (int f = t; f < 128 * kChunksPerRow; f += 32) {
           const int r = f / kChunksPerRow, c = f % kChunksPerRow;
           uint4 w = make_uint4(0, 0, 0, 0);
           if (r < rows) w = __ldg(reinterpret_cast<const uint4*>(src + r * kPackedRow + c * 16));
@@ -446,21 +422,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(bar_q4);
-      Schedule sc = sched0;
+      MergeCursor c = unit_cursor(p, x);
       uint32_t val;
-      int mask, u;
-      int n40 = 0, n41 = 0;  // fills so far of each unit's K4 ring
-      while (sc.next(u, val, mask)) {
+      int mask;
+      for (int n4 = 0; c.next(val, mask);) {
         if ((val >> 28) != TRA_PREC_INT4) continue;
-        const int n4 = u ? n41 : n40;
         const int s = n4 % NS4, use = n4 / NS4;  // the unit's K4 ring slot
-        if (u) ++n41; else ++n40;
+        ++n4;
         if (use > 0 && !mbar_wait(bar_k4free(u, s), (use - 1) & 1, err)) break;
         const int kt = (int)(val & 0x0FFFFFFFu);
-        const uint8_t* ks = p.k4 + ((long long)(TRA_UNIT_FIELD(u, kvh) * p.ntiles +
-                                                TRA_UNIT_FIELD(u, toff) + kt) * kTile) * kPackedRow;
+        const uint8_t* ks = p.k4 + ((long long)(x.kvh * p.ntiles + x.toff + kt) * kTile) * kPackedRow;
         uint8_t* dst = gbase + C::kOffK4 + (u * NS4 + s) * C::kK4Bytes;
-        for (int f = t; f < 64 * kChunksPerRow; f += 64) {
+        for (int f = t; f < 64 * kChunksPerRow; f += 32) {
           const int r = f / kChunksPerRow, cc = f % kChunksPerRow;
           const uint4 w = __ldg(reinterpret_cast<const uint4*>(ks + r * kPackedRow + cc * 16));
           const uint2 e0 = expand_int4x8(w.x), e1 = expand_int4x8(w.y);
@@ -472,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar_k4full(u, s));
       }
     }
-  } else {
+  } else if (warp >= 4 && warp < 12) {
     // ================================================================ softmax / epilogue
     const int u = (warp - 4) >> 2;               // unit of this warpgroup
     const Unit x = make_unit(p, (long long)blockIdx.x * kUnits + u);
@@ -691,7 +664,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-#undef TRA_UNIT_FIELD
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
