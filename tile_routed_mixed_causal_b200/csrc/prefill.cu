@@ -422,27 +422,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(bar_q4);
+      // packed codes of the unit's next INT4 entry are loaded into registers as soon
+      // as the previous one is handed over, so the load overlaps the wait for a slot
+      constexpr int kPer = 64 * kChunksPerRow / 32;  // 16-byte chunks per lane and tile
       MergeCursor c = unit_cursor(p, x);
-      uint32_t val;
-      int mask;
-      for (int n4 = 0; c.next(val, mask);) {
-        if ((val >> 28) != TRA_PREC_INT4) continue;
-        const int s = n4 % NS4, use = n4 / NS4;  // the unit's K4 ring slot
-        ++n4;
-        if (use > 0 && !mbar_wait(bar_k4free(u, s), (use - 1) & 1, err)) break;
-        const int kt = (int)(val & 0x0FFFFFFFu);
+      auto next_int4 = [&](uint32_t& v) -> bool {
+        int mk;
+        while (c.next(v, mk))
+          if ((v >> 28) == TRA_PREC_INT4) return true;
+        return false;
+      };
+      auto load_packed = [&](uint32_t v, uint4 (&w)[kPer]) {
+        const int kt = (int)(v & 0x0FFFFFFFu);
         const uint8_t* ks = p.k4 + ((long long)(x.kvh * p.ntiles + x.toff + kt) * kTile) * kPackedRow;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const int f = t + 32 * j, r = f / kChunksPerRow, cc = f % kChunksPerRow;
+          w[j] = __ldg(reinterpret_cast<const uint4*>(ks + r * kPackedRow + cc * 16));
+        }
+      };
+      uint4 w[kPer];
+      uint32_t val;
+      bool have = next_int4(val);
+      if (have) load_packed(val, w);
+      for (int n4 = 0; have; ++n4) {
+        const int s = n4 % NS4, use = n4 / NS4;  // the unit's K4 ring slot
+        if (use > 0 && !mbar_wait(bar_k4free(u, s), (use - 1) & 1, err)) break;
         uint8_t* dst = gbase + C::kOffK4 + (u * NS4 + s) * C::kK4Bytes;
-        for (int f = t; f < 64 * kChunksPerRow; f += 32) {
-          const int r = f / kChunksPerRow, cc = f % kChunksPerRow;
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(ks + r * kPackedRow + cc * 16));
-          const uint2 e0 = expand_int4x8(w.x), e1 = expand_int4x8(w.y);
-          const uint2 e2 = expand_int4x8(w.z), e3 = expand_int4x8(w.w);
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const int f = t + 32 * j, r = f / kChunksPerRow, cc = f % kChunksPerRow;
+          const uint2 e0 = expand_int4x8(w[j].x), e1 = expand_int4x8(w[j].y);
+          const uint2 e2 = expand_int4x8(w[j].z), e3 = expand_int4x8(w[j].w);
           *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * cc)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
           *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * cc + 1)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
         }
         fence_proxy_async_smem();
         mbar_arrive(bar_k4full(u, s));
+        have = next_int4(val);
+        if (have) load_packed(val, w);
       }
     }
   } else if (warp >= 4 && warp < 12) {
