@@ -369,12 +369,21 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a host float over all ranks (every rank gets it); device tensor under NCCL,
+    host tensor under gloo."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(world, units_per_rank, ms):
+    """Whole-job throughput in units per second x 1e-12 (TOPS for ops): every rank processes
+    units_per_rank in ms, the slowest rank's time being the job's."""
+    return world * units_per_rank / (ms * 1e-3) / 1e12
 
 
 def reference_arm(args, world, rank):
@@ -456,7 +465,7 @@ def main():
     clk = clocks.stop()
     total_ms = max_over_ranks(total_ms, world)
     ms_step = total_ms / args.steps
-    value = world * ops / (ms_step * 1e-3) / 1e12
+    value = whole_job_value(world, ops, ms_step)
 
     attn_avg = sum(attn_ms) / len(attn_ms)
     prep_avg = sum(prep_ms) / len(prep_ms)
@@ -466,13 +475,19 @@ def main():
 
     e2e_ms, h2d, d2h = run_prefill_e2e(S, args.e2e_steps, stream)
     e2e_ms = max_over_ranks(e2e_ms, world)
-    e2e_value = world * ops / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_value(world, ops, e2e_ms)
 
     dec = None
     if not args.no_decode:
         del S["plan"]
         torch.cuda.empty_cache()
         dec = decode_bench(device, args.decode_passes, stream, hbm_gbs)
+        if world > 1:  # whole-job GB/s over the slowest rank's step time
+            ms_dec = max_over_ranks(dec["ms_per_token_step"], world)
+            gbs = whole_job_value(world, dec["bytes_per_step"], ms_dec) * 1e3
+            dec.update(value=round(gbs, 1), ms_per_token_step=round(ms_dec, 4))
+            dec["roofline"].update(achieved=round(gbs / world, 1),
+                                   frac=round(gbs / world / hbm_gbs, 4))
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
