@@ -285,6 +285,20 @@ TRA_API tra_status routed_attention_decode_noalloc(
     const uint32_t* entries, uint16_t* k_tail, uint16_t* v_tail, int32_t* tail_len_dev,
     int32_t tail_cap, float softmax_scale, uint16_t* out, int32_t* status_dev, void* stream);
 
+/*
+ * tra_selftest_bounded_wait -- diagnostic; the pages have no counterpart.  Runs
+ * one small kernel whose mbarrier wait can never complete, through the same
+ * bounded-wait routine every pipeline wait of the prefill and decode kernels
+ * uses, with a limit of limit_ns nanoseconds instead of their 2 s.  The wait
+ * must give up, OR TRA_DEV_TIMEOUT (0x1) into *status_dev and let the kernel
+ * return; a waiter that returns success would OR 0x100 instead.  Nothing is
+ * read or written outside the kernel's shared memory and *status_dev.
+ * status_dev: device int32 (the caller zeroes it).  limit_ns: 1e3 .. 1e9, else
+ * TRA_ERR_INVALID.  stream: cudaStream_t or NULL.  Asynchronous like the other
+ * entry points; a launch failure is returned as TRA_ERR_CUDA.
+ */
+TRA_API tra_status tra_selftest_bounded_wait(int32_t* status_dev, int64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -177,3 +177,13 @@ def test_workload_shapes():
     assert w.bitmask.shape == (32, 512, 4)
     frac = np.mean(np.unpackbits(w.bitmask.view(np.uint8)))
     assert 0.24 < frac < 0.26
+
+
+def test_selftest_argument_errors(lib):
+    """The bounded-wait self-test rejects a missing status word and limits outside
+    [1 us, 1 s] on the host, before anything is launched."""
+    assert lib.tra_selftest_bounded_wait(None, 10**6, None) == 1
+    assert b"status" in lib.tra_last_error()
+    assert lib.tra_selftest_bounded_wait(FAKE, 999, None) == 1
+    assert lib.tra_selftest_bounded_wait(FAKE, 10**9 + 1, None) == 1
+    assert b"limit_ns" in lib.tra_last_error()

@@ -22,7 +22,7 @@ PREC_INT4, PREC_INT8, PREC_BF16 = 1, 2, 3
 POLICY_BOUNDARY, POLICY_BITMASK = 0, 1
 LISTS_PREFILL, LISTS_DECODE_CACHE = 0, 1
 FMT_Q8, FMT_Q4, FMT_K8, FMT_K4, FMT_V8, FMT_V4 = 0x1, 0x2, 0x4, 0x8, 0x10, 0x20
-DEV_TIMEOUT, DEV_TAIL_FULL = 0x1, 0x2
+DEV_TIMEOUT, DEV_TAIL_FULL, DEV_BAD_LIST = 0x1, 0x2, 0x4
 STATUS = {0: "TRA_OK", 1: "TRA_ERR_INVALID", 2: "TRA_ERR_UNSUPPORTED", 3: "TRA_ERR_BUFFER",
           4: "TRA_ERR_CUDA", 5: "TRA_ERR_TIMEOUT"}
 
@@ -76,6 +76,7 @@ def load():
         "tra_decode_workspace_bytes": ([I32, I32, I32, I32], SZ),
         "routed_attention_decode": ([P, P, P, P, P, P, P, P, P, P, P, I32, F, P, P, SZ, P, P], I32),
         "routed_attention_decode_noalloc": ([P, P, P, P, P, P, P, P, P, P, P, I32, F, P, P, P], I32),
+        "tra_selftest_bounded_wait": ([P, I64, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -251,3 +252,9 @@ def routed_attention_decode_noalloc(shape: Shape, policy: Policy, q, k_new, v_ne
         shape.c, policy.c, _ptr(q), _ptr(k_new), _ptr(v_new), cache.c, _ptr(row_ptr),
         _ptr(entries), _ptr(k_tail), _ptr(v_tail), _ptr(tail_len), int(k_tail.shape[2]),
         float(softmax_scale), _ptr(out), _ptr(status), _stream(stream)))
+
+
+def tra_selftest_bounded_wait(status, limit_ns: int, stream=None):
+    """Diagnostic: a kernel whose mbarrier wait never completes must give up after
+    limit_ns and OR DEV_TIMEOUT into the device int32 `status` (see include/tra.h)."""
+    _check(load().tra_selftest_bounded_wait(_ptr(status), int(limit_ns), _stream(stream)))

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       MergeCursor c = unit_cursor(p, x);
       uint32_t val;
       int mask;
-      int nk = 0, nv = 0;  // fills so far of this unit's K and V rings
+      int nk = 0, nv = 0;  // fills issued so far into this unit's K and V rings
       while (c.next(val, mask)) {
         const int sv = nv % NSV, usev = nv / NSV;  // the unit's V ring slot
         const uint32_t prec = val >> 28;
@@ -296,7 +296,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (prec != TRA_PREC_INT4) {
           const int s = nk % NSK, use = nk / NSK;  // the unit's K ring slot
-          ++nk;
           if (use > 0 && !mbar_wait(bar_kfree(u, s), (use - 1) & 1, err)) break;
           const uint32_t dst = sK(u, s);
           if (prec == TRA_PREC_INT8) {
@@ -308,13 +307,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(u, s), sl * 64, x.kvh,
                           x.seq0 + kt * kTile);
           }
+          ++nk;
         }
-        ++nv;
         if (usev > 0 && !mbar_wait(bar_vfree(u, sv), (usev - 1) & 1, err)) break;
         mbar_arrive_expect_tx(bar_vfull(u, sv), 64 * D * 2);
         for (int sl = 0; sl < C::kSlabs; ++sl)
           tma_load_3d(sV(u, sv) + sl * 64 * 128, &m.vb, bar_vfull(u, sv), sl * 64, x.kvh,
                       x.seq0 + kt * kTile);
+        ++nv;
+      }
+      if (*err) {
+        // an abandoned traversal: every load this thread issued lands before the
+        // CTA can exit. Only this thread arrives on a full barrier, so the last
+        // fill of each slot completes its phase as soon as its bytes are in.
+        mbar_wait_drain(bar_q, 0);
+        for (int s = 0; s < NSK && s < nk; ++s)
+          mbar_wait_drain(bar_kfull(u, s), (uint32_t)(((nk - 1 - s) / NSK) & 1));
+        for (int s = 0; s < NSV && s < nv; ++s)
+          mbar_wait_drain(bar_vfull(u, s), (uint32_t)(((nv - 1 - s) / NSV) & 1));
       }
     }
   } else if (warp == 1 || warp == 12) {

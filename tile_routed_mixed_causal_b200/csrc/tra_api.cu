@@ -463,4 +463,14 @@ tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* pol
   return ok();
 }
 
+tra_status tra_selftest_bounded_wait(int32_t* status_dev, int64_t limit_ns, void* stream) {
+  if (!status_dev) return fail(TRA_ERR_INVALID, "status_dev is NULL");
+  if (limit_ns < 1000 || limit_ns > 1000000000)
+    return fail(TRA_ERR_INVALID, "limit_ns must lie in [1e3, 1e9] (got %lld)", (long long)limit_ns);
+  cudaError_t e = tra::launch_wait_selftest(status_dev, (uint64_t)limit_ns,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ok();
+}
+
 }  // extern "C"

@@ -80,19 +80,24 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// sets *err) if the wait exceeds kWaitLimitNs or *err is already set by another
-// role of the CTA, so that every role drains instead of spinning forever.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* err) {
+// sets *err) if the wait exceeds limit_ns (kWaitLimitNs for mbar_wait) or *err
+// is already set by another role of the CTA, so that every role drains instead
+// of spinning forever.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int* err,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
     if (*err) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *err = TRA_DEV_TIMEOUT;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* err) {
+  return mbar_wait_for(bar, parity, err, kWaitLimitNs);
 }
 
 // Bounded wait that ignores the CTA error flag: used where the waiter must not

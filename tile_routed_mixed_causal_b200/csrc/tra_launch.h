@@ -106,6 +106,7 @@ struct DecodeMaps {
 };
 
 int decode_splits(int B, int Hkv);
+cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, const DecodeMaps& m, cudaStream_t s);
 
 // Records `msg` as this thread's tra_last_error() text and returns `st`.
