@@ -11,8 +11,10 @@
 // bank-conflict free.  Each consumer warp takes every fourth tile and keeps its
 // own online-softmax state for all query heads of the GQA group, so the loop has
 // no block barrier and every cached byte is read once per group:
-//   scores: S^T = K Q^T on the tensor cores (mma.sync m16n8k16, f16 codes exact,
-//           fp32 accumulation), K tiles fed by ldmatrix;
+//   scores: S^T = K Q^T on the tensor cores as integer MMAs (mma.sync m16n8k32,
+//           s8 x s8 -> s32): the K codes go in as they are stored (INT4 nibbles
+//           masked in place, worth 16 x code), q as a 16-bit fixed-point pair of
+//           int8 limbs per head; K tiles fed by ldmatrix;
 //   softmax: per head over the warp's fragment lanes, K scale and 1/sqrt(d)
 //           folded into the exponent, V scale folded into P (f16, staged per warp);
 //   P V:    O^T += V^T P^T on the tensor cores, V fed by ldmatrix.trans.
@@ -44,13 +46,14 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 }
 
 // ---------------------------------------------------------------- mma.sync helpers
-// The GQA group's contractions run on the tensor cores as m16n8k16 MMAs (f16
-// inputs, fp32 accumulation): scores S^T = K Q^T (M = 16 keys, N = 8 heads) and
-// O^T += V^T P^T (M = 16 channels, N = 8 heads).  Codes reach f16 exactly: each
-// biased byte / nibble becomes the low mantissa byte of 1024.0h, and one packed
-// subtraction removes the bias.  ldmatrix on the int8 tiles, viewed as 16-bit
-// pairs, hands every thread four consecutive codes; the k (channel or key)
-// order inside an MMA is a permutation applied identically to both operands.
+// The GQA group's contractions run on the tensor cores.  Scores S^T = K Q^T are
+// m16n8k32 integer MMAs (M = 16 keys, N = 8 columns = 4 heads x 2 q limbs, exact
+// int32 accumulation); O^T += V^T P^T are m16n8k16 MMAs (f16 inputs, fp32
+// accumulation; M = 16 channels, N = 8 heads), whose V codes reach f16 exactly:
+// each biased byte / nibble becomes the low mantissa byte of 1024.0h, and one
+// packed subtraction removes the bias.  ldmatrix on the int8 tiles, viewed as
+// 16-bit pairs, hands every thread four consecutive bytes; the k (channel or
+// key) order inside an MMA is a permutation applied identically to both operands.
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -70,6 +73,16 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void mma_s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Four signed INT4 codes of a word's even / odd nibbles as int8 lanes worth
+// 16 x code (exact: the nibble becomes the high half of its byte).
+__device__ __forceinline__ uint32_t i4_even_x16(uint32_t x) { return (x << 4) & 0xF0F0F0F0u; }
+__device__ __forceinline__ uint32_t i4_odd_x16(uint32_t x) { return x & 0xF0F0F0F0u; }
 // Two biased bytes (selected by `sel` from x) -> f16x2 of (byte - bias).
 __device__ __forceinline__ uint32_t h2_from_bytes(uint32_t x, uint32_t sel, uint32_t bias2) {
   uint32_t h = __byte_perm(x, 0x6464u, sel);
@@ -100,17 +113,12 @@ __device__ __forceinline__ void i4x8_to_h2(uint32_t x, uint32_t (&h)[4]) {
   asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h[1]) : "r"(sixteenth), "r"(m72));
   asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h[3]) : "r"(sixteenth), "r"(m72));
 }
-constexpr uint32_t kSel01 = 0x5140, kSel23 = 0x5342, kSel02 = 0x5240, kSel13 = 0x5341;
+constexpr uint32_t kSel02 = 0x5240, kSel13 = 0x5341;
 constexpr uint32_t kBias8 = 0x64806480u;  // f16x2 (1152, 1152) = 1024 + 128
 
 // Named barrier over the whole CTA, usable from different code locations.
 __device__ __forceinline__ void named_sync(int id) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kDecThreads) : "memory");
-}
-
-__device__ __forceinline__ uint32_t f16x2_from(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 template <int D, int GRP>
@@ -124,18 +132,19 @@ struct DecCfg {
   static constexpr int kQBytes = (D / 2) * GRP * 8;
   static constexpr int kOffP = kOffQ + kQBytes;            // P: [warp][8 heads][kPStride] f16
   static constexpr int kPBytes = kConsumers * 8 * kPStride * 2;
-  static constexpr int kOffT = kOffP + kPBytes;            // tail p: [64 keys][GRP] float
-  static constexpr int kTBytes = kTile * GRP * 4;
+  static constexpr int kOffE = kOffP + kPBytes;            // q limb exponents: [GRP] int
+  static constexpr int kEBytes = 32;
   static constexpr int kStates = kConsumers;               // one state per consumer warp
   // merge area [state][GRP][D + 2] floats, aliasing the drained ring
   static constexpr int kOffRed = 0;
   static constexpr int kRedBytes = kStates * GRP * (D + 2) * 4;
   static_assert(kRedBytes <= kDecStages * kStageBytes, "merge area must fit in the ring");
-  static constexpr int kOffBar = kOffT + kTBytes;
+  static constexpr int kOffBar = kOffE + kEBytes;
   static constexpr int kSmem = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
   static constexpr int kCh = D / 32;             // tail P V channels per lane
-  static constexpr int kB8 = D / 16;             // 16-channel blocks (INT8 fragments)
-  static constexpr int kB4 = D / 32;             // 32-channel blocks (INT4 fragments)
+  static constexpr int kB8 = D / 16;             // 16-channel blocks (INT8 V fragments)
+  static constexpr int kB4 = D / 32;             // 32-channel blocks (INT4 V fragments)
+  static constexpr int kQM = GRP > 4 ? 2 : 1;    // score MMAs per K fragment (4 heads each)
 };
 
 template <int D, int GRP>
@@ -241,41 +250,66 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     }
     asm volatile("bar.sync 3, %0;" ::"n"(32 * kConsumers) : "memory");  // consumers only
     const int g = lane >> 2, tq = lane & 3;  // fragment group / thread in group
-    // Power-of-two scale keeping q inside the f16 range (exact: only the exponent moves)
-    float qmax = 0.0f;
-    for (int x = lane; x < (D / 2) * GRP; x += 32) {
-      const float2 v = q2[x];
-      qmax = fmaxf(qmax, fmaxf(fabsf(v.x), fabsf(v.y)));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
-    int qexp = 0;
-    if (qmax > 16384.0f) frexpf(qmax / 16384.0f, &qexp);
-    const float qs = ldexpf(1.0f, -qexp), q_unscale = ldexpf(1.0f, qexp);
-    // B fragments of q for head g (zero for padded heads), in the channel order
-    // the K codes arrive in:
-    //   INT8, 16-channel block j: (16j+4t, +1) and (16j+4t+2, +3)
-    //   INT4, 32-channel block j, half ab: (32j+8t+2ab, +4) and (32j+8t+2ab+1, +5)
-    auto qv = [&](int c) -> float {
-      if (g >= grp) return 0.0f;
-      const float2 v = q2[(c >> 1) * GRP + g];
-      return (c & 1 ? v.y : v.x) * qs;
-    };
-    uint32_t qb8[C::kB8][2], qb4[C::kB4][2][2];
-#pragma unroll
-    for (int j = 0; j < C::kB8; ++j) {
-      const int c = 16 * j + 4 * tq;
-      qb8[j][0] = f16x2_from(qv(c), qv(c + 1));
-      qb8[j][1] = f16x2_from(qv(c + 2), qv(c + 3));
-    }
-#pragma unroll
-    for (int j = 0; j < C::kB4; ++j)
-#pragma unroll
-      for (int ab = 0; ab < 2; ++ab) {
-        const int c = 32 * j + 8 * tq + 2 * ab;
-        qb4[j][ab][0] = f16x2_from(qv(c), qv(c + 4));
-        qb4[j][ab][1] = f16x2_from(qv(c + 1), qv(c + 5));
+    // q of head h as a 16-bit fixed-point integer Q = 256 hi + lo (hi, lo int8)
+    // times the power of two 2^(E_h - 14), where 2^E_h > max_c |q_h[c]|:
+    // |Q| <= 2^14, and each channel is off by at most 2^(E_h - 15), i.e. 2^-14 of
+    // the head's largest |q| (exact for every channel within 2^7 of it).
+    int* const qe = reinterpret_cast<int*>(sm + C::kOffE);
+    for (int hd = warp; hd < GRP; hd += kConsumers) {
+      float mx = 0.0f;
+      for (int cp = lane; cp < D / 2; cp += 32) {
+        const float2 v = q2[cp * GRP + hd];
+        mx = fmaxf(mx, fmaxf(fabsf(v.x), fabsf(v.y)));
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      int e = 0;
+      frexpf(mx, &e);  // mx = f 2^e with f in [0.5, 1), or e = 0 for mx = 0
+      if (lane == 0) qe[hd] = e;
+    }
+    asm volatile("bar.sync 3, %0;" ::"n"(32 * kConsumers) : "memory");
+    // limb `limb` (0: hi, 1: lo) of head hd's Q at channel c; 0 for padded heads
+    auto q_limb = [&](int hd, int limb, int c) -> uint32_t {
+      if (hd >= grp) return 0u;
+      const float2 v = q2[(c >> 1) * GRP + hd];
+      const int Q = __float2int_rn(ldexpf(c & 1 ? v.y : v.x, 14 - qe[hd]));
+      const int hi = (Q + 128) >> 8;
+      return (uint32_t)((limb ? Q - 256 * hi : hi) & 0xFF);
+    };
+    auto pack4 = [&](int hd, int limb, int c, int step) -> uint32_t {
+      return q_limb(hd, limb, c) | q_limb(hd, limb, c + step) << 8 |
+             q_limb(hd, limb, c + 2 * step) << 16 | q_limb(hd, limb, c + 3 * step) << 24;
+    };
+    // B fragments (column g = head (g & 3) + 4 mq, limb g >> 2), in the channel
+    // order the K codes arrive in:
+    //   INT8, 32-channel block cb: k = 4t + i -> channel 32cb + 4t + i, k = 16 + 4t + i
+    //         -> 32cb + 16 + 4t + i
+    //   INT4, 32-channel block 2cb + h: k = 4t + i -> even channel 64cb + 32h + 8t + 2i,
+    //         k = 16 + 4t + i -> the odd channel after it
+    uint32_t qi8[D / 32][C::kQM][2], qi4[D / 64][2][C::kQM][2];
+#pragma unroll
+    for (int mq = 0; mq < C::kQM; ++mq) {
+      const int hc = (g & 3) + 4 * mq, limb = g >> 2;
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        qi8[cb][mq][0] = pack4(hc, limb, 32 * cb + 4 * tq, 1);
+        qi8[cb][mq][1] = pack4(hc, limb, 32 * cb + 16 + 4 * tq, 1);
+      }
+#pragma unroll
+      for (int cb = 0; cb < D / 64; ++cb)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          qi4[cb][h][mq][0] = pack4(hc, limb, 64 * cb + 32 * h + 8 * tq, 2);
+          qi4[cb][h][mq][1] = pack4(hc, limb, 64 * cb + 32 * h + 8 * tq + 1, 2);
+        }
+    }
+    // this lane's heads 2tq, 2tq+1: score = Q-limb integer product x 2^(E - 14)
+    float qsig[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int hd = 2 * tq + hh;
+      qsig[hh] = hd < grp ? ldexpf(1.0f, qe[hd] - 14) : 0.0f;
+    }
 
     // this lane's state for heads 2tq, 2tq+1; O^T fragments: INT8 tiles accumulate in
     // o8 (channels 16j + 2g, +1), INT4 tiles in o4 (channels 32j + 4g + 2ab, +1)
@@ -384,6 +418,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     bool ok = true;
     for (int i = warp; i < ntile; i += kConsumers) {
       const int s = i % kDecStages;
+      // Stage s last held tile i - kDecStages, which another warp consumes.  A
+      // parity wait only tells adjacent phases apart, so this warp first waits for
+      // that tile's release (which the load of tile i needs anyway): only then is the
+      // full barrier's previous phase known to be complete, and its wait exact.
+      if (i >= kDecStages &&
+          !mbar_wait(bar_empty + s * 8, ((i / kDecStages) - 1) & 1, err)) { ok = false; break; }
       if (!mbar_wait(bar_full + s * 8, (i / kDecStages) & 1, err)) { ok = false; break; }
       const uint32_t e = __ldg(p.entries + my0 + i);
       const int kt = (int)(e & 0x0FFFFFFFu);
@@ -393,26 +433,23 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       const uint32_t vb = kb + C::kTileBytes;
       const bool is8 = (e >> 28) == TRA_PREC_INT8;
 
-      // ---- scores: sacc[kb] = S^T fragment of keys 16kb + (g, g+8), heads (2tq, 2tq+1)
-      float sacc[4][4];
+      // ---- scores: si[mq][k] = S^T fragment of keys 16k + (g, g+8), columns (2tq, 2tq+1)
+      int si[C::kQM][4][4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
+      for (int mq = 0; mq < C::kQM; ++mq)
 #pragma unroll
-        for (int x = 0; x < 4; ++x) sacc[k][x] = 0.0f;
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int x = 0; x < 4; ++x) si[mq][k][x] = 0;
       if (is8) {
 #pragma unroll
         for (int cb = 0; cb < D / 32; ++cb)
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            uint32_t r[4];
+            uint32_t r[4];  // keys g / g+8 at channels 32cb + 4tq .. (+16): the A fragment as is
             ldsm_x4(kb + 16 * C::kRow8 * k + off8[cb], r);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {  // channels 32cb + 16h ..
-              const uint32_t u0 = r[2 * h] ^ 0x80808080u, u1 = r[2 * h + 1] ^ 0x80808080u;
-              const uint32_t a[4] = {h2_from_bytes(u0, kSel01, kBias8), h2_from_bytes(u1, kSel01, kBias8),
-                                     h2_from_bytes(u0, kSel23, kBias8), h2_from_bytes(u1, kSel23, kBias8)};
-              mma16816(sacc[k], a, qb8[2 * cb + h][0], qb8[2 * cb + h][1]);
-            }
+            for (int mq = 0; mq < C::kQM; ++mq) mma_s8(si[mq][k], r, qi8[cb][mq][0], qi8[cb][mq][1]);
           }
       } else {
 #pragma unroll
@@ -423,28 +460,32 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             ldsm_x4(kb + 16 * C::kRow4 * k + off4[cb], r);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // packed bytes 16h.. = channels 64cb + 32h ..
-              // codes of keys g / g+8 at channels 8tq .. 8tq+7 as channel pairs (c, c+4)
-              uint32_t c0[4], c1[4];
-              i4x8_to_h2(r[2 * h], c0);
-              i4x8_to_h2(r[2 * h + 1], c1);
+              // keys g / g+8, channels 8tq + (0, 2, 4, 6) and 8tq + (1, 3, 5, 7)
+              const uint32_t a[4] = {i4_even_x16(r[2 * h]), i4_even_x16(r[2 * h + 1]),
+                                     i4_odd_x16(r[2 * h]), i4_odd_x16(r[2 * h + 1])};
 #pragma unroll
-              for (int ab = 0; ab < 2; ++ab) {
-                const uint32_t a[4] = {c0[2 * ab], c1[2 * ab], c0[2 * ab + 1], c1[2 * ab + 1]};
-                mma16816(sacc[k], a, qb4[2 * cb + h][ab][0], qb4[2 * cb + h][ab][1]);
-              }
+              for (int mq = 0; mq < C::kQM; ++mq)
+                mma_s8(si[mq][k], a, qi4[cb][h][mq][0], qi4[cb][h][mq][1]);
             }
           }
       }
       // ---- online softmax for heads 2tq, 2tq+1 over keys 16k + g (+8)
-      const float ks = (is8 ? __ldg(p.sk8 + tile) : __ldg(p.sk4 + tile)) * p.scale_log2 * q_unscale;
+      // This lane's columns 2tq + hh hold limb 0 (tq < 2) or limb 1 (tq >= 2) of head
+      // (2tq + hh) mod 4, plus 4 in MMA 1.  Lane tq wants head 2tq + hh: lanes tq and
+      // tq ^ 2 swap the limb the other one lacks (MMA 0 for tq < 2, MMA 1 above).
+      const float kscale = (is8 ? __ldg(p.sk8 + tile) : __ldg(p.sk4 + tile) * 0.0625f) * p.scale_log2;
       const float vs = is8 ? __ldg(p.sv8 + tile) : __ldg(p.sv4 + tile);
+      const float ks[2] = {kscale * qsig[0], kscale * qsig[1]};
+      const bool lowq = tq < 2;
       float sv[2][8];  // [head][key slot: 2k + (g / g+8)]
 #pragma unroll
       for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          sv[hh][2 * k] = sacc[k][hh] * ks;
-          sv[hh][2 * k + 1] = sacc[k][2 + hh] * ks;
+        for (int x = 0; x < 4; ++x) {
+          const int a0 = si[0][k][x], a1 = si[C::kQM - 1][k][x];
+          const int other = __shfl_xor_sync(0xffffffffu, lowq ? a1 : a0, 2);
+          const int q = lowq ? a0 * 256 + other : other * 256 + a1;
+          sv[x & 1][2 * k + (x >> 1)] = (float)q * ks[x & 1];
         }
       if (nvalid < kTile) {  // a sequence's last tile: keys past its end are masked
 #pragma unroll
