@@ -130,12 +130,18 @@ typedef struct {
 typedef struct {
   int8_t* q8;  uint8_t* q4;         /* [Hq][ntiles][64][d] / [..][d/2] */
   int8_t* k8;  uint8_t* k4;         /* [Hkv][ntiles][64][d] / [..][d/2] */
-  int8_t* v8;  uint8_t* v4;
+  int8_t* v8;  uint8_t* v4;         /* v4: see the V4 byte order below */
   float* sq8;  float* sq4;          /* [Hq][ntiles] */
   float* sk8;  float* sk4;          /* [Hkv][ntiles] */
   float* sv8;  float* sv4;
   uint32_t formats;                 /* TRA_FMT_* bits: which fields are present */
 } tra_qtiles;
+/* Code layout.  Rows are tokens of a 64-token tile; INT8 rows hold channel c in byte c.
+ * INT4 rows pack two signed codes (range -7..7) per byte, the even channel in the low
+ * nibble.  Q4 and K4 rows are row-major: byte j holds channels 2j and 2j + 1.  V4 rows,
+ * read only by the decode, are stored in its MMA fragment order: within each 16-byte
+ * group m, byte 2g + e (g = 0..7, e = 0, 1) holds the pair that row-major order keeps at
+ * byte 16m + 8e + g, i.e. channels 32m + 16e + 2g and 32m + 16e + 2g + 1. */
 
 /* Thread-local description of the last error returned on this thread. */
 TRA_API const char* tra_last_error(void);

@@ -127,6 +127,7 @@ struct DecCfg {
   static constexpr int kRow4 = D / 2;            // INT4 row bytes
   static constexpr int kTileBytes = kTile * D;   // INT8 codes of one K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;
+  static_assert(kConsumers <= kDecStages, "the consumers' parity waits need kConsumers <= kDecStages");
   static constexpr int kPStride = 72;            // f16 per head row of P (bank-conflict free)
   static constexpr int kOffQ = kDecStages * kStageBytes;  // q: [D/2 pairs][GRP] float2
   static constexpr int kQBytes = (D / 2) * GRP * 8;
@@ -142,8 +143,7 @@ struct DecCfg {
   static constexpr int kOffBar = kOffE + kEBytes;
   static constexpr int kSmem = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
   static constexpr int kCh = D / 32;             // tail P V channels per lane
-  static constexpr int kB8 = D / 16;             // 16-channel blocks (INT8 V fragments)
-  static constexpr int kB4 = D / 32;             // 32-channel blocks (INT4 V fragments)
+  static constexpr int kB8 = D / 16;             // 16-channel blocks of the O fragments
   static constexpr int kQM = GRP > 4 ? 2 : 1;    // score MMAs per K fragment (4 heads each)
 };
 
@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   if (warp == kConsumers) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      int issued = 0;
       for (int i = 0; i < ntile; ++i) {
         const int s = i % kDecStages, use = i / kDecStages;
         if (use > 0 && !mbar_wait(bar_empty + s * 8, (use - 1) & 1, err)) break;
@@ -217,6 +218,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
           tma_load_2d(dst, &m.k4, bar_full + s * 8, 0, r0);
           tma_load_2d(dst + C::kTileBytes, &m.v4, bar_full + s * 8, 0, r0);
         }
+        ++issued;
+      }
+      if (*err) {
+        // an abandoned split: every load issued lands before the CTA can exit (this
+        // thread alone arrives on the full barriers, so the last fill of each stage
+        // completes its phase as soon as its bytes are in)
+        for (int s = 0; s < kDecStages && s < issued; ++s)
+          mbar_wait_drain(bar_full + s * 8, (uint32_t)(((issued - 1 - s) / kDecStages) & 1));
       }
     }
     named_sync(1);  // ring drained
@@ -311,20 +320,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       qsig[hh] = hd < grp ? ldexpf(1.0f, qe[hd] - 14) : 0.0f;
     }
 
-    // this lane's state for heads 2tq, 2tq+1; O^T fragments: INT8 tiles accumulate in
-    // o8 (channels 16j + 2g, +1), INT4 tiles in o4 (channels 32j + 4g + 2ab, +1)
+    // this lane's state for heads 2tq, 2tq+1; O^T fragments o8[j]: channels 16j + 2g
+    // (rows g) and 16j + 2g + 1 (rows g + 8), for INT8 and INT4 tiles alike (the V4
+    // cache is stored in this fragment order)
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
-    float o8[C::kB8][4], o4[C::kB4][2][4];
+    float o8[C::kB8][4];
 #pragma unroll
     for (int j = 0; j < C::kB8; ++j)
 #pragma unroll
       for (int k = 0; k < 4; ++k) o8[j][k] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < C::kB4; ++j)
-#pragma unroll
-      for (int ab = 0; ab < 2; ++ab)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) o4[j][ab][k] = 0.0f;
     __half* const pw = reinterpret_cast<__half*>(sm + C::kOffP) + warp * 8 * C::kPStride;
     const uint32_t pw_addr = smem_u32(pw);
     const int mrow = lane & 7, mj = lane >> 3;  // ldmatrix: this lane's row / matrix
@@ -341,13 +345,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       off4[cb] = swz<C::kRow4>(mrow + 8 * (mj & 1), 2 * cb + (mj >> 1));
 
     // bf16 tail (tail CTA): tokens [0, tl) of the tail buffer and the new token at
-    // tl; warp w takes tokens w, w + 4, ..., one per lane, with CUDA-core fp32 math
+    // tl; warp w takes tokens w, w + kConsumers, ..., one per lane, with CUDA-core fp32 math
     // and its own softmax state.  All of a lane's loads are issued before use.
     auto tail_pass = [&](float (&tm)[GRP], float (&tlsum)[GRP], float2 (&to)[GRP][C::kCh / 2]) {
       const long long tbase = ((long long)b * p.Hkv + kvh) * p.tail_cap;
       const long long nbase = ((long long)b * p.Hkv + kvh) * D;
-      for (int c0 = 0; warp + 4 * c0 <= tl; c0 += 32) {  // this warp's next 32 tokens
-        const int pos = warp + 4 * (c0 + lane);
+      for (int c0 = 0; warp + kConsumers * c0 <= tl; c0 += 32) {  // this warp's next 32 tokens
+        const int pos = warp + kConsumers * (c0 + lane);
         const bool valid = pos <= tl;
         float2 acc[GRP];
 #pragma unroll
@@ -393,10 +397,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
           for (int k = 0; k < C::kCh / 2; ++k)
             to[gg][k] = __fmul2_rn(to[gg][k], make_float2(al[gg], al[gg]));
         // P V: this lane's channels lane * kCh .. + kCh, tokens of the chunk in order
-        const int nk = min(32, (tl - warp) / 4 - c0 + 1);
+        const int nk = min(32, (tl - warp) / kConsumers - c0 + 1);
 #pragma unroll 4
         for (int j = 0; j < nk; ++j) {
-          const int pj = warp + 4 * (c0 + j);
+          const int pj = warp + kConsumers * (c0 + j);
           const uint16_t* vr = pj == tl ? p.v_new + nbase : p.v_tail + (tbase + pj) * D;
           uint32_t vw[C::kCh / 2];
 #pragma unroll
@@ -421,7 +425,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       // Stage s last held tile i - kDecStages, which another warp consumes.  A
       // parity wait only tells adjacent phases apart, so this warp first waits for
       // that tile's release (which the load of tile i needs anyway): only then is the
-      // full barrier's previous phase known to be complete, and its wait exact.
+      // full barrier's previous phase known to be complete, and its wait exact.  The
+      // release wait is itself exact: the tile before that one in stage s was released
+      // before tile i - kDecStages was loaded, which happened no later than this
+      // warp's previous tile i - kConsumers (kConsumers <= kDecStages).
       if (i >= kDecStages &&
           !mbar_wait(bar_empty + s * 8, ((i / kDecStages) - 1) & 1, err)) { ok = false; break; }
       if (!mbar_wait(bar_full + s * 8, (i / kDecStages) & 1, err)) { ok = false; break; }
@@ -547,13 +554,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
           o8[j][0] *= alpha[0]; o8[j][1] *= alpha[1];
           o8[j][2] *= alpha[0]; o8[j][3] *= alpha[1];
         }
-#pragma unroll
-        for (int j = 0; j < C::kB4; ++j)
-#pragma unroll
-          for (int ab = 0; ab < 2; ++ab) {
-            o4[j][ab][0] *= alpha[0]; o4[j][ab][1] *= alpha[1];
-            o4[j][ab][2] *= alpha[0]; o4[j][ab][3] *= alpha[1];
-          }
       }
       __syncwarp();
       // ---- O^T += V^T P^T: B fragment = P[head g][keys 16k + 2tq (+1), +8 (+9)]
@@ -581,16 +581,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             uint32_t r[4];
             ldsm_x4_t(vb + 16 * C::kRow4 * k + off4[cp], r);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {  // 32 channels 64cp + 32h .. (4g .. 4g+3)
-              // words: keys (2tq, 2tq+1) / (2tq+8, 2tq+9), channels 4g .. 4g+3; the
-              // conversion yields one key pair per channel 4g + 0 .. 3
+            for (int h = 0; h < 2; ++h) {  // 32 channels 64cp + 32h ..
+              // words: keys (2tq, 2tq+1) / (2tq+8, 2tq+9); nibble n of the lane's 16-bit
+              // column holds channel 64cp + 32h + 16 (n / 2) + 2g + n % 2, so the
+              // conversion yields one key pair per channel of blocks 4cp + 2h (+1)
               uint32_t v0[4], v1[4];
               i4x8_to_h2(r[2 * h], v0);
               i4x8_to_h2(r[2 * h + 1], v1);
               const uint32_t aA[4] = {v0[0], v0[1], v1[0], v1[1]};
-              mma16816(o4[2 * cp + h][0], aA, pb0, pb1);
+              mma16816(o8[4 * cp + 2 * h], aA, pb0, pb1);
               const uint32_t aB[4] = {v0[2], v0[3], v1[2], v1[3]};
-              mma16816(o4[2 * cp + h][1], aB, pb0, pb1);
+              mma16816(o8[4 * cp + 2 * h + 1], aB, pb0, pb1);
             }
           }
         }
@@ -627,8 +628,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       }
     } else {
       named_sync(1);
-      for (int x = lane; x < GRP * (D + 2); x += 32) rw[x] = 0.0f;
-      __syncwarp();
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int hd = 2 * tq + hh;
@@ -642,20 +641,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             rw[hd * (D + 2) + D] = m_run[hh];
             rw[hd * (D + 2) + D + 1] = l_run[hh];
           }
-        }
-      }
-      __syncwarp();
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int hd = 2 * tq + hh;
-        if (hd < GRP) {
-#pragma unroll
-          for (int j = 0; j < C::kB4; ++j)
-#pragma unroll
-            for (int ab = 0; ab < 2; ++ab) {
-              rw[hd * (D + 2) + 32 * j + 4 * g + 2 * ab] += o4[j][ab][hh];
-              rw[hd * (D + 2) + 32 * j + 4 * g + 2 * ab + 1] += o4[j][ab][2 + hh];
-            }
         }
       }
     }

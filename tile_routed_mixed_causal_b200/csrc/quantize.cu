@@ -104,10 +104,21 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p) {
       *reinterpret_cast<uint2*>(t.x8 + (tile_base * kTile + r) * D + c * 8) = make_uint2(o[0], o[1]);
     }
     if (t.x4) {
-      uint32_t o = 0;
+      uint32_t o = 0;  // byte jj: channels 8c + 2jj (low nibble) and 8c + 2jj + 1
 #pragma unroll
       for (int j = 0; j < 8; ++j) o |= (uint32_t)(quant_code(x[j], s4, 7) & 0x0F) << (j * 4);
-      *reinterpret_cast<uint32_t*>(t.x4 + (tile_base * kTile + r) * (D / 2) + c * 4) = o;
+      uint8_t* row = t.x4 + (tile_base * kTile + r) * (D / 2);
+      if (!t.perm4) {
+        *reinterpret_cast<uint32_t*>(row + c * 4) = o;
+      } else {
+        // decode order: in each 16-byte group m, byte 2g + e holds the byte that
+        // row-major order keeps at 16m + 8e + g.  Chunks c and c ^ 2 (lanes t, t ^ 2)
+        // fill the same 8 bytes, even positions from e = 0 and odd from e = 1.
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, o, 2);
+        const int e = (c >> 1) & 1;
+        const uint32_t w = e ? __byte_perm(o, other, 0x3726) : __byte_perm(o, other, 0x5140);
+        *reinterpret_cast<uint32_t*>(row + 16 * (c >> 2) + 8 * (c & 1) + 4 * e) = w;
+      }
     }
   }
 }

@@ -18,6 +18,7 @@ struct QuantTensor {
   uint8_t* x4;         // nullable
   float* s8;
   float* s4;
+  int perm4;           // x4 in the decode's V fragment order (V), else row-major
 };
 
 struct QuantParams {
