@@ -289,8 +289,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       return q_limb(hd, limb, c) | q_limb(hd, limb, c + step) << 8 |
              q_limb(hd, limb, c + 2 * step) << 16 | q_limb(hd, limb, c + 3 * step) << 24;
     };
-    // B fragments (column g = head (g & 3) + 4 mq, limb g >> 2), in the channel
-    // order the K codes arrive in:
+    // B fragments (column g = head (g >> 1) + 4 mq, limb g & 1, so that lane tq's
+    // accumulator columns 2tq, 2tq + 1 are both limbs of head tq + 4 mq), in the
+    // channel order the K codes arrive in:
     //   INT8, 32-channel block cb: k = 4t + i -> channel 32cb + 4t + i, k = 16 + 4t + i
     //         -> 32cb + 16 + 4t + i
     //   INT4, 32-channel block 2cb + h: k = 4t + i -> even channel 64cb + 32h + 8t + 2i,
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     uint32_t qi8[D / 32][C::kQM][2], qi4[D / 64][2][C::kQM][2];
 #pragma unroll
     for (int mq = 0; mq < C::kQM; ++mq) {
-      const int hc = (g & 3) + 4 * mq, limb = g >> 2;
+      const int hc = (g >> 1) + 4 * mq, limb = g & 1;
 #pragma unroll
       for (int cb = 0; cb < D / 32; ++cb) {
         qi8[cb][mq][0] = pack4(hc, limb, 32 * cb + 4 * tq, 1);
@@ -312,18 +313,26 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
           qi4[cb][h][mq][1] = pack4(hc, limb, 64 * cb + 32 * h + 8 * tq + 1, 2);
         }
     }
-    // this lane's heads 2tq, 2tq+1: score = Q-limb integer product x 2^(E - 14)
-    float qsig[2];
+    // Softmax heads of this lane ("slots"): tq + 4 mq, score = Q-limb integer product
+    // x 2^(E - 14).  O heads of this lane: 2tq, 2tq + 1 (the P V MMA's columns).
+    float qsig[C::kQM];
+    bool real[C::kQM];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int hd = 2 * tq + hh;
-      qsig[hh] = hd < grp ? ldexpf(1.0f, qe[hd] - 14) : 0.0f;
+    for (int mq = 0; mq < C::kQM; ++mq) {
+      const int hd = tq + 4 * mq;
+      real[mq] = hd < grp;
+      qsig[mq] = real[mq] ? ldexpf(1.0f, qe[hd] - 14) : 0.0f;
     }
 
-    // this lane's state for heads 2tq, 2tq+1; O^T fragments o8[j]: channels 16j + 2g
-    // (rows g) and 16j + 2g + 1 (rows g + 8), for INT8 and INT4 tiles alike (the V4
-    // cache is stored in this fragment order)
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+    // softmax state per slot; O^T fragments o8[j]: channels 16j + 2g (rows g) and
+    // 16j + 2g + 1 (rows g + 8), for INT8 and INT4 tiles alike (the V4 cache is stored
+    // in this fragment order)
+    float m_run[C::kQM], l_run[C::kQM];
+#pragma unroll
+    for (int mq = 0; mq < C::kQM; ++mq) {
+      m_run[mq] = -INFINITY;
+      l_run[mq] = 0.0f;
+    }
     float o8[C::kB8][4];
 #pragma unroll
     for (int j = 0; j < C::kB8; ++j)
@@ -476,69 +485,64 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             }
           }
       }
-      // ---- online softmax for heads 2tq, 2tq+1 over keys 16k + g (+8)
-      // This lane's columns 2tq + hh hold limb 0 (tq < 2) or limb 1 (tq >= 2) of head
-      // (2tq + hh) mod 4, plus 4 in MMA 1.  Lane tq wants head 2tq + hh: lanes tq and
-      // tq ^ 2 swap the limb the other one lacks (MMA 0 for tq < 2, MMA 1 above).
+      // ---- online softmax for this lane's slots over keys 16k + g (+8): accumulator
+      // columns 2tq, 2tq + 1 hold the hi and lo limb products of head tq + 4 mq
       const float kscale = (is8 ? __ldg(p.sk8 + tile) : __ldg(p.sk4 + tile) * 0.0625f) * p.scale_log2;
       const float vs = is8 ? __ldg(p.sv8 + tile) : __ldg(p.sv4 + tile);
-      const float ks[2] = {kscale * qsig[0], kscale * qsig[1]};
-      const bool lowq = tq < 2;
-      float sv[2][8];  // [head][key slot: 2k + (g / g+8)]
+      float sv[C::kQM][8];  // [slot][key slot: 2k + (g / g+8)]
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
+      for (int mq = 0; mq < C::kQM; ++mq) {
+        const float ks = kscale * qsig[mq];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int a0 = si[0][k][x], a1 = si[C::kQM - 1][k][x];
-          const int other = __shfl_xor_sync(0xffffffffu, lowq ? a1 : a0, 2);
-          const int q = lowq ? a0 * 256 + other : other * 256 + a1;
-          sv[x & 1][2 * k + (x >> 1)] = (float)q * ks[x & 1];
+        for (int k = 0; k < 4; ++k) {
+          sv[mq][2 * k] = (float)(si[mq][k][0] * 256 + si[mq][k][1]) * ks;
+          sv[mq][2 * k + 1] = (float)(si[mq][k][2] * 256 + si[mq][k][3]) * ks;
         }
+      }
       if (nvalid < kTile) {  // a sequence's last tile: keys past its end are masked
 #pragma unroll
         for (int k = 0; k < 4; ++k)
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            if (16 * k + g >= nvalid) sv[hh][2 * k] = -INFINITY;
-            if (16 * k + g + 8 >= nvalid) sv[hh][2 * k + 1] = -INFINITY;
+          for (int mq = 0; mq < C::kQM; ++mq) {
+            if (16 * k + g >= nvalid) sv[mq][2 * k] = -INFINITY;
+            if (16 * k + g + 8 >= nvalid) sv[mq][2 * k + 1] = -INFINITY;
           }
       }
-      float mt[2], alpha[2] = {1.0f, 1.0f};
+      float mt[C::kQM], alpha[C::kQM];
       bool need = false;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float x = sv[hh][0];
+      for (int mq = 0; mq < C::kQM; ++mq) {
+        float x = sv[mq][0];
 #pragma unroll
-        for (int k = 1; k < 8; ++k) x = fmaxf(x, sv[hh][k]);
+        for (int k = 1; k < 8; ++k) x = fmaxf(x, sv[mq][k]);
         x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
         x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
         x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
-        mt[hh] = x;
-        need |= fmaxf(m_run[hh], x) > m_run[hh] + 8.0f;  // true for the first finite max
+        mt[mq] = x;
+        alpha[mq] = 1.0f;
+        need |= fmaxf(m_run[mq], x) > m_run[mq] + 8.0f;  // true for the first finite max
       }
       // lazy rescaling: the reference max moves only when it grew by more than 2^8
       const bool warp_need = __any_sync(0xffffffffu, need);
       if (warp_need) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const float m_new = fmaxf(m_run[hh], mt[hh]);
-          if (m_new > m_run[hh]) {
-            alpha[hh] = ex2(m_run[hh] - m_new);  // -inf -> 0
-            m_run[hh] = m_new;
+        for (int mq = 0; mq < C::kQM; ++mq) {
+          const float m_new = fmaxf(m_run[mq], mt[mq]);
+          if (m_new > m_run[mq]) {
+            alpha[mq] = ex2(m_run[mq] - m_new);  // -inf -> 0
+            m_run[mq] = m_new;
           }
         }
       }
-      const bool real0 = 2 * tq < grp, real1 = 2 * tq + 1 < grp;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const float mb = m_run[hh] == -INFINITY ? 0.0f : m_run[hh];
-        const bool real = hh == 0 ? real0 : real1;
+      for (int mq = 0; mq < C::kQM; ++mq) {
+        const float mb = m_run[mq] == -INFINITY ? 0.0f : m_run[mq];
         float ps = 0.0f;
-        __half* prow = pw + (2 * tq + hh) * C::kPStride;
+        __half* prow = pw + (tq + 4 * mq) * C::kPStride;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float p0 = real ? ex2(sv[hh][2 * k] - mb) : 0.0f;
-          const float p1 = real ? ex2(sv[hh][2 * k + 1] - mb) : 0.0f;
+          const float p0 = real[mq] ? ex2(sv[mq][2 * k] - mb) : 0.0f;
+          const float p1 = real[mq] ? ex2(sv[mq][2 * k + 1] - mb) : 0.0f;
           ps += p0 + p1;
           prow[16 * k + g] = __float2half_rn(p0 * vs);
           prow[16 * k + g + 8] = __float2half_rn(p1 * vs);
@@ -546,13 +550,22 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         ps += __shfl_xor_sync(0xffffffffu, ps, 4);
         ps += __shfl_xor_sync(0xffffffffu, ps, 8);
         ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-        l_run[hh] = l_run[hh] * alpha[hh] + ps;
+        l_run[mq] = l_run[mq] * alpha[mq] + ps;
       }
       if (warp_need) {
+        // O head 2tq + hh is softmax slot (2tq + hh) / 4 of lane 4g + (2tq + hh) % 4
+        float ao[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int hd = 2 * tq + hh, src = (lane & ~3) | (hd & 3);
+          const float a0 = __shfl_sync(0xffffffffu, alpha[0], src);
+          const float a1 = __shfl_sync(0xffffffffu, alpha[C::kQM - 1], src);
+          ao[hh] = hd >= 4 ? a1 : a0;
+        }
 #pragma unroll
         for (int j = 0; j < C::kB8; ++j) {
-          o8[j][0] *= alpha[0]; o8[j][1] *= alpha[1];
-          o8[j][2] *= alpha[0]; o8[j][3] *= alpha[1];
+          o8[j][0] *= ao[0]; o8[j][1] *= ao[1];
+          o8[j][2] *= ao[0]; o8[j][3] *= ao[1];
         }
       }
       __syncwarp();
@@ -637,10 +650,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             rw[hd * (D + 2) + 16 * j + 2 * g] = o8[j][hh];
             rw[hd * (D + 2) + 16 * j + 2 * g + 1] = o8[j][2 + hh];
           }
-          if (g == 0) {
-            rw[hd * (D + 2) + D] = m_run[hh];
-            rw[hd * (D + 2) + D + 1] = l_run[hh];
-          }
+        }
+      }
+#pragma unroll
+      for (int mq = 0; mq < C::kQM; ++mq) {
+        const int hd = tq + 4 * mq;
+        if (hd < GRP && g == 0) {
+          rw[hd * (D + 2) + D] = m_run[mq];
+          rw[hd * (D + 2) + D + 1] = l_run[mq];
         }
       }
     }
