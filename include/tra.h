@@ -136,7 +136,9 @@ typedef struct {
   float* sv8;  float* sv4;
   uint32_t formats;                 /* TRA_FMT_* bits: which fields are present */
 } tra_qtiles;
-/* Code layout.  Rows are tokens of a 64-token tile; INT8 rows hold channel c in byte c.
+/* Code layout.  Rows are tokens of a 64-token tile; INT8 rows hold channel c in byte c,
+ * as two's complement for Q8 and K8 and offset-binary (code + 128) for V8, which only
+ * the decode reads.
  * INT4 rows pack two signed codes (range -7..7) per byte, the even channel in the low
  * nibble.  Q4 and K4 rows are row-major: byte j holds channels 2j and 2j + 1.  V4 rows,
  * read only by the decode, are stored in its MMA fragment order: within each 16-byte

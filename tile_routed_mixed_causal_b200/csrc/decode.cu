@@ -324,7 +324,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       qsig[mq] = real[mq] ? ldexpf(1.0f, qe[hd] - 14) : 0.0f;
     }
 
-    // softmax state per slot; O^T fragments o8[j]: channels 16j + 2g (rows g) and
+    // softmax state per slot (l_run: this lane's partial sum over its keys, reduced
+    // over the lanes once at the end); O^T fragments o8[j]: channels 16j + 2g (rows g) and
     // 16j + 2g + 1 (rows g + 8), for INT8 and INT4 tiles alike (the V4 cache is stored
     // in this fragment order)
     float m_run[C::kQM], l_run[C::kQM];
@@ -547,9 +548,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
           prow[16 * k + g] = __float2half_rn(p0 * vs);
           prow[16 * k + g + 8] = __float2half_rn(p1 * vs);
         }
-        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
         l_run[mq] = l_run[mq] * alpha[mq] + ps;
       }
       if (warp_need) {
@@ -582,7 +580,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             ldsm_x4_t(vb + 16 * C::kRow8 * k + off8[cp], r);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // channels 32cp + 16h + (2g, 2g+1)
-              const uint32_t u0 = r[2 * h] ^ 0x80808080u, u1 = r[2 * h + 1] ^ 0x80808080u;
+              // V8 codes are stored offset-binary (code + 128)
+              const uint32_t u0 = r[2 * h], u1 = r[2 * h + 1];
               const uint32_t a[4] = {h2_from_bytes(u0, kSel02, kBias8), h2_from_bytes(u0, kSel13, kBias8),
                                      h2_from_bytes(u1, kSel02, kBias8), h2_from_bytes(u1, kSel13, kBias8)};
               mma16816(o8[2 * cp + h], a, pb0, pb1);
@@ -640,6 +639,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         }
       }
     } else {
+#pragma unroll
+      for (int mq = 0; mq < C::kQM; ++mq)
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) l_run[mq] += __shfl_xor_sync(0xffffffffu, l_run[mq], o);
       named_sync(1);
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {

@@ -97,10 +97,13 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p) {
     }
     // rows past the sequence end were loaded as 0 and quantise to code 0
     if (t.x8) {
+      const uint32_t flip = t.bias8 ? 0x80808080u : 0u;  // offset-binary: code + 128
       uint32_t o[2] = {0, 0};
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         o[j >> 2] |= (uint32_t)(quant_code(x[j], s8, 127) & 0xFF) << ((j & 3) * 8);
+      o[0] ^= flip;
+      o[1] ^= flip;
       *reinterpret_cast<uint2*>(t.x8 + (tile_base * kTile + r) * D + c * 8) = make_uint2(o[0], o[1]);
     }
     if (t.x4) {

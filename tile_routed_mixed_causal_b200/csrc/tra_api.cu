@@ -214,6 +214,7 @@ tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const u
       t.s8 = want8 ? s8[i] : nullptr;
       t.x4 = want4 ? o4[i] : nullptr;
       t.perm4 = i == 2;  // V4 is read only by the decode, in its MMA fragment order
+      t.bias8 = i == 2;  // so is V8, kept offset-binary for its f16 conversion
       t.s4 = want4 ? s4[i] : nullptr;
     }
     p.cta_begin[i + 1] = p.cta_begin[i] + (t.x ? (long long)t.H * nt : 0);

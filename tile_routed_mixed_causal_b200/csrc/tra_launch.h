@@ -19,6 +19,7 @@ struct QuantTensor {
   float* s8;
   float* s4;
   int perm4;           // x4 in the decode's V fragment order (V), else row-major
+  int bias8;           // x8 codes stored offset-binary, code + 128 (V), else two's complement
 };
 
 struct QuantParams {
