@@ -296,8 +296,8 @@ def decode_bench(device, passes, stream, hbm_gbs):
         "bytes_per_step": int(pass_bytes / steps),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                      "frac": round(gbs / hbm_gbs, 4), "traffic": profiled_traffic("decode.cu"),
-                     "kernel": "decode_split_kernel + decode_combine_kernel (one ABI call)"},
-        "gpu_launches_per_step": 2,
+                     "kernel": "decode_split_kernel (one ABI call, one launch)"},
+        "gpu_launches_per_step": 1,
     }
 
 

@@ -246,7 +246,11 @@ TRA_API size_t tra_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, in
  * row_ptr/entries: TRA_LISTS_DECODE_CACHE lists;
  * k_tail/v_tail: device bf16 [B][Hkv][tail_cap][d]; tail_len_dev: device
  * int32 [B] (read, then incremented by one); out: device bf16 [B][Hq][d];
- * workspace: device, >= tra_decode_workspace_bytes(B, Hq, Hkv, d).
+ * workspace: device, >= tra_decode_workspace_bytes(B, Hq, Hkv, d), zero-filled
+ * before its first use and not written by anything else between calls: it starts
+ * with per-(sequence, KV head) arrival counters, which every call leaves at zero
+ * (at a fixed place for every shape with B * (Hkv + 1) <= 16384, so one workspace
+ * may serve several shapes), followed by the splits' partial results.
  * A sequence whose tail is full sets TRA_DEV_TAIL_FULL and leaves its output
  * and tail untouched.
  */

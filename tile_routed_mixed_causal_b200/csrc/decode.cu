@@ -21,7 +21,8 @@
 // The bf16 tail (earlier decode tokens + the new one) is a split of its own:
 // CTA x = 0 of every (sequence, KV head), scheduled first, whose four warps
 // share the tail keys on the CUDA cores.  The four warps' states are merged per
-// CTA, and a small combine kernel merges the splits and advances tail_len.
+// CTA; the last split of each (sequence, KV head) to finish merges the splits
+// into the output, and the last such row of a sequence advances tail_len.
 #include "tra_device.cuh"
 #include "tra_launch.h"
 
@@ -140,6 +141,8 @@ struct DecCfg {
   static constexpr int kOffRed = 0;
   static constexpr int kRedBytes = kStates * GRP * (D + 2) * 4;
   static_assert(kRedBytes <= kDecStages * kStageBytes, "merge area must fit in the ring");
+  static_assert((2 * TRA_MAX_DECODE_SPLITS + 1) * GRP * 4 <= kDecStages * kStageBytes,
+                "split weights must fit in the ring");
   static constexpr int kOffBar = kOffE + kEBytes;
   static constexpr int kSmem = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
   static constexpr int kCh = D / 32;             // tail P V channels per lane
@@ -171,14 +174,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   const int T = __ldg(p.cu + b + 1) - seq0;
   const int toff = seq_tile_offset(p.cu, b);
   const int tl = __ldg(p.tail_len + b);
-  if (tl >= p.tail_cap) {
-    if (tail_cta && kvh == 0 && t == 0) {
-      atomicOr(p.status, TRA_DEV_TAIL_FULL);
-      p.skip[b] = 1;
-    }
+  if (tl >= p.tail_cap) {  // every CTA of sequence b leaves: output and tail untouched
+    if (tail_cta && kvh == 0 && t == 0) atomicOr(p.status, TRA_DEV_TAIL_FULL);
     return;
   }
-  if (tail_cta && kvh == 0 && t == 0) p.skip[b] = 0;
   int my0 = 0, ntile = 0;
   if (!tail_cta) {
     const long long row = (long long)b * p.Hkv + kvh;
@@ -689,33 +688,61 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     }
   }
   if (t == 0 && *err) atomicOr(p.status, *err);
-}
 
-// One block per (sequence, query head): merge the splits' partials.
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
-  const int bh = blockIdx.x;
-  const int b = bh / p.Hq;
-  if (p.skip[b]) return;  // full tail: output and tail untouched
-  const long long pi = (long long)bh * p.splits;
-  float M = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, p.part_ml[(pi + s) * 2]);
-  float L = 0.0f;
-  for (int s = 0; s < p.splits; ++s) {
-    const float m = p.part_ml[(pi + s) * 2];
-    if (m != -INFINITY) L += p.part_ml[(pi + s) * 2 + 1] * ex2(m - M);
+  // The last split of row (b, kvh) to finish merges the row's partials into the
+  // output of its query heads (a release / acquire pair of fences around the
+  // arrival count); the last row of sequence b advances tail_len[b], which every
+  // CTA of the sequence has read by then.
+  volatile int* const last = err + 1;
+  const long long row = (long long)b * p.Hkv + kvh;
+  __threadfence();
+  __syncthreads();
+  if (t == 0) *last = atomicAdd(p.row_count + row, 1) == p.splits - 1;
+  __syncthreads();
+  if (!*last) return;
+  __threadfence();
+  // (m, l) of the row's (head, split) partials into shared memory (the ring is
+  // free), then per head the max M, the weights 2^(m - M) and 1/L, then O
+  const int S = p.splits;
+  const long long hb = (long long)b * p.Hq + kvh * grp;  // first query head of the row
+  float* const wm = reinterpret_cast<float*>(sm);        // [grp][S] m, then weights
+  float* const wl = wm + GRP * TRA_MAX_DECODE_SPLITS;    // [grp][S] l
+  float* const winv = wl + GRP * TRA_MAX_DECODE_SPLITS;  // [grp] 1 / L
+  for (int x = t; x < grp * S; x += kDecThreads) {
+    wm[x] = __ldcg(p.part_ml + (hb * S + x) * 2);
+    wl[x] = __ldcg(p.part_ml + (hb * S + x) * 2 + 1);
   }
-  const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-  for (int c = threadIdx.x; c < p.d; c += blockDim.x) {
-    float o = 0.0f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float m = p.part_ml[(pi + s) * 2];
-      if (m != -INFINITY) o += p.part_o[(pi + s) * p.d + c] * ex2(m - M);
+  __syncthreads();
+  if (t < grp) {
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, wm[t * S + s]);
+    float L = 0.0f;
+    for (int s = 0; s < S; ++s) {
+      const float m = wm[t * S + s];
+      const float wt = m == -INFINITY ? 0.0f : ex2(m - M);
+      wm[t * S + s] = wt;
+      L += wl[t * S + s] * wt;
     }
-    const __nv_bfloat16 r = __float2bfloat16_rn(o * inv);
-    p.out[(long long)bh * p.d + c] = *reinterpret_cast<const uint16_t*>(&r);
+    winv[t] = L > 0.0f ? 1.0f / L : 0.0f;
   }
-  // only this block touches tail_len[b]; every split has read it already
-  if (threadIdx.x == 0 && bh % p.Hq == 0) p.tail_len[b] += 1;
+  __syncthreads();
+  for (int x = t; x < grp * D; x += kDecThreads) {
+    const int gg = x / D, c = x % D;
+    const float* po = p.part_o + (hb + gg) * S * D + c;
+    float o = 0.0f;
+#pragma unroll 4
+    for (int s = 0; s < S; ++s) o += __ldcg(po + (long long)s * D) * wm[gg * S + s];
+    const __nv_bfloat16 r = __float2bfloat16_rn(o * winv[gg]);
+    p.out[(hb + gg) * D + c] = *reinterpret_cast<const uint16_t*>(&r);
+  }
+  if (t == 0) {
+    p.row_count[row] = 0;
+    __threadfence();
+    if (atomicAdd(p.seq_count + b, 1) == p.Hkv - 1) {
+      p.seq_count[b] = 0;
+      p.tail_len[b] += 1;
+    }
+  }
 }
 
 template <int D, int GRP>
@@ -726,9 +753,6 @@ cudaError_t launch_dec(const DecodeParams& p, const DecodeMaps& m, cudaStream_t 
   if (e != cudaSuccess) return e;
   dim3 grid(p.splits, p.Hkv, p.B);
   decode_split_kernel<D, GRP><<<grid, kDecThreads, C::kSmem, s>>>(p, m);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<p.B * p.Hq, 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -745,7 +769,9 @@ cudaError_t launch_dec_d(const DecodeParams& p, const DecodeMaps& m, cudaStream_
 
 // Partials per (sequence, KV head): the data splits plus the bf16-tail split.
 int decode_splits(int B, int Hkv) {
-  const int target = 512;  // under two waves of two CTAs per SM: long CTAs, little set-up
+  // about 256 data CTAs (plus one tail CTA per row): long CTAs, little set-up and a
+  // short merge, about 1.3 waves of two CTAs per SM at batch 16 x 8 KV heads
+  const int target = 256;
   const int rows = B * Hkv;
   int s = (target + rows - 1) / rows;
   if (s < 1) s = 1;

@@ -64,9 +64,10 @@ extern "C" tra_status routed_attention_decode_noalloc(
   void* scratch = nullptr;
   tra_status st = scratch_address(&scratch);
   if (st != TRA_OK) return st;
-  // Nothing in the scratch has to start at zero: every split writes its partial
-  // before the combine kernel reads it.  The regular entry point validates all
-  // other arguments and enqueues the same kernels.
+  // The scratch starts zero-filled (static storage) and every call leaves its
+  // arrival counters at zero again; the partials behind them are written before
+  // they are read.  The regular entry point validates all other arguments and
+  // enqueues the same kernel.
   return routed_attention_decode(prefill_shape, policy, q, k_new, v_new, cache, row_ptr, entries,
                                  k_tail, v_tail, tail_len_dev, tail_cap, softmax_scale, out,
                                  scratch, TRA_NOALLOC_SCRATCH_BYTES, status_dev, stream);

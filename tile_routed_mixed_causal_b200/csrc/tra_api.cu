@@ -379,11 +379,20 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
   return ok();
 }
 
+// Decode workspace: arrival counters first, in a region of fixed size for every
+// shape up to kCounterInts of them (so that a workspace reused across shapes keeps
+// them at zero: the partials never land there), then the splits' partials.
+constexpr size_t kCounterInts = 16384;
+size_t decode_counter_bytes(int32_t B, int32_t Hkv) {
+  const size_t n = (size_t)B * (Hkv + 1);
+  return round256(4 * (n > kCounterInts ? n : kCounterInts));
+}
+
 size_t tra_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t d) {
   if (B < 1 || Hq < 1 || Hkv < 1 || d < 1) return 0;
   const size_t S = (size_t)tra::decode_splits(B, Hkv);
-  return round256((size_t)B * Hq * S * 2 * 4) + round256((size_t)B * Hq * S * d * 4) +
-         round256((size_t)B * 4);
+  return decode_counter_bytes(B, Hkv) + round256((size_t)B * Hq * S * 2 * 4) +
+         round256((size_t)B * Hq * S * d * 4);
 }
 
 tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* policy,
@@ -444,12 +453,12 @@ tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* pol
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.out = out;
   const size_t S = (size_t)p.splits;
-  p.part_ml = reinterpret_cast<float*>(workspace);
-  p.part_o = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
-                                      round256((size_t)shape->B * shape->Hq * S * 2 * 4));
-  p.skip = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(workspace) +
-                                      round256((size_t)shape->B * shape->Hq * S * 2 * 4) +
-                                      round256((size_t)shape->B * shape->Hq * S * shape->d * 4));
+  uint8_t* const ws = reinterpret_cast<uint8_t*>(workspace);
+  p.row_count = reinterpret_cast<int32_t*>(ws);
+  p.seq_count = p.row_count + (size_t)shape->B * shape->Hkv;
+  const size_t off_ml = decode_counter_bytes(shape->B, shape->Hkv);
+  p.part_ml = reinterpret_cast<float*>(ws + off_ml);
+  p.part_o = reinterpret_cast<float*>(ws + off_ml + round256((size_t)shape->B * shape->Hq * S * 2 * 4));
   p.status = status_dev;
   tra::DecodeMaps m;
   memset(&m, 0, sizeof m);

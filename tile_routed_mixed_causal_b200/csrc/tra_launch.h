@@ -98,7 +98,8 @@ struct DecodeParams {
   uint16_t* out;           // [B][Hq][d]
   float* part_ml;          // [B][Hq][splits][2]
   float* part_o;           // [B][Hq][splits][d]
-  int32_t* skip;           // [B]: 1 when the sequence's tail is full this step
+  int32_t* row_count;      // [B][Hkv] splits finished this step (zero between calls)
+  int32_t* seq_count;      // [B] rows finished this step (zero between calls)
   int32_t* status;
 };
 
