@@ -68,8 +68,8 @@ def parse():
 # source that has changed since reports null.  Captures: profiles/prefill_kernel_bitmask_32k.md
 # and profiles/decode_split_kernel_b16_32k.md.
 PROFILED_TRAFFIC = {
-    "prefill.cu": ("006591d5deb101dc", 3_384_843_776),
-    "decode.cu": ("fbb72974b738b53e", 663_281_408),
+    "prefill.cu": ("bad45a2b16f93e23", 3_372_927_232),
+    "decode.cu": ("a0ae0cc01c87ca66", 663_556_096),
 }
 
 
