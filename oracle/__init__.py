@@ -61,6 +61,8 @@ def _load():
             lib.orc_lists_boundary.restype = L
             lib.orc_lists_bitmask.argtypes = [P, I, I, P, I, I, P, P]
             lib.orc_lists_bitmask.restype = L
+            lib.orc_lists_mixed.argtypes = [P, I, I, P, P, P, I, I, P, P]
+            lib.orc_lists_mixed.restype = L
             lib.orc_lists_decode.argtypes = [P, I, I, I, I, P, P, P, P]
             lib.orc_lists_decode.restype = L
             lib.orc_int_tile.argtypes = [I, I, P, P, P, P, P]
@@ -140,6 +142,25 @@ def lists_bitmask(cu_seqlens, bitmask, G):
     row_ptr = np.zeros(Hq * num_tiles(cu) + 1, np.int32)
     entries = np.zeros(max(nnz, 1), np.uint32)
     lib.orc_lists_bitmask(_p(cu), B, Hq, _p(bm), G, W, _p(row_ptr), _p(entries))
+    return row_ptr, entries[:nnz]
+
+
+def lists_mixed(cu_seqlens, b1, b2, bitmask, G):
+    """Four-way rows: boundaries give skip / INT4 / INT8, a set bitmask bit of a
+    kept tile's group promotes it to BF16 (a reading combining both pages)."""
+    cu = _c(cu_seqlens, np.int32)
+    b1 = _c(b1, np.int32)
+    b2 = _c(b2, np.int32)
+    bm = _c(bitmask, np.uint32)
+    Hq, _, W = bm.shape
+    lib = _load()
+    B = len(cu) - 1
+    nnz = lib.orc_lists_mixed(_p(cu), B, Hq, _p(b1), _p(b2), _p(bm), G, W, None, None)
+    if nnz < 0:
+        raise ValueError("invalid mixed policy")
+    row_ptr = np.zeros(Hq * num_tiles(cu) + 1, np.int32)
+    entries = np.zeros(max(nnz, 1), np.uint32)
+    lib.orc_lists_mixed(_p(cu), B, Hq, _p(b1), _p(b2), _p(bm), G, W, _p(row_ptr), _p(entries))
     return row_ptr, entries[:nnz]
 
 

@@ -241,6 +241,44 @@ int64_t orc_lists_bitmask(const int32_t* cu, int B, int Hq, const uint32_t* bitm
   return pos;
 }
 
+/* mixed: the boundary rule decides skip / INT4 / INT8 by distance, and the
+ * bitmask bit of a kept tile's group (bit g covers k-tiles [gG, gG+G), as in
+ * orc_lists_bitmask) promotes it to BF16.  This combination of the two pages'
+ * policies is a reading; neither page describes it. */
+int64_t orc_lists_mixed(const int32_t* cu, int B, int Hq, const int32_t* b1, const int32_t* b2,
+                        const uint32_t* bitmask, int G, int W, int32_t* row_ptr,
+                        uint32_t* entries) {
+  if (G < 1) return -1;
+  int64_t ntiles = orc_num_tiles(cu, B);
+  int64_t pos = 0, row = 0;
+  int nt_max = 0;
+  for (int b = 0; b < B; ++b) if (ceil_tiles(cu[b + 1] - cu[b]) > nt_max) nt_max = ceil_tiles(cu[b + 1] - cu[b]);
+  if ((int64_t)W * 32 < (nt_max + G - 1) / G) return -1;
+  int* prec = (int*)malloc(sizeof(int) * (size_t)(nt_max + 1));
+  for (int h = 0; h < Hq; ++h) {
+    if (b1[h] < 1 || b2[h] < b1[h]) { free(prec); return -1; }
+    int64_t gt0 = 0;
+    for (int b = 0; b < B; ++b) {
+      int nt = ceil_tiles(cu[b + 1] - cu[b]);
+      for (int qt = 0; qt < nt; ++qt, ++row) {
+        const uint32_t* words = bitmask + ((int64_t)h * ntiles + gt0 + qt) * W;
+        if (row_ptr) row_ptr[row] = (int32_t)pos;
+        for (int kt = 0; kt <= qt; ++kt) {
+          int pr = boundary_prec(qt - kt, b1[h], b2[h]);
+          int g = kt / G;
+          if (pr != ORC_SKIP && ((words[g / 32] >> (g % 32)) & 1u)) pr = ORC_BF16;
+          prec[kt] = pr;
+        }
+        pos = emit_row(prec, qt + 1, entries, pos);
+      }
+      gt0 += nt;
+    }
+  }
+  if (row_ptr) row_ptr[row] = (int32_t)pos;
+  free(prec);
+  return pos;
+}
+
 /* Decode-cache lists: rows (b, kvh).  mode 0 = boundary (b1,b2 per q head),
  * mode 1 = bitmask (every prefill tile cached as INT8). */
 int64_t orc_lists_decode(const int32_t* cu, int B, int Hq, int Hkv, int mode,

@@ -174,6 +174,57 @@ def test_lists_bitmask_closed_form():
             gt += nt
 
 
+def _mixed_case(seed=5):
+    lengths = [64 * 30 + 7, 64, 64 * 11]
+    G = 2
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    nts = [(L + 63) // 64 for L in lengths]
+    b1 = [1, 3, 2, 5]
+    b2 = [4, 3, 9, 40]
+    rng = np.random.default_rng(seed)
+    bm = rng.integers(0, 2**32, size=(len(b1), sum(nts), 1), dtype=np.uint64).astype(np.uint32)
+    return lengths, nts, cu, b1, b2, bm, G
+
+
+def test_lists_mixed_closed_form():
+    """Four-way rows: kept tiles min(qt+1, b2) as in the boundary rule, each promoted to
+    BF16 when its group's bit is set; INT4 block, then INT8, then BF16, each ascending."""
+    lengths, nts, cu, b1, b2, bm, G = _mixed_case()
+    rp, en = oracle.lists_mixed(cu, b1, b2, bm, G)
+    prec, kt = _decode_entries(en)
+    row = 0
+    for h in range(len(b1)):
+        gt = 0
+        for nt in nts:
+            for qt in range(nt):
+                word = int(bm[h, gt + qt, 0])
+                kept = range(max(0, qt - b2[h] + 1), qt + 1)
+                hi = [j for j in kept if (word >> (j // G)) & 1]
+                t4 = [j for j in kept if not (word >> (j // G)) & 1 and qt - j >= b1[h]]
+                t8 = [j for j in kept if not (word >> (j // G)) & 1 and qt - j < b1[h]]
+                s, e = rp[row], rp[row + 1]
+                assert e - s == min(qt + 1, b2[h])
+                assert list(kt[s:e]) == t4 + t8 + hi
+                assert list(prec[s:e]) == [1] * len(t4) + [2] * len(t8) + [3] * len(hi)
+                row += 1
+            gt += nt
+    assert rp[-1] == len(en)
+
+
+def test_lists_mixed_reduces_to_each_policy():
+    """No bit set: the boundary policy's lists.  b1 = b2 >= every tile count (nothing
+    skipped, no INT4): the bitmask policy's lists."""
+    lengths, nts, cu, b1, b2, bm, G = _mixed_case(seed=6)
+    zero = np.zeros_like(bm)
+    rp_m, en_m = oracle.lists_mixed(cu, b1, b2, zero, G)
+    rp_b, en_b = oracle.lists_boundary(cu, b1, b2)
+    assert np.array_equal(rp_m, rp_b) and np.array_equal(en_m, en_b)
+    big = [max(nts)] * len(b1)
+    rp_m, en_m = oracle.lists_mixed(cu, big, big, bm, G)
+    rp_k, en_k = oracle.lists_bitmask(cu, bm, G)
+    assert np.array_equal(rp_m, rp_k) and np.array_equal(en_m, en_k)
+
+
 def test_lists_decode_closed_form():
     lengths = [64 * 20, 64 * 7 + 5]
     Hq, Hkv = 4, 2
