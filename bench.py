@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part only (used for profiler captures); prints a reduced line")
-    ap.add_argument("--workload", choices=["bitmask_32k", "llama8b_8k", "varlen_8"],
+    ap.add_argument("--workload", choices=["bitmask_32k", "llama8b_8k", "varlen_8", "mixed_8k"],
                     default="bitmask_32k",
                     help="prefill workload for --only prefill (the full bench line always uses "
                          "bitmask_32k)")
@@ -155,6 +155,9 @@ def prefill_setup(device, workload="bitmask_32k"):
     if w.mode == "bitmask":
         bitmask = torch.from_numpy(w.bitmask.view(np.int32)).to(device)
         pol = tra.Policy.from_bitmask(bitmask, w.G)
+    elif w.mode == "mixed":
+        bitmask = torch.from_numpy(w.bitmask.view(np.int32)).to(device)
+        pol = tra.Policy.mixed(w.b1, w.b2, bitmask, w.G)
     else:
         bitmask = torch.zeros(1, dtype=torch.int32, device=device)
         pol = tra.Policy.boundary(w.b1, w.b2)

@@ -89,6 +89,13 @@ typedef enum {
 
 #define TRA_POLICY_BOUNDARY 0
 #define TRA_POLICY_BITMASK 1
+/* Both at once (four-way): the boundaries decide skip / INT4 / INT8 by distance
+ * and a set bitmask bit of a kept tile's group promotes it to BF16.  Neither page
+ * describes the combination; it joins TriAttention's boundary rule (abstract) and
+ * TileMix's bitmask (abstract).  Decode caches of a mixed policy follow its
+ * boundaries.  The prefill runs one work unit per CTA in this mode (its operand
+ * buffers do not fit twice), so it is slower per tile than the other two. */
+#define TRA_POLICY_MIXED 2
 
 #define TRA_LISTS_PREFILL 0
 #define TRA_LISTS_DECODE_CACHE 1
@@ -119,11 +126,11 @@ typedef struct {
 } tra_shape;
 
 typedef struct {
-  int32_t mode;                     /* TRA_POLICY_BOUNDARY or TRA_POLICY_BITMASK */
-  const int32_t* b1;                /* host [Hq] (boundary mode) */
-  const int32_t* b2;                /* host [Hq] (boundary mode) */
-  const uint32_t* bitmask_dev;      /* device [Hq][ntiles][W] (bitmask mode) */
-  int32_t G;                        /* k-tiles per bit (bitmask mode), >= 1 */
+  int32_t mode;                     /* TRA_POLICY_BOUNDARY, _BITMASK or _MIXED */
+  const int32_t* b1;                /* host [Hq] (boundary and mixed modes) */
+  const int32_t* b2;                /* host [Hq] (boundary and mixed modes) */
+  const uint32_t* bitmask_dev;      /* device [Hq][ntiles][W] (bitmask and mixed modes) */
+  int32_t G;                        /* k-tiles per bit (bitmask and mixed modes), >= 1 */
   int32_t W;                        /* words per bitmask row, W*32*G >= max nt */
 } tra_policy;
 

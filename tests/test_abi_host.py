@@ -187,3 +187,38 @@ def test_selftest_argument_errors(lib):
     assert lib.tra_selftest_bounded_wait(FAKE, 999, None) == 1
     assert lib.tra_selftest_bounded_wait(FAKE, 10**9 + 1, None) == 1
     assert b"limit_ns" in lib.tra_last_error()
+
+
+def test_mixed_policy_sizes_and_validation(lib):
+    """A mixed policy keeps the boundary rule's tile counts (the bitmask only changes
+    precisions), its decode caches follow the boundaries, and both halves of the
+    policy are validated."""
+    import torch
+    lengths = [64 * 40 + 3, 65, 64 * 9]
+    b1, b2 = [1, 2, 1, 3], [4, 2, 9, 40]
+    s = _shape(lengths, Hq=4, Hkv=2)
+    nt = sum((L_ + 63) // 64 for L_ in lengths)
+    rng = np.random.default_rng(11)
+    bm = torch.from_numpy(rng.integers(0, 2**31, size=(4, nt, 1), dtype=np.int64).astype(np.int32))
+    pol = L.Policy.mixed(b1, b2, bm, 2)
+    assert pol.has_int4
+    rows, nnz = L.tile_lists_size(s, pol, L.LISTS_PREFILL)
+    rp, en = oracle.lists_mixed(s.cu_host, b1, b2, bm.numpy().view(np.uint32), 2)
+    assert rows == len(rp) - 1 and nnz == len(en)
+    rows, nnz = L.tile_lists_size(s, pol, L.LISTS_DECODE_CACHE)
+    rp, en = oracle.lists_decode(s.cu_host, 4, 2, b1, b2)
+    assert rows == len(rp) - 1 and nnz == len(en)
+    with pytest.raises(L.TraError):                      # boundary half: b2 < b1
+        L.tile_lists_size(s, L.Policy.mixed([2, 1, 1, 1], [1, 1, 1, 1], bm, 2))
+    with pytest.raises(L.TraError):                      # bitmask half: G < 1
+        L.tile_lists_size(s, L.Policy.mixed(b1, b2, bm, 0))
+    bad = L.Policy.mixed(b1, b2, bm, 1)
+    bad._c.W = 1                                         # 41 tiles / G=1 > 32 bits
+    with pytest.raises(L.TraError) as e:
+        L.tile_lists_size(s, bad)
+    assert "words" in str(e.value)
+    odd = L.Policy.mixed(b1, b2, bm, 2)
+    odd._c.mode = 7
+    with pytest.raises(L.TraError) as e:
+        L.tile_lists_size(s, odd)
+    assert "unknown policy mode" in str(e.value)

@@ -68,6 +68,9 @@ class Case:
         self.shape = tra.Shape(w.cu_seqlens, w.Hq, w.Hkv, w.d)
         if w.mode == "boundary":
             self.policy = tra.Policy.boundary(w.b1, w.b2)
+        elif w.mode == "mixed":
+            self.bitmask = torch.from_numpy(w.bitmask.view(np.int32)).cuda()
+            self.policy = tra.Policy.mixed(w.b1, w.b2, self.bitmask, w.G)
         else:
             self.bitmask = torch.from_numpy(w.bitmask.view(np.int32)).cuda()
             self.policy = tra.Policy.from_bitmask(self.bitmask, w.G)
@@ -75,6 +78,9 @@ class Case:
     def oracle_lists(self):
         if self.w.mode == "boundary":
             return oracle.lists_boundary(self.w.cu_seqlens, self.w.b1, self.w.b2)
+        if self.w.mode == "mixed":
+            return oracle.lists_mixed(self.w.cu_seqlens, self.w.b1, self.w.b2, self.w.bitmask,
+                                      self.w.G)
         return oracle.lists_bitmask(self.w.cu_seqlens, self.w.bitmask, self.w.G)
 
 
@@ -89,6 +95,10 @@ SMALL = [
     wl.custom("m_d64_g3", [1500], 2, 2, 64, 36, "bitmask", G=3, p_bf16=0.5),
     wl.custom("m_d128_allbf16", [513], 4, 4, 128, 37, "bitmask", G=2, p_bf16=1.0),
     wl.custom("m_d128_all8", [777], 4, 2, 128, 38, "bitmask", G=4, p_bf16=0.0),
+    # four-way: boundaries (skip / INT4 / INT8) with a bitmask promoting kept tiles to BF16
+    wl.custom("x_d128_gqa4", [1500, 300, 64], 8, 2, 128, 60, "mixed",
+              b1=[1, 2, 3, 1, 4, 1, 2, 8], b2=[3, 5, 9, 30, 4, 1, 20, 8], G=2, p_bf16=0.3),
+    wl.custom("x_d64_ragged", [900, 65, 1], 4, 4, 64, 61, "mixed", G=3, p_bf16=0.5),
 ]
 
 
@@ -151,7 +161,7 @@ def test_lists_bit_exact(w):
     rp, en = c.oracle_lists()
     assert np.array_equal(plan.row_ptr.cpu().numpy(), rp)
     assert np.array_equal(to_np_u32(plan.entries)[:plan.nnz], en)
-    if w.mode == "boundary":
+    if w.mode in ("boundary", "mixed"):  # decode caches follow the boundaries
         dp = api.DecodePlan(c.shape, c.policy, None, 4)
         dp.build()
         torch.cuda.synchronize()
@@ -248,6 +258,7 @@ FULL = {
     "llama8b_8k": (wl.llama8b_8k, [0, 13, 31], lambda nt: [0, 1, 7, 64, nt - 2, nt - 1]),
     "bitmask_32k": (wl.bitmask_32k, [0, 17, 31], lambda nt: [0, 3, 255, nt - 1]),
     "varlen": (wl.varlen_8, [0, 27], lambda nt: [0, nt // 2, nt - 1]),
+    "mixed_8k": (wl.mixed_8k, [0, 21, 31], lambda nt: [0, 2, 64, nt - 1]),
 }
 
 

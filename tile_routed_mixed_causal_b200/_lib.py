@@ -19,7 +19,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "tra.h")
 
 TILE = 64
 PREC_INT4, PREC_INT8, PREC_BF16 = 1, 2, 3
-POLICY_BOUNDARY, POLICY_BITMASK = 0, 1
+POLICY_BOUNDARY, POLICY_BITMASK, POLICY_MIXED = 0, 1, 2
 LISTS_PREFILL, LISTS_DECODE_CACHE = 0, 1
 FMT_Q8, FMT_Q4, FMT_K8, FMT_K4, FMT_V8, FMT_V4 = 0x1, 0x2, 0x4, 0x8, 0x10, 0x20
 DEV_TIMEOUT, DEV_TAIL_FULL, DEV_BAD_LIST = 0x1, 0x2, 0x4
@@ -145,7 +145,8 @@ class Shape:
 
 
 class Policy:
-    """Boundary policy (host b1/b2 per head) or bitmask policy (device words, G)."""
+    """Boundary policy (host b1/b2 per head), bitmask policy (device words, G), or
+    both at once (mixed: boundaries decide skip / INT4 / INT8, a set bit BF16)."""
 
     def __init__(self, mode, b1=None, b2=None, bitmask=None, G=1):
         self.mode = mode
@@ -168,13 +169,17 @@ class Policy:
     def from_bitmask(cls, bitmask: torch.Tensor, G: int):
         return cls(POLICY_BITMASK, bitmask=bitmask, G=G)
 
+    @classmethod
+    def mixed(cls, b1, b2, bitmask: torch.Tensor, G: int):
+        return cls(POLICY_MIXED, b1=b1, b2=b2, bitmask=bitmask, G=G)
+
     @property
     def c(self):
         return ctypes.byref(self._c)
 
     @property
     def has_int4(self) -> bool:
-        return self.mode == POLICY_BOUNDARY and bool(np.any(self.b2 > self.b1))
+        return self.mode != POLICY_BITMASK and bool(np.any(self.b2 > self.b1))
 
 
 class QTiles:

@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(256) lists_kernel(const ListParams p) {
       long long tot = 0;
       for (long long i = lane; i < (long long)p.Hq * p.B; i += 32) {
         const int h = (int)(i / p.B), b = (int)(i % p.B);
-        const long long c = p.mode == TRA_POLICY_BOUNDARY ? p.b2[h] : cap_none;
+        const long long c = p.mode != TRA_POLICY_BITMASK ? p.b2[h] : cap_none;
         tot += tri_capped(seq_tiles(p.cu, b), c);
       }
       tot = warp_sum(tot);
@@ -63,12 +63,12 @@ __global__ void __launch_bounds__(256) lists_kernel(const ListParams p) {
       toff += nt;
     }
     const int qt = gt - toff;
-    const long long c = p.mode == TRA_POLICY_BOUNDARY ? p.b2[h] : cap_none;
+    const long long c = p.mode != TRA_POLICY_BITMASK ? p.b2[h] : cap_none;
     // offset = all earlier heads + earlier sequences of this head + earlier rows
     long long off = 0;
     for (long long i = lane; i < (long long)h * p.B + b; i += 32) {
       const int hh = (int)(i / p.B), bb = (int)(i % p.B);
-      const long long cc = p.mode == TRA_POLICY_BOUNDARY ? p.b2[hh] : cap_none;
+      const long long cc = p.mode != TRA_POLICY_BITMASK ? p.b2[hh] : cap_none;
       off += tri_capped(seq_tiles(p.cu, bb), cc);
     }
     off = warp_sum(off) + tri_capped(qt, c);
@@ -81,6 +81,40 @@ __global__ void __launch_bounds__(256) lists_kernel(const ListParams p) {
       for (int i = lane; i < n; i += 32) {
         const uint32_t prec = i < n4 ? TRA_PREC_INT4 : TRA_PREC_INT8;
         e[i] = (prec << 28) | (uint32_t)(qt - n + 1 + i);
+      }
+    } else if (p.mode == TRA_POLICY_MIXED) {
+      // kept tiles qt-n+1 .. qt as under boundaries; a set bit promotes one to BF16.
+      // Pass 1 counts the INT4 and INT8 tiles, pass 2 writes each group ascending.
+      const int n = min(qt + 1, p.b2[h]);
+      const int k0 = qt - n + 1;
+      const uint32_t* words = p.bitmask + ((long long)h * p.ntiles + gt) * p.W;
+      auto class_of = [&](int kt) -> int {  // 1 INT4, 2 INT8, 3 BF16
+        const int g = kt / p.G;
+        if ((__ldg(words + (g >> 5)) >> (g & 31)) & 1u) return TRA_PREC_BF16;
+        return qt - kt < p.b1[h] ? TRA_PREC_INT8 : TRA_PREC_INT4;
+      };
+      int n4 = 0, n8 = 0;
+      for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        const int cl = i < n ? class_of(k0 + i) : 0;
+        n4 += __popc(__ballot_sync(0xffffffffu, cl == TRA_PREC_INT4));
+        n8 += __popc(__ballot_sync(0xffffffffu, cl == TRA_PREC_INT8));
+      }
+      int c4 = 0, c8 = 0, c16 = 0;
+      for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        const int cl = i < n ? class_of(k0 + i) : 0;
+        const uint32_t m4 = __ballot_sync(0xffffffffu, cl == TRA_PREC_INT4);
+        const uint32_t m8 = __ballot_sync(0xffffffffu, cl == TRA_PREC_INT8);
+        const uint32_t m16 = __ballot_sync(0xffffffffu, cl == TRA_PREC_BF16);
+        const uint32_t below = (1u << lane) - 1u;
+        const uint32_t v = ((uint32_t)cl << 28) | (uint32_t)(k0 + i);
+        if (cl == TRA_PREC_INT4) e[c4 + __popc(m4 & below)] = v;
+        if (cl == TRA_PREC_INT8) e[n4 + c8 + __popc(m8 & below)] = v;
+        if (cl == TRA_PREC_BF16) e[n4 + n8 + c16 + __popc(m16 & below)] = v;
+        c4 += __popc(m4);
+        c8 += __popc(m8);
+        c16 += __popc(m16);
       }
     } else {
       const uint32_t* words = p.bitmask + ((long long)h * p.ntiles + gt) * p.W;
@@ -124,7 +158,7 @@ __global__ void __launch_bounds__(256) lists_kernel(const ListParams p) {
   const int grp = p.Hq / p.Hkv;
   auto row_count = [&](int bb, int kk) -> long long {
     const int nt = seq_tiles(p.cu, bb);
-    if (p.mode != TRA_POLICY_BOUNDARY) return nt;
+    if (p.mode == TRA_POLICY_BITMASK) return nt;
     return min(nt, group_max_b(p.b2, kk, grp));
   };
   long long off = 0;
@@ -135,7 +169,7 @@ __global__ void __launch_bounds__(256) lists_kernel(const ListParams p) {
   const int b = (int)(row / p.Hkv), kvh = (int)(row % p.Hkv);
   const int nt = seq_tiles(p.cu, b);
   uint32_t* e = p.entries + off;
-  if (p.mode == TRA_POLICY_BOUNDARY) {
+  if (p.mode != TRA_POLICY_BITMASK) {  // boundaries (mixed policies too)
     const int n = min(nt, group_max_b(p.b2, kvh, grp));
     const int n8 = min(nt, group_max_b(p.b1, kvh, grp));
     for (int i = lane; i < n; i += 32) {

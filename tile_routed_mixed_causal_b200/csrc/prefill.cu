@@ -56,26 +56,34 @@ constexpr int kSmemLimit = 232448;         // max dynamic shared memory per CTA 
 
 template <int D, int MODE>
 struct Cfg {
+  static constexpr bool kHasBf16 = MODE != TRA_POLICY_BOUNDARY;  // bf16 Q and K operands
+  static constexpr bool kHasInt4 = MODE != TRA_POLICY_BITMASK;   // expanded INT4 operands
+  // work units per CTA: two, or one under a mixed policy, whose operand buffers
+  // (int8, expanded INT4 and bf16 Q, bf16-sized K slots, the K4 ring) do not fit twice
+  static constexpr int kCtaUnits = MODE == TRA_POLICY_MIXED ? 1 : 2;
   static constexpr int kQ8Bytes = 128 * D;                                    // int8 Q codes
-  static constexpr int kQxBytes = MODE == TRA_POLICY_BITMASK ? 128 * D * 2 : 128 * D;
-  static constexpr int kQUnitBytes = kQ8Bytes + kQxBytes;
-  // K slot: BF16 or INT8 codes under a bitmask policy, INT8 codes only under boundaries
-  static constexpr int kKBytes = MODE == TRA_POLICY_BITMASK ? 64 * D * 2 : 64 * D;
+  static constexpr int kQ4Bytes = kHasInt4 ? 128 * D : 0;                     // expanded INT4 Q
+  static constexpr int kQbBytes = kHasBf16 ? 128 * D * 2 : 0;                 // bf16 Q
+  static constexpr int kQUnitBytes = kQ8Bytes + kQ4Bytes + kQbBytes;
+  // K slot: BF16 or INT8 codes when bf16 tiles occur, INT8 codes only under boundaries
+  static constexpr int kKBytes = kHasBf16 ? 64 * D * 2 : 64 * D;
   static constexpr int kK4Bytes = 64 * D;                                     // expanded INT4 K
   static constexpr int kVBytes = 64 * D * 2;
   // ring depths per unit (every ring belongs to one unit)
   static constexpr int kStagesK = 2;
-  static constexpr int kStagesK4 = MODE == TRA_POLICY_BOUNDARY ? 2 : 0;
-  static constexpr int kFixed = kUnits * (kQUnitBytes + kStagesK * kKBytes + kStagesK4 * kK4Bytes) +
-                                2048;                                         // + barriers, slack
-  static constexpr int kStagesVFit = (kSmemLimit - kFixed) / (kUnits * kVBytes);
+  static constexpr int kStagesK4 = kHasInt4 ? 2 : 0;
+  static constexpr int kFixed =
+      kCtaUnits * (kQUnitBytes + kStagesK * kKBytes + kStagesK4 * kK4Bytes) + 2048;  // + barriers
+  static constexpr int kStagesVFit = (kSmemLimit - kFixed) / (kCtaUnits * kVBytes);
   static constexpr int kStagesV = kStagesVFit > 4 ? 4 : kStagesVFit;
   static_assert(kStagesV >= 2, "shared memory too small for the V rings");
   static constexpr int kOffQ = 0;                                             // unit u at u * kQUnitBytes
-  static constexpr int kOffK = kUnits * kQUnitBytes;                          // [unit][slot]
-  static constexpr int kOffK4 = kOffK + kUnits * kStagesK * kKBytes;
-  static constexpr int kOffV = kOffK4 + kUnits * kStagesK4 * kK4Bytes;
-  static constexpr int kOffBar = kOffV + kUnits * kStagesV * kVBytes;
+  static constexpr int kOffK = kCtaUnits * kQUnitBytes;                       // [unit][slot]
+  static constexpr int kOffK4 = kOffK + kCtaUnits * kStagesK * kKBytes;
+  static constexpr int kOffV = kOffK4 + kCtaUnits * kStagesK4 * kK4Bytes;
+  static constexpr int kOffBar = kOffV + kCtaUnits * kStagesV * kVBytes;
+  // (barriers exist for two units in every mode; a CTA's missing second unit has
+  // no entries and touches none of the buffers above)
   static constexpr int kUnitBars = 2 * kStagesK + 2 * kStagesK4 + 2 * kStagesV + 6;
   static constexpr int kNumBars = 2 + kUnits * kUnitBars + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -188,18 +196,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NS4 = NS4R > 0 ? NS4R : 1;  // (no K4 ring without INT4)
   extern __shared__ uint8_t smem_raw[];
 
-  // ---- the CTA's two work units
-  const Unit un0 = make_unit(p, (long long)blockIdx.x * kUnits);
-  const Unit un1 = make_unit(p, (long long)blockIdx.x * kUnits + 1);
+  // ---- the CTA's work units (the second is absent under a mixed policy)
+  auto unit_of = [&](int u) {
+    const long long none = (long long)p.jmax * p.B * p.Hq;  // an id past the last unit
+    return make_unit(p, u < C::kCtaUnits ? (long long)blockIdx.x * C::kCtaUnits + u : none);
+  };
+  const Unit un0 = unit_of(0);
+  const Unit un1 = unit_of(1);
   if (!un0.valid && !un1.valid) return;  // uniform exit, before any barrier or TMEM use
-  // INT4 operands exist only for boundary policies with an INT4 region; a list
-  // entry asking for INT4 without them is reported, never read
-  const bool int4 = MODE == TRA_POLICY_BOUNDARY && p.has_int4;
+  // INT4 operands exist only for policies with an INT4 region; a list entry asking
+  // for INT4 without them is reported, never read
+  const bool int4 = C::kHasInt4 && p.has_int4;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (base - smem_u32(smem_raw));
   auto sQ8 = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes; };
-  auto sQx = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes; };
+  auto sQ4 = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes; };
+  auto sQb = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes + C::kQ4Bytes; };
   auto sK = [&](int u, int s) { return base + C::kOffK + (u * NSK + s) * C::kKBytes; };
   auto sK4 = [&](int u, int s) { return base + C::kOffK4 + (u * NS4 + s) * C::kK4Bytes; };
   auto sV = [&](int u, int s) { return base + C::kOffV + (u * NSV + s) * C::kVBytes; };
@@ -272,13 +285,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const int u = warp == 0 ? 0 : 1;
       const Unit x = u ? un1 : un0;
-      constexpr uint32_t kQBytes = C::kQ8Bytes + (MODE == TRA_POLICY_BITMASK ? 128 * D * 2 : 0);
+      constexpr uint32_t kQBytes = C::kQ8Bytes + C::kQbBytes;
       mbar_arrive_expect_tx(bar_q, x.valid ? kQBytes : 0u);
       if (x.valid) {
         tma_load_2d(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
-        if (MODE == TRA_POLICY_BITMASK) {
+        if (C::kHasBf16) {
           for (int sl = 0; sl < C::kSlabs; ++sl)
-            tma_load_3d(sQx(u) + sl * 128 * 128, &m.qb, bar_q, sl * 64, x.h,
+            tma_load_3d(sQb(u) + sl * 128 * 128, &m.qb, bar_q, sl * 64, x.h,
                         x.seq0 + x.qt0 * kTile);
         }
       }
@@ -382,12 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const int sl = kk >> 2, off = (kk & 3) * 32;
-              const uint64_t a = smem_desc(sQx(mu) + sl * 128 * 128 + off, 16, 1024, kSwz128);
+              const uint64_t a = smem_desc(sQb(mu) + sl * 128 * 128 + off, 16, 1024, kSwz128);
               const uint64_t bd = smem_desc(kb + sl * 64 * 128 + off, 16, 1024, kSwz128);
               mma_bf16(tSb, a, bd, kIdQK16, kk > 0 ? 1u : 0u);
             }
           } else {
-            const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(mu) : sQx(mu);
+            const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(mu) : sQ4(mu);
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk) {
               const uint64_t a = smem_desc(qa + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
@@ -476,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4 && warp < 12) {
     // ================================================================ softmax / epilogue
     const int u = (warp - 4) >> 2;               // unit of this warpgroup
-    const Unit x = make_unit(p, (long long)blockIdx.x * kUnits + u);
+    const Unit x = unit_of(u);
     const int r = (threadIdx.x - 128) & 127;     // query row of the unit = TMEM lane
     const int q4 = warp & 3;                     // TMEM lane quarter of this warp
     const int half = r >> 6, rr = r & 63;
@@ -703,7 +716,7 @@ template <int D, int MODE>
 cudaError_t launch_one(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s) {
   using C = Cfg<D, MODE>;
   const long long units = (long long)p.jmax * p.B * p.Hq;
-  const long long ctas = (units + kUnits - 1) / kUnits;
+  const long long ctas = (units + C::kCtaUnits - 1) / C::kCtaUnits;
   if (ctas == 0) return cudaSuccess;
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, MODE>,
@@ -715,12 +728,15 @@ cudaError_t launch_one(const PrefillParams& p, const PrefillMaps& m, cudaStream_
 
 }  // namespace
 
+template <int D>
+cudaError_t launch_d(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s) {
+  if (p.mode == TRA_POLICY_BITMASK) return launch_one<D, TRA_POLICY_BITMASK>(p, m, s);
+  if (p.mode == TRA_POLICY_MIXED) return launch_one<D, TRA_POLICY_MIXED>(p, m, s);
+  return launch_one<D, TRA_POLICY_BOUNDARY>(p, m, s);
+}
+
 cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s) {
-  if (p.d == 128)
-    return p.mode == TRA_POLICY_BITMASK ? launch_one<128, TRA_POLICY_BITMASK>(p, m, s)
-                                        : launch_one<128, TRA_POLICY_BOUNDARY>(p, m, s);
-  return p.mode == TRA_POLICY_BITMASK ? launch_one<64, TRA_POLICY_BITMASK>(p, m, s)
-                                      : launch_one<64, TRA_POLICY_BOUNDARY>(p, m, s);
+  return p.d == 128 ? launch_d<128>(p, m, s) : launch_d<64>(p, m, s);
 }
 
 }  // namespace tra

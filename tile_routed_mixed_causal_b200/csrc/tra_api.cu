@@ -69,29 +69,32 @@ int64_t tri_capped(int64_t n, int64_t c) {
   return c * (c + 1) / 2 + (n - c) * c;
 }
 
+bool uses_boundaries(const tra_policy* p) { return p->mode != TRA_POLICY_BITMASK; }
+bool uses_bitmask(const tra_policy* p) { return p->mode != TRA_POLICY_BOUNDARY; }
+
 tra_status check_policy(const tra_shape* s, const tra_policy* p, int64_t nt_max) {
   if (!p) return fail(TRA_ERR_INVALID, "policy is NULL");
-  if (p->mode == TRA_POLICY_BOUNDARY) {
+  if (p->mode != TRA_POLICY_BOUNDARY && p->mode != TRA_POLICY_BITMASK && p->mode != TRA_POLICY_MIXED)
+    return fail(TRA_ERR_INVALID, "unknown policy mode %d", p->mode);
+  if (uses_boundaries(p)) {
     if (!p->b1 || !p->b2) return fail(TRA_ERR_INVALID, "boundary policy needs host b1 and b2");
     for (int h = 0; h < s->Hq; ++h) {
       if (p->b1[h] < 1) return fail(TRA_ERR_INVALID, "b1[%d] = %d < 1", h, p->b1[h]);
       if (p->b2[h] < p->b1[h]) return fail(TRA_ERR_INVALID, "b2[%d] = %d < b1 = %d", h, p->b2[h], p->b1[h]);
     }
-    return TRA_OK;
   }
-  if (p->mode == TRA_POLICY_BITMASK) {
+  if (uses_bitmask(p)) {
     if (p->G < 1) return fail(TRA_ERR_INVALID, "G must be >= 1 (got %d)", p->G);
     if (p->W < 1) return fail(TRA_ERR_INVALID, "W must be >= 1");
     const int64_t groups = (nt_max + p->G - 1) / p->G;
     if ((int64_t)p->W * 32 < groups)
       return fail(TRA_ERR_INVALID, "W = %d words cannot hold %lld groups", p->W, (long long)groups);
-    return TRA_OK;
   }
-  return fail(TRA_ERR_INVALID, "unknown policy mode %d", p->mode);
+  return TRA_OK;
 }
 
 bool policy_has_int4(const tra_shape* s, const tra_policy* p) {
-  if (p->mode != TRA_POLICY_BOUNDARY) return false;
+  if (!uses_boundaries(p)) return false;
   for (int h = 0; h < s->Hq; ++h)
     if (p->b2[h] > p->b1[h]) return true;
   return false;
@@ -244,7 +247,7 @@ tra_status tra_tile_lists_size(const tra_shape* shape, const tra_policy* policy,
     for (int h = 0; h < shape->Hq; ++h)
       for (int b = 0; b < shape->B; ++b) {
         const int64_t n = ceil_tiles(cu[b + 1] - cu[b]);
-        total += tri_capped(n, policy->mode == TRA_POLICY_BOUNDARY ? policy->b2[h] : (1ll << 40));
+        total += tri_capped(n, uses_boundaries(policy) ? policy->b2[h] : (1ll << 40));
       }
   } else if (list_kind == TRA_LISTS_DECODE_CACHE) {
     *rows = (int64_t)shape->B * shape->Hkv;
@@ -252,7 +255,7 @@ tra_status tra_tile_lists_size(const tra_shape* shape, const tra_policy* policy,
     for (int b = 0; b < shape->B; ++b) {
       const int64_t n = ceil_tiles(cu[b + 1] - cu[b]);
       for (int kvh = 0; kvh < shape->Hkv; ++kvh) {
-        if (policy->mode != TRA_POLICY_BOUNDARY) {
+        if (!uses_boundaries(policy)) {
           total += n;
           continue;
         }
@@ -280,7 +283,7 @@ tra_status build_tile_lists(const tra_shape* shape, const tra_policy* policy, in
     return fail(TRA_ERR_INVALID, "row_ptr/entries not 16-byte aligned");
   if (row_ptr_len < rows + 1) return fail(TRA_ERR_BUFFER, "row_ptr needs %lld entries", (long long)(rows + 1));
   if (entries_cap < nnz) return fail(TRA_ERR_BUFFER, "entries needs %lld entries", (long long)nnz);
-  if (policy->mode == TRA_POLICY_BITMASK && list_kind == TRA_LISTS_PREFILL) {
+  if (uses_bitmask(policy) && list_kind == TRA_LISTS_PREFILL) {
     if (!policy->bitmask_dev || (reinterpret_cast<uintptr_t>(policy->bitmask_dev) & 3u))
       return fail(TRA_ERR_INVALID, "bitmask_dev NULL or misaligned");
   }
@@ -300,7 +303,7 @@ tra_status build_tile_lists(const tra_shape* shape, const tra_policy* policy, in
   p.row_ptr = row_ptr;
   p.entries = entries;
   p.rows = rows;
-  if (policy->mode == TRA_POLICY_BOUNDARY)
+  if (uses_boundaries(policy))
     for (int h = 0; h < shape->Hq; ++h) {
       p.b1[h] = policy->b1[h];
       p.b2[h] = policy->b2[h];

@@ -40,7 +40,7 @@ class Workload:
     lengths: list
     seed: int
     outliers: bool
-    mode: str                      # "boundary" or "bitmask"
+    mode: str                      # "boundary", "bitmask" or "mixed" (both)
     b1: Optional[np.ndarray] = None
     b2: Optional[np.ndarray] = None
     bitmask: Optional[np.ndarray] = None   # uint32 [Hq, ntiles, W]
@@ -140,6 +140,19 @@ def llama8b_8k(seed: int = 1) -> Workload:
     return w
 
 
+def mixed_8k(seed: int = 5) -> Workload:
+    """Both policies at once on the Llama-3-8B shape (32/8 heads, d 128, 8192 tokens):
+    per-head boundaries as in llama8b_8k, then a G = 4 bitmask with 25% of bits set
+    promoting kept tiles to BF16."""
+    w = Workload("mixed_prefill_t8192_g4", 1, 32, 8, 128, [8192], seed, True, "mixed", G=4)
+    rng = np.random.default_rng(seed + 1000)
+    w.b1 = rng.integers(1, 9, size=w.Hq).astype(np.int32)
+    w.b2 = np.array([rng.integers(b, 65) for b in w.b1], np.int32)
+    W = _bitmask_words(w.ntiles, w.G)
+    w.bitmask = _draw_bitmask(rng, w.Hq, w.ntiles, W, 0.25)
+    return w
+
+
 def bitmask_32k(seed: int = 2, T: int = 32768) -> Workload:
     """Bitmask mode: 32/8 heads, d 128, 32K tokens, G = 4, 25% of bits BF16."""
     w = Workload(f"bitmask_prefill_t{T}_g4", 1, 32, 8, 128, [T], seed, True, "bitmask", G=4)
@@ -199,18 +212,19 @@ def decode_32k(seed: int = 4, B: int = 16, T: int = 32768, steps: int = 64,
 
 def custom(name, lengths, Hq, Hkv, d, seed, mode, *, b1=None, b2=None, G=1,
            p_bf16=0.25, outliers=True, decode_steps=0, tail_cap=0) -> Workload:
-    """Small ad-hoc workload for tests (ragged lengths, GQA, either policy)."""
+    """Small ad-hoc workload for tests (ragged lengths, GQA, any policy; a mixed one
+    draws its boundaries first, then its bitmask)."""
     w = Workload(name, len(lengths), Hq, Hkv, d, list(lengths), seed, outliers, mode,
                  decode_steps=decode_steps, tail_cap=tail_cap, G=G)
     rng = np.random.default_rng(seed + 1000)
-    if mode == "boundary":
+    if mode in ("boundary", "mixed"):
         if b1 is None:
             w.b1 = rng.integers(1, 4, size=Hq).astype(np.int32)
             w.b2 = np.array([rng.integers(b, b + 5) for b in w.b1], np.int32)
         else:
             w.b1 = np.asarray(b1, np.int32)
             w.b2 = np.asarray(b2, np.int32)
-    else:
+    if mode in ("bitmask", "mixed"):
         W = _bitmask_words(max(w.tiles_per_seq), G)
         w.bitmask = _draw_bitmask(rng, Hq, w.ntiles, W, p_bf16)
     return w
