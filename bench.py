@@ -68,7 +68,7 @@ def parse():
 # source that has changed since reports null.  Captures: profiles/prefill_kernel_bitmask_32k.md
 # and profiles/decode_split_kernel_b16_32k.md.
 PROFILED_TRAFFIC = {
-    "prefill.cu": ("bad45a2b16f93e23", 3_372_927_232),
+    "prefill.cu": ("e07280ea9221a6e1", 3_425_659_392),
     "decode.cu": ("a0ae0cc01c87ca66", 663_556_096),
 }
 
