@@ -54,8 +54,9 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
-                    help="run one part only (used for profiler captures); prints a reduced line")
+    ap.add_argument("--only", choices=["prefill", "decode", "allocate"], default=None,
+                    help="run one part only (used for profiler captures); prints a reduced line. "
+                         "allocate: measured complete-tile cost model + boundary allocator demo")
     ap.add_argument("--workload", choices=["bitmask_32k", "llama8b_8k", "varlen_8", "mixed_8k"],
                     default="bitmask_32k",
                     help="prefill workload for --only prefill (the full bench line always uses "
@@ -243,6 +244,94 @@ def run_prefill_e2e(S, steps, stream):
         end.record(stream)
         stream.synchronize()
     return start.elapsed_time(end) / steps, h2d, d2h
+
+
+# ----------------------------------------------------------------------------- allocator
+def allocate_bench(device, stream, budget_frac=0.5, units=4096, seed=7):
+    """Complete-tile cost model and model-wide boundary allocation on the Llama-3-8B
+    prefill shape (TriAttention abstract: candidate pairs weighed by calibration errors
+    and complete-tile execution costs, an allocator choosing each head's pair under a
+    shared budget).  Per-tile INT8 and INT4 times and a fixed term are fitted from three
+    uniform policies; the errors are a seeded synthetic table (no model here); the budget
+    is budget_frac of the all-INT8 cost.  The allocated policy's predicted kernel time is
+    then compared with its measured time."""
+    import math
+    import tile_routed_mixed_causal_b200 as tra
+    from tile_routed_mixed_causal_b200 import api
+    from tile_routed_mixed_causal_b200 import workloads as wl
+
+    w = wl.llama8b_8k()
+    t = wl.make_inputs(w, device)
+    q, k, v = t["q"], t["k"], t["v"]
+    shape = tra.Shape(w.cu_seqlens, w.Hq, w.Hkv, w.d, device=device)
+    nt = w.tiles_per_seq[0]
+    out = torch.empty_like(q)
+
+    def kernel_ms(b1, b2, reps=20):
+        plan = api.PrefillPlan(shape, tra.Policy.boundary(b1, b2), device=device)
+        with torch.cuda.stream(stream):
+            plan.run(q, k, v, out, stream=stream)
+            for _ in range(3):
+                plan.attend(q, k, v, out, stream=stream)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                plan.attend(q, k, v, out, stream=stream)
+            b.record(stream)
+            stream.synchronize()
+        assert int(plan.status.item()) == 0
+        return a.elapsed_time(b) / reps
+
+    def counts(b1, b2):
+        n8 = n4 = 0
+        for h in range(w.Hq):
+            c8, c4 = tra.boundary_tile_counts(shape, b1[h], b2[h])
+            n8, n4 = n8 + c8, n4 + c4
+        return n8, n4
+
+    H = w.Hq
+    full = [nt] * H
+    half = [nt // 2] * H
+    pol = {"int8_all": (full, full), "int8_half": (half, half), "int4_all": ([1] * H, full)}
+    meas = {name: kernel_ms(*bb) for name, bb in pol.items()}
+    cnt = {name: counts(*bb) for name, bb in pol.items()}
+    w8 = (meas["int8_all"] - meas["int8_half"]) / (cnt["int8_all"][0] - cnt["int8_half"][0])
+    t0 = meas["int8_all"] - cnt["int8_all"][0] * w8
+    w4 = (meas["int4_all"] - t0 - cnt["int4_all"][0] * w8) / cnt["int4_all"][1]
+
+    # candidates: b1 in powers of two, b2 in b1 x powers of two, up to nt
+    cands = [(b1, b2) for b1 in [1 << i for i in range(8) if (1 << i) <= nt]
+             for b2 in [b1 << j for j in range(8) if (b1 << j) <= nt]]
+    C = len(cands)
+    cost_ms = np.zeros((H, C))
+    for c, (b1, b2) in enumerate(cands):
+        n8, n4 = tra.boundary_tile_counts(shape, b1, b2)
+        cost_ms[:, c] = n8 * w8 + n4 * w4
+    quantum = cnt["int8_all"][0] * w8 / units          # all-INT8 cost = `units` units
+    cost = np.ceil(cost_ms / quantum).astype(np.int64)
+    err = wl.synthetic_boundary_errors(H, cands, nt, seed)
+    budget = int(budget_frac * units)
+    t_a = time.perf_counter()
+    choice, total_err, total_units = tra.allocate_boundaries(err, cost, budget)
+    alloc_ms = (time.perf_counter() - t_a) * 1e3
+    # best single pair for every head within the same budget
+    uni = [c for c in range(C) if cost[:, c].sum() <= budget]
+    uni_c = min(uni, key=lambda c: err[:, c].sum())
+    b1 = [cands[c][0] for c in choice]
+    b2 = [cands[c][1] for c in choice]
+    predicted = t0 + float(sum(cost_ms[h, choice[h]] for h in range(H)))
+    measured = kernel_ms(b1, b2)
+    return {
+        "shape": w.name, "tile_ms_model": {"int8_per_tile_ns": w8 * 1e6, "int4_per_tile_ns": w4 * 1e6,
+                                           "fixed_ms": t0},
+        "fit_points_ms": meas, "candidates_per_head": C, "budget_frac_of_all_int8": budget_frac,
+        "budget_units": budget, "allocator_ms": alloc_ms, "total_err": total_err,
+        "uniform_best_err": float(err[:, uni_c].sum()), "uniform_best_pair": list(cands[uni_c]),
+        "used_units": int(total_units), "predicted_kernel_ms": predicted,
+        "measured_kernel_ms": measured, "predicted_over_measured": predicted / measured,
+        "b1": b1, "b2": b2,
+    }
 
 
 # ----------------------------------------------------------------------------- decode
@@ -439,6 +528,10 @@ def main():
         if rank == 0:
             print(json.dumps({"only": "decode", **decode_bench(device, args.decode_passes, stream,
                                                               hbm_gbs)}), flush=True)
+        return
+    if args.only == "allocate":
+        if rank == 0:
+            print(json.dumps({"only": "allocate", **allocate_bench(device, stream)}), flush=True)
         return
     if args.only == "prefill":
         S = prefill_setup(device, args.workload)

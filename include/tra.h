@@ -304,6 +304,31 @@ TRA_API tra_status routed_attention_decode_noalloc(
     const uint32_t* entries, uint16_t* k_tail, uint16_t* v_tail, int32_t* tail_len_dev,
     int32_t tail_cap, float softmax_scale, uint16_t* out, int32_t* status_dev, void* stream);
 
+/* Complete-tile counts of one head's boundary pair over a batch (TriAttention
+ * abstract: candidate boundary pairs are weighed by complete-tile execution costs):
+ * n8 = sum over every sequence's q-tiles qt of min(qt + 1, b1), n4 = the sum of
+ * min(qt + 1, b2) minus n8; the cost of the pair is n8 and n4 times the per-tile
+ * times of the two precisions.  Host only.  TRA_ERR_INVALID for an invalid shape,
+ * NULL outputs, or not 1 <= b1 <= b2. */
+TRA_API tra_status tra_boundary_tile_counts(const tra_shape* shape, int32_t b1, int32_t b2,
+                                            int64_t* n8, int64_t* n4);
+
+/* Model-wide boundary allocation (TriAttention abstract: an allocator selects each
+ * head's boundaries to minimise calibration error under a shared computation budget).
+ * Host only.  err [n_heads][n_cand] (finite) and cost [n_heads][n_cand] (>= 0, integer
+ * units chosen by the caller, e.g. tile counts times per-tile times, rounded up) describe
+ * each head's candidate pairs; choice [n_heads] receives, per head, the index of the
+ * candidate that minimises the total error with total cost <= budget.  Exact: candidates
+ * beaten on both cost and error are dropped, then a dynamic programme runs over the
+ * integer budget (O(n_heads x n_cand x budget) time, one byte per head and budget unit of
+ * host memory); ties between equal totals are broken deterministically.
+ * total_err / total_cost (nullable) receive the sums.  TRA_ERR_INVALID for bad arguments
+ * or when no choice fits the budget; TRA_ERR_UNSUPPORTED when n_heads x (budget + 1)
+ * exceeds 2^27 (use coarser cost units).  1 <= n_cand <= 255. */
+TRA_API tra_status tra_allocate_boundaries(int32_t n_heads, int32_t n_cand, const double* err,
+                                           const int64_t* cost, int64_t budget, int32_t* choice,
+                                           double* total_err, int64_t* total_cost);
+
 /*
  * tra_selftest_bounded_wait -- diagnostic; the pages have no counterpart.  Runs
  * one small kernel whose mbarrier wait can never complete, through the same

@@ -273,3 +273,26 @@ def decode_step(qd_bits, cu_seqlens, Hkv, cache: Quantised, row_ptr, entries,
     if rc != 0:
         raise ValueError("oracle decode failed")
     return out
+
+
+def allocate_boundaries(err, cost, budget):
+    """Model-wide boundary allocation by enumeration (TriAttention abstract: an allocator
+    selects each head's boundaries to minimise calibration error under a shared
+    computation budget).  err / cost [heads][candidates]; every combination of one
+    candidate per head is tried, the least total error with total cost <= budget wins
+    (ties: the lexicographically smallest choice).  Small cases only: the work is
+    candidates ** heads.  Returns (choice, total_err, total_cost), or None when nothing
+    fits the budget."""
+    import itertools
+    err = np.asarray(err, np.float64)
+    cost = np.asarray(cost, np.int64)
+    H, C = err.shape
+    best = None
+    for pick in itertools.product(range(C), repeat=H):
+        c = sum(int(cost[h, pick[h]]) for h in range(H))
+        if c > budget:
+            continue
+        e = sum(float(err[h, pick[h]]) for h in range(H))
+        if best is None or e < best[1]:
+            best = (list(pick), e, c)
+    return best

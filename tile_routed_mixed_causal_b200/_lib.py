@@ -77,6 +77,8 @@ def load():
         "routed_attention_decode": ([P, P, P, P, P, P, P, P, P, P, P, I32, F, P, P, SZ, P, P], I32),
         "routed_attention_decode_noalloc": ([P, P, P, P, P, P, P, P, P, P, P, I32, F, P, P, P], I32),
         "tra_selftest_bounded_wait": ([P, I64, P], I32),
+        "tra_boundary_tile_counts": ([P, I32, I32, P, P], I32),
+        "tra_allocate_boundaries": ([I32, I32, P, P, I64, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -263,3 +265,26 @@ def tra_selftest_bounded_wait(status, limit_ns: int, stream=None):
     """Diagnostic: a kernel whose mbarrier wait never completes must give up after
     limit_ns and OR DEV_TIMEOUT into the device int32 `status` (see include/tra.h)."""
     _check(load().tra_selftest_bounded_wait(_ptr(status), int(limit_ns), _stream(stream)))
+
+
+def boundary_tile_counts(shape: Shape, b1: int, b2: int):
+    """(INT8 tiles, INT4 tiles) of one head's boundary pair over the batch."""
+    n8, n4 = ctypes.c_int64(), ctypes.c_int64()
+    _check(load().tra_boundary_tile_counts(shape.c, int(b1), int(b2), ctypes.byref(n8),
+                                           ctypes.byref(n4)))
+    return n8.value, n4.value
+
+
+def allocate_boundaries(err, cost, budget: int):
+    """One candidate per head minimising the total error with total cost <= budget.
+    err float64 [heads][candidates], cost int64 (same shape).  Returns (choice int32
+    [heads], total error, total cost)."""
+    err = np.ascontiguousarray(np.asarray(err, np.float64))
+    cost = np.ascontiguousarray(np.asarray(cost, np.int64))
+    H, C = err.shape
+    assert cost.shape == (H, C)
+    choice = np.zeros(H, np.int32)
+    te, tc = ctypes.c_double(), ctypes.c_int64()
+    _check(load().tra_allocate_boundaries(H, C, _ptr(err), _ptr(cost), int(budget), _ptr(choice),
+                                          ctypes.byref(te), ctypes.byref(tc)))
+    return choice, te.value, tc.value

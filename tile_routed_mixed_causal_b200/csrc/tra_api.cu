@@ -4,6 +4,7 @@
 // or synchronises the device.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -474,6 +475,97 @@ tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* pol
   if (!good) return fail(TRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
   cudaError_t e = tra::launch_decode(p, m, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+tra_status tra_boundary_tile_counts(const tra_shape* shape, int32_t b1, int32_t b2, int64_t* n8,
+                                    int64_t* n4) {
+  tra_status st = check_shape(shape, nullptr, nullptr, nullptr);
+  if (st != TRA_OK) return st;
+  if (!n8 || !n4) return fail(TRA_ERR_INVALID, "n8/n4 outputs are NULL");
+  if (b1 < 1 || b2 < b1) return fail(TRA_ERR_INVALID, "need 1 <= b1 <= b2 (got %d, %d)", b1, b2);
+  const int32_t* cu = shape->cu_seqlens_host;
+  int64_t kept8 = 0, kept = 0;
+  for (int b = 0; b < shape->B; ++b) {
+    const int64_t n = ceil_tiles(cu[b + 1] - cu[b]);
+    kept8 += tri_capped(n, b1);
+    kept += tri_capped(n, b2);
+  }
+  *n8 = kept8;
+  *n4 = kept - kept8;
+  return ok();
+}
+
+tra_status tra_allocate_boundaries(int32_t n_heads, int32_t n_cand, const double* err,
+                                   const int64_t* cost, int64_t budget, int32_t* choice,
+                                   double* total_err, int64_t* total_cost) {
+  if (n_heads < 1 || n_cand < 1 || n_cand > 255)
+    return fail(TRA_ERR_INVALID, "need n_heads >= 1 and 1 <= n_cand <= 255 (got %d, %d)", n_heads, n_cand);
+  if (!err || !cost || !choice) return fail(TRA_ERR_INVALID, "err, cost and choice are required");
+  if (budget < 0) return fail(TRA_ERR_INVALID, "budget < 0");
+  if ((double)n_heads * ((double)budget + 1.0) > (double)(1ll << 27))
+    return fail(TRA_ERR_UNSUPPORTED, "n_heads x (budget + 1) = %.0f exceeds 2^27: use coarser cost units",
+                (double)n_heads * ((double)budget + 1.0));
+  const size_t nh = (size_t)n_heads, nc = (size_t)n_cand, nb = (size_t)budget + 1;
+  for (size_t i = 0; i < nh * nc; ++i) {
+    if (!std::isfinite(err[i])) return fail(TRA_ERR_INVALID, "err[%zu] is not finite", i);
+    if (cost[i] < 0) return fail(TRA_ERR_INVALID, "cost[%zu] < 0", i);
+  }
+  // per head, the candidates no other one beats on both cost and error, by rising cost
+  std::vector<std::vector<int>> front(nh);
+  for (size_t h = 0; h < nh; ++h) {
+    std::vector<int> idx(nc);
+    for (size_t c = 0; c < nc; ++c) idx[c] = (int)c;
+    const double* e = err + h * nc;
+    const int64_t* k = cost + h * nc;
+    std::sort(idx.begin(), idx.end(), [&](int a, int b) {
+      if (k[a] != k[b]) return k[a] < k[b];
+      if (e[a] != e[b]) return e[a] < e[b];
+      return a < b;
+    });
+    double best = INFINITY;
+    for (int c : idx)
+      if (e[c] < best && k[c] <= budget) {
+        front[h].push_back(c);
+        best = e[c];
+      }
+    if (front[h].empty())
+      return fail(TRA_ERR_INVALID, "head %zu has no candidate within the budget", h);
+  }
+  // f[B]: least total error of the heads so far with total cost <= B
+  std::vector<double> f(nb, 0.0), g(nb);
+  std::vector<uint8_t> pick(nh * nb);
+  for (size_t h = 0; h < nh; ++h) {
+    const double* e = err + h * nc;
+    const int64_t* k = cost + h * nc;
+    for (size_t B = 0; B < nb; ++B) {
+      double v = INFINITY;
+      uint8_t pk = 0;
+      for (size_t j = 0; j < front[h].size(); ++j) {
+        const int c = front[h][j];
+        if ((size_t)k[c] > B) break;  // the front rises in cost
+        const double t = e[c] + f[B - (size_t)k[c]];
+        if (t < v) {
+          v = t;
+          pk = (uint8_t)j;
+        }
+      }
+      g[B] = v;
+      pick[h * nb + B] = pk;
+    }
+    f.swap(g);
+  }
+  if (!(f[nb - 1] < INFINITY)) return fail(TRA_ERR_INVALID, "no choice of candidates fits the budget");
+  size_t B = nb - 1;
+  int64_t spent = 0;
+  for (size_t h = nh; h-- > 0;) {
+    const int c = front[h][pick[h * nb + B]];
+    choice[h] = c;
+    B -= (size_t)cost[h * nc + c];
+    spent += cost[h * nc + c];
+  }
+  if (total_err) *total_err = f[nb - 1];
+  if (total_cost) *total_cost = spent;
   return ok();
 }
 

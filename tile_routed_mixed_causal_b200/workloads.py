@@ -230,6 +230,24 @@ def custom(name, lengths, Hq, Hkv, d, seed, mode, *, b1=None, b2=None, G=1,
     return w
 
 
+def synthetic_boundary_errors(Hq: int, cands, nt: int, seed: int) -> np.ndarray:
+    """Seeded synthetic calibration errors [Hq][len(cands)] for boundary pairs (b1, b2):
+    a skip term that falls as b2 keeps more distant tiles and an INT4 term that grows with
+    the INT4 band (b2 - b1) and falls as b1 keeps more tiles in INT8, each with per-head
+    sensitivities.  Stands in for the normalised projected-output errors that an offline
+    calibration of a real model would measure."""
+    rng = np.random.default_rng(seed)
+    a = np.exp(rng.uniform(np.log(0.05), np.log(2.0), Hq))      # skip sensitivity
+    tau = rng.uniform(0.05, 0.5, Hq) * nt                        # reach of useful context
+    c = np.exp(rng.uniform(np.log(0.01), np.log(0.5), Hq))      # INT4 sensitivity
+    sig = rng.uniform(1.0, 16.0, Hq)
+    err = np.zeros((Hq, len(cands)))
+    for j, (b1, b2) in enumerate(cands):
+        err[:, j] = (a * np.exp(-b2 / tau)
+                     + c * (b2 - b1) / b2 * np.exp(-b1 / sig))
+    return err
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama8b_8k": llama8b_8k,
