@@ -326,6 +326,34 @@ def test_decode_matches_oracle(w):
     assert np.array_equal(wl.bf16_bits(dp.k_tail[:, :, :w.decode_steps]), kt[:, :, :w.decode_steps])
 
 
+def test_decode_workspace_shared_across_shapes():
+    """The decode's arrival counters sit at a fixed place of the workspace and every call
+    leaves them at zero, so one zero-filled workspace serves two shapes in turn: steps of
+    both, interleaved on it, match steps on separate workspaces bit for bit."""
+    runs = {}
+    for w in DEC[:2]:
+        own = _decode_case(w)
+        shared = _decode_case(w)
+        runs[w.name] = (w, own, shared)
+    nbytes = max(r[2][2].workspace.numel() for r in runs.values())
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    for _, (_, _, sh) in runs.items():
+        sh[2].workspace = ws
+    steps = min(w.decode_steps for w, _, _ in runs.values())
+    for step in range(steps):
+        for name, (w, own, sh) in runs.items():
+            outs = []
+            for c, cache, dp, qs, kn, vn in (own, sh):
+                out = torch.zeros((w.B, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
+                dp.step(qs[step], kn[step], vn[step], out)
+                outs.append(out)
+            torch.cuda.synchronize()
+            assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16)), (name, step)
+    for _, (_, own, sh) in runs.items():
+        assert int(own[2].status.item()) == 0 and int(sh[2].status.item()) == 0
+    assert int(ws[:4 * 16384].count_nonzero().item()) == 0   # counters back at zero
+
+
 def test_decode_tail_full_sets_status():
     w = wl.custom("dec_full", [128], 2, 1, 64, 53, "boundary", b1=[1, 1], b2=[2, 2],
                   decode_steps=2, tail_cap=1)
