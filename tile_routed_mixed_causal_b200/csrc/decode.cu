@@ -18,9 +18,9 @@
 //   softmax: per head over the warp's fragment lanes, K scale and 1/sqrt(d)
 //           folded into the exponent, V scale folded into P (f16, staged per warp);
 //   P V:    O^T += V^T P^T on the tensor cores, V fed by ldmatrix.trans.
-// The bf16 tail (earlier decode tokens + the new one) is a split of its own:
-// CTA x = 0 of every (sequence, KV head), scheduled first, whose four warps
-// share the tail keys on the CUDA cores.  The four warps' states are merged per
+// The bf16 tail (earlier decode tokens + the new one) goes to the last data split
+// of every (sequence, KV head): after its cached tiles, its four warps share the
+// tail keys on the CUDA cores, so the grid holds data splits only.  The four warps' states are merged per
 // CTA; the last split of each (sequence, KV head) to finish merges the splits
 // into the output, and the last such row of a sequence advances tail_len.
 #include "tra_device.cuh"
@@ -136,7 +136,7 @@ struct DecCfg {
   static constexpr int kPBytes = kConsumers * 8 * kPStride * 2;
   static constexpr int kOffE = kOffP + kPBytes;            // q limb exponents: [GRP] int
   static constexpr int kEBytes = 32;
-  static constexpr int kStates = kConsumers;               // one state per consumer warp
+  static constexpr int kStates = 2 * kConsumers;           // tile + tail state per warp
   // merge area [state][GRP][D + 2] floats, aliasing the drained ring
   static constexpr int kOffRed = 0;
   static constexpr int kRedBytes = kStates * GRP * (D + 2) * 4;
@@ -164,10 +164,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   volatile int* const err =
       reinterpret_cast<volatile int*>(sm + C::kOffBar + 2 * kDecStages * 8);
 
-  // x = 0: the bf16 tail of (b, kvh); x = 1 .. splits-1: data split x - 1
+  // x: data split x of (b, kvh); the last one also attends over the bf16 tail
   const int kvh = blockIdx.y, b = blockIdx.z;
-  const bool tail_cta = blockIdx.x == 0;
-  const int nsplit = p.splits - 1, split = (int)blockIdx.x - 1;
+  const int nsplit = p.splits, split = (int)blockIdx.x;
+  const bool tail_cta = split == nsplit - 1;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int grp = p.Hq / p.Hkv;
   const int seq0 = __ldg(p.cu + b);
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     return;
   }
   int my0 = 0, ntile = 0;
-  if (!tail_cta) {
+  {
     const long long row = (long long)b * p.Hkv + kvh;
     const int rs = __ldg(p.row_ptr + row), re = __ldg(p.row_ptr + row + 1);
     const int n = re - rs;
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     named_sync(2);  // merge area written
   } else {
     // ------------------------------------------------------------ consumers
-    // append the new token to the tail (tail CTA; the tail slot tl is read by nobody)
+    // append the new token to the tail (tail split; the tail slot tl is read by nobody)
     if (tail_cta) {
       const long long src = ((long long)b * p.Hkv + kvh) * D;
       const long long dst = (((long long)b * p.Hkv + kvh) * p.tail_cap + tl) * D;
@@ -613,8 +613,33 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     }
 
     // ---- the shared-memory merge; the merge area aliases the ring, so every warp
-    // must be done with the ring first.  Tail CTAs fill the slots from the tail pass.
+    // must be done with the ring first.  Slot w holds warp w's tile state, slot
+    // kConsumers + w (the tail split only) its tail state.
     float* rw = red + warp * GRP * (D + 2);
+#pragma unroll
+    for (int mq = 0; mq < C::kQM; ++mq)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) l_run[mq] += __shfl_xor_sync(0xffffffffu, l_run[mq], o);
+    named_sync(1);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int hd = 2 * tq + hh;
+      if (hd < GRP) {
+#pragma unroll
+        for (int j = 0; j < C::kB8; ++j) {
+          rw[hd * (D + 2) + 16 * j + 2 * g] = o8[j][hh];
+          rw[hd * (D + 2) + 16 * j + 2 * g + 1] = o8[j][2 + hh];
+        }
+      }
+    }
+#pragma unroll
+    for (int mq = 0; mq < C::kQM; ++mq) {
+      const int hd = tq + 4 * mq;
+      if (hd < GRP && g == 0) {
+        rw[hd * (D + 2) + D] = m_run[mq];
+        rw[hd * (D + 2) + D + 1] = l_run[mq];
+      }
+    }
     if (tail_cta) {
       float tm[GRP], tlsum[GRP];
       float2 to[GRP][C::kCh / 2];
@@ -626,55 +651,29 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         for (int k = 0; k < C::kCh / 2; ++k) to[gg][k] = make_float2(0.0f, 0.0f);
       }
       tail_pass(tm, tlsum, to);
-      named_sync(1);
+      float* rt = red + (kConsumers + warp) * GRP * (D + 2);
 #pragma unroll
       for (int gg = 0; gg < GRP; ++gg) {
 #pragma unroll
         for (int k = 0; k < C::kCh / 2; ++k)
-          *reinterpret_cast<float2*>(rw + gg * (D + 2) + lane * C::kCh + 2 * k) = to[gg][k];
+          *reinterpret_cast<float2*>(rt + gg * (D + 2) + lane * C::kCh + 2 * k) = to[gg][k];
         if (lane == 0) {
-          rw[gg * (D + 2) + D] = tm[gg];
-          rw[gg * (D + 2) + D + 1] = tlsum[gg];
-        }
-      }
-    } else {
-#pragma unroll
-      for (int mq = 0; mq < C::kQM; ++mq)
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) l_run[mq] += __shfl_xor_sync(0xffffffffu, l_run[mq], o);
-      named_sync(1);
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int hd = 2 * tq + hh;
-        if (hd < GRP) {
-#pragma unroll
-          for (int j = 0; j < C::kB8; ++j) {
-            rw[hd * (D + 2) + 16 * j + 2 * g] = o8[j][hh];
-            rw[hd * (D + 2) + 16 * j + 2 * g + 1] = o8[j][2 + hh];
-          }
-        }
-      }
-#pragma unroll
-      for (int mq = 0; mq < C::kQM; ++mq) {
-        const int hd = tq + 4 * mq;
-        if (hd < GRP && g == 0) {
-          rw[hd * (D + 2) + D] = m_run[mq];
-          rw[hd * (D + 2) + D + 1] = l_run[mq];
+          rt[gg * (D + 2) + D] = tm[gg];
+          rt[gg * (D + 2) + D + 1] = tlsum[gg];
         }
       }
     }
     named_sync(2);
   }
-  // merge the consumer warps into this split's partial (m, l, o)
+  // merge the consumer warps' states into this split's partial (m, l, o)
+  const int nstates = tail_cta ? C::kStates : kConsumers;
   for (int x = t; x < GRP * D; x += kDecThreads) {
     const int gg = x / D, c = x % D;
     if (gg >= grp) continue;
     float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < C::kStates; ++w) M = fmaxf(M, red[(w * GRP + gg) * (D + 2) + D]);
+    for (int w = 0; w < nstates; ++w) M = fmaxf(M, red[(w * GRP + gg) * (D + 2) + D]);
     float L = 0.0f, o = 0.0f;
-#pragma unroll
-    for (int w = 0; w < C::kStates; ++w) {
+    for (int w = 0; w < nstates; ++w) {
       const float* r = red + (w * GRP + gg) * (D + 2);
       const float wt = r[D] == -INFINITY ? 0.0f : ex2(r[D] - M);
       L += r[D + 1] * wt;
@@ -767,16 +766,16 @@ cudaError_t launch_dec_d(const DecodeParams& p, const DecodeMaps& m, cudaStream_
 
 }  // namespace
 
-// Partials per (sequence, KV head): the data splits plus the bf16-tail split.
+// Splits (partials) per (sequence, KV head); the last one also takes the tail.
 int decode_splits(int B, int Hkv) {
-  // about 256 data CTAs (plus one tail CTA per row): long CTAs, little set-up and a
-  // short merge, about 1.3 waves of two CTAs per SM at batch 16 x 8 KV heads
+  // about 256 CTAs: long CTAs, little set-up and a short merge, one wave of two CTAs
+  // per SM at batch 16 x 8 KV heads
   const int target = 256;
   const int rows = B * Hkv;
   int s = (target + rows - 1) / rows;
   if (s < 1) s = 1;
-  if (s > TRA_MAX_DECODE_SPLITS - 1) s = TRA_MAX_DECODE_SPLITS - 1;
-  return s + 1;
+  if (s > TRA_MAX_DECODE_SPLITS) s = TRA_MAX_DECODE_SPLITS;
+  return s;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodeMaps& m, cudaStream_t s) {
