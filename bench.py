@@ -70,7 +70,7 @@ def parse():
 # and profiles/decode_split_kernel_b16_32k.md.
 PROFILED_TRAFFIC = {
     "prefill.cu": ("e07280ea9221a6e1", 3_425_659_392),
-    "decode.cu": ("a0ae0cc01c87ca66", 663_556_096),
+    "decode.cu": ("681e247ef97b3884", 662_413_568),
 }
 
 
