@@ -499,7 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_valid = half_valid && tq < x.T;
     const long long qtile = (long long)x.h * p.ntiles + x.toff + qt;
     const float sq8 = half_valid ? __ldg(p.sq8 + qtile) : 0.0f;
-    const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) : 0.0f;
+    // expanded INT4 operands are 16 x code, so INT4 accumulators are 256 x the code
+    // product: the power of two goes into the row's INT4 scale (exact)
+    const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) * (1.0f / 256.0f) : 0.0f;
     const uint32_t lane_addr = ((uint32_t)(q4 * 32) << 16) + (uint32_t)(u * 256);
     const uint32_t tU = tmem + lane_addr, tO = tU + 128;  // S/P buffer b at tU + 64 * b
     float m_run = -INFINITY, l_run = 0.0f;
@@ -559,7 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (__ldg(dc) == x.b && __ldg(dc + 1) == x.h && __ldg(dc + 2) == qt &&
                 __ldg(dc + 3) == kt) {
               int32_t* dst = p.dump_out + ((long long)di * 64 + rr) * 64;
-              for (int cc = 0; cc < 64; ++cc) dst[cc] = (int32_t)sr[cc];
+              const int sh = prec == TRA_PREC_INT4 ? 8 : 0;  // INT4: 256 x the code product
+              for (int cc = 0; cc < 64; ++cc) dst[cc] = (int32_t)sr[cc] >> sh;
             }
           }
         }

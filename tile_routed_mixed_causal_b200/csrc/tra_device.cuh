@@ -248,11 +248,12 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 // ----------------------------------------------------------------- small helpers
-// Sign-extend the eight INT4 codes of a 32-bit word (byte i = channels 2i, 2i+1,
-// even channel in the low nibble) into eight int8 codes in channel order.
+// The eight INT4 codes of a 32-bit word (byte i = channels 2i, 2i+1, even channel
+// in the low nibble) as eight int8 values 16 x code in channel order: each nibble
+// becomes the high half of its byte, which is exact and stays within int8.
 __device__ __forceinline__ uint2 expand_int4x8(uint32_t w) {
-  const uint32_t lo = __vsub4((w & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
-  const uint32_t hi = __vsub4(((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+  const uint32_t lo = (w << 4) & 0xF0F0F0F0u;  // even channels in the high nibbles
+  const uint32_t hi = w & 0xF0F0F0F0u;         // odd channels, already there
   return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
