@@ -69,7 +69,7 @@ def parse():
 # source that has changed since reports null.  Captures: profiles/prefill_kernel_bitmask_32k.md
 # and profiles/decode_split_kernel_b16_32k.md.
 PROFILED_TRAFFIC = {
-    "prefill.cu": ("e07280ea9221a6e1", 3_425_659_392),
+    "prefill.cu": ("701cf6b01ac2f0b3", 3_403_118_848),
     "decode.cu": ("681e247ef97b3884", 662_413_568),
 }
 
