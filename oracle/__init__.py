@@ -296,3 +296,115 @@ def allocate_boundaries(err, cost, budget):
         if best is None or e < best[1]:
             best = (list(pick), e, c)
     return best
+
+
+# --------------------------------------------------------------- token-level hybrid
+# HyQuant ("The observation behind the method"; "How HyQuant works"): a small set of
+# important key positions and a recent window keep high precision, the rest of the
+# context is quantised.  Readings: per (sequence, KV head) the ceil(frac * T) most
+# important prefix tokens and every key within `window` positions of the query stay
+# bf16; the other keys and values use their tile's INT4 codes times the tile scale;
+# queries stay bf16.  Plain numpy in fp64.
+
+def _f64(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _int4_values(x4, s4, cu, H):
+    """Dequantised INT4 codes [ntok, H, d] in token order (fp64)."""
+    cu = _c(cu, np.int32)
+    nib = np.stack([x4 & 0xF, x4 >> 4], -1).reshape(*x4.shape[:-1], -1).astype(np.int64)
+    codes = np.where(nib >= 8, nib - 16, nib).astype(np.float64)      # [H, nt, 64, d]
+    ntok = int(cu[-1])
+    out = np.zeros((ntok, H, codes.shape[-1]), np.float64)
+    gt = 0
+    for b in range(len(cu) - 1):
+        L = int(cu[b + 1] - cu[b])
+        for t in range((L + TILE - 1) // TILE):
+            n = min(TILE, L - t * TILE)
+            for h in range(H):
+                out[cu[b] + t * TILE: cu[b] + t * TILE + n, h] = codes[h, gt, :n] * np.float64(s4[h, gt])
+            gt += 1
+    return out
+
+
+def hybrid_select(importance, cu_seqlens, frac=0.05):
+    """bool [ntok, Hkv]: per sequence and KV head, the ceil(frac * T) tokens of largest
+    importance (ties: the earlier position)."""
+    imp = np.asarray(importance, np.float64)
+    cu = _c(cu_seqlens, np.int32)
+    sel = np.zeros(imp.shape, bool)
+    for b in range(len(cu) - 1):
+        s, e = int(cu[b]), int(cu[b + 1])
+        n = int(np.ceil(frac * (e - s)))
+        for h in range(imp.shape[1]):
+            order = sorted(range(s, e), key=lambda j: (-imp[j, h], j))
+            sel[order[:n], h] = True
+    return sel
+
+
+def hybrid_prefill(q_bits, k_bits, v_bits, cu_seqlens, kv: Quantised, selected, window,
+                   scale=None):
+    """fp64 output [ntok, Hq, d]: causal attention in which query i reads key j <= i (same
+    sequence) at bf16 when j is selected or i - j < window, else from its INT4 tile."""
+    q = _f64(q_bits); k = _f64(k_bits); v = _f64(v_bits)
+    cu = _c(cu_seqlens, np.int32)
+    ntok, Hq, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    k4 = _int4_values(kv.k4, kv.sk4, cu, Hkv)
+    v4 = _int4_values(kv.v4, kv.sv4, cu, Hkv)
+    out = np.zeros((ntok, Hq, d), np.float64)
+    for b in range(len(cu) - 1):
+        s, e = int(cu[b]), int(cu[b + 1])
+        T = e - s
+        if T == 0:
+            continue
+        i = np.arange(T)[:, None]
+        j = np.arange(T)[None, :]
+        causal = j <= i
+        for h in range(Hq):
+            kh = h // g
+            hi = selected[s:e, kh][None, :] | (i - j < window)
+            s_hi = q[s:e, h] @ k[s:e, kh].T
+            s_lo = q[s:e, h] @ k4[s:e, kh].T
+            sc = np.where(hi, s_hi, s_lo) * scale
+            sc = np.where(causal, sc, -np.inf)
+            p = np.exp(sc - sc.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            out[s:e, h] = (p * hi) @ v[s:e, kh] + (p * ~hi) @ v4[s:e, kh]
+    return out
+
+
+def hybrid_decode_step(qd_bits, k_bits, v_bits, cu_seqlens, kv: Quantised, selected, window,
+                       k_tail_bits, v_tail_bits, tail_len, scale=None):
+    """fp64 output [B, Hq, d] of one decode step: the query, at position T_b + tail_len_b - 1,
+    reads every prefix token (bf16 when selected or within `window` positions of it, else
+    from its INT4 tile) and the bf16 tail tokens [0, tail_len_b), which hold the new one."""
+    qd = _f64(qd_bits); k = _f64(k_bits); v = _f64(v_bits)
+    kt = _f64(k_tail_bits); vt = _f64(v_tail_bits)
+    cu = _c(cu_seqlens, np.int32)
+    B, Hq, d = qd.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    k4 = _int4_values(kv.k4, kv.sk4, cu, Hkv)
+    v4 = _int4_values(kv.v4, kv.sv4, cu, Hkv)
+    out = np.zeros((B, Hq, d), np.float64)
+    for b in range(B):
+        s, e = int(cu[b]), int(cu[b + 1])
+        tl = int(tail_len[b])
+        pos = (e - s) + tl - 1
+        j = np.arange(e - s)
+        for h in range(Hq):
+            kh = h // g
+            hi = selected[s:e, kh] | (pos - j < window)
+            kp = np.where(hi[:, None], k[s:e, kh], k4[s:e, kh])
+            vp = np.where(hi[:, None], v[s:e, kh], v4[s:e, kh])
+            keys = np.concatenate([kp, kt[b, kh, :tl]])
+            vals = np.concatenate([vp, vt[b, kh, :tl]])
+            sc = keys @ qd[b, h] * scale
+            p = np.exp(sc - sc.max())
+            out[b, h] = p @ vals / p.sum()
+    return out

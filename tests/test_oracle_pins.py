@@ -508,3 +508,99 @@ def test_decode_matches_naive_dense_softmax():
                 p = np.exp(s - s.max())
                 p /= p.sum()
                 assert np.max(np.abs(got[b, h] - p @ V)) < 1e-12
+
+
+# --------------------------------------------------------------------------- token-level hybrid
+def _hybrid_case():
+    w = wl.custom("hybrid", [300, 64, 1, 200], 4, 2, 64, 71, "boundary")
+    q, k, v = _inputs(w)
+    cu = w.cu_seqlens
+    kv = oracle.Quantised(None, k, v, cu)
+    return w, q, k, v, cu, kv
+
+
+def test_hybrid_select_top_fraction():
+    """ceil(frac * T) positions per sequence and KV head, none less important than any
+    position left out (ties to the earlier position)."""
+    w, q, k, v, cu, kv = _hybrid_case()
+    imp = wl.hybrid_importance(w, 3)
+    imp[5, 0] = imp[6, 0] = imp[:300, 0].max() + 1.0        # a tie at the top
+    sel = oracle.hybrid_select(imp, cu, 0.05)
+    for b in range(len(cu) - 1):
+        s, e = cu[b], cu[b + 1]
+        for h in range(w.Hkv):
+            n = int(np.ceil(0.05 * (e - s)))
+            assert int(sel[s:e, h].sum()) == n
+            if 0 < n < e - s:
+                assert imp[s:e, h][sel[s:e, h]].min() >= imp[s:e, h][~sel[s:e, h]].max()
+    assert sel[5, 0] and sel[6, 0]
+
+
+def test_hybrid_prefill_reduces_to_dense_attention():
+    """Everything kept in bf16 (all selected, or a window covering every key) is textbook
+    causal attention; nothing kept is textbook attention over the INT4-dequantised K and V."""
+    w, q, k, v, cu, kv = _hybrid_case()
+    qv, kvv, vv = val_of(q), val_of(k), val_of(v)
+    dense = _dense_causal(qv, kvv, vv, cu, w.Hq, w.Hkv)
+    every = np.ones((w.ntok, w.Hkv), bool)
+    none = np.zeros((w.ntok, w.Hkv), bool)
+    assert np.max(np.abs(oracle.hybrid_prefill(q, k, v, cu, kv, every, 0) - dense)) < 1e-12
+    assert np.max(np.abs(oracle.hybrid_prefill(q, k, v, cu, kv, none, 10**6) - dense)) < 1e-12
+    k4 = _dequant_tokens(_unpack4(kv.k4), kv.sk4, cu, w.d, w.Hkv)
+    v4 = _dequant_tokens(_unpack4(kv.v4), kv.sv4, cu, w.d, w.Hkv)
+    low = _dense_causal(qv, k4, v4, cu, w.Hq, w.Hkv)
+    assert np.max(np.abs(oracle.hybrid_prefill(q, k, v, cu, kv, none, 0) - low)) < 1e-12
+
+
+def test_hybrid_prefill_mixes_per_key_and_rows_sum_to_one():
+    """A key's precision depends only on its selection and its distance to the query: with
+    V = 1 every output is a convex combination of 1 (bf16 keys) and 7 fl32(1/7) (the same
+    value read from INT4), so the weights sum to one; changing the precision of one
+    unselected, distant key moves only the rows that read it from INT4."""
+    w, q, k, v, cu, kv = _hybrid_case()
+    sel = oracle.hybrid_select(wl.hybrid_importance(w, 4), cu, 0.05)
+    ones = np.full_like(v, 0x3F80)                            # bf16 1.0
+    kv1 = oracle.Quantised(None, k, ones, cu)
+    out = oracle.hybrid_prefill(q, k, ones, cu, kv1, sel, 16)
+    lo4 = 7.0 * np.float64(np.float32(1.0) / np.float32(7.0))
+    assert out.min() >= min(1.0, lo4) - 1e-12 and out.max() <= max(1.0, lo4) + 1e-12
+    assert np.max(np.abs(out - 1.0)) > 0.0                    # some rows did read INT4
+    base = oracle.hybrid_prefill(q, k, v, cu, kv, sel, 16)
+    j = int(np.flatnonzero(~sel[:300, 0])[0])                 # an unselected key of sequence 0
+    sel2 = sel.copy()
+    sel2[j, 0] = True
+    moved = oracle.hybrid_prefill(q, k, v, cu, kv, sel2, 16)
+    diff = np.abs(moved - base).max(axis=2)                   # [ntok, Hq]
+    heads = [h for h in range(w.Hq) if h // (w.Hq // w.Hkv) == 0]
+    for i in range(w.ntok):
+        reads_lo = 0 <= i - j < 300 - j and i - j >= 16 and i < 300
+        for h in range(w.Hq):
+            if not (reads_lo and h in heads):
+                assert diff[i, h] == 0.0
+    assert diff[j + 16:300, heads].max() > 0.0
+
+
+def test_hybrid_decode_reduces_to_dense_softmax():
+    """One decode step: all prefix keys in bf16 gives the textbook softmax over the prefix
+    plus the tail; none gives it over the INT4-dequantised prefix plus the tail."""
+    w, q, k, v, cu, kv = _hybrid_case()
+    B, Hq, Hkv, d = w.B, w.Hq, w.Hkv, w.d
+    rng = np.random.default_rng(9)
+    qd = wl.bf16_bits(torch.from_numpy(rng.standard_normal((B, Hq, d)).astype(np.float32)).bfloat16())
+    cap, tl = 4, np.array([1, 3, 2, 4], np.int32)
+    kt = wl.bf16_bits(torch.from_numpy(rng.standard_normal((B, Hkv, cap, d)).astype(np.float32)).bfloat16())
+    vt = wl.bf16_bits(torch.from_numpy(rng.standard_normal((B, Hkv, cap, d)).astype(np.float32)).bfloat16())
+    every = np.ones((w.ntok, Hkv), bool)
+    none = np.zeros((w.ntok, Hkv), bool)
+    k4 = _dequant_tokens(_unpack4(kv.k4), kv.sk4, cu, d, Hkv)
+    v4 = _dequant_tokens(_unpack4(kv.v4), kv.sv4, cu, d, Hkv)
+    for sel, kk, vv_ in ((every, val_of(k), val_of(v)), (none, k4, v4)):
+        got = oracle.hybrid_decode_step(qd, k, v, cu, kv, sel, 0, kt, vt, tl)
+        for b in range(B):
+            for h in range(Hq):
+                kh = h // (Hq // Hkv)
+                keys = np.concatenate([kk[cu[b]:cu[b + 1], kh], val_of(kt[b, kh, :tl[b]])])
+                vals = np.concatenate([vv_[cu[b]:cu[b + 1], kh], val_of(vt[b, kh, :tl[b]])])
+                sc = keys @ val_of(qd[b, h]) / np.sqrt(d)
+                p = np.exp(sc - sc.max())
+                assert np.max(np.abs(got[b, h] - p @ vals / p.sum())) < 1e-12

@@ -248,6 +248,13 @@ def synthetic_boundary_errors(Hq: int, cands, nt: int, seed: int) -> np.ndarray:
     return err
 
 
+def hybrid_importance(w: "Workload", seed: int) -> np.ndarray:
+    """Seeded synthetic importance [ntok, Hkv] of key positions for the token-level hybrid
+    (heavy-tailed, so that a few positions stand out as vertical lines would)."""
+    rng = np.random.default_rng(seed + 3000)
+    return rng.pareto(1.5, size=(w.ntok, w.Hkv))
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama8b_8k": llama8b_8k,
