@@ -3,9 +3,11 @@
 TEST INFRASTRUCTURE ONLY: the test-suite, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg are the only callers.  The product path (the CUDA
 library and its Python binding) never imports this package, and this package
-never imports the product.  All arithmetic lives in ``tra_oracle.c`` (plain C,
-fp64, IEEE fp32 for the quantiser); this module only compiles it with gcc and
-marshals numpy arrays.
+never imports the product.  The arithmetic of the hot path lives in
+``tra_oracle.c`` (plain C, fp64, IEEE fp32 for the quantiser), which this module
+compiles with gcc and calls with numpy arrays; the boundary allocator's
+enumeration and the token-level hybrid (HyQuant) are plain numpy / Python below,
+fp64.
 
 Sources (page titles): "TriAttention: Unified Sparse Mixed-Precision Attention
 for Long-Context LLM Inference" (abstract), "TileMix: Tile-Centric
