@@ -39,6 +39,8 @@
  *    diagonal tile is always kept in INT8.  Storage 8*Hq bytes at any length.
  *  - Bitmask policy: uint32 [Hq][ntiles][W]; bit g of row (h, q-tile) (word
  *    g/32, bit g%32) covers k-tiles [g*G, g*G+G): 1 -> BF16, 0 -> INT8; no skip.
+ *  - Mixed policy: both of the above; the boundaries decide skip / INT4 / INT8
+ *    and a set bit promotes a kept tile to BF16 (see TRA_POLICY_MIXED).
  *  - Traversal lists (CSR): prefill rows are (h, global q-tile), h-major;
  *    decode-cache rows are (b, kv-head), b-major.  entry = (prec << 28) | kt,
  *    kt local to the sequence, prec = TRA_PREC_*; a row lists its INT4 tiles
@@ -47,7 +49,8 @@
  *  - GQA: query head h reads KV head h / (Hq/Hkv).
  *
  * Memory and streams: every buffer is caller-owned device memory unless a
- * parameter says "host".  The library allocates nothing, never synchronises the
+ * parameter says "host".  The library allocates no device memory (the host-only
+ * boundary allocator keeps its tables in host memory), never synchronises the
  * device, and enqueues all work on the given stream (a cudaStream_t passed as
  * void*; NULL = legacy default stream).  Pointers to device buffers must be
  * 16-byte aligned.  Every call validates its arguments on the host before any
