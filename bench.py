@@ -19,6 +19,11 @@ The same run also measures:
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 launch with torch.distributed.run; every rank runs an independent
 replica (the method has no cross-GPU exchange) and rank 0 prints one JSON line.
+
+Reduced lines (--only): "prefill" times one prefill workload (--workload
+bitmask_32k | llama8b_8k | varlen_8 | mixed_8k), "decode" the decode alone,
+"allocate" fits the complete-tile cost model and runs the boundary allocator on
+synthetic error tables, then times the allocated policy.
 """
 from __future__ import annotations
 
