@@ -3,7 +3,9 @@
 ``PrefillPlan``: quantize_qkv_tiles -> build_tile_lists -> routed_attention_prefill.
 ``DecodePlan``:  build_tile_lists (decode-cache kind, once) -> routed_attention_decode
 per step, over the K/V tiles a PrefillPlan (or quantize_qkv_tiles) produced.
-Buffers are allocated once per plan; ``run``/``step`` only enqueue kernels.
+Buffers are allocated once per plan; ``run``/``step`` only enqueue kernels.  The
+decode workspace is zero-filled once (the decode's arrival counters need that, and
+every step leaves them at zero).
 """
 from __future__ import annotations
 
