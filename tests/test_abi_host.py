@@ -222,3 +222,13 @@ def test_mixed_policy_sizes_and_validation(lib):
     with pytest.raises(L.TraError) as e:
         L.tile_lists_size(s, odd)
     assert "unknown policy mode" in str(e.value)
+
+
+def test_mixed_policy_needs_its_bitmask(lib):
+    """build_tile_lists rejects a mixed policy without device bitmask words, on the host."""
+    s = _shape([300], Hq=4, Hkv=2)
+    pol = L.Policy(L.POLICY_MIXED, b1=[1, 1, 1, 1], b2=[3, 3, 3, 3], G=2)
+    pol._c.W = 1
+    rows, nnz = L.tile_lists_size(s, pol, L.LISTS_PREFILL)
+    st = lib.build_tile_lists(s.c, pol.c, L.LISTS_PREFILL, FAKE, rows + 1, FAKE, nnz, None)
+    assert st == 1 and b"bitmask" in lib.tra_last_error()
