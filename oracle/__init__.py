@@ -39,7 +39,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call([
-            "gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+            "gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
             "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
@@ -55,6 +55,8 @@ def _load():
             I = ctypes.c_int
             L = ctypes.c_int64
             D = ctypes.c_double
+            lib.orc_set_threads.argtypes = [I]
+            lib.orc_set_threads.restype = I
             lib.orc_num_tiles.argtypes = [P, I]
             lib.orc_num_tiles.restype = L
             lib.orc_quantize.argtypes = [P, P, I, I, I, P, P, P, P]
@@ -87,6 +89,12 @@ def _p(a):
 
 def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
+
+
+def set_threads(n: int) -> int:
+    """Threads prefill_rows spreads its independent rows over (n < 1: every core);
+    returns the count set.  Results do not depend on it."""
+    return int(_load().orc_set_threads(int(n)))
 
 
 def num_tiles(cu_seqlens) -> int:

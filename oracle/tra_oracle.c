@@ -7,9 +7,12 @@
  * CPU-baseline leg use it.  It shares no code, header, table or constant with
  * the CUDA library; neither side includes the other.
  *
- * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC
  *        (no -ffast-math: the quantiser relies on IEEE fp32 divide and
- *         round-half-even under the default rounding mode).
+ *         round-half-even under the default rounding mode).  OpenMP only
+ *         spreads independent traversal rows over threads; every row is
+ *         computed by one thread in the same order, so results do not depend
+ *         on the thread count.
  *
  * Sources followed (page titles; the pages print no formulas, so each rule
  * below is the plainest reading of the cited sentence):
@@ -49,6 +52,7 @@
  *    bitmask mode every cached tile is INT8.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -81,6 +85,13 @@ static int64_t tile_offsets(const int32_t* cu, int B, int64_t* off /* [B+1] */) 
   off[0] = 0;
   for (int b = 0; b < B; ++b) off[b + 1] = off[b] + ceil_tiles(cu[b + 1] - cu[b]);
   return off[B];
+}
+
+/* Threads used by orc_prefill_rows (independent rows); n < 1 selects all cores. */
+int orc_set_threads(int n) {
+  if (n < 1) n = omp_get_num_procs();
+  omp_set_num_threads(n);
+  return n;
 }
 
 int64_t orc_num_tiles(const int32_t* cu, int B) {
@@ -362,8 +373,13 @@ int orc_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   int64_t ntiles = tile_offsets(cu, B, off);
   int nt_max = 0;
   for (int b = 0; b < B; ++b) if (ceil_tiles(cu[b + 1] - cu[b]) > nt_max) nt_max = ceil_tiles(cu[b + 1] - cu[b]);
+  int bad = 0;
+#pragma omp parallel
+  {
+  /* per-thread score and key buffers; each row is handled by one thread */
   double* s = (double*)malloc(sizeof(double) * (size_t)(nt_max + 1) * 2 * ORC_TILE);
   int64_t* key = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nt_max + 1) * 2 * ORC_TILE);
+#pragma omp for schedule(dynamic, 1)
   for (int i = 0; i < nrows; ++i) {
     int64_t row = rows[i];
     int h = (int)(row / ntiles);
@@ -408,8 +424,9 @@ int orc_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
               sc = (double)acc * (double)sq4[(int64_t)h * ntiles + gq] *
                    (double)sk4[(int64_t)kvh * ntiles + gk] * scale;
             } else {
-              free(off); free(s); free(key);
-              return -2;
+#pragma omp atomic write
+              bad = 1;
+              sc = 0.0;
             }
           }
           s[ns] = sc;
@@ -431,8 +448,10 @@ int orc_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
       if (lse) lse[(int64_t)i * ORC_TILE + r] = m + log(l);
     }
   }
-  free(off); free(s); free(key);
-  return 0;
+  free(s); free(key);
+  }
+  free(off);
+  return bad ? -2 : 0;
 }
 
 /* ---------------------------------------------------------------------------

@@ -344,9 +344,22 @@ def test_prefill_all_bf16_is_dense_attention():
     w = wl.custom("allbf16", [130, 64, 1, 200], 4, 2, 64, 5, "bitmask", G=2, p_bf16=1.0)
     q, k, v = _inputs(w)
     cu = w.cu_seqlens
-    got, _, _ = _run_oracle_all_rows(w, q, k, v, cu)
+    got, _, lse = _run_oracle_all_rows(w, q, k, v, cu)
     ref = _dense_causal(val_of(q), val_of(k), val_of(v), cu, w.Hq, w.Hkv)
     assert np.max(np.abs(got - ref)) < 1e-12
+    # lse against scipy's logsumexp of the masked textbook scores
+    from scipy.special import logsumexp
+    qv, kv = val_of(q), val_of(k)
+    grp = w.Hq // w.Hkv
+    ref_lse = np.zeros((cu[-1], w.Hq))
+    for b in range(len(cu) - 1):
+        s0, s1 = cu[b], cu[b + 1]
+        L = s1 - s0
+        for h in range(w.Hq):
+            S = qv[s0:s1, h] @ kv[s0:s1, h // grp].T / np.sqrt(q.shape[-1])
+            S = np.where(np.tril(np.ones((L, L), bool)), S, -np.inf)
+            ref_lse[s0:s1, h] = logsumexp(S, axis=1)
+    assert np.max(np.abs(_lse_tokens(lse, cu, w.Hq) - ref_lse)) < 1e-10
 
 
 def test_prefill_block_local():
@@ -384,8 +397,10 @@ def test_prefill_all_int8_is_dense_over_dequantised_scores():
     assert np.max(np.abs(got - ref)) < 1e-12
 
 
-def _brute_force_prefill(w, q, k, v, qz):
-    """Per (query, key) pair: pick the precision by the boundary/bitmask rule directly."""
+def _brute_force_prefill(w, q, k, v, qz, with_lse=False):
+    """Per (query, key) pair: pick the precision by the boundary/bitmask rule directly.
+    With with_lse, also the natural-log logsumexp of each query's scaled scores
+    [ntok, Hq], written out as log(sum(exp(s))) with a shift for range only."""
     cu = w.cu_seqlens
     d = q.shape[-1]
     grp = w.Hq // w.Hkv
@@ -395,6 +410,7 @@ def _brute_force_prefill(w, q, k, v, qz):
     q4 = _dequant_tokens(_unpack4(qz.q4), qz.sq4, cu, d, w.Hq) if qz.q4 is not None else None
     k4 = _dequant_tokens(_unpack4(qz.k4), qz.sk4, cu, d, w.Hkv) if qz.k4 is not None else None
     out = np.zeros((cu[-1], w.Hq, d))
+    lse = np.zeros((cu[-1], w.Hq))
     gt0 = 0
     for b in range(len(cu) - 1):
         L = cu[b + 1] - cu[b]
@@ -423,10 +439,29 @@ def _brute_force_prefill(w, q, k, v, qz):
                     s.append(sc / np.sqrt(d))
                     keys.append(j)
                 s = np.array(s)
+                shift = s[0]                      # any finite shift; the first key's score
+                lse[cu[b] + i, h] = shift + np.log(np.sum(np.exp(s - shift)))
                 p = np.exp(s - s.max())
                 p /= p.sum()
                 out[cu[b] + i, h] = p @ vv[cu[b] + np.array(keys), kvh]
         gt0 += (L + 63) // 64
+    return (out, lse) if with_lse else out
+
+
+def _lse_tokens(lse_rows, cu, Hq):
+    """Oracle lse [rows, 64] (rows h-major over global q-tiles) -> [ntok, Hq]."""
+    cu = np.asarray(cu, np.int64)
+    nts = [(int(cu[b + 1] - cu[b]) + 63) // 64 for b in range(len(cu) - 1)]
+    ntiles = sum(nts)
+    out = np.full((int(cu[-1]), Hq), np.nan)
+    for h in range(Hq):
+        g = 0
+        for b, nt in enumerate(nts):
+            T = int(cu[b + 1] - cu[b])
+            for qt in range(nt):
+                n = min(64, T - qt * 64)
+                out[cu[b] + qt * 64: cu[b] + qt * 64 + n, h] = lse_rows[h * ntiles + g, :n]
+                g += 1
     return out
 
 
@@ -434,17 +469,20 @@ def test_prefill_brute_force_tiny_config():
     """The tiny configuration (1 x 2 heads x 256 tokens, (b1, b2) = (1, 3)), brute force."""
     w = wl.tiny()
     q, k, v = _inputs(w)
-    got, qz, _ = _run_oracle_all_rows(w, q, k, v, w.cu_seqlens)
-    ref = _brute_force_prefill(w, q, k, v, qz)
+    got, qz, lse = _run_oracle_all_rows(w, q, k, v, w.cu_seqlens)
+    ref, ref_lse = _brute_force_prefill(w, q, k, v, qz, with_lse=True)
     assert np.max(np.abs(got - ref)) < 1e-12
+    # lse: natural log of the sum of exp over the kept, scaled scores of each query
+    assert np.max(np.abs(_lse_tokens(lse, w.cu_seqlens, w.Hq) - ref_lse)) < 1e-10
 
 
 def test_prefill_brute_force_bitmask_gqa_varlen():
     w = wl.custom("bm", [190, 70], 4, 2, 64, 12, "bitmask", G=2, p_bf16=0.4)
     q, k, v = _inputs(w)
-    got, qz, _ = _run_oracle_all_rows(w, q, k, v, w.cu_seqlens)
-    ref = _brute_force_prefill(w, q, k, v, qz)
+    got, qz, lse = _run_oracle_all_rows(w, q, k, v, w.cu_seqlens)
+    ref, ref_lse = _brute_force_prefill(w, q, k, v, qz, with_lse=True)
     assert np.max(np.abs(got - ref)) < 1e-12
+    assert np.max(np.abs(_lse_tokens(lse, w.cu_seqlens, w.Hq) - ref_lse)) < 1e-10
 
 
 def test_prefill_rows_sum_to_one():
