@@ -55,11 +55,13 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--decode-passes", type=int, default=3)
+    ap.add_argument("--decode-passes", type=int, default=5)
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-configuration prefill records and the allocator record")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--only", choices=["prefill", "decode", "allocate"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "allocate", "hybrid"], default=None,
                     help="run one part only (used for profiler captures); prints a reduced line. "
                          "allocate: measured complete-tile cost model + boundary allocator demo")
     ap.add_argument("--workload", choices=["bitmask_32k", "llama8b_8k", "varlen_8", "mixed_8k"],
@@ -71,8 +73,7 @@ def parse():
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
 # each dominant kernel, keyed by the SHA-256 prefix of the kernel source that was captured; a
-# source that has changed since reports null.  Captures: profiles/prefill_kernel_bitmask_32k.md
-# and profiles/decode_split_kernel_b16_32k.md.
+# source that has changed since reports null.
 PROFILED_TRAFFIC = {
     "prefill.cu": ("701cf6b01ac2f0b3", 3_403_118_848),
     "decode.cu": ("681e247ef97b3884", 662_413_568),
@@ -219,36 +220,118 @@ def run_prefill_bench(S, steps, warmup, stream):
 
 
 def run_prefill_e2e(S, steps, stream):
-    """Same path with pinned-host inputs copied in and the output copied out per step."""
-    plan, shape = S["plan"], S["shape"]
+    """Same path with pinned-host inputs copied in and the output copied out every step.
+    Copies run on their own streams and are double-buffered, so step i's output copy and
+    step i+1's input copy overlap step i's and i+1's kernels; the timed region spans the
+    first input copy to the last output copy."""
+    plan = S["plan"]
     hq = S["q"].cpu().pin_memory()
     hk = S["k"].cpu().pin_memory()
     hv = S["v"].cpu().pin_memory()
     hbm = S["bitmask"].cpu().pin_memory()
-    hout = torch.empty(S["out"].shape, dtype=S["out"].dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(S["q"]), torch.empty_like(S["k"]), torch.empty_like(S["v"])
+    hout = [torch.empty(S["out"].shape, dtype=S["out"].dtype).pin_memory() for _ in range(2)]
+    sets = [dict(q=torch.empty_like(S["q"]), k=torch.empty_like(S["k"]), v=torch.empty_like(S["v"]),
+                 out=torch.empty_like(S["out"])) for _ in range(2)]
     dbm = S["bitmask"]
-    dout = torch.empty_like(S["out"])
     h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + hbm.numel() * 4
-    d2h = hout.numel() * 2
-    with torch.cuda.stream(stream):
-        def one():
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            dbm.copy_(hbm, non_blocking=True)
-            plan.run(dq, dk, dv, dout, stream=stream)
-            hout.copy_(dout, non_blocking=True)
-        one()
-        stream.synchronize()
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
-        start.record(stream)
-        for _ in range(steps):
-            one()
-        end.record(stream)
-        stream.synchronize()
+    d2h = hout[0].numel() * 2
+    s_in, s_out = torch.cuda.Stream(stream.device), torch.cuda.Stream(stream.device)
+    ev = lambda: torch.cuda.Event()
+
+    def run(nsteps):
+        loaded = [None, None]      # set i: its inputs are in
+        computed = [None, None]    # set i: its kernels are done
+        drained = [ev(), ev()]     # set i: its output copy is done (inputs free again)
+        for e in drained:
+            e.record(s_out)
+        for i in range(nsteps):
+            b = i % 2
+            st = sets[b]
+            s_in.wait_event(drained[b])
+            if computed[b] is not None:
+                s_in.wait_event(computed[b])
+            with torch.cuda.stream(s_in):
+                st["q"].copy_(hq, non_blocking=True)
+                st["k"].copy_(hk, non_blocking=True)
+                st["v"].copy_(hv, non_blocking=True)
+                if i == 0:
+                    dbm.copy_(hbm, non_blocking=True)
+            loaded[b] = ev()
+            loaded[b].record(s_in)
+            stream.wait_event(loaded[b])
+            plan.run(st["q"], st["k"], st["v"], st["out"], stream=stream)
+            computed[b] = ev()
+            computed[b].record(stream)
+            s_out.wait_event(computed[b])
+            with torch.cuda.stream(s_out):
+                hout[b].copy_(st["out"], non_blocking=True)
+            drained[b] = ev()
+            drained[b].record(s_out)
+
+    run(2)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    stream.wait_event(start)
+    s_out.wait_event(start)
+    run(steps)
+    s_out.wait_stream(stream)
+    s_out.wait_stream(s_in)
+    end.record(s_out)
+    torch.cuda.synchronize()
     return start.elapsed_time(end) / steps, h2d, d2h
+
+
+def quantize_bench(S, stream, reps=20):
+    """quantize_qkv_tiles alone on the workload (its formats): ms and GB/s of algorithmic
+    bytes (bf16 inputs read once, codes and scales written once)."""
+    plan, q, k, v = S["plan"], S["q"], S["k"], S["v"]
+    w = S["w"]
+    nt = w.ntiles
+    tiles = plan.tiles
+    fm = tiles.formats
+    bytes_ = 0
+    for bit8, bit4, H, x in ((0x1, 0x2, w.Hq, q), (0x4, 0x8, w.Hkv, k), (0x10, 0x20, w.Hkv, v)):
+        if fm & (bit8 | bit4):
+            bytes_ += x.numel() * 2
+            if fm & bit8:
+                bytes_ += H * nt * 64 * w.d + H * nt * 4
+            if fm & bit4:
+                bytes_ += H * nt * 64 * w.d // 2 + H * nt * 4
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            plan.quantize(q, k, v, stream=stream)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            plan.quantize(q, k, v, stream=stream)
+        b.record(stream)
+        stream.synchronize()
+    ms = a.elapsed_time(b) / reps
+    return {"ms": round(ms, 4), "bytes": int(bytes_), "GB/s": round(bytes_ / (ms * 1e-3) / 1e9, 1)}
+
+
+def workload_records(device, stream, bf16_tflops, names=("llama8b_8k", "varlen_8", "mixed_8k"),
+                     steps=10, warmup=3):
+    """The other prefill configurations: kernel time, TOPS and tile-mix roofline fraction."""
+    recs = {}
+    for name in names:
+        S = prefill_setup(device, name)
+        total_ms, attn_ms, prep_ms = run_prefill_bench(S, steps, warmup, stream)
+        ops = prefill_ops(S)
+        kern = statistics.median(attn_ms)
+        t_roof = roofline_time(S, bf16_tflops)
+        recs[name] = {"workload": S["w"].name, "prefill_kernel_ms": round(kern, 4),
+                      "ms_per_step": round(total_ms / steps, 4),
+                      "kernel_TOPS": round(ops / (kern * 1e-3) / 1e12, 2),
+                      "roofline_frac": round(t_roof / (kern * 1e-3), 4),
+                      "tiles": S["tiles"], "bf16_tiles": S["n16"], "int8_tiles": S["n8"],
+                      "int4_tiles": S["n4"], "prep_ms": round(statistics.median(prep_ms), 4)}
+        del S
+        torch.cuda.empty_cache()
+    return recs
 
 
 # ----------------------------------------------------------------------------- allocator
@@ -382,7 +465,7 @@ def decode_bench(device, passes, stream, hbm_gbs):
             if it > 0:
                 times.append(s0.elapsed_time(s1))
     assert int(dp.status.item()) == 0, "decode reported a device error"
-    ms = min(times)
+    ms = statistics.median(times)
     gbs = pass_bytes / (ms * 1e-3) / 1e9
     return {
         "metric": "decode KV-cache GB/s",
@@ -390,12 +473,76 @@ def decode_bench(device, passes, stream, hbm_gbs):
         "unit": "GB/s",
         "workload": w.name + f" (b1~U[64,192], b2~U[b1+128,480]; {n8} INT8 + {n4} INT4 cached tiles)",
         "ms_per_token_step": round(ms / steps, 4),
+        "passes": len(times), "pass_ms": [round(t, 3) for t in times], "stat": "median of passes",
         "bytes_per_step": int(pass_bytes / steps),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                      "frac": round(gbs / hbm_gbs, 4), "traffic": profiled_traffic("decode.cu"),
-                     "kernel": "decode_split_kernel (one ABI call, one launch)"},
-        "gpu_launches_per_step": 1,
+                     "kernel": "decode_split_kernel (one ABI call: the two- and three-limb launches, each group in one)"},
+        "gpu_launches_per_step": 2,
     }
+
+
+# ----------------------------------------------------------------------------- hybrid decode
+def hybrid_bench(device, passes, stream, hbm_gbs, frac=0.05, window=128):
+    """Token-level hybrid decode (HyQuant, "How HyQuant works") on the decode workload:
+    every prefix tile streamed in INT4 with the 5% selected and the in-window keys read
+    from a bf16 side cache; 64 steps.  GB/s of algorithmic bytes."""
+    import tile_routed_mixed_causal_b200 as tra
+    from tile_routed_mixed_causal_b200 import api
+    from tile_routed_mixed_causal_b200 import workloads as wl
+
+    w = wl.decode_32k()
+    t = wl.make_inputs(w, device, need_q=False)
+    shape = tra.Shape(w.cu_seqlens, w.Hq, w.Hkv, w.d, device=device)
+    cache = tra.QTiles(shape, tra.FMT_K4 | tra.FMT_V4, device)
+    tra.quantize_qkv_tiles(shape, None, t["k"], t["v"], cache)
+    imp = torch.from_numpy(wl.hybrid_importance(w, 7).astype(np.float32)).to(device)
+    hp = api.HybridDecodePlan(shape, cache, frac, window, w.tail_cap, device)
+    torch.cuda.synchronize()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s0.record(stream)
+        hp.select(imp, t["k"], t["v"], stream=stream)
+        s1.record(stream)
+    stream.synchronize()
+    select_ms = s0.elapsed_time(s1)
+    del t
+    qs, kn, vn = wl.make_decode_inputs(w, device)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=device)
+    d, nt = w.d, w.tiles_per_seq[0]
+    nsel = int(np.ceil(frac * w.lengths[0]))
+    steps = w.decode_steps
+    int4_bytes = w.B * w.Hkv * nt * (2 * 64 * d // 2 + 8 + 8)   # codes, scales, key mask
+    fixed = w.B * w.Hq * d * 2 * 2 + w.B * w.Hkv * d * 2 * 4      # q, out, new token
+    pass_bytes = 0
+    for s in range(steps):
+        in_win = sum(1 for x in range(window) if (w.lengths[0] + s) - (w.lengths[0] - window + x) < window)
+        hi_rows = nsel + in_win                                    # upper bound: overlaps counted twice
+        pass_bytes += int4_bytes + fixed + w.B * w.Hkv * (hi_rows + s + 1) * d * 2 * 2
+    times = []
+    with torch.cuda.stream(stream):
+        for it in range(passes + 1):
+            hp.tail_len.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for s in range(steps):
+                hp.step(qs[s], kn[s], vn[s], out, stream=stream)
+            b.record(stream)
+            stream.synchronize()
+            if it > 0:
+                times.append(a.elapsed_time(b))
+    assert int(hp.status.item()) == 0, "hybrid decode reported a device error"
+    ms = statistics.median(times)
+    gbs = pass_bytes / (ms * 1e-3) / 1e9
+    return {"metric": "hybrid decode KV-cache GB/s", "value": round(gbs, 1), "unit": "GB/s",
+            "workload": w.name + f" (token-level hybrid: every tile INT4, {nsel} selected + "
+                                 f"{window}-token window bf16 per sequence and KV head)",
+            "ms_per_token_step": round(ms / steps, 4), "bytes_per_step": int(pass_bytes / steps),
+            "select_ms": round(select_ms, 4), "stat": "median of passes",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": round(gbs / hbm_gbs, 4)}}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -422,26 +569,40 @@ def oracle_sample(w, q, k, v, qtiles, head=0):
     return 2 * tiles * TILE_OPS_PER_GEMM * w.d, dt, tiles
 
 
-def cpu_baseline(S, budget_s=12.0):
+def cpu_baseline(S, budget_s=10.0):
+    """The oracle as it stands on a bounded sample of the 32K workload's q-tile rows of head 0:
+    first single-threaded, then with its rows spread over every host core."""
+    import oracle
     w = S["w"]
     nt = w.ntiles
-    rows = []
-    ops = secs = tiles = 0
-    # q-tiles spread over the sequence (heavy late rows first), until the time budget is used
     order = [nt - 1, 3 * nt // 4, nt // 2, nt // 4]
     order += [int(x) for x in np.random.default_rng(7).permutation(nt) if int(x) not in order]
-    for qt in order:
-        o, s, t = oracle_sample(w, S["q"], S["k"], S["v"], [qt])
-        rows.append(qt)
-        ops += o
-        secs += s
-        tiles += t
-        if secs > budget_s:
-            break
-    return {"value": round(ops / secs / 1e12, 8), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"head 0, {len(rows)} q-tile rows (first {rows[:6]}, then a seeded "
-                      f"permutation) of the 32K bitmask workload ({tiles} kept tiles, "
-                      f"quantisation + traversal + fp64 attention), {secs:.1f} s single-threaded"}
+    res = {}
+    cores = os.cpu_count() or 1
+    for label, threads in (("single", 1), ("all", cores)):
+        oracle.set_threads(threads)
+        rows = []
+        ops = secs = tiles = 0
+        pos = 0
+        while secs <= budget_s and pos < len(order):
+            batch = order[pos:pos + threads]
+            pos += len(batch)
+            o, s_, t = oracle_sample(w, S["q"], S["k"], S["v"], batch)
+            rows += batch
+            ops += o
+            secs += s_
+            tiles += t
+        res[label] = {"value": round(ops / secs / 1e12, 8), "cores": threads, "rows": len(rows),
+                      "tiles": tiles, "seconds": round(secs, 2)}
+    oracle.set_threads(1)
+    a = res["all"]
+    return {"value": a["value"], "unit": UNIT, "cores": a["cores"], "kind": "oracle",
+            "single_thread": res["single"],
+            "sample": f"head 0 q-tile rows of the 32K bitmask workload (first {order[:4]}, then a "
+                      f"seeded permutation): all {a['cores']} host cores took {a['rows']} rows "
+                      f"({a['tiles']} kept tiles) in {a['seconds']} s, one core took "
+                      f"{res['single']['rows']} rows ({res['single']['tiles']} tiles) in "
+                      f"{res['single']['seconds']} s; quantisation + traversal + fp64 attention"}
 
 
 # ----------------------------------------------------------------------------- main
@@ -488,15 +649,19 @@ def reference_arm(args, world, rank):
     if rank != 0:
         return
     from tile_routed_mixed_causal_b200 import workloads as wl
+    import oracle
     w = wl.bitmask_32k()
     t = wl.make_inputs(w, "cpu")
     nt = w.ntiles
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
     cycle = [nt // 4, nt // 3, nt // 2, nt // 5]
+    rows_of = lambda i: [(cycle[i % len(cycle)] + 7 * j) % nt for j in range(cores)]
     for i in range(args.warmup):
-        oracle_sample(w, t["q"], t["k"], t["v"], [cycle[i % len(cycle)]])
+        oracle_sample(w, t["q"], t["k"], t["v"], rows_of(i))
     ops = secs = tiles = 0
     for i in range(args.steps):
-        o, s, tl = oracle_sample(w, t["q"], t["k"], t["v"], [cycle[i % len(cycle)]])
+        o, s, tl = oracle_sample(w, t["q"], t["k"], t["v"], rows_of(i))
         ops += o
         secs += s
         tiles += tl
@@ -508,9 +673,10 @@ def reference_arm(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": 1, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
                    "seq_len": w.lengths[0], "G": w.G, "bf16_bit_fraction": 0.25},
-        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"one q-tile row of head 0 per step ({tiles} kept tiles over "
-                                   f"{args.steps} steps), quantisation + traversal + fp64 attention"},
+        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{cores} q-tile rows of head 0 per step, one per core "
+                                   f"({tiles} kept tiles over {args.steps} steps), quantisation + "
+                                   f"traversal + fp64 attention"},
         "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -532,6 +698,11 @@ def main():
     if args.only == "decode":
         if rank == 0:
             print(json.dumps({"only": "decode", **decode_bench(device, args.decode_passes, stream,
+                                                              hbm_gbs)}), flush=True)
+        return
+    if args.only == "hybrid":
+        if rank == 0:
+            print(json.dumps({"only": "hybrid", **hybrid_bench(device, args.decode_passes, stream,
                                                               hbm_gbs)}), flush=True)
         return
     if args.only == "allocate":
@@ -577,10 +748,12 @@ def main():
     e2e_ms, h2d, d2h = run_prefill_e2e(S, args.e2e_steps, stream)
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_value = whole_job_value(world, ops, e2e_ms)
+    quant = quantize_bench(S, stream)
+    quant["frac_of_hbm"] = round(quant["GB/s"] / hbm_gbs, 4)
 
     dec = None
     if not args.no_decode:
-        del S["plan"]
+        S.pop("plan", None)
         torch.cuda.empty_cache()
         dec = decode_bench(device, args.decode_passes, stream, hbm_gbs)
         if world > 1:  # whole-job GB/s over the slowest rank's step time
@@ -589,6 +762,17 @@ def main():
             dec.update(value=round(gbs, 1), ms_per_token_step=round(ms_dec, 4))
             dec["roofline"].update(achieved=round(gbs / world, 1),
                                    frac=round(gbs / world / hbm_gbs, 4))
+
+    recs = alloc = hyb = None
+    if not args.no_decode:
+        torch.cuda.empty_cache()
+        hyb = hybrid_bench(device, args.decode_passes, stream, hbm_gbs)
+    if not args.no_workloads:
+        base_S = S.pop("plan", None)
+        del base_S
+        torch.cuda.empty_cache()
+        recs = workload_records(device, stream, bf16_tflops)
+        alloc = allocate_bench(device, stream)
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -627,12 +811,21 @@ def main():
                               f"int8 = 2x bf16 (nominal ratio)",
             },
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+                    "copies": "pinned host buffers, copy-in and copy-out streams double-buffered "
+                              "against the compute stream"},
             "gpu_launches": 3 * args.steps,
             "clocks": clk,
         }
+        line["quantize"] = quant
         if dec is not None:
             line["decode"] = dec
+        if recs is not None:
+            line["workloads"] = recs
+        if alloc is not None:
+            line["allocate"] = alloc
+        if hyb is not None:
+            line["hybrid_decode"] = hyb
         if base is not None:
             line["cpu_baseline"] = base
         print(json.dumps(line), flush=True)

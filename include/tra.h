@@ -110,6 +110,13 @@ typedef enum {
 #define TRA_FMT_K4 0x08u
 #define TRA_FMT_V8 0x10u
 #define TRA_FMT_V4 0x20u
+/* INT4 codes of Q / K expanded to the int8 values 16 x code, row-major [H][ntiles][64][d]:
+ * the tensor-core operand form the prefill streams for INT4 tiles (sm_100 has no integer
+ * 4-bit MMA, so INT4 tiles run as int8 MMAs on these; the factor 256 of a product is
+ * taken out of the INT4 scales exactly).  They share the sq4 / sk4 scales with Q4 / K4.
+ * The packed Q4 / K4 formats stay the compact cache for decoding. */
+#define TRA_FMT_Q4X 0x40u
+#define TRA_FMT_K4X 0x80u
 
 /* device status word bits */
 #define TRA_DEV_TIMEOUT 0x1      /* a bounded pipeline wait expired */
@@ -145,6 +152,7 @@ typedef struct {
   float* sk8;  float* sk4;          /* [Hkv][ntiles] */
   float* sv8;  float* sv4;
   uint32_t formats;                 /* TRA_FMT_* bits: which fields are present */
+  int8_t* q4x; int8_t* k4x;         /* [Hq|Hkv][ntiles][64][d]: 16 x INT4 code (TRA_FMT_Q4X/K4X) */
 } tra_qtiles;
 /* Code layout.  Rows are tokens of a 64-token tile; INT8 rows hold channel c in byte c,
  * as two's complement for Q8 and K8 and offset-binary (code + 128) for V8, which only
@@ -219,7 +227,8 @@ TRA_API tra_status build_tile_lists(const tra_shape* shape, const tra_policy* po
  * TileMix abstract: the high- and low-precision paths share one online-softmax
  * state.)
  * q/k/v: device bf16 as above; tiles: output of quantize_qkv_tiles (Q8/K8
- * always, Q4/K4 when the policy has INT4 tiles); row_ptr/entries: prefill
+ * always, Q4X/K4X and the INT4 scales when the policy has INT4 tiles);
+ * row_ptr/entries: prefill
  * lists; out: device bf16 [ntok][Hq][d]; lse: device float [Hq][ntok] natural-
  * log logsumexp of the scaled scores, or NULL.
  * Integer-accumulator dump (debug; n_dump = 0 disables): dump_coords device
@@ -289,23 +298,95 @@ TRA_API tra_status routed_attention_decode(const tra_shape* prefill_shape, const
  * routed_attention_decode, minus workspace/workspace_bytes.
  * Limits and rules:
  *  - problems needing more than TRA_NOALLOC_SCRATCH_BYTES of scratch
- *    (tra_decode_workspace_bytes(B, Hq, Hkv, d)) are rejected with
+ *    (tra_decode_workspace_bytes(B, Hq, Hkv, d)), or with
+ *    B * (Hkv + 1) > TRA_NOALLOC_MAX_COUNTERS, are rejected with
  *    TRA_ERR_UNSUPPORTED;
  *  - the first call on each device looks up the array's device address with
  *    that device current; make that first call before any stream capture;
  *  - all calls on a device share the one array, which keeps whatever the last
  *    call left there; calls whose kernels overlap on the GPU (for example on
  *    two streams at once) race on it and give wrong results, so issue them on
- *    one stream or otherwise order them.  No part of the array needs to start
- *    at zero.
+ *    one stream or otherwise order them;
+ *  - the array starts zero-filled (static storage).  Its first 64 KiB hold the
+ *    decode's per-(sequence, KV head) and per-sequence arrival counters, which
+ *    must be zero when a call starts; every call leaves them at zero again, and
+ *    for every accepted shape (B * (Hkv + 1) <= TRA_NOALLOC_MAX_COUNTERS) they
+ *    stay inside that area, so calls of different shapes may follow one another.
+ *    The partial results behind the counters are written before they are read.
  */
 #define TRA_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define TRA_NOALLOC_MAX_COUNTERS 16384
 
 TRA_API tra_status routed_attention_decode_noalloc(
     const tra_shape* prefill_shape, const tra_policy* policy, const uint16_t* q,
     const uint16_t* k_new, const uint16_t* v_new, const tra_qtiles* cache, const int32_t* row_ptr,
     const uint32_t* entries, uint16_t* k_tail, uint16_t* v_tail, int32_t* tail_len_dev,
     int32_t tail_cap, float softmax_scale, uint16_t* out, int32_t* status_dev, void* stream);
+
+/*
+ * Token-level hybrid (HyQuant Uses Hybrid Precision to Compress LLM Attention, "The
+ * observation behind the method" and "How HyQuant works": a small set of important
+ * key positions and a window of recent tokens keep high precision, the rest of the
+ * context is read from quantised storage; selection and the decode kernel run on the
+ * GPU).  Reading adopted here: per (sequence, KV head) the n = ceil(frac * T) prefix
+ * positions of largest importance (ties to the earlier position) and every key within
+ * `window` positions of the query keep bf16 K and V; all other prefix keys and values
+ * are read from their tile's INT4 codes (K4 / V4 of quantize_qkv_tiles) times the
+ * tile scale; queries stay bf16.  A decode query sits at position T + tail_len,
+ * after the prefix and the tail tokens before it.
+ * All arrays are caller-owned device memory:
+ *   sel_count int32 [B]                 n of each sequence (written by the selection)
+ *   sel_pos   int32 [B][Hkv][cap]       selected positions (0 .. T-1), ascending
+ *   sel_mask  uint64 [Hkv][ntiles]      bit c of tile kt: token kt*64 + c is selected
+ *   k_sel, v_sel bf16 [B][Hkv][cap][d]  K / V rows of the selected positions
+ *   k_win, v_win bf16 [B][Hkv][window][d] K / V of prefix tokens T - window .. T - 1
+ *                                       (rows before the sequence start are zero)
+ * cap >= tra_hybrid_capacity(shape, frac); window >= 0.
+ */
+typedef struct {
+  int32_t window;
+  int32_t cap;
+  int32_t* sel_count;
+  int32_t* sel_pos;
+  uint64_t* sel_mask;
+  uint16_t* k_sel;
+  uint16_t* v_sel;
+  uint16_t* k_win;
+  uint16_t* v_win;
+} tra_hybrid;
+
+/* max over sequences of ceil(frac * T); -1 for an invalid shape or frac outside [0, 1]. */
+TRA_API int32_t tra_hybrid_capacity(const tra_shape* shape, double frac);
+
+/*
+ * hybrid_select_tokens -- the high-precision side of the hybrid cache.  importance:
+ * device float [ntok][Hkv] (finite), one score per key position and KV head (the
+ * signal that marks "vertical lines"; synthetic in this library's tests);
+ * k, v: device bf16 [ntok][Hkv][d].  Writes every array of *hy (layouts above).
+ * TRA_ERR_INVALID for bad pointers, frac outside [0, 1], window < 0;
+ * TRA_ERR_BUFFER if hy->cap is below tra_hybrid_capacity.
+ */
+TRA_API tra_status hybrid_select_tokens(const tra_shape* shape, const float* importance, double frac,
+                                        const uint16_t* k, const uint16_t* v, const tra_hybrid* hy,
+                                        void* stream);
+
+/*
+ * hybrid_attention_decode -- one decode step of the token-level hybrid: every prefix
+ * tile of (b, kv-head) is streamed in INT4 (cache: K4 / V4 and their scales) with
+ * its selected and in-window keys masked out, those keys are read from the bf16 side
+ * arrays of *hy instead, and the bf16 tail (earlier decode tokens and the new one,
+ * appended at tail position tail_len[b]) is attended as in routed_attention_decode;
+ * one softmax per query head; then tail_len[b] is incremented.  Arguments as
+ * routed_attention_decode (same workspace size and rules), with *hy from
+ * hybrid_select_tokens on the same shape.  Hq / Hkv <= 8.
+ */
+TRA_API tra_status hybrid_attention_decode(const tra_shape* prefill_shape, const tra_hybrid* hy,
+                                           const uint16_t* q, const uint16_t* k_new,
+                                           const uint16_t* v_new, const tra_qtiles* cache,
+                                           uint16_t* k_tail, uint16_t* v_tail, int32_t* tail_len_dev,
+                                           int32_t tail_cap, float softmax_scale, uint16_t* out,
+                                           void* workspace, size_t workspace_bytes,
+                                           int32_t* status_dev, void* stream);
 
 /* Complete-tile counts of one head's boundary pair over a batch (TriAttention
  * abstract: candidate boundary pairs are weighed by complete-tile execution costs):

@@ -232,3 +232,32 @@ def test_mixed_policy_needs_its_bitmask(lib):
     rows, nnz = L.tile_lists_size(s, pol, L.LISTS_PREFILL)
     st = lib.build_tile_lists(s.c, pol.c, L.LISTS_PREFILL, FAKE, rows + 1, FAKE, nnz, None)
     assert st == 1 and b"bitmask" in lib.tra_last_error()
+
+
+def test_hybrid_capacity_and_validation(lib):
+    """Token-level hybrid: the selected-token capacity is max_b ceil(frac * T_b) (in double,
+    as the oracle computes it); bad fractions, windows and short capacities are rejected
+    before any launch."""
+    lengths = [300, 64, 1, 257]
+    s = _shape(lengths)
+    for frac in (0.0, 0.05, 0.2, 1.0, 1.0 / 3.0):
+        want = max(min(T, int(np.ceil(frac * T))) for T in lengths)
+        assert lib.tra_hybrid_capacity(s.c, frac) == want
+    assert lib.tra_hybrid_capacity(s.c, -0.1) == -1
+    assert lib.tra_hybrid_capacity(s.c, 1.5) == -1
+    cap = lib.tra_hybrid_capacity(s.c, 0.05)
+    hy = L._Hybrid(128, cap, *([1 << 20] * 7))
+    hy.cap = cap - 1            # (only calls that validation rejects: nothing is launched)
+    st = lib.hybrid_select_tokens(s.c, FAKE, ctypes.c_double(0.05), FAKE, FAKE, ctypes.byref(hy), None)
+    assert st == 3 and b"cap" in lib.tra_last_error()
+    hy.cap, hy.window = cap, -1
+    st = lib.hybrid_select_tokens(s.c, FAKE, ctypes.c_double(0.05), FAKE, FAKE, ctypes.byref(hy), None)
+    assert st == 1 and b"window" in lib.tra_last_error()
+    hy.window = 128
+    st = lib.hybrid_select_tokens(s.c, FAKE, ctypes.c_double(1.5), FAKE, FAKE, ctypes.byref(hy), None)
+    assert st == 1 and b"frac" in lib.tra_last_error()
+    # decode: K4 / V4 cache tiles are required
+    qt = L._QTiles(*([None] * 12), L.FMT_K8 | L.FMT_V8)
+    args = [s.c, ctypes.byref(hy), FAKE, FAKE, FAKE, ctypes.byref(qt), FAKE, FAKE, FAKE, 4, 0.1,
+            FAKE, FAKE, 1 << 30, FAKE, None]
+    assert lib.hybrid_attention_decode(*args) == 1 and b"K4" in lib.tra_last_error()

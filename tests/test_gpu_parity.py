@@ -116,11 +116,15 @@ def _run_prefill(c: Case, with_lse=True):
 @pytest.mark.parametrize("w", SMALL[:5], ids=lambda w: w.name)
 def test_quantize_bit_exact(w):
     c = Case(w)
-    qt = tra.QTiles(c.shape, 0x3F)
+    qt = tra.QTiles(c.shape, 0xFF)
     tra.quantize_qkv_tiles(c.shape, c.q, c.k, c.v, qt)
     torch.cuda.synchronize()
     for name, bits in (("q", c.qb), ("k", c.kb), ("v", c.vb)):
         x8, x4, s8, s4 = oracle.quantize(bits, w.cu_seqlens)
+        if name != "v":  # INT4 codes in the int8 operand form: 16 x the signed code
+            nib = np.stack([x4 & 0xF, x4 >> 4], -1).reshape(*x4.shape[:-1], -1).astype(np.int16)
+            codes = np.where(nib >= 8, nib - 16, nib)
+            assert np.array_equal(qt[name + "4x"].cpu().numpy().astype(np.int16), 16 * codes), name + "4x"
         got8 = qt[name + "8"].cpu().numpy()
         if name == "v":  # V8 is stored offset-binary: code + 128
             got8 = (got8.view(np.uint8) ^ 0x80).view(np.int8)
@@ -161,13 +165,16 @@ def test_lists_bit_exact(w):
     rp, en = c.oracle_lists()
     assert np.array_equal(plan.row_ptr.cpu().numpy(), rp)
     assert np.array_equal(to_np_u32(plan.entries)[:plan.nnz], en)
-    if w.mode in ("boundary", "mixed"):  # decode caches follow the boundaries
-        dp = api.DecodePlan(c.shape, c.policy, None, 4)
-        dp.build()
-        torch.cuda.synchronize()
+    # decode caches follow the boundaries; a bitmask-only policy caches every tile in INT8
+    dp = api.DecodePlan(c.shape, c.policy, None, 4)
+    dp.build()
+    torch.cuda.synchronize()
+    if w.mode in ("boundary", "mixed"):
         rp, en = oracle.lists_decode(w.cu_seqlens, w.Hq, w.Hkv, w.b1, w.b2)
-        assert np.array_equal(dp.row_ptr.cpu().numpy(), rp)
-        assert np.array_equal(to_np_u32(dp.entries)[:dp.nnz], en)
+    else:
+        rp, en = oracle.lists_decode(w.cu_seqlens, w.Hq, w.Hkv)
+    assert np.array_equal(dp.row_ptr.cpu().numpy(), rp)
+    assert np.array_equal(to_np_u32(dp.entries)[:dp.nnz], en)
 
 
 # ---------------------------------------------------------------- prefill
@@ -241,6 +248,94 @@ def test_prefill_integer_accumulator_dump():
         else:
             ref = oracle.int_tile(prec, q4t=qz.q4[h, qt], k4t=qz.k4[h, kt])
         assert np.array_equal(dump[i].cpu().numpy(), ref), (h, qt, kt, prec)
+
+
+def _dump_coords(c: Case, rows_hq, per_prec=6, limit=64):
+    """Dump coordinates (b, h, qt, kt) for integer tiles of the oracle's lists at the given
+    (h, b, qt) rows: up to per_prec INT8 and per_prec INT4 entries per row (first, last and
+    evenly spread between), at most `limit` in all."""
+    w = c.w
+    rp, en = c.oracle_lists()
+    off = np.concatenate([[0], np.cumsum(w.tiles_per_seq)])
+    coords = []
+    for h, b, qt in rows_hq:
+        row = h * int(off[-1]) + int(off[b]) + qt
+        ent = en[rp[row]:rp[row + 1]]
+        for prec in (oracle.INT8, oracle.INT4):
+            sel = ent[(ent >> 28) == prec]
+            if len(sel) == 0:
+                continue
+            idx = np.unique(np.linspace(0, len(sel) - 1, min(per_prec, len(sel))).astype(int))
+            for i in idx:
+                coords.append((b, h, qt, int(sel[i] & 0x0FFFFFFF), prec))
+    return coords[:limit]
+
+
+def _check_dump(c: Case, coords, gen_device="cpu"):
+    """Run the prefill with an integer dump of `coords`; every dumped tile must equal the
+    oracle's own int32 Q-code x K-code^T product bit for bit."""
+    w = c.w
+    plan = api.PrefillPlan(c.shape, c.policy)
+    plan.quantize(c.q, c.k, c.v)
+    plan.lists()
+    dc = torch.tensor([x[:4] for x in coords], dtype=torch.int32, device="cuda")
+    dump = torch.full((len(coords), 64, 64), -7, dtype=torch.int32, device="cuda")
+    out = torch.zeros_like(c.q)
+    plan.attend(c.q, c.k, c.v, out, dump_coords=dc, dump_out=dump)
+    torch.cuda.synchronize()
+    assert int(plan.status.item()) == 0
+    qz = oracle.Quantised(c.qb, c.kb, None, w.cu_seqlens)
+    off = np.concatenate([[0], np.cumsum(w.tiles_per_seq)])
+    got = dump.cpu().numpy()
+    for i, (b, h, qt, kt, prec) in enumerate(coords):
+        gq, gk = int(off[b]) + qt, int(off[b]) + kt
+        kvh = h // (w.Hq // w.Hkv)
+        if prec == oracle.INT8:
+            ref = oracle.int_tile(prec, q8t=qz.q8[h, gq], k8t=qz.k8[kvh, gk])
+        else:
+            ref = oracle.int_tile(prec, q4t=qz.q4[h, gq], k4t=qz.k4[kvh, gk])
+        # rows past the sequence end hold no query: the kernel writes only valid rows
+        n = min(64, w.lengths[b] - qt * 64)
+        assert np.array_equal(got[i, :n], ref[:n]), (b, h, qt, kt, prec)
+    return out
+
+
+DUMP_FULL = {
+    # d = 128 at full size: INT8 and INT4 tiles (128-byte swizzle, INT4 as 16 x code)
+    "llama8b_8k": (wl.llama8b_8k, [(0, 0, 127), (13, 0, 64), (31, 0, 9), (7, 0, 126)]),
+    "bitmask_32k": (wl.bitmask_32k, [(0, 0, 511), (17, 0, 300), (31, 0, 3)]),
+    "mixed_8k": (wl.mixed_8k, [(0, 0, 127), (21, 0, 70), (31, 0, 5), (9, 0, 100)]),
+    "varlen": (wl.varlen_8, [(0, 0, 20), (27, 3, 5), (13, 7, 0)]),
+}
+
+
+@pytest.mark.parametrize("name", list(DUMP_FULL))
+def test_prefill_integer_dump_full_size(name):
+    """Bit-exact int32 accumulators of sampled INT8 / INT4 tiles at full size (d = 128) under
+    boundary, bitmask and mixed policies, in the launch configuration the benchmark uses."""
+    make, rows = DUMP_FULL[name]
+    w = make()
+    c = Case(w, gen_device="cuda")
+    rows = [(h, b, min(qt, w.tiles_per_seq[b] - 1)) for h, b, qt in rows]
+    coords = _dump_coords(c, rows)
+    assert any(x[4] == oracle.INT8 for x in coords)
+    if w.mode != "bitmask":
+        assert any(x[4] == oracle.INT4 for x in coords)
+    _check_dump(c, coords)
+
+
+@pytest.mark.parametrize("w", [x for x in SMALL if x.d == 128 and x.mode != "bitmask"] +
+                         [SMALL[6]], ids=lambda w: w.name)
+def test_prefill_integer_dump_small(w):
+    """Every integer tile of a few rows of the small d = 128 (and a d = 64 bitmask) cases."""
+    c = Case(w)
+    rows = []
+    for h in range(min(w.Hq, 4)):
+        for b, nt in enumerate(w.tiles_per_seq):
+            rows.append((h, b, nt - 1))
+    coords = _dump_coords(c, rows, per_prec=3)
+    if coords:
+        _check_dump(c, coords)
 
 
 def _sampled_rows(w, heads, qtiles_per_seq):
@@ -326,6 +421,72 @@ def test_decode_matches_oracle(w):
     assert np.array_equal(wl.bf16_bits(dp.k_tail[:, :, :w.decode_steps]), kt[:, :, :w.decode_steps])
 
 
+def _decode_vs_oracle(w, c, dp, qs, kn, vn, steps, cu_lists=None):
+    """Run `steps` decode steps and compare each with the oracle (full batch)."""
+    cu = w.cu_seqlens
+    ocache = oracle.Quantised(None, c.kb, c.vb, cu)
+    if w.mode == "bitmask":
+        rp, en = oracle.lists_decode(cu, w.Hq, w.Hkv)
+    else:
+        rp, en = oracle.lists_decode(cu, w.Hq, w.Hkv, w.b1, w.b2)
+    assert np.array_equal(dp.row_ptr.cpu().numpy(), rp)
+    assert np.array_equal(to_np_u32(dp.entries)[:dp.nnz], en)
+    kt = np.zeros((w.B, w.Hkv, w.tail_cap, w.d), np.uint16)
+    vt = np.zeros_like(kt)
+    out = torch.zeros((w.B, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
+    for step in range(steps):
+        dp.step(qs[step], kn[step], vn[step], out)
+        torch.cuda.synchronize()
+        kt[:, :, step] = wl.bf16_bits(kn[step])
+        vt[:, :, step] = wl.bf16_bits(vn[step])
+        ref = oracle.decode_step(wl.bf16_bits(qs[step]), cu, w.Hkv, ocache, rp, en, kt, vt,
+                                 np.full(w.B, step + 1, np.int32))
+        assert_close(out.float().cpu().numpy(), ref, f"{w.name} step {step}")
+    assert int(dp.status.item()) == 0
+
+
+def test_decode_after_bitmask_prefill():
+    """TileMix's INT8 K/V cache: a bitmask-policy prefill quantises K/V; its decode-cache
+    lists hold every tile in INT8 (no b1/b2); decode steps over that cache vs the oracle."""
+    w = wl.custom("bm_prefill_decode", [64 * 21 + 7, 64 * 9, 64 * 4], 8, 2, 128, 70, "bitmask",
+                  G=4, p_bf16=0.25, decode_steps=3, tail_cap=5)
+    c = Case(w)
+    plan = api.PrefillPlan(c.shape, c.policy, keep_v_cache=True)
+    out = torch.zeros_like(c.q)
+    plan.run(c.q, c.k, c.v, out)
+    dp = api.DecodePlan(c.shape, c.policy, plan.tiles, w.tail_cap)
+    dp.build()
+    qs, kn, vn = (x.cuda() for x in wl.make_decode_inputs(w, "cpu"))
+    torch.cuda.synchronize()
+    assert int(plan.status.item()) == 0
+    _decode_vs_oracle(w, c, dp, qs, kn, vn, w.decode_steps)
+
+
+@pytest.mark.parametrize("where", ["every_head", "one_group"])
+def test_decode_query_high_dynamic_range(where):
+    """Queries whose channels span far more than 2^7 within a head: per head one channel
+    x 1e3 (or x 30) and several x 1e-3.  The decode must still follow the bf16 query
+    within the output tolerance.  one_group: only the heads of (sequence 0, KV head 0)
+    get such a query, so that one step mixes groups of small and large queries."""
+    w = wl.custom("dec_hdr", [64 * 40, 64 * 33 + 17], 8, 2, 128, 71, "boundary",
+                  b1=[3, 1, 9, 2, 1, 1, 4, 2], b2=[20, 5, 9, 30, 1, 2, 4, 16], decode_steps=3,
+                  tail_cap=4)
+    c, cache, dp, qs, kn, vn = _decode_case(w)
+    g = torch.Generator().manual_seed(123)
+    q = qs.float().cpu()
+    grp = w.Hq // w.Hkv
+    for h in range(w.Hq):
+        ch = torch.randperm(w.d, generator=g)[:7]
+        bs = slice(None) if where == "every_head" else slice(0, 1)
+        if where == "one_group" and h >= grp:
+            continue
+        q[:, bs, h, ch[0]] *= 1e3 if h % 2 == 0 else 30.0
+        q[:, bs, h, ch[1:]] *= 1e-3
+    qs = q.to(torch.bfloat16).cuda()
+    _decode_vs_oracle(w, c, dp, qs, kn, vn, w.decode_steps)
+    assert np.array_equal(dp.tail_len.cpu().numpy(), np.full(w.B, w.decode_steps))
+
+
 def test_decode_workspace_shared_across_shapes():
     """The decode's arrival counters sit at a fixed place of the workspace and every call
     leaves them at zero, so one zero-filled workspace serves two shapes in turn: steps of
@@ -370,9 +531,12 @@ def test_decode_tail_full_sets_status():
     assert torch.equal(out, first)
 
 
-def test_decode_full_size_sampled():
-    """Batch 16 over a 32K prefix, 64 steps as benchmarked; sampled sequences vs the oracle."""
-    w = wl.decode_32k()
+@pytest.mark.parametrize("literal", [False, True], ids=["headline", "literal_1_3"])
+def test_decode_full_size_sampled(literal):
+    """Batch 16 over a 32K prefix, 64 steps as benchmarked; sampled sequences vs the oracle.
+    literal: the cache of the (b1, b2) = (1, 3) rule for every head (INT8 tile 511, INT4
+    tiles 509-510 of each sequence); headline: the per-head HBM-sized cache."""
+    w = wl.decode_32k(literal=literal)
     c, cache, dp, qs, kn, vn = _decode_case(w, gen_device="cuda")
     out = torch.zeros((w.B, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
     check_steps = {0, 31, 63}

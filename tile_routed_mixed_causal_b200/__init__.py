@@ -13,7 +13,7 @@ from ._lib import (  # noqa: F401
     TraError, Shape, Policy, QTiles, load, quantize_qkv_tiles, tile_lists_size,
     build_tile_lists, routed_attention_prefill, routed_attention_decode,
     decode_workspace_bytes, PREC_INT4, PREC_INT8, PREC_BF16, POLICY_BOUNDARY, POLICY_BITMASK, POLICY_MIXED,
-    LISTS_PREFILL, LISTS_DECODE_CACHE, FMT_Q8, FMT_Q4, FMT_K8, FMT_K4, FMT_V8, FMT_V4,
+    LISTS_PREFILL, LISTS_DECODE_CACHE, FMT_Q8, FMT_Q4, FMT_K8, FMT_K4, FMT_V8, FMT_V4, FMT_Q4X, FMT_K4X,
     DEV_TIMEOUT, DEV_TAIL_FULL, DEV_BAD_LIST, tra_selftest_bounded_wait, boundary_tile_counts,
-    allocate_boundaries,
+    allocate_boundaries, Hybrid, hybrid_select_tokens, hybrid_attention_decode,
 )

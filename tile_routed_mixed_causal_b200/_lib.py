@@ -22,6 +22,7 @@ PREC_INT4, PREC_INT8, PREC_BF16 = 1, 2, 3
 POLICY_BOUNDARY, POLICY_BITMASK, POLICY_MIXED = 0, 1, 2
 LISTS_PREFILL, LISTS_DECODE_CACHE = 0, 1
 FMT_Q8, FMT_Q4, FMT_K8, FMT_K4, FMT_V8, FMT_V4 = 0x1, 0x2, 0x4, 0x8, 0x10, 0x20
+FMT_Q4X, FMT_K4X = 0x40, 0x80
 DEV_TIMEOUT, DEV_TAIL_FULL, DEV_BAD_LIST = 0x1, 0x2, 0x4
 STATUS = {0: "TRA_OK", 1: "TRA_ERR_INVALID", 2: "TRA_ERR_UNSUPPORTED", 3: "TRA_ERR_BUFFER",
           4: "TRA_ERR_CUDA", 5: "TRA_ERR_TIMEOUT"}
@@ -44,10 +45,16 @@ class _Policy(ctypes.Structure):
                 ("bitmask_dev", ctypes.c_void_p), ("G", ctypes.c_int32), ("W", ctypes.c_int32)]
 
 
+class _Hybrid(ctypes.Structure):
+    _fields_ = [("window", ctypes.c_int32), ("cap", ctypes.c_int32)] + \
+               [(n, ctypes.c_void_p) for n in
+                ("sel_count", "sel_pos", "sel_mask", "k_sel", "v_sel", "k_win", "v_win")]
+
+
 class _QTiles(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("q8", "q4", "k8", "k4", "v8", "v4", "sq8", "sq4", "sk8", "sk4", "sv8", "sv4")] + \
-               [("formats", ctypes.c_uint32)]
+               [("formats", ctypes.c_uint32), ("q4x", ctypes.c_void_p), ("k4x", ctypes.c_void_p)]
 
 
 _lib = None
@@ -79,6 +86,9 @@ def load():
         "tra_selftest_bounded_wait": ([P, I64, P], I32),
         "tra_boundary_tile_counts": ([P, I32, I32, P, P], I32),
         "tra_allocate_boundaries": ([I32, I32, P, P, I64, P, P, P], I32),
+        "tra_hybrid_capacity": ([P, ctypes.c_double], I32),
+        "hybrid_select_tokens": ([P, P, ctypes.c_double, P, P, P, P], I32),
+        "hybrid_attention_decode": ([P, P, P, P, P, P, P, P, P, I32, F, P, P, SZ, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -198,10 +208,15 @@ class QTiles:
                 self.t["s" + name + "8"] = torch.zeros((H, nt), dtype=torch.float32, device=device)
             if formats & (FMT_Q4 << (2 * i)):
                 self.t[name + "4"] = torch.zeros((H, nt, TILE, d // 2), dtype=torch.uint8, device=device)
+            x4 = {"q": FMT_Q4X, "k": FMT_K4X}.get(name, 0)
+            if formats & x4:
+                self.t[name + "4x"] = torch.zeros((H, nt, TILE, d), dtype=torch.int8, device=device)
+            if formats & ((FMT_Q4 << (2 * i)) | x4):
                 self.t["s" + name + "4"] = torch.zeros((H, nt), dtype=torch.float32, device=device)
-        self._c = _QTiles(*[self.t[n].data_ptr() if n in self.t else None for n in
-                            ("q8", "q4", "k8", "k4", "v8", "v4",
-                             "sq8", "sq4", "sk8", "sk4", "sv8", "sv4")], formats)
+        ptr = lambda n: self.t[n].data_ptr() if n in self.t else None
+        self._c = _QTiles(*[ptr(n) for n in ("q8", "q4", "k8", "k4", "v8", "v4",
+                                             "sq8", "sq4", "sk8", "sk4", "sv8", "sv4")],
+                          formats, ptr("q4x"), ptr("k4x"))
 
     def __getitem__(self, k):
         return self.t[k]
@@ -265,6 +280,47 @@ def tra_selftest_bounded_wait(status, limit_ns: int, stream=None):
     """Diagnostic: a kernel whose mbarrier wait never completes must give up after
     limit_ns and OR DEV_TIMEOUT into the device int32 `status` (see include/tra.h)."""
     _check(load().tra_selftest_bounded_wait(_ptr(status), int(limit_ns), _stream(stream)))
+
+
+class Hybrid:
+    """Device arrays of the token-level hybrid's high-precision side (torch-allocated):
+    per (sequence, KV head) the ceil(frac * T) selected positions, their tile masks and
+    bf16 K / V rows, and the bf16 K / V of the last `window` prefix tokens."""
+
+    def __init__(self, shape: Shape, frac: float, window: int, device="cuda"):
+        cap = int(load().tra_hybrid_capacity(shape.c, float(frac)))
+        if cap < 0:
+            raise TraError(1, "invalid shape or frac")
+        B, Hkv, d, nt = shape.B, shape.Hkv, shape.d, shape.ntiles
+        self.frac, self.window, self.cap = float(frac), int(window), cap
+        c1, w1 = max(cap, 1), max(window, 1)
+        self.sel_count = torch.zeros(B, dtype=torch.int32, device=device)
+        self.sel_pos = torch.zeros((B, Hkv, c1), dtype=torch.int32, device=device)
+        self.sel_mask = torch.zeros((Hkv, max(nt, 1)), dtype=torch.int64, device=device)
+        self.k_sel = torch.zeros((B, Hkv, c1, d), dtype=torch.bfloat16, device=device)
+        self.v_sel = torch.zeros_like(self.k_sel)
+        self.k_win = torch.zeros((B, Hkv, w1, d), dtype=torch.bfloat16, device=device)
+        self.v_win = torch.zeros_like(self.k_win)
+        self._c = _Hybrid(self.window, cap, *[getattr(self, n).data_ptr() for n in
+                                             ("sel_count", "sel_pos", "sel_mask", "k_sel", "v_sel",
+                                              "k_win", "v_win")])
+
+    @property
+    def c(self):
+        return ctypes.byref(self._c)
+
+
+def hybrid_select_tokens(shape: Shape, importance, frac: float, k, v, hy: Hybrid, stream=None):
+    _check(load().hybrid_select_tokens(shape.c, _ptr(importance), float(frac), _ptr(k), _ptr(v),
+                                       hy.c, _stream(stream)))
+
+
+def hybrid_attention_decode(shape: Shape, hy: Hybrid, q, k_new, v_new, cache: QTiles, k_tail,
+                            v_tail, tail_len, softmax_scale, out, workspace, status, stream=None):
+    _check(load().hybrid_attention_decode(
+        shape.c, hy.c, _ptr(q), _ptr(k_new), _ptr(v_new), cache.c, _ptr(k_tail), _ptr(v_tail),
+        _ptr(tail_len), int(k_tail.shape[2]), float(softmax_scale), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
 
 
 def boundary_tile_counts(shape: Shape, b1: int, b2: int):

@@ -3,6 +3,9 @@
 ``PrefillPlan``: quantize_qkv_tiles -> build_tile_lists -> routed_attention_prefill.
 ``DecodePlan``:  build_tile_lists (decode-cache kind, once) -> routed_attention_decode
 per step, over the K/V tiles a PrefillPlan (or quantize_qkv_tiles) produced.
+``HybridDecodePlan``: hybrid_select_tokens (once, over the prefix) ->
+hybrid_attention_decode per step (token-level hybrid: INT4 tiles plus bf16 selected
+and recent tokens).
 Buffers are allocated once per plan; ``run``/``step`` only enqueue kernels.  The
 decode workspace is zero-filled once (the decode's arrival counters need that, and
 every step leaves them at zero).
@@ -22,7 +25,7 @@ class PrefillPlan:
         self.shape, self.policy = shape, policy
         fm = L.FMT_Q8 | L.FMT_K8
         if policy.has_int4:
-            fm |= L.FMT_Q4 | L.FMT_K4
+            fm |= L.FMT_Q4X | L.FMT_K4X     # INT4 codes in the tensor-core operand form
         if keep_v_cache:
             fm |= L.FMT_K4 | L.FMT_V8 | L.FMT_V4
         self.tiles = L.QTiles(shape, fm, device)
@@ -77,3 +80,26 @@ class DecodePlan:
         L.routed_attention_decode(self.shape, self.policy, q, k_new, v_new, self.cache,
                                   self.row_ptr, self.entries, self.k_tail, self.v_tail,
                                   self.tail_len, scale, out, self.workspace, self.status, stream)
+
+
+class HybridDecodePlan:
+    def __init__(self, shape: L.Shape, cache: L.QTiles, frac: float, window: int, tail_cap: int,
+                 device="cuda"):
+        self.shape, self.cache = shape, cache
+        self.hy = L.Hybrid(shape, frac, window, device)
+        B, Hkv, d = shape.B, shape.Hkv, shape.d
+        self.k_tail = torch.zeros((B, Hkv, tail_cap, d), dtype=torch.bfloat16, device=device)
+        self.v_tail = torch.zeros_like(self.k_tail)
+        self.tail_len = torch.zeros(B, dtype=torch.int32, device=device)
+        nbytes = L.decode_workspace_bytes(B, shape.Hq, Hkv, d)
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def select(self, importance, k, v, stream=None):
+        L.hybrid_select_tokens(self.shape, importance, self.hy.frac, k, v, self.hy, stream)
+
+    def step(self, q, k_new, v_new, out, scale=None, stream=None):
+        scale = 1.0 / math.sqrt(self.shape.d) if scale is None else scale
+        L.hybrid_attention_decode(self.shape, self.hy, q, k_new, v_new, self.cache, self.k_tail,
+                                  self.v_tail, self.tail_len, scale, out, self.workspace,
+                                  self.status, stream)

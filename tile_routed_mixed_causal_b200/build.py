@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libtra.so")
 BUILD = os.path.join(PKG, "_build")
 SOURCES = ["tra_api.cu", "quantize.cu", "lists.cu", "prefill.cu", "decode.cu",
-           "decode_noalloc.cu", "selftest.cu"]
+           "decode_noalloc.cu", "selftest.cu", "hybrid.cu"]
 HEADERS = ["tra_device.cuh", "tra_launch.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

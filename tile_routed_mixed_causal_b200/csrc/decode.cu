@@ -13,7 +13,7 @@
 // no block barrier and every cached byte is read once per group:
 //   scores: S^T = K Q^T on the tensor cores as integer MMAs (mma.sync m16n8k32,
 //           s8 x s8 -> s32): the K codes go in as they are stored (INT4 nibbles
-//           masked in place, worth 16 x code), q as a 16-bit fixed-point pair of
+//           masked in place, worth 16 x code), q as a 24-bit fixed-point triple of
 //           int8 limbs per head; K tiles fed by ldmatrix;
 //   softmax: per head over the warp's fragment lanes, K scale and 1/sqrt(d)
 //           folded into the exponent, V scale folded into P (f16, staged per warp);
@@ -23,6 +23,8 @@
 // tail keys on the CUDA cores, so the grid holds data splits only.  The four warps' states are merged per
 // CTA; the last split of each (sequence, KV head) to finish merges the splits
 // into the output, and the last such row of a sequence advances tail_len.
+#include <type_traits>
+
 #include "tra_device.cuh"
 #include "tra_launch.h"
 
@@ -32,6 +34,10 @@ namespace {
 constexpr int kConsumers = 4;
 constexpr int kDecThreads = 32 * (kConsumers + 1);
 constexpr int kDecStages = 6;
+// Two q limbs serve a CTA whose query heads all have max |q| < 2^kTwoLimbMaxE.  Measured
+// on a decode cache with x10 outlier K channels, the output error of two limbs against
+// exact q stays below about 1e-3 up to there and doubles with every further power of two.
+constexpr int kTwoLimbMaxE = 4;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -48,7 +54,7 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 
 // ---------------------------------------------------------------- mma.sync helpers
 // The GQA group's contractions run on the tensor cores.  Scores S^T = K Q^T are
-// m16n8k32 integer MMAs (M = 16 keys, N = 8 columns = 4 heads x 2 q limbs, exact
+// m16n8k32 integer MMAs (M = 16 keys, N = 8 columns of (head, q limb) pairs, exact
 // int32 accumulation); O^T += V^T P^T are m16n8k16 MMAs (f16 inputs, fp32
 // accumulation; M = 16 channels, N = 8 heads), whose V codes reach f16 exactly:
 // each biased byte / nibble becomes the low mantissa byte of 1024.0h, and one
@@ -147,10 +153,10 @@ struct DecCfg {
   static constexpr int kSmem = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
   static constexpr int kCh = D / 32;             // tail P V channels per lane
   static constexpr int kB8 = D / 16;             // 16-channel blocks of the O fragments
-  static constexpr int kQM = GRP > 4 ? 2 : 1;    // score MMAs per K fragment (4 heads each)
+  static constexpr int kQM = GRP > 4 ? 2 : 1;    // (hi, mid) limb MMAs per K fragment (4 heads each)
 };
 
-template <int D, int GRP>
+template <int D, int GRP, int NL, bool HYB>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     const DecodeParams p, const __grid_constant__ DecodeMaps m) {
   using C = DecCfg<D, GRP>;
@@ -173,6 +179,49 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   const int seq0 = __ldg(p.cu + b);
   const int T = __ldg(p.cu + b + 1) - seq0;
   const int toff = seq_tile_offset(p.cu, b);
+  // q of the group's heads as fp32 channel pairs q2[pair][g] (tail path and fragments)
+  for (int x = t; x < (D / 2) * GRP; x += kDecThreads) {
+    const int cp = x / GRP, gq = x % GRP;
+    float2 v = make_float2(0.0f, 0.0f);
+    if (gq < grp) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(
+          p.q + ((long long)b * p.Hq + kvh * grp + gq) * D + 2 * cp);
+      v = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    }
+    q2[cp * GRP + gq] = v;
+  }
+  __syncthreads();
+  // q of head h as a fixed-point integer Q of NL int8 limbs (balanced base-256
+  // digits) times the power of two 2^(E_h - F), where 2^E_h > max_c |q_h[c]|:
+  //   NL = 2, F = 14:   Q = 256 hi + lo, |Q| <= 2^14; a channel is off by at most
+  //                    2^(E_h - 15) (exact within 2^7 of the head's largest |q|);
+  //   NL = 3, F = 22:   Q = 65536 hi + 256 mid + lo, |Q| <= 2^22, off by at most
+  //                    2^(E_h - 23) (exact within 2^15 of the largest |q|).
+  // The error of two limbs grows with |q| in absolute terms, so they serve only groups
+  // whose heads all have max |q| < 2^kTwoLimbMaxE.  Every step launches the kernel for
+  // both limb counts; each (sequence, KV head) group takes part in exactly one of them,
+  // and a CTA of the other leaves here, before it touches the tail or any counter.
+  int* const qe = reinterpret_cast<int*>(sm + C::kOffE);
+  for (int hd = warp; hd < GRP; hd += kConsumers + 1) {
+    float mx = 0.0f;
+    for (int cp = lane; cp < D / 2; cp += 32) {
+      const float2 v = q2[cp * GRP + hd];
+      mx = fmaxf(mx, fmaxf(fabsf(v.x), fabsf(v.y)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    int e = 0;
+    frexpf(mx, &e);  // mx = f 2^e with f in [0.5, 1), or e = 0 for mx = 0
+    if (lane == 0) qe[hd] = e;
+  }
+  __syncthreads();
+  {
+    bool three = false;
+    for (int hd = 0; hd < grp; ++hd) three |= qe[hd] > kTwoLimbMaxE;
+    if (three != (NL == 3)) return;  // uniform over the CTA
+  }
+  constexpr int F = NL == 3 ? 22 : 14;             // fraction bits of Q
+  constexpr int QL = NL == 3 ? C::kQM + 1 : C::kQM;  // score MMAs per K fragment
   const int tl = __ldg(p.tail_len + b);
   if (tl >= p.tail_cap) {  // every CTA of sequence b leaves: output and tail untouched
     if (tail_cta && kvh == 0 && t == 0) atomicOr(p.status, TRA_DEV_TAIL_FULL);
@@ -180,12 +229,21 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   }
   int my0 = 0, ntile = 0;
   {
-    const long long row = (long long)b * p.Hkv + kvh;
-    const int rs = __ldg(p.row_ptr + row), re = __ldg(p.row_ptr + row + 1);
-    const int n = re - rs;
+    // cached tiles of (b, kvh): the decode-cache list row, or (hybrid) every prefix
+    // tile in INT4, my0 then being the split's first k-tile
+    int rs = 0, n = (T + kTile - 1) / kTile;
+    if (!HYB) {
+      const long long row = (long long)b * p.Hkv + kvh;
+      rs = __ldg(p.row_ptr + row);
+      n = __ldg(p.row_ptr + row + 1) - rs;
+    }
     my0 = rs + (int)((long long)n * split / nsplit);
     ntile = rs + (int)((long long)n * (split + 1) / nsplit) - my0;
   }
+  // entry i of this split: (precision << 28) | kt
+  auto entry_of = [&](int i) -> uint32_t {
+    return HYB ? ((uint32_t)TRA_PREC_INT4 << 28) | (uint32_t)(my0 + i) : __ldg(p.entries + my0 + i);
+  };
   // barriers first, so that the producer's first copies overlap the consumers' set-up
   if (t == 0) {
     for (int s = 0; s < kDecStages; ++s) {
@@ -204,7 +262,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       for (int i = 0; i < ntile; ++i) {
         const int s = i % kDecStages, use = i / kDecStages;
         if (use > 0 && !mbar_wait(bar_empty + s * 8, (use - 1) & 1, err)) break;
-        const uint32_t e = __ldg(p.entries + my0 + i);
+        const uint32_t e = entry_of(i);
         const int kt = (int)(e & 0x0FFFFFFFu);
         const int r0 = (kvh * p.ntiles + toff + kt) * kTile;
         const uint32_t dst = base + s * C::kStageBytes;
@@ -240,17 +298,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         p.v_tail[dst + c] = p.v_new[src + c];
       }
     }
-    // q of the group's heads as fp32 channel pairs q2[pair][g] (tail path and fragments)
-    for (int x = t; x < (D / 2) * GRP; x += 32 * kConsumers) {
-      const int cp = x / GRP, gq = x % GRP;
-      float2 v = make_float2(0.0f, 0.0f);
-      if (gq < grp) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(
-            p.q + ((long long)b * p.Hq + kvh * grp + gq) * D + 2 * cp);
-        v = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-      }
-      q2[cp * GRP + gq] = v;
-    }
     // zero the P rows of padded heads (never written; N = 8 heads per MMA)
     {
       __half* pz = reinterpret_cast<__half*>(sm + C::kOffP);
@@ -258,71 +305,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     }
     asm volatile("bar.sync 3, %0;" ::"n"(32 * kConsumers) : "memory");  // consumers only
     const int g = lane >> 2, tq = lane & 3;  // fragment group / thread in group
-    // q of head h as a 16-bit fixed-point integer Q = 256 hi + lo (hi, lo int8)
-    // times the power of two 2^(E_h - 14), where 2^E_h > max_c |q_h[c]|:
-    // |Q| <= 2^14, and each channel is off by at most 2^(E_h - 15), i.e. 2^-14 of
-    // the head's largest |q| (exact for every channel within 2^7 of it).
-    int* const qe = reinterpret_cast<int*>(sm + C::kOffE);
-    for (int hd = warp; hd < GRP; hd += kConsumers) {
-      float mx = 0.0f;
-      for (int cp = lane; cp < D / 2; cp += 32) {
-        const float2 v = q2[cp * GRP + hd];
-        mx = fmaxf(mx, fmaxf(fabsf(v.x), fabsf(v.y)));
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      int e = 0;
-      frexpf(mx, &e);  // mx = f 2^e with f in [0.5, 1), or e = 0 for mx = 0
-      if (lane == 0) qe[hd] = e;
-    }
-    asm volatile("bar.sync 3, %0;" ::"n"(32 * kConsumers) : "memory");
-    // limb `limb` (0: hi, 1: lo) of head hd's Q at channel c; 0 for padded heads
-    auto q_limb = [&](int hd, int limb, int c) -> uint32_t {
-      if (hd >= grp) return 0u;
-      const float2 v = q2[(c >> 1) * GRP + hd];
-      const int Q = __float2int_rn(ldexpf(c & 1 ? v.y : v.x, 14 - qe[hd]));
-      const int hi = (Q + 128) >> 8;
-      return (uint32_t)((limb ? Q - 256 * hi : hi) & 0xFF);
-    };
-    auto pack4 = [&](int hd, int limb, int c, int step) -> uint32_t {
-      return q_limb(hd, limb, c) | q_limb(hd, limb, c + step) << 8 |
-             q_limb(hd, limb, c + 2 * step) << 16 | q_limb(hd, limb, c + 3 * step) << 24;
-    };
-    // B fragments (column g = head (g >> 1) + 4 mq, limb g & 1, so that lane tq's
-    // accumulator columns 2tq, 2tq + 1 are both limbs of head tq + 4 mq), in the
-    // channel order the K codes arrive in:
-    //   INT8, 32-channel block cb: k = 4t + i -> channel 32cb + 4t + i, k = 16 + 4t + i
-    //         -> 32cb + 16 + 4t + i
-    //   INT4, 32-channel block 2cb + h: k = 4t + i -> even channel 64cb + 32h + 8t + 2i,
-    //         k = 16 + 4t + i -> the odd channel after it
-    uint32_t qi8[D / 32][C::kQM][2], qi4[D / 64][2][C::kQM][2];
-#pragma unroll
-    for (int mq = 0; mq < C::kQM; ++mq) {
-      const int hc = (g >> 1) + 4 * mq, limb = g & 1;
-#pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
-        qi8[cb][mq][0] = pack4(hc, limb, 32 * cb + 4 * tq, 1);
-        qi8[cb][mq][1] = pack4(hc, limb, 32 * cb + 16 + 4 * tq, 1);
-      }
-#pragma unroll
-      for (int cb = 0; cb < D / 64; ++cb)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          qi4[cb][h][mq][0] = pack4(hc, limb, 64 * cb + 32 * h + 8 * tq, 2);
-          qi4[cb][h][mq][1] = pack4(hc, limb, 64 * cb + 32 * h + 8 * tq + 1, 2);
-        }
-    }
-    // Softmax heads of this lane ("slots"): tq + 4 mq, score = Q-limb integer product
-    // x 2^(E - 14).  O heads of this lane: 2tq, 2tq + 1 (the P V MMA's columns).
-    float qsig[C::kQM];
     bool real[C::kQM];
 #pragma unroll
-    for (int mq = 0; mq < C::kQM; ++mq) {
-      const int hd = tq + 4 * mq;
-      real[mq] = hd < grp;
-      qsig[mq] = real[mq] ? ldexpf(1.0f, qe[hd] - 14) : 0.0f;
-    }
-
+    for (int mq = 0; mq < C::kQM; ++mq) real[mq] = tq + 4 * mq < grp;
     // softmax state per slot (l_run: this lane's partial sum over its keys, reduced
     // over the lanes once at the end); O^T fragments o8[j]: channels 16j + 2g (rows g) and
     // 16j + 2g + 1 (rows g + 8), for INT8 and INT4 tiles alike (the V4 cache is stored
@@ -353,20 +338,22 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     for (int cb = 0; cb < D / 64; ++cb)
       off4[cb] = swz<C::kRow4>(mrow + 8 * (mj & 1), 2 * cb + (mj >> 1));
 
-    // bf16 tail (tail CTA): tokens [0, tl) of the tail buffer and the new token at
-    // tl; warp w takes tokens w, w + kConsumers, ..., one per lane, with CUDA-core fp32 math
+    // bf16 rows: the tail (tail CTA: tokens [0, tl) of the tail buffer and the new
+    // token at tl) and, for the hybrid, the split's share of the selected and in-window
+    // prefix rows.  row(x, kr, vr) gives row x's K and V and whether it takes part.
+    // Warp w takes rows w, w + kConsumers, ..., one per lane, with CUDA-core fp32 math
     // and its own softmax state.  All of a lane's loads are issued before use.
-    auto tail_pass = [&](float (&tm)[GRP], float (&tlsum)[GRP], float2 (&to)[GRP][C::kCh / 2]) {
-      const long long tbase = ((long long)b * p.Hkv + kvh) * p.tail_cap;
-      const long long nbase = ((long long)b * p.Hkv + kvh) * D;
-      for (int c0 = 0; warp + kConsumers * c0 <= tl; c0 += 32) {  // this warp's next 32 tokens
-        const int pos = warp + kConsumers * (c0 + lane);
-        const bool valid = pos <= tl;
+    auto row_pass = [&](int count, auto row, float (&tm)[GRP], float (&tlsum)[GRP],
+                        float2 (&to)[GRP][C::kCh / 2]) {
+      for (int c0 = 0; warp + kConsumers * c0 < count; c0 += 32) {  // this warp's next 32 rows
+        const int x = warp + kConsumers * (c0 + lane);
+        const uint16_t* kr = nullptr;
+        const uint16_t* vr0 = nullptr;
+        const bool valid = x < count && row(x, kr, vr0);
         float2 acc[GRP];
 #pragma unroll
         for (int gg = 0; gg < GRP; ++gg) acc[gg] = make_float2(0.0f, 0.0f);
         if (valid) {
-          const uint16_t* kr = pos == tl ? p.k_new + nbase : p.k_tail + (tbase + pos) * D;
           uint4 kw[D / 8];
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) kw[c] = *reinterpret_cast<const uint4*>(kr + c * 8);
@@ -405,12 +392,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 #pragma unroll
           for (int k = 0; k < C::kCh / 2; ++k)
             to[gg][k] = __fmul2_rn(to[gg][k], make_float2(al[gg], al[gg]));
-        // P V: this lane's channels lane * kCh .. + kCh, tokens of the chunk in order
-        const int nk = min(32, (tl - warp) / kConsumers - c0 + 1);
+        // P V: this lane's channels lane * kCh .. + kCh, rows of the chunk in order
+        const int nk = min(32, (count - 1 - warp) / kConsumers - c0 + 1);
 #pragma unroll 4
         for (int j = 0; j < nk; ++j) {
           const int pj = warp + kConsumers * (c0 + j);
-          const uint16_t* vr = pj == tl ? p.v_new + nbase : p.v_tail + (tbase + pj) * D;
+          const uint16_t* kr_unused = nullptr;
+          const uint16_t* vr = nullptr;
+          if (!row(pj, kr_unused, vr)) continue;  // (uniform over the warp)
           uint32_t vw[C::kCh / 2];
 #pragma unroll
           for (int k = 0; k < C::kCh / 2; ++k)
@@ -429,6 +418,56 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     };
 
     bool ok = true;
+    // limb `limb` of head hd's Q at channel c (two limbs: 0 hi, 1 lo; three: 0 hi,
+    // 1 mid, 2 lo; each in [-128, 127]); 0 for padded heads
+    auto q_limb = [&](int hd, int limb, int c) -> uint32_t {
+      if (hd >= grp) return 0u;
+      const float2 v = q2[(c >> 1) * GRP + hd];
+      const int Q = __float2int_rn(ldexpf(c & 1 ? v.y : v.x, F - qe[hd]));
+      const int lo = ((Q + 128) & 0xFF) - 128;
+      const int q1 = (Q - lo) >> 8;
+      if (NL == 2) return (uint32_t)((limb == 0 ? q1 : lo) & 0xFF);
+      const int mid = ((q1 + 128) & 0xFF) - 128;
+      const int hi = (q1 - mid) >> 8;
+      return (uint32_t)((limb == 0 ? hi : limb == 1 ? mid : lo) & 0xFF);
+    };
+    auto pack4 = [&](int hd, int limb, int c, int step) -> uint32_t {
+      return q_limb(hd, limb, c) | q_limb(hd, limb, c + step) << 8 |
+             q_limb(hd, limb, c + 2 * step) << 16 | q_limb(hd, limb, c + 3 * step) << 24;
+    };
+    // B fragments.  MMA mq < kQM: column g = (head (g >> 1) + 4 mq, limb g & 1), so
+    // lane tq's accumulator columns 2tq, 2tq + 1 are the first two limb products (hi,
+    // lo for two limbs; hi, mid for three) of head tq + 4 mq.  With three limbs, MMA
+    // kQM: column g = lo limb of head (g >> 1) + 4 (g & 1), so lane tq's columns hold
+    // the lo products of heads tq and tq + 4.
+    // Channel order as the K codes arrive:
+    //   INT8, 32-channel block cb: k = 4t + i -> channel 32cb + 4t + i, k = 16 + 4t + i
+    //         -> 32cb + 16 + 4t + i
+    //   INT4, 32-channel block 2cb + h: k = 4t + i -> even channel 64cb + 32h + 8t + 2i,
+    //         k = 16 + 4t + i -> the odd channel after it
+    uint32_t qi8[D / 32][QL][2], qi4[D / 64][2][QL][2];
+  #pragma unroll
+    for (int mq = 0; mq < QL; ++mq) {
+      const bool lo_mma = NL == 3 && mq == C::kQM;
+      const int hc = lo_mma ? (g >> 1) + 4 * (g & 1) : (g >> 1) + 4 * mq;
+      const int limb = lo_mma ? 2 : (g & 1);
+  #pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        qi8[cb][mq][0] = pack4(hc, limb, 32 * cb + 4 * tq, 1);
+        qi8[cb][mq][1] = pack4(hc, limb, 32 * cb + 16 + 4 * tq, 1);
+      }
+  #pragma unroll
+      for (int cb = 0; cb < D / 64; ++cb)
+  #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          qi4[cb][h][mq][0] = pack4(hc, limb, 64 * cb + 32 * h + 8 * tq, 2);
+          qi4[cb][h][mq][1] = pack4(hc, limb, 64 * cb + 32 * h + 8 * tq + 1, 2);
+        }
+    }
+    float qsig[C::kQM];  // 2^(E - F) of the lane's softmax heads tq + 4 mq
+#pragma unroll
+    for (int mq = 0; mq < C::kQM; ++mq)
+      qsig[mq] = real[mq] ? ldexpf(1.0f, qe[tq + 4 * mq] - F) : 0.0f;
     for (int i = warp; i < ntile; i += kConsumers) {
       const int s = i % kDecStages;
       // Stage s last held tile i - kDecStages, which another warp consumes.  A
@@ -441,7 +480,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       if (i >= kDecStages &&
           !mbar_wait(bar_empty + s * 8, ((i / kDecStages) - 1) & 1, err)) { ok = false; break; }
       if (!mbar_wait(bar_full + s * 8, (i / kDecStages) & 1, err)) { ok = false; break; }
-      const uint32_t e = __ldg(p.entries + my0 + i);
+      const uint32_t e = entry_of(i);
       const int kt = (int)(e & 0x0FFFFFFFu);
       const long long tile = (long long)kvh * p.ntiles + toff + kt;
       const int nvalid = min(kTile, T - kt * kTile);
@@ -450,59 +489,84 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       const bool is8 = (e >> 28) == TRA_PREC_INT8;
 
       // ---- scores: si[mq][k] = S^T fragment of keys 16k + (g, g+8), columns (2tq, 2tq+1)
-      int si[C::kQM][4][4];
-#pragma unroll
-      for (int mq = 0; mq < C::kQM; ++mq)
-#pragma unroll
+      int si[QL][4][4];
+  #pragma unroll
+      for (int mq = 0; mq < QL; ++mq)
+  #pragma unroll
         for (int k = 0; k < 4; ++k)
-#pragma unroll
+  #pragma unroll
           for (int x = 0; x < 4; ++x) si[mq][k][x] = 0;
       if (is8) {
-#pragma unroll
+  #pragma unroll
         for (int cb = 0; cb < D / 32; ++cb)
-#pragma unroll
+  #pragma unroll
           for (int k = 0; k < 4; ++k) {
             uint32_t r[4];  // keys g / g+8 at channels 32cb + 4tq .. (+16): the A fragment as is
             ldsm_x4(kb + 16 * C::kRow8 * k + off8[cb], r);
-#pragma unroll
-            for (int mq = 0; mq < C::kQM; ++mq) mma_s8(si[mq][k], r, qi8[cb][mq][0], qi8[cb][mq][1]);
+  #pragma unroll
+            for (int mq = 0; mq < QL; ++mq) mma_s8(si[mq][k], r, qi8[cb][mq][0], qi8[cb][mq][1]);
           }
       } else {
-#pragma unroll
+  #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb)
-#pragma unroll
+  #pragma unroll
           for (int k = 0; k < 4; ++k) {
             uint32_t r[4];
             ldsm_x4(kb + 16 * C::kRow4 * k + off4[cb], r);
-#pragma unroll
+  #pragma unroll
             for (int h = 0; h < 2; ++h) {  // packed bytes 16h.. = channels 64cb + 32h ..
               // keys g / g+8, channels 8tq + (0, 2, 4, 6) and 8tq + (1, 3, 5, 7)
               const uint32_t a[4] = {i4_even_x16(r[2 * h]), i4_even_x16(r[2 * h + 1]),
                                      i4_odd_x16(r[2 * h]), i4_odd_x16(r[2 * h + 1])};
-#pragma unroll
-              for (int mq = 0; mq < C::kQM; ++mq)
+  #pragma unroll
+              for (int mq = 0; mq < QL; ++mq)
                 mma_s8(si[mq][k], a, qi4[cb][h][mq][0], qi4[cb][h][mq][1]);
             }
           }
       }
       // ---- online softmax for this lane's slots over keys 16k + g (+8): accumulator
-      // columns 2tq, 2tq + 1 hold the hi and lo limb products of head tq + 4 mq
+      // columns 2tq, 2tq + 1 of MMA mq hold the hi and mid limb products of head
+      // tq + 4 mq, column 2tq + mq of MMA kQM its lo limb products
       const float kscale = (is8 ? __ldg(p.sk8 + tile) : __ldg(p.sk4 + tile) * 0.0625f) * p.scale_log2;
       const float vs = is8 ? __ldg(p.sv8 + tile) : __ldg(p.sv4 + tile);
       float sv[C::kQM][8];  // [slot][key slot: 2k + (g / g+8)]
-#pragma unroll
+  #pragma unroll
       for (int mq = 0; mq < C::kQM; ++mq) {
         const float ks = kscale * qsig[mq];
-#pragma unroll
+  #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          sv[mq][2 * k] = (float)(si[mq][k][0] * 256 + si[mq][k][1]) * ks;
-          sv[mq][2 * k + 1] = (float)(si[mq][k][2] * 256 + si[mq][k][3]) * ks;
+          if (NL == 2) {
+            sv[mq][2 * k] = (float)(si[mq][k][0] * 256 + si[mq][k][1]) * ks;
+            sv[mq][2 * k + 1] = (float)(si[mq][k][2] * 256 + si[mq][k][3]) * ks;
+          } else {
+            // hi x 65536 is exact in fp32 (|hi| < 2^21); mid x 256 + lo fits int32
+            sv[mq][2 * k] = fmaf((float)si[mq][k][0], 65536.0f,
+                                 (float)(si[mq][k][1] * 256 + si[QL - 1][k][mq])) * ks;
+            sv[mq][2 * k + 1] = fmaf((float)si[mq][k][2], 65536.0f,
+                                     (float)(si[mq][k][3] * 256 + si[QL - 1][k][2 + mq])) * ks;
+          }
+        }
+      }
+      if (HYB) {
+        // selected keys and keys within the window of the query (position T + tl) are
+        // read in bf16 by the row pass: masked out of their INT4 tile here
+        uint64_t hi = __ldg(p.sel_mask + tile);
+        const int wlo = T + tl - p.window + 1 - kt * kTile;  // first in-window key of the tile
+        if (p.window > 0 && wlo < kTile) hi |= wlo <= 0 ? ~0ull : (~0ull << wlo);
+        if (hi) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int mq = 0; mq < C::kQM; ++mq) {
+              if ((hi >> (16 * k + g)) & 1) sv[mq][2 * k] = -INFINITY;
+              if ((hi >> (16 * k + g + 8)) & 1) sv[mq][2 * k + 1] = -INFINITY;
+            }
         }
       }
       if (nvalid < kTile) {  // a sequence's last tile: keys past its end are masked
-#pragma unroll
+  #pragma unroll
         for (int k = 0; k < 4; ++k)
-#pragma unroll
+  #pragma unroll
           for (int mq = 0; mq < C::kQM; ++mq) {
             if (16 * k + g >= nvalid) sv[mq][2 * k] = -INFINITY;
             if (16 * k + g + 8 >= nvalid) sv[mq][2 * k + 1] = -INFINITY;
@@ -510,10 +574,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       }
       float mt[C::kQM], alpha[C::kQM];
       bool need = false;
-#pragma unroll
+  #pragma unroll
       for (int mq = 0; mq < C::kQM; ++mq) {
         float x = sv[mq][0];
-#pragma unroll
+  #pragma unroll
         for (int k = 1; k < 8; ++k) x = fmaxf(x, sv[mq][k]);
         x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
         x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
@@ -525,7 +589,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       // lazy rescaling: the reference max moves only when it grew by more than 2^8
       const bool warp_need = __any_sync(0xffffffffu, need);
       if (warp_need) {
-#pragma unroll
+  #pragma unroll
         for (int mq = 0; mq < C::kQM; ++mq) {
           const float m_new = fmaxf(m_run[mq], mt[mq]);
           if (m_new > m_run[mq]) {
@@ -534,12 +598,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
           }
         }
       }
-#pragma unroll
+  #pragma unroll
       for (int mq = 0; mq < C::kQM; ++mq) {
         const float mb = m_run[mq] == -INFINITY ? 0.0f : m_run[mq];
         float ps = 0.0f;
         __half* prow = pw + (tq + 4 * mq) * C::kPStride;
-#pragma unroll
+  #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float p0 = real[mq] ? ex2(sv[mq][2 * k] - mb) : 0.0f;
           const float p1 = real[mq] ? ex2(sv[mq][2 * k + 1] - mb) : 0.0f;
@@ -552,14 +616,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       if (warp_need) {
         // O head 2tq + hh is softmax slot (2tq + hh) / 4 of lane 4g + (2tq + hh) % 4
         float ao[2];
-#pragma unroll
+  #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int hd = 2 * tq + hh, src = (lane & ~3) | (hd & 3);
           const float a0 = __shfl_sync(0xffffffffu, alpha[0], src);
           const float a1 = __shfl_sync(0xffffffffu, alpha[C::kQM - 1], src);
           ao[hh] = hd >= 4 ? a1 : a0;
         }
-#pragma unroll
+  #pragma unroll
         for (int j = 0; j < C::kB8; ++j) {
           o8[j][0] *= ao[0]; o8[j][1] *= ao[1];
           o8[j][2] *= ao[0]; o8[j][3] *= ao[1];
@@ -567,17 +631,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       }
       __syncwarp();
       // ---- O^T += V^T P^T: B fragment = P[head g][keys 16k + 2tq (+1), +8 (+9)]
-#pragma unroll
+  #pragma unroll
       for (int k = 0; k < 4; ++k) {
         uint32_t pb0, pb1;
         asm volatile("ld.shared.b32 %0, [%1];" : "=r"(pb0) : "r"(pw_addr + (g * C::kPStride + 16 * k + 2 * tq) * 2));
         asm volatile("ld.shared.b32 %0, [%1];" : "=r"(pb1) : "r"(pw_addr + (g * C::kPStride + 16 * k + 2 * tq + 8) * 2));
         if (is8) {
-#pragma unroll
+  #pragma unroll
           for (int cp = 0; cp < D / 32; ++cp) {
             uint32_t r[4];
             ldsm_x4_t(vb + 16 * C::kRow8 * k + off8[cp], r);
-#pragma unroll
+  #pragma unroll
             for (int h = 0; h < 2; ++h) {  // channels 32cp + 16h + (2g, 2g+1)
               // V8 codes are stored offset-binary (code + 128)
               const uint32_t u0 = r[2 * h], u1 = r[2 * h + 1];
@@ -587,11 +651,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             }
           }
         } else {
-#pragma unroll
+  #pragma unroll
           for (int cp = 0; cp < D / 64; ++cp) {
             uint32_t r[4];
             ldsm_x4_t(vb + 16 * C::kRow4 * k + off4[cp], r);
-#pragma unroll
+  #pragma unroll
             for (int h = 0; h < 2; ++h) {  // 32 channels 64cp + 32h ..
               // words: keys (2tq, 2tq+1) / (2tq+8, 2tq+9); nibble n of the lane's 16-bit
               // column holds channel 64cp + 32h + 16 (n / 2) + 2g + n % 2, so the
@@ -640,7 +704,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         rw[hd * (D + 2) + D + 1] = l_run[mq];
       }
     }
-    if (tail_cta) {
+    if (HYB || tail_cta) {
       float tm[GRP], tlsum[GRP];
       float2 to[GRP][C::kCh / 2];
 #pragma unroll
@@ -650,7 +714,44 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 #pragma unroll
         for (int k = 0; k < C::kCh / 2; ++k) to[gg][k] = make_float2(0.0f, 0.0f);
       }
-      tail_pass(tm, tlsum, to);
+      const long long tbase = ((long long)b * p.Hkv + kvh) * p.tail_cap;
+      const long long nbase = ((long long)b * p.Hkv + kvh) * D;
+      auto tail_row = [&](int x, const uint16_t*& kr, const uint16_t*& vr) -> bool {
+        kr = x == tl ? p.k_new + nbase : p.k_tail + (tbase + x) * D;
+        vr = x == tl ? p.v_new + nbase : p.v_tail + (tbase + x) * D;
+        return true;
+      };
+      const int ntail = tail_cta ? tl + 1 : 0;
+      if (!HYB) {
+        row_pass(ntail, tail_row, tm, tlsum, to);
+      } else {
+        // hybrid bf16 rows: n_sel selected rows, then `window` rows of the last prefix
+        // tokens (a window row takes part if it is still in the query's window and not
+        // selected); split x takes rows [R x / S, R (x + 1) / S) of the R, then the tail
+        const int nsel = __ldg(p.sel_count + b);
+        const int R = nsel + p.window;
+        const int x0 = (int)((long long)R * split / nsplit);
+        const int nh = (int)((long long)R * (split + 1) / nsplit) - x0;
+        const long long sbase = ((long long)b * p.Hkv + kvh) * p.sel_cap;
+        const long long wbase = ((long long)b * p.Hkv + kvh) * p.window;
+        const int qpos = T + tl;  // the query's position
+        auto hy_row = [&](int x, const uint16_t*& kr, const uint16_t*& vr) -> bool {
+          if (x >= nh) return tail_row(x - nh, kr, vr);
+          const int hx = x0 + x;
+          if (hx < nsel) {
+            kr = p.k_sel + (sbase + hx) * D;
+            vr = p.v_sel + (sbase + hx) * D;
+            return true;
+          }
+          const int w = hx - nsel, j = T - p.window + w;
+          kr = p.k_win + (wbase + w) * D;
+          vr = p.v_win + (wbase + w) * D;
+          if (j < 0 || qpos - j >= p.window) return false;
+          const uint64_t sm_ = __ldg(p.sel_mask + (long long)kvh * p.ntiles + toff + j / kTile);
+          return ((sm_ >> (j % kTile)) & 1) == 0;
+        };
+        row_pass(nh + ntail, hy_row, tm, tlsum, to);
+      }
       float* rt = red + (kConsumers + warp) * GRP * (D + 2);
 #pragma unroll
       for (int gg = 0; gg < GRP; ++gg) {
@@ -666,7 +767,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     named_sync(2);
   }
   // merge the consumer warps' states into this split's partial (m, l, o)
-  const int nstates = tail_cta ? C::kStates : kConsumers;
+  const int nstates = (HYB || tail_cta) ? C::kStates : kConsumers;
   for (int x = t; x < GRP * D; x += kDecThreads) {
     const int gg = x / D, c = x % D;
     if (gg >= grp) continue;
@@ -744,15 +845,25 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   }
 }
 
-template <int D, int GRP>
-cudaError_t launch_dec(const DecodeParams& p, const DecodeMaps& m, cudaStream_t s) {
+template <int D, int GRP, bool HYB>
+cudaError_t launch_dec_h(const DecodeParams& p, const DecodeMaps& m, cudaStream_t s) {
   using C = DecCfg<D, GRP>;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GRP>,
+  dim3 grid(p.splits, p.Hkv, p.B);
+  // two limbs first (the common case), then three; each group runs in one of them
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GRP, 2, HYB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.splits, p.Hkv, p.B);
-  decode_split_kernel<D, GRP><<<grid, kDecThreads, C::kSmem, s>>>(p, m);
+  decode_split_kernel<D, GRP, 2, HYB><<<grid, kDecThreads, C::kSmem, s>>>(p, m);
+  e = cudaFuncSetAttribute(decode_split_kernel<D, GRP, 3, HYB>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  decode_split_kernel<D, GRP, 3, HYB><<<grid, kDecThreads, C::kSmem, s>>>(p, m);
   return cudaGetLastError();
+}
+
+template <int D, int GRP>
+cudaError_t launch_dec(const DecodeParams& p, const DecodeMaps& m, cudaStream_t s) {
+  return p.sel_mask ? launch_dec_h<D, GRP, true>(p, m, s) : launch_dec_h<D, GRP, false>(p, m, s);
 }
 
 template <int D>

@@ -51,6 +51,18 @@ extern "C" tra_status routed_attention_decode_noalloc(
     const uint32_t* entries, uint16_t* k_tail, uint16_t* v_tail, int32_t* tail_len_dev,
     int32_t tail_cap, float softmax_scale, uint16_t* out, int32_t* status_dev, void* stream) {
   if (!prefill_shape) return tra::report_error(TRA_ERR_INVALID, "shape is NULL");
+  // The arrival counters sit in a fixed area at the start of the array for every shape
+  // with B * (Hkv + 1) <= TRA_NOALLOC_MAX_COUNTERS; a larger shape would put them where
+  // earlier calls left partial results, which need not be zero.
+  if ((long long)prefill_shape->B * ((long long)prefill_shape->Hkv + 1) > TRA_NOALLOC_MAX_COUNTERS) {
+    char msg[256];
+    snprintf(msg, sizeof msg,
+             "B * (Hkv + 1) = %lld exceeds %d, the arrival counters the fixed scratch keeps at "
+             "zero; use routed_attention_decode with a caller workspace",
+             (long long)prefill_shape->B * ((long long)prefill_shape->Hkv + 1),
+             (int)TRA_NOALLOC_MAX_COUNTERS);
+    return tra::report_error(TRA_ERR_UNSUPPORTED, msg);
+  }
   const size_t need = tra_decode_workspace_bytes(prefill_shape->B, prefill_shape->Hq,
                                                  prefill_shape->Hkv, prefill_shape->d);
   if (need > TRA_NOALLOC_SCRATCH_BYTES) {
@@ -65,8 +77,8 @@ extern "C" tra_status routed_attention_decode_noalloc(
   tra_status st = scratch_address(&scratch);
   if (st != TRA_OK) return st;
   // The scratch starts zero-filled (static storage) and every call leaves its
-  // arrival counters at zero again; the partials behind them are written before
-  // they are read.  The regular entry point validates all other arguments and
+  // arrival counters at zero again (they stay in the fixed counter area checked
+  // above); the partials behind them are written before they are read.  The regular entry point validates all other arguments and
   // enqueues the same kernel.
   return routed_attention_decode(prefill_shape, policy, q, k_new, v_new, cache, row_ptr, entries,
                                  k_tail, v_tail, tail_len_dev, tail_cap, softmax_scale, out,

@@ -5,36 +5,34 @@
 // paths update the same online-softmax state).
 //
 // Work unit: one query head h of one sequence b and one pair of q-tiles
-// (2j, 2j+1) = 128 query rows, the M of one tcgen05 MMA.  The two rows' CSR
-// traversals (each sorted by (precision, kt)) are merged on the fly into one
-// stream of (kt, precision, half-mask) entries; an entry whose tile appears in
-// only one q-tile's list (or with a different precision) is computed for all
-// 128 rows and masked to -inf in the other half, so routing stays exact.
+// (2j, 2j+1) = 128 query rows, the M of one tcgen05 MMA (rows 0-63 q-tile 2j =
+// TMEM lanes 0-63, rows 64-127 q-tile 2j+1 = lanes 64-127).  The two q-tiles'
+// CSR traversals (each sorted by (precision, kt): three ascending runs) are
+// merged into one stream of key tiles in ascending kt; an entry carries the
+// precision each q-tile gives the tile (or none).  When the two precisions
+// differ, the entry computes both score products into the same S block, each
+// MMA writing only its own q-tile's 64 lanes (tcgen05.mma output-lane mask), so
+// every entry has one S block, one softmax pass over all 128 rows and one P V.
 //
-// Two work units share one CTA (448 threads) so that one unit's softmax runs
+// Two work units share one CTA (384 threads) so that one unit's softmax runs
 // while the tensor core works on the other's tiles:
-//   warps 0, 13 TMA producers, one per unit: the unit's Q tiles once, then in
-//               traversal order K (INT8 codes or BF16) into the unit's K ring
-//               and V (BF16) into its V ring (K slots free up right after QK,
-//               V slots only after P V);
-//   warps 1, 12 MMA issuers, one per unit (warp 1 also owns TMEM): S = Q K^T
-//               with kind::i8 (INT8/INT4, exact int32) or kind::f16 (BF16,
-//               fp32) into one of the unit's two S buffers in TMEM, then
-//               O += P V with P read from TMEM (bf16) and V from shared memory;
-//   warps 2, 3  INT4 expanders of units 0, 1: packed INT4 codes (Q once, K per
-//               INT4 entry)
-//               sign-extended to int8 in the swizzled operand layout (tcgen05
-//               has no integer 4-bit MMA, so INT4 tiles run as int8 MMAs), into
-//               the unit's K4 ring.  Every ring belongs to one unit: one filler
-//               and one consumer (the unit's MMA issuer), both taking its slots
-//               in order, so no parity wait on a full or free barrier can
-//               alias a phase two uses away;
+//   warps 0, 2  TMA producers of units 0, 1: the unit's Q operands once (INT8
+//               codes; INT4 codes in their int8 operand form, 16 x code, as the
+//               quantiser writes them; BF16), then per entry one K tile per
+//               precision the entry needs into the unit's K ring and the BF16 V
+//               tile into its V ring;
+//   warps 1, 3  MMA issuers of units 0, 1 (warp 1 also owns TMEM): S = Q K^T with
+//               kind::i8 (INT8 / INT4, exact int32) or kind::f16 (BF16, fp32) into
+//               one of the unit's two S blocks in TMEM, then O += P V with P read
+//               from TMEM (bf16, written over S) and V from shared memory;
 //   warps 4-7   softmax / epilogue of unit 0, warps 8-11 of unit 1: one thread
 //               per query row (TMEM lane): S -> log2-domain scores -> mask ->
 //               online softmax with lazy rescaling of O -> bf16 P into TMEM;
-//               finally O / l.  P(i) overwrites S(i) in its TMEM buffer; with
-//               two buffers QK(i+1) runs while entry i is in the softmax, and
-//               the softmax never waits for a P V except to rescale O.
+//               finally O / l.  With two S blocks, QK(i+1) runs while entry i is
+//               in the softmax.
+// Every ring belongs to one unit: one filler and one consumer, both taking its
+// slots in order, so no parity wait can alias a phase two uses away.  All waits
+// are bounded (2 s); on expiry a role records TRA_DEV_TIMEOUT and all drain.
 #include <type_traits>
 
 #include "tra_device.cuh"
@@ -43,8 +41,7 @@
 namespace tra {
 namespace {
 
-constexpr int kThreads = 448;
-constexpr int kProdWarp1 = 13;  // TMA producer of unit 1 (warp 0: unit 0)
+constexpr int kThreads = 384;
 constexpr int kUnits = 2;
 // log2 units: O and l are rescaled only once the running max has grown by more
 // than 2^16.  Until then P (bf16, exponent range of fp32) may reach 2^16, and
@@ -52,40 +49,39 @@ constexpr int kUnits = 2;
 // inside fp32; rarer rescales matter because each one waits for the previous
 // P V to complete.
 constexpr float kRescaleThreshold = 16.0f;
-constexpr int kSmemLimit = 232448;         // max dynamic shared memory per CTA on sm_100
+constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
+constexpr uint32_t kNoKt = 0x0FFFFFFFu;
 
 template <int D, int MODE>
 struct Cfg {
   static constexpr bool kHasBf16 = MODE != TRA_POLICY_BOUNDARY;  // bf16 Q and K operands
-  static constexpr bool kHasInt4 = MODE != TRA_POLICY_BITMASK;   // expanded INT4 operands
+  static constexpr bool kHasInt4 = MODE != TRA_POLICY_BITMASK;   // INT4 operands (int8 form)
   // work units per CTA: two, or one under a mixed policy, whose operand buffers
-  // (int8, expanded INT4 and bf16 Q, bf16-sized K slots, the K4 ring) do not fit twice
+  // (int8, INT4 and bf16 Q, bf16-sized K slots) do not fit twice
   static constexpr int kCtaUnits = MODE == TRA_POLICY_MIXED ? 1 : 2;
-  static constexpr int kQ8Bytes = 128 * D;                                    // int8 Q codes
-  static constexpr int kQ4Bytes = kHasInt4 ? 128 * D : 0;                     // expanded INT4 Q
-  static constexpr int kQbBytes = kHasBf16 ? 128 * D * 2 : 0;                 // bf16 Q
+  static constexpr int kQ8Bytes = 128 * D;                     // int8 Q codes
+  static constexpr int kQ4Bytes = kHasInt4 ? 128 * D : 0;      // INT4 Q codes as int8
+  static constexpr int kQbBytes = kHasBf16 ? 128 * D * 2 : 0;  // bf16 Q
   static constexpr int kQUnitBytes = kQ8Bytes + kQ4Bytes + kQbBytes;
-  // K slot: BF16 or INT8 codes when bf16 tiles occur, INT8 codes only under boundaries
+  // K slot: one K tile, BF16 or int8 codes (INT8 or INT4 in int8 form)
   static constexpr int kKBytes = kHasBf16 ? 64 * D * 2 : 64 * D;
-  static constexpr int kK4Bytes = 64 * D;                                     // expanded INT4 K
   static constexpr int kVBytes = 64 * D * 2;
-  // ring depths per unit (every ring belongs to one unit)
-  static constexpr int kStagesK = 2;
-  static constexpr int kStagesK4 = kHasInt4 ? 2 : 0;
-  static constexpr int kFixed =
-      kCtaUnits * (kQUnitBytes + kStagesK * kKBytes + kStagesK4 * kK4Bytes) + 2048;  // + barriers
-  static constexpr int kStagesVFit = (kSmemLimit - kFixed) / (kCtaUnits * kVBytes);
+  static constexpr int kBase = kCtaUnits * kQUnitBytes + 2048 + 1024;  // + barriers, slack
+  // ring depths per unit: as many of both as fit, K first (up to 4 each)
+  static constexpr int kRoom = (kSmemLimit - kBase) / kCtaUnits;
+  static constexpr int kStagesK = kRoom >= 4 * kKBytes + 4 * kVBytes ? 4
+                                  : kRoom >= 3 * kKBytes + 3 * kVBytes ? 3 : 2;
+  static constexpr int kStagesVFit = (kRoom - kStagesK * kKBytes) / kVBytes;
   static constexpr int kStagesV = kStagesVFit > 4 ? 4 : kStagesVFit;
   static_assert(kStagesV >= 2, "shared memory too small for the V rings");
   static constexpr int kOffQ = 0;                                             // unit u at u * kQUnitBytes
   static constexpr int kOffK = kCtaUnits * kQUnitBytes;                       // [unit][slot]
-  static constexpr int kOffK4 = kOffK + kCtaUnits * kStagesK * kKBytes;
-  static constexpr int kOffV = kOffK4 + kCtaUnits * kStagesK4 * kK4Bytes;
+  static constexpr int kOffV = kOffK + kCtaUnits * kStagesK * kKBytes;
   static constexpr int kOffBar = kOffV + kCtaUnits * kStagesV * kVBytes;
   // (barriers exist for two units in every mode; a CTA's missing second unit has
   // no entries and touches none of the buffers above)
-  static constexpr int kUnitBars = 2 * kStagesK + 2 * kStagesK4 + 2 * kStagesV + 6;
-  static constexpr int kNumBars = 2 + kUnits * kUnitBars + 1;
+  static constexpr int kUnitBars = 2 * kStagesK + 2 * kStagesV + 6;
+  static constexpr int kNumBars = 1 + kUnits * kUnitBars + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= kSmemLimit, "shared memory budget");
@@ -98,30 +94,60 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = 512;
 };
 
-// Byte offset of 16-byte chunk `c` of row `r` in a swizzled K-major int8 tile.
-template <int D>
-__device__ __forceinline__ uint32_t i8_swz_offset(int r, int c) {
-  if (D == 128) return r * 128 + ((c ^ (r & 7)) << 4);
-  return r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
-}
-
-// Merge of two sorted CSR rows (entry = (prec << 28) | kt): yields each
-// distinct entry once with a mask of the rows (bit 0: first, bit 1: second)
-// that contain it.
-struct MergeCursor {
+// The two q-tiles' rows of a unit merged in ascending kt.  A row lists its INT4,
+// INT8 and BF16 tiles as three ascending runs (sorted as whole entries); next()
+// yields each kt of either row once with the precision each row gives it (0: the
+// row does not list it).
+struct KtMerge {
   const uint32_t* e;
-  int p0, e0, p1, e1;
-  __device__ __forceinline__ bool next(uint32_t& val, int& mask) {
-    const uint32_t a = p0 < e0 ? __ldg(e + p0) : 0xFFFFFFFFu;
-    const uint32_t b = p1 < e1 ? __ldg(e + p1) : 0xFFFFFFFFu;
-    if (a == 0xFFFFFFFFu && b == 0xFFFFFFFFu) return false;
-    if (a < b) {
-      val = a; mask = 1; ++p0;
-    } else if (b < a) {
-      val = b; mask = 2; ++p1;
-    } else {
-      val = a; mask = 3; ++p0; ++p1;
+  int pos[2][3], end[2][3];
+  uint32_t head[2][3];  // current kt of each run, kNoKt when exhausted
+
+  __device__ __forceinline__ void load(int r, int g) {
+    head[r][g] = pos[r][g] < end[r][g] ? (__ldg(e + pos[r][g]) & kNoKt) : kNoKt;
+  }
+  __device__ __forceinline__ static int lower_bound(const uint32_t* e, int lo, int hi, uint32_t key) {
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(e + mid) < key) lo = mid + 1; else hi = mid;
     }
+    return lo;
+  }
+  // rows [rs[r], re[r]) of the entry array; an absent row is empty
+  __device__ __forceinline__ void init(const uint32_t* entries, const int (&rs)[2], const int (&re)[2]) {
+    e = entries;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int b8 = lower_bound(e, rs[r], re[r], (uint32_t)TRA_PREC_INT8 << 28);
+      const int bb = lower_bound(e, b8, re[r], (uint32_t)TRA_PREC_BF16 << 28);
+      pos[r][0] = rs[r]; end[r][0] = b8;
+      pos[r][1] = b8;    end[r][1] = bb;
+      pos[r][2] = bb;    end[r][2] = re[r];
+#pragma unroll
+      for (int g = 0; g < 3; ++g) load(r, g);
+    }
+  }
+  // next entry: kt and each row's precision (TRA_PREC_*, or 0)
+  __device__ __forceinline__ bool next(int& kt, int& p0, int& p1) {
+    uint32_t k = kNoKt;
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int g = 0; g < 3; ++g) k = min(k, head[r][g]);
+    if (k == kNoKt) return false;
+    int pr[2] = {0, 0};
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int g = 0; g < 3; ++g)
+        if (head[r][g] == k) {
+          pr[r] = g + 1;  // TRA_PREC_INT4 = 1, INT8 = 2, BF16 = 3
+          ++pos[r][g];
+          load(r, g);
+        }
+    kt = (int)k;
+    p0 = pr[0];
+    p1 = pr[1];
     return true;
   }
 };
@@ -157,24 +183,49 @@ __device__ __forceinline__ Unit make_unit(const PrefillParams& p, long long id) 
   return x;
 }
 
-__device__ __forceinline__ MergeCursor unit_cursor(const PrefillParams& p, const Unit& x) {
-  MergeCursor c;
-  c.e = p.entries;
+__device__ __forceinline__ KtMerge unit_merge(const PrefillParams& p, const Unit& x) {
+  KtMerge c;
+  int rs[2] = {0, 0}, re[2] = {0, 0};
   if (x.valid) {
-    c.p0 = __ldg(p.row_ptr + x.row0);
-    c.e0 = __ldg(p.row_ptr + x.row0 + 1);
-    c.p1 = c.e0;
-    c.e1 = x.has_second ? __ldg(p.row_ptr + x.row0 + 2) : c.e0;
-  } else {
-    c.p0 = c.e0 = c.p1 = c.e1 = 0;
+    rs[0] = __ldg(p.row_ptr + x.row0);
+    re[0] = rs[1] = __ldg(p.row_ptr + x.row0 + 1);
+    re[1] = x.has_second ? __ldg(p.row_ptr + x.row0 + 2) : rs[1];
   }
+  c.init(p.entries, rs, re);
   return c;
+}
+
+// The K tiles of an entry: one per distinct precision, q-tile 2j's first.
+__device__ __forceinline__ int entry_fills(int p0, int p1) { return (p0 && p1 && p0 != p1) ? 2 : 1; }
+__device__ __forceinline__ int entry_fill_prec(int p0, int p1, int f) {
+  return f == 0 ? (p0 ? p0 : p1) : p1;
 }
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// tcgen05.mma with an output-lane mask: lanes whose bit is set in m0..m3 (lane
+// 32 w + i <-> bit i of m_w) keep their contents.
+__device__ __forceinline__ void mma_i8_mask(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate, const uint32_t (&m)[4]) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(m[0]), "r"(m[1]), "r"(m[2]), "r"(m[3])
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_mask(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t accumulate, const uint32_t (&m)[4]) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(m[0]), "r"(m[1]), "r"(m[2]), "r"(m[3])
+      : "memory");
 }
 
 // O += P V with the 128 x 16 bf16 A operand (P) read from TMEM.
@@ -192,8 +243,7 @@ template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps m) {
   using C = Cfg<D, MODE>;
-  constexpr int NSK = C::kStagesK, NSV = C::kStagesV, NS4R = C::kStagesK4;
-  constexpr int NS4 = NS4R > 0 ? NS4R : 1;  // (no K4 ring without INT4)
+  constexpr int NSK = C::kStagesK, NSV = C::kStagesV;
   extern __shared__ uint8_t smem_raw[];
 
   // ---- the CTA's work units (the second is absent under a mixed policy)
@@ -214,28 +264,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sQ4 = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes; };
   auto sQb = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes + C::kQ4Bytes; };
   auto sK = [&](int u, int s) { return base + C::kOffK + (u * NSK + s) * C::kKBytes; };
-  auto sK4 = [&](int u, int s) { return base + C::kOffK4 + (u * NS4 + s) * C::kK4Bytes; };
   auto sV = [&](int u, int s) { return base + C::kOffV + (u * NSV + s) * C::kVBytes; };
   const uint32_t bars = base + C::kOffBar;
-  const uint32_t bar_q = bars + 0 * 8;
-  const uint32_t bar_q4 = bars + 1 * 8;
-  // barriers of unit u: K ring full/free, K4 ring full/free, V ring full/free, then
-  // S full (2), P full (2), O full, O final
-  auto ubar = [&](int u, int k) { return bars + (2 + u * C::kUnitBars + k) * 8; };
+  const uint32_t bar_q = bars;
+  // barriers of unit u: K ring full/free, V ring full/free, then S full (2),
+  // P full (2), O full, O final
+  auto ubar = [&](int u, int k) { return bars + (1 + u * C::kUnitBars + k) * 8; };
   auto bar_kfull = [&](int u, int s) { return ubar(u, s); };
   auto bar_kfree = [&](int u, int s) { return ubar(u, NSK + s); };
-  auto bar_k4full = [&](int u, int s) { return ubar(u, 2 * NSK + s); };
-  auto bar_k4free = [&](int u, int s) { return ubar(u, 2 * NSK + NS4R + s); };
-  constexpr int kVB = 2 * NSK + 2 * NS4R;  // first V ring barrier of a unit
-  auto bar_vfull = [&](int u, int s) { return ubar(u, kVB + s); };
-  auto bar_vfree = [&](int u, int s) { return ubar(u, kVB + NSV + s); };
-  constexpr int kSB = kVB + 2 * NSV;       // first S/P/O barrier of a unit
+  auto bar_vfull = [&](int u, int s) { return ubar(u, 2 * NSK + s); };
+  auto bar_vfree = [&](int u, int s) { return ubar(u, 2 * NSK + NSV + s); };
+  constexpr int kSB = 2 * NSK + 2 * NSV;  // first S/P/O barrier of a unit
   auto bar_sfull = [&](int u, int sb) { return ubar(u, kSB + sb); };
   auto bar_pfull = [&](int u, int sb) { return ubar(u, kSB + 2 + sb); };
   auto bar_ofull = [&](int u) { return ubar(u, kSB + 4); };
   // completes once every MMA of unit u (its last P V included) is done
   auto bar_ofinal = [&](int u) { return ubar(u, kSB + 5); };
-  const uint32_t bar_done = bars + (2 + kUnits * C::kUnitBars) * 8;
+  const uint32_t bar_done = bars + (1 + kUnits * C::kUnitBars) * 8;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kOffMisc);
   volatile int* const err = reinterpret_cast<volatile int*>(gbase + C::kOffMisc + 16);
 
@@ -244,15 +289,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, kUnits);  // one arrival (with its byte count) per producer
-    mbar_init(bar_q4, 64);  // both expander warps, each after its unit's Q
     for (int u = 0; u < kUnits; ++u) {
       for (int s = 0; s < NSK; ++s) {
         mbar_init(bar_kfull(u, s), 1);
         mbar_init(bar_kfree(u, s), 1);
-      }
-      for (int s = 0; s < NS4R; ++s) {
-        mbar_init(bar_k4full(u, s), 32);  // the unit's expander warp
-        mbar_init(bar_k4free(u, s), 1);
       }
       for (int s = 0; s < NSV; ++s) {
         mbar_init(bar_vfull(u, s), 1);
@@ -278,50 +318,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-
-  if (warp == 0 || warp == kProdWarp1) {
+  if (warp == 0 || warp == 2) {
     // ================================================================ TMA producers
-    // one per unit, each walking its own unit's traversal into its own rings
+    // one per unit, each walking its own unit's merged stream into its own rings
     if (lane == 0) {
-      const int u = warp == 0 ? 0 : 1;
+      const int u = warp >> 1;
       const Unit x = u ? un1 : un0;
-      constexpr uint32_t kQBytes = C::kQ8Bytes + C::kQbBytes;
-      mbar_arrive_expect_tx(bar_q, x.valid ? kQBytes : 0u);
+      const uint32_t qbytes = x.valid ? C::kQ8Bytes + (int4 ? C::kQ4Bytes : 0) + C::kQbBytes : 0u;
+      mbar_arrive_expect_tx(bar_q, qbytes);
       if (x.valid) {
         tma_load_2d(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
+        if (int4) tma_load_2d(sQ4(u), &m.q4x, bar_q, 0, x.row0 * kTile);
         if (C::kHasBf16) {
           for (int sl = 0; sl < C::kSlabs; ++sl)
             tma_load_3d(sQb(u) + sl * 128 * 128, &m.qb, bar_q, sl * 64, x.h,
                         x.seq0 + x.qt0 * kTile);
         }
       }
-      MergeCursor c = unit_cursor(p, x);
-      uint32_t val;
-      int mask;
+      KtMerge c = unit_merge(p, x);
+      int kt, p0, p1;
       int nk = 0, nv = 0;  // fills issued so far into this unit's K and V rings
-      while (c.next(val, mask)) {
-        const int sv = nv % NSV, usev = nv / NSV;  // the unit's V ring slot
-        const uint32_t prec = val >> 28;
-        const int kt = (int)(val & 0x0FFFFFFFu);
-        if (prec == TRA_PREC_INT4 && !int4) {
+      while (c.next(kt, p0, p1)) {
+        if ((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) {
           *err = TRA_DEV_BAD_LIST;
           break;
         }
-        if (prec != TRA_PREC_INT4) {
+        bool ok = true;
+        const int nf = entry_fills(p0, p1);
+        for (int f = 0; f < nf; ++f) {
+          const int prec = entry_fill_prec(p0, p1, f);
           const int s = nk % NSK, use = nk / NSK;  // the unit's K ring slot
-          if (use > 0 && !mbar_wait(bar_kfree(u, s), (use - 1) & 1, err)) break;
+          if (use > 0 && !mbar_wait(bar_kfree(u, s), (use - 1) & 1, err)) { ok = false; break; }
           const uint32_t dst = sK(u, s);
-          if (prec == TRA_PREC_INT8) {
-            mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D);
-            tma_load_2d(dst, &m.k8, bar_kfull(u, s), 0, (x.kvh * p.ntiles + x.toff + kt) * kTile);
-          } else {
+          const int krow = (x.kvh * p.ntiles + x.toff + kt) * kTile;
+          if (prec == TRA_PREC_BF16) {
             mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D * 2);
             for (int sl = 0; sl < C::kSlabs; ++sl)
               tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(u, s), sl * 64, x.kvh,
                           x.seq0 + kt * kTile);
+          } else {
+            mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D);
+            tma_load_2d(dst, prec == TRA_PREC_INT8 ? &m.k8 : &m.k4x, bar_kfull(u, s), 0, krow);
           }
           ++nk;
         }
+        if (!ok) break;
+        const int sv = nv % NSV, usev = nv / NSV;  // the unit's V ring slot
         if (usev > 0 && !mbar_wait(bar_vfree(u, sv), (usev - 1) & 1, err)) break;
         mbar_arrive_expect_tx(bar_vfull(u, sv), 64 * D * 2);
         for (int sl = 0; sl < C::kSlabs; ++sl)
@@ -340,16 +382,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait_drain(bar_vfull(u, s), (uint32_t)(((nv - 1 - s) / NSV) & 1));
       }
     }
-  } else if (warp == 1 || warp == 12) {
+  } else if (warp == 1 || warp == 3) {
     // ================================================================ MMA issuers
     if (lane == 0) {
-      const int mu = warp == 1 ? 0 : 1;  // the unit this thread issues for
+      const int mu = warp >> 1;  // the unit this thread issues for
       constexpr uint32_t kIdI8 = instr_desc(2, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdQK16 = instr_desc(1, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdPV = instr_desc(1, 1, 0, 1, D, 128);
       const uint32_t tU = tmem + mu * 256;
       bool ok = mbar_wait(bar_q, 0, err);
-      if (ok && int4) ok = mbar_wait(bar_q4, 0, err);
       tc_fence_after();
       // O += P(idx) V(idx): P from TMEM buffer idx & 1, V (MN-major) from the unit's
       // V ring, which holds one tile per entry of the unit, in order
@@ -369,47 +410,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       if (ok) {
-        int nk = 0, n4 = 0;           // this unit's K / K4 ring fills consumed so far
-        int i = 0;                    // entries of this unit issued so far
-        MergeCursor c = unit_cursor(p, mu ? un1 : un0);
-        uint32_t val;
-        int mask;
-        while (c.next(val, mask)) {
-          const uint32_t prec = val >> 28;
-          if (prec == TRA_PREC_INT4 && !int4) {
+        int nk = 0;  // this unit's K ring fills consumed so far
+        int i = 0;   // entries of this unit issued so far
+        KtMerge c = unit_merge(p, mu ? un1 : un0);
+        int kt, p0, p1;
+        while (c.next(kt, p0, p1)) {
+          if ((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) {
             *err = TRA_DEV_BAD_LIST;
             ok = false;
             break;
           }
-          const bool is4 = prec == TRA_PREC_INT4;
-          const int s = is4 ? n4 % NS4 : nk % NSK;
-          const uint32_t ph = (uint32_t)((is4 ? n4 / NS4 : nk / NSK) & 1);
-          if (is4) ++n4; else ++nk;
           // S buffer i & 1 last held entry i-2, whose P V this thread has already
           // issued; MMAs of one thread run in order, so QK(i) cannot overtake it
-          if (!mbar_wait(is4 ? bar_k4full(mu, s) : bar_kfull(mu, s), ph, err)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t tSb = tU + (i & 1) * 64;
-          const uint32_t kb = is4 ? sK4(mu, s) : sK(mu, s);
-          if (prec == TRA_PREC_BF16) {
+          const int nf = entry_fills(p0, p1);
+          for (int f = 0; f < nf; ++f) {
+            const int prec = entry_fill_prec(p0, p1, f);
+            const int s = nk % NSK;
+            if (!mbar_wait(bar_kfull(mu, s), (uint32_t)((nk / NSK) & 1), err)) { ok = false; break; }
+            tc_fence_after();
+            // lanes written: all for a single-precision entry; for two precisions the
+            // first MMA writes q-tile 2j's lanes 0-63, the second q-tile 2j+1's 64-127
+            const uint32_t keep = nf == 1 ? 0u : 0xFFFFFFFFu;
+            const uint32_t msk[4] = {f == 1 ? keep : 0u, f == 1 ? keep : 0u, f == 0 ? keep : 0u,
+                                     f == 0 ? keep : 0u};
+            const uint32_t kb = sK(mu, s);
+            if (prec == TRA_PREC_BF16) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const int sl = kk >> 2, off = (kk & 3) * 32;
-              const uint64_t a = smem_desc(sQb(mu) + sl * 128 * 128 + off, 16, 1024, kSwz128);
-              const uint64_t bd = smem_desc(kb + sl * 64 * 128 + off, 16, 1024, kSwz128);
-              mma_bf16(tSb, a, bd, kIdQK16, kk > 0 ? 1u : 0u);
-            }
-          } else {
-            const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(mu) : sQ4(mu);
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const int sl = kk >> 2, off = (kk & 3) * 32;
+                const uint64_t a = smem_desc(sQb(mu) + sl * 128 * 128 + off, 16, 1024, kSwz128);
+                const uint64_t bd = smem_desc(kb + sl * 64 * 128 + off, 16, 1024, kSwz128);
+                mma_bf16_mask(tSb, a, bd, kIdQK16, kk > 0 ? 1u : 0u, msk);
+              }
+            } else {
+              const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(mu) : sQ4(mu);
 #pragma unroll
-            for (int kk = 0; kk < D / 32; ++kk) {
-              const uint64_t a = smem_desc(qa + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
-              const uint64_t bd = smem_desc(kb + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
-              mma_i8(tSb, a, bd, kIdI8, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < D / 32; ++kk) {
+                const uint64_t a = smem_desc(qa + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
+                const uint64_t bd = smem_desc(kb + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
+                mma_i8_mask(tSb, a, bd, kIdI8, kk > 0 ? 1u : 0u, msk);
+              }
             }
+            mma_commit(bar_kfree(mu, s));
+            ++nk;
           }
+          if (!ok) break;
           mma_commit(bar_sfull(mu, i & 1));
-          mma_commit(is4 ? bar_k4free(mu, s) : bar_kfree(mu, s));
           if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
           ++i;
         }
@@ -419,128 +466,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar_done);
       mbar_wait_drain(bar_done, 0);
     }
-  } else if (warp == 2 || warp == 3) {
-    // ================================================================ INT4 expanders
-    // warp 2 for unit 0, warp 3 for unit 1, each walking its own unit's traversal
-    const int u = warp - 2;
-    const int t = lane;
-    const Unit x = u ? un1 : un0;
-    constexpr int kPackedRow = D / 2;          // bytes per packed row
-    constexpr int kChunksPerRow = kPackedRow / 16;
-    if (int4) {
-      // Q: 128 rows (two q-tiles); rows of a missing q-tile stay zero
-      if (x.valid) {
-        const uint8_t* src = p.q4 + (long long)x.row0 * kTile * kPackedRow;
-        const int rows = x.has_second ? 128 : 64;
-        uint8_t* dst = gbase + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes;
-        for (int f = t; f < 128 * kChunksPerRow; f += 32) {
-          const int r = f / kChunksPerRow, c = f % kChunksPerRow;
-          uint4 w = make_uint4(0, 0, 0, 0);
-          if (r < rows) w = __ldg(reinterpret_cast<const uint4*>(src + r * kPackedRow + c * 16));
-          const uint2 e0 = expand_int4x8(w.x), e1 = expand_int4x8(w.y);
-          const uint2 e2 = expand_int4x8(w.z), e3 = expand_int4x8(w.w);
-          *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * c)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
-          *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * c + 1)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar_q4);
-      // packed codes of the unit's next INT4 entry are loaded into registers as soon
-      // as the previous one is handed over, so the load overlaps the wait for a slot
-      constexpr int kPer = 64 * kChunksPerRow / 32;  // 16-byte chunks per lane and tile
-      MergeCursor c = unit_cursor(p, x);
-      auto next_int4 = [&](uint32_t& v) -> bool {
-        int mk;
-        while (c.next(v, mk))
-          if ((v >> 28) == TRA_PREC_INT4) return true;
-        return false;
-      };
-      auto load_packed = [&](uint32_t v, uint4 (&w)[kPer]) {
-        const int kt = (int)(v & 0x0FFFFFFFu);
-        const uint8_t* ks = p.k4 + ((long long)(x.kvh * p.ntiles + x.toff + kt) * kTile) * kPackedRow;
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-          const int f = t + 32 * j, r = f / kChunksPerRow, cc = f % kChunksPerRow;
-          w[j] = __ldg(reinterpret_cast<const uint4*>(ks + r * kPackedRow + cc * 16));
-        }
-      };
-      uint4 w[kPer];
-      uint32_t val;
-      bool have = next_int4(val);
-      if (have) load_packed(val, w);
-      for (int n4 = 0; have; ++n4) {
-        const int s = n4 % NS4, use = n4 / NS4;  // the unit's K4 ring slot
-        if (use > 0 && !mbar_wait(bar_k4free(u, s), (use - 1) & 1, err)) break;
-        uint8_t* dst = gbase + C::kOffK4 + (u * NS4 + s) * C::kK4Bytes;
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-          const int f = t + 32 * j, r = f / kChunksPerRow, cc = f % kChunksPerRow;
-          const uint2 e0 = expand_int4x8(w[j].x), e1 = expand_int4x8(w[j].y);
-          const uint2 e2 = expand_int4x8(w[j].z), e3 = expand_int4x8(w[j].w);
-          *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * cc)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
-          *reinterpret_cast<uint4*>(dst + i8_swz_offset<D>(r, 2 * cc + 1)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(bar_k4full(u, s));
-        have = next_int4(val);
-        if (have) load_packed(val, w);
-      }
-    }
   } else if (warp >= 4 && warp < 12) {
     // ================================================================ softmax / epilogue
     const int u = (warp - 4) >> 2;               // unit of this warpgroup
     const Unit x = unit_of(u);
     const int r = (threadIdx.x - 128) & 127;     // query row of the unit = TMEM lane
     const int q4 = warp & 3;                     // TMEM lane quarter of this warp
-    const int half = r >> 6, rr = r & 63;
+    const int half = r >> 6, rr = r & 63;        // q-tile of the row (uniform per warp)
     const int qt = x.qt0 + half;
     const bool half_valid = x.valid && qt < x.nt;
     const int tq = qt * kTile + rr;              // query position in the sequence
     const bool row_valid = half_valid && tq < x.T;
     const long long qtile = (long long)x.h * p.ntiles + x.toff + qt;
     const float sq8 = half_valid ? __ldg(p.sq8 + qtile) : 0.0f;
-    // expanded INT4 operands are 16 x code, so INT4 accumulators are 256 x the code
-    // product: the power of two goes into the row's INT4 scale (exact)
+    // INT4 operands are 16 x code, so INT4 accumulators are 256 x the code product:
+    // the power of two goes into the row's INT4 scale (exact)
     const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) * (1.0f / 256.0f) : 0.0f;
     const uint32_t lane_addr = ((uint32_t)(q4 * 32) << 16) + (uint32_t)(u * 256);
     const uint32_t tU = tmem + lane_addr, tO = tU + 128;  // S/P buffer b at tU + 64 * b
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     int i = 0;
-    MergeCursor c = unit_cursor(p, x);
-    // K-tile scale of an entry (1 for BF16), loaded one entry ahead
-    auto kscale = [&](uint32_t v) -> float {
-      const uint32_t pr = v >> 28;
-      const long long kt_ = (long long)x.kvh * p.ntiles + x.toff + (int)(v & 0x0FFFFFFFu);
-      if (pr == TRA_PREC_INT8) return __ldg(p.sk8 + kt_);
-      if (pr == TRA_PREC_INT4 && int4) return __ldg(p.sk4 + kt_);
+    KtMerge c = unit_merge(p, x);
+    // the K-tile scale of this row's precision of an entry (1 for BF16), loaded one
+    // entry ahead
+    auto kscale = [&](int kt_, int pr) -> float {
+      const long long t_ = (long long)x.kvh * p.ntiles + x.toff + kt_;
+      if (pr == TRA_PREC_INT8) return __ldg(p.sk8 + t_);
+      if (pr == TRA_PREC_INT4 && int4) return __ldg(p.sk4 + t_);
       return 1.0f;
     };
-    uint32_t nval = 0;
-    int nmask = 0;
-    bool have = c.next(nval, nmask);
-    float nsk = have ? kscale(nval) : 0.0f;
+    int nkt = 0, np0 = 0, np1 = 0;
+    bool have = c.next(nkt, np0, np1);
+    float nsk = have ? kscale(nkt, half ? np1 : np0) : 0.0f;
     for (; have; ++i) {
-      const uint32_t val = nval;
-      const int mask = nmask;
+      const int kt = nkt, pa = np0, pb = np1;
       const float skt = nsk;
-      have = c.next(nval, nmask);  // look-ahead: list value and scale of the next entry
-      if (have) nsk = kscale(nval);
+      have = c.next(nkt, np0, np1);  // look-ahead: next entry and its scale
+      if (have) nsk = kscale(nkt, half ? np1 : np0);
       const int sb = i & 1;
       const uint32_t tS = tU + sb * 64;
       if (!mbar_wait(bar_sfull(u, sb), (i >> 1) & 1, err)) { ok = false; break; }
-      const uint32_t prec = val >> 28;
-      const int kt = (int)(val & 0x0FFFFFFFu);
-      if (prec == TRA_PREC_INT4 && !int4) {
+      if ((pa == TRA_PREC_INT4 || pb == TRA_PREC_INT4) && !int4) {
         *err = TRA_DEV_BAD_LIST;
         ok = false;
         break;
       }
-      // A half (64 rows = 2 warps) whose q-tile does not list this entry adds
-      // P = 0: its warps skip the TMEM read and every exponential.
-      const bool half_applies = ((mask >> half) & 1) && half_valid;
+      const int prec = half ? pb : pa;  // this row's precision (0: its q-tile skips kt)
+      // A q-tile that does not list this tile adds P = 0: its warps skip the TMEM
+      // read and every exponential.
+      const bool half_applies = prec != 0 && half_valid;
       uint32_t pk[32];
-      bool warp_need = false, warp_rescale_o = false;
+      bool warp_rescale_o = false;
       float alpha = 1.0f;
       if (!half_applies) {
 #pragma unroll
@@ -615,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float m_tile = mx == -INFINITY ? -INFINITY : mx * f;  // f > 0 keeps the argmax
           const float m_new = fmaxf(m_run, m_tile);
           const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
-          warp_need = __any_sync(0xffffffffu, need);
+          const bool warp_need = __any_sync(0xffffffffu, need);
           // O rows that have seen no key yet are exactly zero: no rescale
           warp_rescale_o = __any_sync(0xffffffffu, need && m_run != -INFINITY);
           if (warp_need && m_new > m_run) {
@@ -631,13 +608,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < 64; cc += 2) {
             const float2 arg = __ffma2_rn(make_float2(xs[cc], xs[cc + 1]), f2, nm2);
-            float p0 = ex2(arg.x);
-            float p1 = ex2(arg.y);
+            float q0 = ex2(arg.x);
+            float q1 = ex2(arg.y);
             if (!kFull) {  // masked columns of a row whose max is still -inf
-              p0 = cc < nvalid ? p0 : 0.0f;
-              p1 = cc + 1 < nvalid ? p1 : 0.0f;
+              q0 = cc < nvalid ? q0 : 0.0f;
+              q1 = cc + 1 < nvalid ? q1 : 0.0f;
             }
-            const __nv_bfloat162 pbf = __floats2bfloat162_rn(p0, p1);
+            const __nv_bfloat162 pbf = __floats2bfloat162_rn(q0, q1);
             const uint32_t w = *reinterpret_cast<const uint32_t*>(&pbf);
             ls[(cc >> 1) & 3] = __fadd2_rn(
                 ls[(cc >> 1) & 3],

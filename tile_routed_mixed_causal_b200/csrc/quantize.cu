@@ -4,8 +4,10 @@
 //
 // One CTA per (tensor, head, tile): the 64 x d bf16 tile is read once with
 // 16-byte loads into registers, the absolute maximum is reduced with warp
-// shuffles, and the INT8 codes, packed INT4 codes and both scales are written
-// tile-major.  HBM-bound: 2*64*d bytes in, (1 + 1/2)*64*d bytes + 8 out.
+// shuffles, and the INT8 codes, packed INT4 codes, INT4 codes expanded to the
+// int8 operand form (16 x code) and both scales are written tile-major.
+// HBM-bound: 2*64*d bytes in, per requested format 64*d (INT8, expanded INT4) or
+// 64*d/2 (packed INT4) bytes + 4 (scale) out.
 // Arithmetic: s = fl32(amax / qmax) and code = rne(fl32(x / s)) with IEEE
 // division (__fdiv_rn) and round-half-even conversion (__float2int_rn).
 #include "tra_device.cuh"
@@ -105,6 +107,13 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p) {
       o[0] ^= flip;
       o[1] ^= flip;
       *reinterpret_cast<uint2*>(t.x8 + (tile_base * kTile + r) * D + c * 8) = make_uint2(o[0], o[1]);
+    }
+    if (t.x4x) {  // INT4 codes as int8 operand values 16 x code (exact, |16 x code| <= 112)
+      uint32_t o[2] = {0, 0};
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        o[j >> 2] |= (uint32_t)((quant_code(x[j], s4, 7) * 16) & 0xFF) << ((j & 3) * 8);
+      *reinterpret_cast<uint2*>(t.x4x + (tile_base * kTile + r) * D + c * 8) = make_uint2(o[0], o[1]);
     }
     if (t.x4) {
       uint32_t o = 0;  // byte jj: channels 8c + 2jj (low nibble) and 8c + 2jj + 1

@@ -174,12 +174,21 @@ size_t tra_qtiles_bytes(const tra_shape* shape, uint32_t formats) {
   if (check_shape(shape, &nt, nullptr, nullptr) != TRA_OK) return 0;
   const size_t d = shape->d;
   size_t total = 0;
-  const struct { uint32_t bit; int H; size_t per_row; } f[6] = {
-      {TRA_FMT_Q8, shape->Hq, d}, {TRA_FMT_Q4, shape->Hq, d / 2}, {TRA_FMT_K8, shape->Hkv, d},
-      {TRA_FMT_K4, shape->Hkv, d / 2}, {TRA_FMT_V8, shape->Hkv, d}, {TRA_FMT_V4, shape->Hkv, d / 2}};
-  for (const auto& x : f)
-    if (formats & x.bit)
-      total += round256((size_t)x.H * nt * TRA_TILE * x.per_row) + round256((size_t)x.H * nt * 4);
+  // codes of each format; scales once per (tensor, precision): Q4X / K4X share the
+  // INT4 scales of Q4 / K4
+  const struct { uint32_t bit, scale_bits; int H; size_t per_row; } f[8] = {
+      {TRA_FMT_Q8, TRA_FMT_Q8, shape->Hq, d},
+      {TRA_FMT_Q4, TRA_FMT_Q4 | TRA_FMT_Q4X, shape->Hq, d / 2},
+      {TRA_FMT_K8, TRA_FMT_K8, shape->Hkv, d},
+      {TRA_FMT_K4, TRA_FMT_K4 | TRA_FMT_K4X, shape->Hkv, d / 2},
+      {TRA_FMT_V8, TRA_FMT_V8, shape->Hkv, d},
+      {TRA_FMT_V4, TRA_FMT_V4, shape->Hkv, d / 2},
+      {TRA_FMT_Q4X, 0, shape->Hq, d},
+      {TRA_FMT_K4X, 0, shape->Hkv, d}};
+  for (const auto& x : f) {
+    if (formats & x.bit) total += round256((size_t)x.H * nt * TRA_TILE * x.per_row);
+    if (formats & x.scale_bits) total += round256((size_t)x.H * nt * 4);
+  }
   return total;
 }
 
@@ -190,19 +199,23 @@ tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const u
   if (st != TRA_OK) return st;
   if (!out) return fail(TRA_ERR_INVALID, "out is NULL");
   const uint32_t f = out->formats;
-  if (f & ~0x3Fu) return fail(TRA_ERR_INVALID, "unknown format bits 0x%x", f);
+  if (f & ~0xFFu) return fail(TRA_ERR_INVALID, "unknown format bits 0x%x", f);
   tra::QuantParams p{};
   const uint16_t* src[3] = {q, k, v};
   const int H[3] = {shape->Hq, shape->Hkv, shape->Hkv};
   int8_t* o8[3] = {out->q8, out->k8, out->v8};
   uint8_t* o4[3] = {out->q4, out->k4, out->v4};
+  int8_t* o4x[3] = {out->q4x, out->k4x, nullptr};
+  const uint32_t fx[3] = {TRA_FMT_Q4X, TRA_FMT_K4X, 0u};
   float* s8[3] = {out->sq8, out->sk8, out->sv8};
   float* s4[3] = {out->sq4, out->sk4, out->sv4};
   const char* nm[3] = {"q", "k", "v"};
   p.cta_begin[0] = 0;
   for (int i = 0; i < 3; ++i) {
     const bool want8 = f & (TRA_FMT_Q8 << (2 * i));
-    const bool want4 = f & (TRA_FMT_Q4 << (2 * i));
+    const bool wantp = f & (TRA_FMT_Q4 << (2 * i));  // packed INT4
+    const bool wantx = (f & fx[i]) != 0;              // INT4 as int8 16 x code
+    const bool want4 = wantp || wantx;
     tra::QuantTensor& t = p.t[i];
     t = tra::QuantTensor{};
     if (want8 || want4) {
@@ -210,13 +223,18 @@ tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const u
       if (!aligned16(src[i])) return fail(TRA_ERR_INVALID, "%s not 16-byte aligned", nm[i]);
       if (want8 && (!o8[i] || !s8[i] || !aligned16(o8[i]) || !aligned16(s8[i])))
         return fail(TRA_ERR_INVALID, "%s8 codes/scales missing or misaligned", nm[i]);
-      if (want4 && (!o4[i] || !s4[i] || !aligned16(o4[i]) || !aligned16(s4[i])))
-        return fail(TRA_ERR_INVALID, "%s4 codes/scales missing or misaligned", nm[i]);
+      if (want4 && (!s4[i] || !aligned16(s4[i])))
+        return fail(TRA_ERR_INVALID, "%s4 scales missing or misaligned", nm[i]);
+      if (wantp && (!o4[i] || !aligned16(o4[i])))
+        return fail(TRA_ERR_INVALID, "%s4 codes missing or misaligned", nm[i]);
+      if (wantx && (!o4x[i] || !aligned16(o4x[i])))
+        return fail(TRA_ERR_INVALID, "%s4x codes missing or misaligned", nm[i]);
       t.x = src[i];
       t.H = H[i];
       t.x8 = want8 ? o8[i] : nullptr;
       t.s8 = want8 ? s8[i] : nullptr;
-      t.x4 = want4 ? o4[i] : nullptr;
+      t.x4 = wantp ? o4[i] : nullptr;
+      t.x4x = wantx ? o4x[i] : nullptr;
       t.perm4 = i == 2;  // V4 is read only by the decode, in its MMA fragment order
       t.bias8 = i == 2;  // so is V8, kept offset-binary for its f16 conversion
       t.s4 = want4 ? s4[i] : nullptr;
@@ -333,12 +351,15 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
   if ((tiles->formats & need8) != need8 || !tiles->q8 || !tiles->k8 || !tiles->sq8 || !tiles->sk8)
     return fail(TRA_ERR_INVALID, "prefill needs Q8 and K8 tiles");
   if (!aligned16(tiles->q8) || !aligned16(tiles->k8)) return fail(TRA_ERR_INVALID, "Q8/K8 misaligned");
-  if (policy_has_int4(shape, policy)) {
-    const uint32_t need4 = TRA_FMT_Q4 | TRA_FMT_K4;
-    if ((tiles->formats & need4) != need4 || !tiles->q4 || !tiles->k4 || !tiles->sq4 || !tiles->sk4)
-      return fail(TRA_ERR_INVALID, "the policy has INT4 tiles: Q4 and K4 tiles are required");
-    if (!aligned16(tiles->q4) || !aligned16(tiles->k4)) return fail(TRA_ERR_INVALID, "Q4/K4 misaligned");
+  const bool has4 = policy_has_int4(shape, policy);
+  if (has4) {
+    const uint32_t need4 = TRA_FMT_Q4X | TRA_FMT_K4X;
+    if ((tiles->formats & need4) != need4 || !tiles->q4x || !tiles->k4x || !tiles->sq4 || !tiles->sk4)
+      return fail(TRA_ERR_INVALID,
+                  "the policy has INT4 tiles: Q4X and K4X tiles (INT4 as int8 operands) are required");
+    if (!aligned16(tiles->q4x) || !aligned16(tiles->k4x)) return fail(TRA_ERR_INVALID, "Q4X/K4X misaligned");
   }
+  if (nt_max >= (1ll << 24)) return fail(TRA_ERR_UNSUPPORTED, "a sequence has more than 2^24 tiles");
   if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
     return fail(TRA_ERR_INVALID, "softmax_scale must be positive and finite");
   if (n_dump < 0 || n_dump > TRA_MAX_DUMP) return fail(TRA_ERR_INVALID, "n_dump must be in [0, %d]", TRA_MAX_DUMP);
@@ -356,8 +377,6 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
   p.jmax = (int)((nt_max + 1) / 2);
   p.row_ptr = row_ptr;
   p.entries = entries;
-  p.q4 = tiles->q4;
-  p.k4 = tiles->k4;
   p.sq8 = tiles->sq8;
   p.sq4 = tiles->sq4;
   p.sk8 = tiles->sk8;
@@ -372,8 +391,10 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
   tra::PrefillMaps m;
   memset(&m, 0, sizeof m);
   const int d = shape->d;
-  bool good = map_i8(&m.q8, tiles->q8, d, (int64_t)shape->Hq * nt * TRA_TILE, 128) &&
-              map_i8(&m.k8, tiles->k8, d, (int64_t)shape->Hkv * nt * TRA_TILE, 64) &&
+  const int64_t qrows = (int64_t)shape->Hq * nt * TRA_TILE, krows = (int64_t)shape->Hkv * nt * TRA_TILE;
+  bool good = map_i8(&m.q8, tiles->q8, d, qrows, 128) && map_i8(&m.k8, tiles->k8, d, krows, 64) &&
+              (!has4 || (map_i8(&m.q4x, tiles->q4x, d, qrows, 128) &&
+                         map_i8(&m.k4x, tiles->k4x, d, krows, 64))) &&
               map_bf16(&m.qb, q, d, shape->Hq, ntok, 128) &&
               map_bf16(&m.kb, k, d, shape->Hkv, ntok, 64) &&
               map_bf16(&m.vb, v, d, shape->Hkv, ntok, 64);
@@ -386,7 +407,7 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
 // Decode workspace: arrival counters first, in a region of fixed size for every
 // shape up to kCounterInts of them (so that a workspace reused across shapes keeps
 // them at zero: the partials never land there), then the splits' partials.
-constexpr size_t kCounterInts = 16384;
+constexpr size_t kCounterInts = TRA_NOALLOC_MAX_COUNTERS;
 size_t decode_counter_bytes(int32_t B, int32_t Hkv) {
   const size_t n = (size_t)B * (Hkv + 1);
   return round256(4 * (n > kCounterInts ? n : kCounterInts));
@@ -475,6 +496,148 @@ tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* pol
   if (!good) return fail(TRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
   cudaError_t e = tra::launch_decode(p, m, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+int32_t tra_hybrid_capacity(const tra_shape* shape, double frac) {
+  if (check_shape(shape, nullptr, nullptr, nullptr) != TRA_OK) return -1;
+  if (!(frac >= 0.0 && frac <= 1.0)) return -1;
+  int64_t m = 0;
+  for (int b = 0; b < shape->B; ++b) {
+    const int64_t T = (int64_t)shape->cu_seqlens_host[b + 1] - shape->cu_seqlens_host[b];
+    const int64_t n = std::min<int64_t>(T, (int64_t)std::ceil(frac * (double)T));
+    m = std::max(m, n);
+  }
+  return (int32_t)m;
+}
+
+static tra_status check_hybrid(const tra_shape* shape, const tra_hybrid* hy, int64_t nt) {
+  if (!hy) return fail(TRA_ERR_INVALID, "hybrid arrays are NULL");
+  if (hy->window < 0) return fail(TRA_ERR_INVALID, "window must be >= 0 (got %d)", hy->window);
+  if (hy->cap < 0) return fail(TRA_ERR_INVALID, "cap must be >= 0");
+  if (!hy->sel_count || !hy->sel_pos || !hy->sel_mask || (hy->cap > 0 && (!hy->k_sel || !hy->v_sel)) ||
+      (hy->window > 0 && (!hy->k_win || !hy->v_win)))
+    return fail(TRA_ERR_INVALID, "a hybrid array is NULL");
+  if (!aligned16(hy->sel_mask) || !aligned16(hy->sel_pos) || (hy->k_sel && !aligned16(hy->k_sel)) ||
+      (hy->v_sel && !aligned16(hy->v_sel)) || (hy->k_win && !aligned16(hy->k_win)) ||
+      (hy->v_win && !aligned16(hy->v_win)))
+    return fail(TRA_ERR_INVALID, "hybrid arrays must be 16-byte aligned");
+  (void)shape;
+  (void)nt;
+  return TRA_OK;
+}
+
+tra_status hybrid_select_tokens(const tra_shape* shape, const float* importance, double frac,
+                                const uint16_t* k, const uint16_t* v, const tra_hybrid* hy,
+                                void* stream) {
+  int64_t nt = 0, ntok = 0;
+  tra_status st = check_shape(shape, &nt, &ntok, nullptr);
+  if (st != TRA_OK) return st;
+  if (!(frac >= 0.0 && frac <= 1.0)) return fail(TRA_ERR_INVALID, "frac must lie in [0, 1]");
+  if (!importance || !k || !v) return fail(TRA_ERR_INVALID, "importance, k and v are required");
+  if (!aligned16(k) || !aligned16(v) || (reinterpret_cast<uintptr_t>(importance) & 3u))
+    return fail(TRA_ERR_INVALID, "k / v must be 16-byte aligned, importance 4-byte aligned");
+  st = check_hybrid(shape, hy, nt);
+  if (st != TRA_OK) return st;
+  const int32_t need = tra_hybrid_capacity(shape, frac);
+  if (hy->cap < need) return fail(TRA_ERR_BUFFER, "cap %d < %d selected tokens", hy->cap, need);
+  if (nt == 0) return ok();
+  tra::HybridSelectParams p{};
+  p.cu = shape->cu_seqlens_dev;
+  p.B = shape->B;
+  p.Hkv = shape->Hkv;
+  p.d = shape->d;
+  p.ntiles = (int)nt;
+  p.cap = hy->cap;
+  p.window = hy->window;
+  p.frac = frac;
+  p.imp = importance;
+  p.k = k;
+  p.v = v;
+  p.sel_count = hy->sel_count;
+  p.sel_pos = hy->sel_pos;
+  p.sel_mask = hy->sel_mask;
+  p.k_sel = hy->k_sel;
+  p.v_sel = hy->v_sel;
+  p.k_win = hy->k_win;
+  p.v_win = hy->v_win;
+  cudaError_t e = tra::launch_hybrid_select(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hybrid select launch");
+  return ok();
+}
+
+tra_status hybrid_attention_decode(const tra_shape* shape, const tra_hybrid* hy, const uint16_t* q,
+                                   const uint16_t* k_new, const uint16_t* v_new,
+                                   const tra_qtiles* cache, uint16_t* k_tail, uint16_t* v_tail,
+                                   int32_t* tail_len_dev, int32_t tail_cap, float softmax_scale,
+                                   uint16_t* out, void* workspace, size_t workspace_bytes,
+                                   int32_t* status_dev, void* stream) {
+  int64_t nt = 0, ntok = 0, nt_max = 0;
+  tra_status st = check_shape(shape, &nt, &ntok, &nt_max);
+  if (st != TRA_OK) return st;
+  st = check_hybrid(shape, hy, nt);
+  if (st != TRA_OK) return st;
+  if (shape->Hq / shape->Hkv > 8) return fail(TRA_ERR_UNSUPPORTED, "decode supports Hq/Hkv <= 8");
+  if (!q || !k_new || !v_new || !cache || !k_tail || !v_tail || !tail_len_dev || !out || !workspace ||
+      !status_dev)
+    return fail(TRA_ERR_INVALID, "a required pointer is NULL");
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_tail) ||
+      !aligned16(v_tail) || !aligned16(out) || !aligned16(workspace))
+    return fail(TRA_ERR_INVALID, "q/k_new/v_new/tails/out/workspace must be 16-byte aligned");
+  if (tail_cap < 1) return fail(TRA_ERR_INVALID, "tail_cap must be >= 1");
+  const uint32_t need4 = TRA_FMT_K4 | TRA_FMT_V4;
+  if ((cache->formats & need4) != need4 || !cache->k4 || !cache->v4 || !cache->sk4 || !cache->sv4)
+    return fail(TRA_ERR_INVALID, "the hybrid decode reads K4 and V4 cache tiles");
+  if (!aligned16(cache->k4) || !aligned16(cache->v4)) return fail(TRA_ERR_INVALID, "K4/V4 misaligned");
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
+    return fail(TRA_ERR_INVALID, "softmax_scale must be positive and finite");
+  const size_t need = tra_decode_workspace_bytes(shape->B, shape->Hq, shape->Hkv, shape->d);
+  if (workspace_bytes < need) return fail(TRA_ERR_BUFFER, "workspace needs %zu bytes", need);
+  tra::DecodeParams p{};
+  p.cu = shape->cu_seqlens_dev;
+  p.B = shape->B;
+  p.Hq = shape->Hq;
+  p.Hkv = shape->Hkv;
+  p.d = shape->d;
+  p.ntiles = (int)nt;
+  p.splits = tra::decode_splits(shape->B, shape->Hkv);
+  p.q = q;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.sk4 = cache->sk4;
+  p.sv4 = cache->sv4;
+  p.k_tail = k_tail;
+  p.v_tail = v_tail;
+  p.tail_len = tail_len_dev;
+  p.tail_cap = tail_cap;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  const size_t S = (size_t)p.splits;
+  uint8_t* const ws = reinterpret_cast<uint8_t*>(workspace);
+  p.row_count = reinterpret_cast<int32_t*>(ws);
+  p.seq_count = p.row_count + (size_t)shape->B * shape->Hkv;
+  const size_t off_ml = decode_counter_bytes(shape->B, shape->Hkv);
+  p.part_ml = reinterpret_cast<float*>(ws + off_ml);
+  p.part_o = reinterpret_cast<float*>(ws + off_ml + round256((size_t)shape->B * shape->Hq * S * 2 * 4));
+  p.status = status_dev;
+  p.sel_count = hy->sel_count;
+  p.sel_mask = hy->sel_mask;
+  p.k_sel = hy->k_sel;
+  p.v_sel = hy->v_sel;
+  p.k_win = hy->k_win;
+  p.v_win = hy->v_win;
+  p.sel_cap = hy->cap;
+  p.window = hy->window;
+  tra::DecodeMaps m;
+  memset(&m, 0, sizeof m);
+  const int64_t rows = (int64_t)shape->Hkv * nt * TRA_TILE;
+  bool good = map_i8(&m.k4, cache->k4, shape->d / 2, rows, 64) &&
+              map_i8(&m.v4, cache->v4, shape->d / 2, rows, 64);
+  m.k8 = m.k4;  // (INT8 maps unused: every prefix tile is read in INT4)
+  m.v8 = m.v4;
+  if (!good) return fail(TRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  cudaError_t e = tra::launch_decode(p, m, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hybrid decode launch");
   return ok();
 }
 

@@ -16,6 +16,7 @@ struct QuantTensor {
   int H;
   int8_t* x8;          // nullable
   uint8_t* x4;         // nullable
+  int8_t* x4x;         // nullable: INT4 codes as int8 values 16 x code, row-major
   float* s8;
   float* s4;
   int perm4;           // x4 in the decode's V fragment order (V), else row-major
@@ -51,12 +52,10 @@ struct PrefillParams {
   const int32_t* cu;
   int B, Hq, Hkv, d, ntiles;
   int mode;              // TRA_POLICY_*
-  int has_int4;          // Q4/K4 tiles present (boundary policies with some b1 < b2)
+  int has_int4;          // Q4X/K4X tiles present (boundary policies with some b1 < b2)
   int jmax;              // max over sequences of ceil(nt/2) (q-tile pairs)
   const int32_t* row_ptr;
   const uint32_t* entries;
-  const uint8_t* q4;     // packed INT4 codes [Hq][ntiles][64][d/2]
-  const uint8_t* k4;     // [Hkv][ntiles][64][d/2]
   const float* sq8;
   const float* sq4;
   const float* sk8;
@@ -72,6 +71,7 @@ struct PrefillParams {
 
 struct PrefillMaps {
   CUtensorMap q8, k8;    // int8 tiles, 2-D (d bytes x rows)
+  CUtensorMap q4x, k4x;  // expanded INT4 tiles (int8 16 x code), 2-D like q8 / k8
   CUtensorMap qb, kb, vb;  // bf16, 3-D (d, H, ntok)
 };
 
@@ -101,12 +101,40 @@ struct DecodeParams {
   int32_t* row_count;      // [B][Hkv] splits finished this step (zero between calls)
   int32_t* seq_count;      // [B] rows finished this step (zero between calls)
   int32_t* status;
+  // token-level hybrid (hybrid_attention_decode; null otherwise): every prefix tile is
+  // read in INT4 except its selected / in-window keys, which come from the bf16 side
+  const int32_t* sel_count;
+  const uint64_t* sel_mask;
+  const uint16_t* k_sel;
+  const uint16_t* v_sel;
+  const uint16_t* k_win;
+  const uint16_t* v_win;
+  int sel_cap, window;
 };
 
 struct DecodeMaps {
   CUtensorMap k8, v8;      // int8 codes, 2-D (d bytes x rows), box 64 rows
   CUtensorMap k4, v4;      // packed INT4 codes (d/2 bytes x rows)
 };
+
+// ------------------------------------------------------------ token-level hybrid
+struct HybridSelectParams {
+  const int32_t* cu;
+  int B, Hkv, d, ntiles, cap, window;
+  double frac;
+  const float* imp;        // [ntok][Hkv]
+  const uint16_t* k;       // [ntok][Hkv][d] bf16
+  const uint16_t* v;
+  int32_t* sel_count;      // [B]
+  int32_t* sel_pos;        // [B][Hkv][cap]
+  uint64_t* sel_mask;      // [Hkv][ntiles]
+  uint16_t* k_sel;         // [B][Hkv][cap][d]
+  uint16_t* v_sel;
+  uint16_t* k_win;         // [B][Hkv][window][d]
+  uint16_t* v_win;
+};
+
+cudaError_t launch_hybrid_select(const HybridSelectParams& p, cudaStream_t s);
 
 int decode_splits(int B, int Hkv);
 cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t s);
