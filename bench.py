@@ -23,7 +23,8 @@ replica (the method has no cross-GPU exchange) and rank 0 prints one JSON line.
 Reduced lines (--only): "prefill" times one prefill workload (--workload
 bitmask_32k | llama8b_8k | varlen_8 | mixed_8k), "decode" the decode alone,
 "allocate" fits the complete-tile cost model and runs the boundary allocator on
-synthetic error tables, then times the allocated policy.
+synthetic error tables, then times the allocated policy; "hybrid" times the
+token-level hybrid decode and prefill.
 """
 from __future__ import annotations
 
@@ -410,7 +411,18 @@ def allocate_bench(device, stream, budget_frac=0.5, units=4096, seed=7):
     b2 = [cands[c][1] for c in choice]
     predicted = t0 + float(sum(cost_ms[h, choice[h]] for h in range(H)))
     measured = kernel_ms(b1, b2)
+    # the library's scheduling-aware model: per-entry time and fixed cost fitted on the
+    # same three uniform policies, evaluated on the allocated policy
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    alt = [nt if h % 2 == 0 else nt // 8 for h in range(H)]
+    fitpol = [pol["int8_all"], pol["int8_half"], (alt, alt)]
+    fit_ms = [meas["int8_all"], meas["int8_half"], kernel_ms(alt, alt)]
+    per_entry, fixed, solo = tra.fit_prefill_cost_model(shape, fitpol, fit_ms, n_sm=sms)
+    model_pred = per_entry * tra.prefill_cost_model(shape, b1, b2, solo=solo, n_sm=sms)[0] + fixed
     return {
+        "makespan_model": {"per_entry_us": per_entry * 1e3, "fixed_ms": fixed, "solo": solo,
+                           "predicted_kernel_ms": model_pred,
+                           "predicted_over_measured": model_pred / measured},
         "shape": w.name, "tile_ms_model": {"int8_per_tile_ns": w8 * 1e6, "int4_per_tile_ns": w4 * 1e6,
                                            "fixed_ms": t0},
         "fit_points_ms": meas, "candidates_per_head": C, "budget_frac_of_all_int8": budget_frac,
@@ -543,6 +555,55 @@ def hybrid_bench(device, passes, stream, hbm_gbs, frac=0.05, window=128):
             "select_ms": round(select_ms, 4), "stat": "median of passes",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                          "frac": round(gbs / hbm_gbs, 4)}}
+
+
+def hybrid_prefill_bench(device, stream, bf16_tflops, frac=0.05, window=128, reps=10):
+    """Token-level hybrid prefill (HyQuant, "How HyQuant works": prefill support) on the
+    32K, 32/8-head, d 128 shape: every causal key tile on the tensor cores in bf16, keys
+    outside the 128-token window read from their INT4 codes unless among the 5% selected.
+    Times one hybrid_attention_prefill call (mixed-operand build + attention) with inputs
+    larger than L2; roofline: dense causal QK + PV ops at the measured bf16 rate."""
+    import tile_routed_mixed_causal_b200 as tra
+    from tile_routed_mixed_causal_b200 import api
+    from tile_routed_mixed_causal_b200 import workloads as wl
+
+    w = wl.bitmask_32k()
+    t = wl.make_inputs(w, device)
+    shape = tra.Shape(w.cu_seqlens, w.Hq, w.Hkv, w.d, device=device)
+    plan = api.HybridPrefillPlan(shape, frac, window, device)
+    imp = torch.from_numpy(wl.hybrid_importance(w, 7).astype(np.float32)).to(device)
+    out = torch.empty_like(t["q"])
+    with torch.cuda.stream(stream):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        plan.prepare(t["k"], t["v"], imp, stream=stream)
+        b.record(stream)
+        times = []
+        for it in range(reps + 3):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            plan.attend(t["q"], t["k"], t["v"], out, stream=stream)
+            e1.record(stream)
+            stream.synchronize()
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+    assert int(plan.status.item()) == 0, "hybrid prefill reported a device error"
+    prep_ms = a.elapsed_time(b)
+    ms = statistics.median(times)
+    tiles = sum(n * (n + 1) // 2 for n in w.tiles_per_seq) * w.Hq
+    ops = tiles * 2 * (2 * 64 * 64 * w.d)
+    t_roof = ops / (bf16_tflops * 1e12)
+    achieved = ops / (ms * 1e-3) / 1e12
+    return {"metric": "hybrid prefill TOPS", "value": round(achieved, 1), "unit": "TOPS",
+            "workload": f"hybrid_prefill_t{w.lengths[0]}_h{w.Hq}_{w.Hkv}_d{w.d} ({frac:.0%} "
+                        f"selected, {window}-token window bf16, other keys INT4)",
+            "ms": round(ms, 4), "prep_ms": round(prep_ms, 4), "causal_tiles": tiles,
+            "stat": "median of calls",
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_tflops,
+                         "unit": "TFLOP/s", "frac": round(t_roof / (ms * 1e-3), 4),
+                         "kernel": "hybrid_mix_kernel + prefill_kernel<128, hybrid> (one ABI call)"}}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -704,6 +765,9 @@ def main():
         if rank == 0:
             print(json.dumps({"only": "hybrid", **hybrid_bench(device, args.decode_passes, stream,
                                                               hbm_gbs)}), flush=True)
+            torch.cuda.empty_cache()
+            print(json.dumps({"only": "hybrid_prefill",
+                              **hybrid_prefill_bench(device, stream, bf16_tflops)}), flush=True)
         return
     if args.only == "allocate":
         if rank == 0:
@@ -763,10 +827,13 @@ def main():
             dec["roofline"].update(achieved=round(gbs / world, 1),
                                    frac=round(gbs / world / hbm_gbs, 4))
 
-    recs = alloc = hyb = None
+    recs = alloc = hyb = hyp = None
     if not args.no_decode:
         torch.cuda.empty_cache()
         hyb = hybrid_bench(device, args.decode_passes, stream, hbm_gbs)
+    if not args.no_workloads:
+        torch.cuda.empty_cache()
+        hyp = hybrid_prefill_bench(device, stream, bf16_tflops)
     if not args.no_workloads:
         base_S = S.pop("plan", None)
         del base_S
@@ -826,6 +893,8 @@ def main():
             line["allocate"] = alloc
         if hyb is not None:
             line["hybrid_decode"] = hyb
+        if hyp is not None:
+            line["hybrid_prefill"] = hyp
         if base is not None:
             line["cpu_baseline"] = base
         print(json.dumps(line), flush=True)

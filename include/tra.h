@@ -388,6 +388,31 @@ TRA_API tra_status hybrid_attention_decode(const tra_shape* prefill_shape, const
                                            void* workspace, size_t workspace_bytes,
                                            int32_t* status_dev, void* stream);
 
+/*
+ * hybrid_attention_prefill -- causal prefill attention of the token-level hybrid
+ * (HyQuant Uses Hybrid Precision to Compress LLM Attention, "How HyQuant works":
+ * prefill support with dedicated kernels).  Query i of a sequence reads key j <= i
+ * with bf16 K and V when j is selected (hy->sel_mask, from hybrid_select_tokens on
+ * the same shape) or i - j < hy->window, and from the INT4 codes of j's tile times
+ * the tile scale (K4 and V4 of quantize_qkv_tiles) otherwise; one softmax per row.
+ *   q bf16 [ntok][Hq][d]; k, v bf16 [ntok][Hkv][d]; kv: the INT4 scales sk4 and sv4
+ *   (formats K4 or K4X, and V4; the codes are not read: they are recomputed from k,
+ *   v and those scales exactly as the quantiser computes them);
+ *   k_mix, v_mix: caller-owned scratch, bf16 [ntok][Hkv][d], written by this call:
+ *   each row is the token's bf16 row when it is selected, else its INT4 codes as
+ *   bf16 integers (the operands of the tiles outside the window);
+ *   out bf16 [ntok][Hq][d]; lse fp32 [Hq][ntok] (natural log of the row's sum of
+ *   exp of scaled scores) or NULL.  Two launches (operand build, attention), no
+ *   synchronisation.  Device-side errors (a bounded wait expired) are OR-ed into
+ *   *status_dev.  TRA_ERR_INVALID for NULL or misaligned pointers, a missing
+ *   scale array, window < 0 or a bad softmax_scale.
+ */
+TRA_API tra_status hybrid_attention_prefill(const tra_shape* shape, const tra_hybrid* hy,
+                                            const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                            const tra_qtiles* kv, uint16_t* k_mix, uint16_t* v_mix,
+                                            float softmax_scale, uint16_t* out, float* lse,
+                                            int32_t* status_dev, void* stream);
+
 /* Complete-tile counts of one head's boundary pair over a batch (TriAttention
  * abstract: candidate boundary pairs are weighed by complete-tile execution costs):
  * n8 = sum over every sequence's q-tiles qt of min(qt + 1, b1), n4 = the sum of
@@ -396,6 +421,24 @@ TRA_API tra_status hybrid_attention_decode(const tra_shape* prefill_shape, const
  * NULL outputs, or not 1 <= b1 <= b2. */
 TRA_API tra_status tra_boundary_tile_counts(const tra_shape* shape, int32_t b1, int32_t b2,
                                             int64_t* n8, int64_t* n4);
+
+/* Complete-tile cost model of routed_attention_prefill under a boundary policy (TriAttention
+ * abstract: candidate boundary pairs are weighed by complete-tile execution costs).  Host
+ * only.  The prefill runs one work unit per (query head, sequence, q-tile pair) and two
+ * units per CTA; a unit's work is its entries -- the k-tiles either of its two q-tiles
+ * lists -- counting dual_weight for an entry the two q-tiles give different precisions
+ * (two score products, one P V) and 1 for the others; the two units of a CTA run side by
+ * side until the lighter one ends, then the heavier one runs alone, `solo` times as long
+ * per entry (it no longer shares the SM): CTA time = min(w0, w1) + solo * |w0 - w1|;
+ * CTAs are placed in launch order on n_sm SMs, each on the SM that frees first.
+ * *makespan receives the resulting time in entry units and *entries the total entry
+ * count, so that a kernel time is predicted as entry_time * makespan + fixed with
+ * entry_time, fixed and solo fitted from measured launches.  b1 / b2: host [Hq].
+ * TRA_ERR_INVALID for an invalid shape or policy, dual_weight < 1, solo not in (0, 1]
+ * or n_sm < 1. */
+TRA_API tra_status tra_prefill_cost_model(const tra_shape* shape, const int32_t* b1, const int32_t* b2,
+                                          double dual_weight, double solo, int32_t n_sm,
+                                          double* makespan, double* entries);
 
 /* Model-wide boundary allocation (TriAttention abstract: an allocator selects each
  * head's boundaries to minimise calibration error under a shared computation budget).

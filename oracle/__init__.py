@@ -354,9 +354,12 @@ def hybrid_select(importance, cu_seqlens, frac=0.05):
 
 
 def hybrid_prefill(q_bits, k_bits, v_bits, cu_seqlens, kv: Quantised, selected, window,
-                   scale=None):
+                   scale=None, rows=None, with_lse=False):
     """fp64 output [ntok, Hq, d]: causal attention in which query i reads key j <= i (same
-    sequence) at bf16 when j is selected or i - j < window, else from its INT4 tile."""
+    sequence) at bf16 when j is selected or i - j < window, else from its INT4 tile.
+    rows: optional global query-token indices; only those rows are computed (the others
+    stay zero), each exactly as in the full computation.  with_lse: also return lse
+    [Hq, ntok], the natural log of the row's sum of exp of the scaled scores."""
     q = _f64(q_bits); k = _f64(k_bits); v = _f64(v_bits)
     cu = _c(cu_seqlens, np.int32)
     ntok, Hq, d = q.shape
@@ -365,26 +368,35 @@ def hybrid_prefill(q_bits, k_bits, v_bits, cu_seqlens, kv: Quantised, selected, 
     scale = 1.0 / np.sqrt(d) if scale is None else scale
     k4 = _int4_values(kv.k4, kv.sk4, cu, Hkv)
     v4 = _int4_values(kv.v4, kv.sv4, cu, Hkv)
+    want = np.ones(ntok, bool)
+    if rows is not None:
+        want = np.zeros(ntok, bool)
+        want[np.asarray(rows, np.int64)] = True
     out = np.zeros((ntok, Hq, d), np.float64)
+    lse = np.zeros((Hq, ntok), np.float64)
     for b in range(len(cu) - 1):
         s, e = int(cu[b]), int(cu[b + 1])
         T = e - s
-        if T == 0:
+        ii = np.nonzero(want[s:e])[0]
+        if T == 0 or len(ii) == 0:
             continue
-        i = np.arange(T)[:, None]
+        i = ii[:, None]
         j = np.arange(T)[None, :]
         causal = j <= i
         for h in range(Hq):
             kh = h // g
             hi = selected[s:e, kh][None, :] | (i - j < window)
-            s_hi = q[s:e, h] @ k[s:e, kh].T
-            s_lo = q[s:e, h] @ k4[s:e, kh].T
+            s_hi = q[s + ii, h] @ k[s:e, kh].T
+            s_lo = q[s + ii, h] @ k4[s:e, kh].T
             sc = np.where(hi, s_hi, s_lo) * scale
             sc = np.where(causal, sc, -np.inf)
-            p = np.exp(sc - sc.max(axis=1, keepdims=True))
-            p /= p.sum(axis=1, keepdims=True)
-            out[s:e, h] = (p * hi) @ v[s:e, kh] + (p * ~hi) @ v4[s:e, kh]
-    return out
+            mx = sc.max(axis=1, keepdims=True)
+            p = np.exp(sc - mx)
+            tot = p.sum(axis=1, keepdims=True)
+            lse[h, s + ii] = (mx + np.log(tot))[:, 0]
+            p /= tot
+            out[s + ii, h] = (p * hi) @ v[s:e, kh] + (p * ~hi) @ v4[s:e, kh]
+    return (out, lse) if with_lse else out
 
 
 def hybrid_decode_step(qd_bits, k_bits, v_bits, cu_seqlens, kv: Quantised, selected, window,

@@ -97,3 +97,55 @@ def test_allocator_validation(lib):
     with pytest.raises(L.TraError) as e:                       # table too large
         L.allocate_boundaries(err, cost, 1 << 27)
     assert e.value.status == 2
+
+
+def test_prefill_cost_model_counts_entries_of_the_oracle_lists():
+    """The cost model's entries are the k-tiles either q-tile of a unit lists (from the
+    oracle's traversal lists), duals those the two q-tiles give different precisions; with
+    one SM the makespan is the sum over CTAs (two units each) of the heavier unit's work."""
+    import oracle
+    from tile_routed_mixed_causal_b200 import _lib as L
+    lengths = [300, 64, 1, 700]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    Hq, Hkv = 4, 2
+    b1 = np.array([1, 2, 3, 1], np.int32)
+    b2 = np.array([4, 2, 9, 6], np.int32)
+    shape = L.Shape(cu, Hq, Hkv, 64, device=None)
+    rp, en = oracle.lists_boundary(cu, b1, b2)
+    nts = [(int(x) + 63) // 64 for x in lengths]
+    off = np.concatenate([[0], np.cumsum(nts)])
+    ntiles = int(off[-1])
+    jmax = (max(nts) + 1) // 2
+    dw = 1.5
+
+    def row(h, b, qt):
+        if qt >= nts[b]:
+            return {}
+        r = h * ntiles + off[b] + qt
+        return {int(e & 0x0FFFFFFF): int(e >> 28) for e in en[rp[r]:rp[r + 1]]}
+
+    def unit(uid):
+        h, b, j = uid % Hq, (uid // Hq) % len(lengths), jmax - 1 - uid // (Hq * len(lengths))
+        r0, r1 = row(h, b, 2 * j), row(h, b, 2 * j + 1)
+        kts = set(r0) | set(r1)
+        w = sum(dw if (kt in r0 and kt in r1 and r0[kt] != r1[kt]) else 1.0 for kt in kts)
+        return w, len(kts)
+
+    units = jmax * len(lengths) * Hq
+    total = sum(unit(u)[1] for u in range(units))
+    serial = sum(max(unit(2 * c)[0], unit(2 * c + 1)[0] if 2 * c + 1 < units else 0.0)
+                 for c in range((units + 1) // 2))
+    ms, ne = L.prefill_cost_model(shape, b1, b2, dual_weight=dw, solo=1.0, n_sm=1)
+    assert ne == total and abs(ms - serial) < 1e-9
+    ms_many, _ = L.prefill_cost_model(shape, b1, b2, dual_weight=dw, solo=1.0, n_sm=1000)
+    assert ms_many == max(max(unit(2 * c)[0], unit(2 * c + 1)[0] if 2 * c + 1 < units else 0.0)
+                          for c in range((units + 1) // 2))
+    # a CTA's lighter unit ends first; the rest of the heavier one runs `solo` times as long
+    solo = 0.6
+    ms_solo, _ = L.prefill_cost_model(shape, b1, b2, dual_weight=dw, solo=solo, n_sm=1)
+
+    def cta(c):
+        w0 = unit(2 * c)[0]
+        w1 = unit(2 * c + 1)[0] if 2 * c + 1 < units else 0.0
+        return min(w0, w1) + solo * abs(w0 - w1)
+    assert abs(ms_solo - sum(cta(c) for c in range((units + 1) // 2))) < 1e-9

@@ -1,6 +1,7 @@
 """GPU parity of the token-level hybrid (HyQuant Uses Hybrid Precision to Compress LLM
-Attention, "How HyQuant works"): token selection bit-exact against the oracle's
-selection, decode steps within the output tolerance of the other GPU parity tests.
+Attention, "How HyQuant works"): token selection and the prefill's mixed operands
+bit-exact against the oracle's selection and codes, prefill rows and decode steps within
+the output tolerance of the other GPU parity tests.
 
 Selection: per (sequence, KV head) the ceil(frac * T) positions of largest importance,
 ties to the earlier position; importance is handed to both sides in fp32.
@@ -43,9 +44,10 @@ def _importance(w, seed, ties=False):
 
 
 class HybridCase:
-    def __init__(self, w, frac, window, seed, gen_device="cpu", ties=False):
+    def __init__(self, w, frac, window, seed, gen_device="cpu", ties=False, need_q=False):
         self.w, self.frac, self.window = w, frac, window
-        t = wl.make_inputs(w, gen_device, need_q=False)
+        t = wl.make_inputs(w, gen_device, need_q=need_q)
+        self.q = t["q"].cuda() if need_q else None
         self.k, self.v = t["k"].cuda(), t["v"].cuda()
         self.kb, self.vb = wl.bf16_bits(t["k"]), wl.bf16_bits(t["v"])
         self.shape = tra.Shape(w.cu_seqlens, w.Hq, w.Hkv, w.d)
@@ -151,3 +153,106 @@ def test_hybrid_decode_full_size_sampled():
             ref = oracle.hybrid_decode_step(wl.bf16_bits(qs[step, b:b + 1]), kb, vb, cu1, kv, sel,
                                             128, kt, vt, np.array([step + 1], np.int32))
             _assert_close(outs[step][b], ref[0], f"hybrid b={b} step={step}")
+
+
+# --------------------------------------------------------------------------- prefill
+LSE_TOL = 2.0 ** -8
+
+
+def _codes4(x4):
+    """[H][nt][64][d/2] packed INT4 (even channel in the low nibble) -> int codes [H][nt][64][d]."""
+    x4 = np.asarray(x4, np.uint8)
+    lo = (x4 & 0xF).astype(np.int16)
+    hi = (x4 >> 4).astype(np.int16)
+    out = np.empty(x4.shape[:-1] + (2 * x4.shape[-1],), np.int16)
+    out[..., 0::2] = np.where(lo > 7, lo - 16, lo)
+    out[..., 1::2] = np.where(hi > 7, hi - 16, hi)
+    return out
+
+
+def _tiles_to_tokens(codes, cu):
+    """[H][ntiles][64][d] -> [ntok][H][d] (rows past a sequence's end dropped)."""
+    rows = []
+    t0 = 0
+    for b in range(len(cu) - 1):
+        T = int(cu[b + 1] - cu[b])
+        nt = (T + 63) // 64
+        rows.append(codes[:, t0:t0 + nt].reshape(codes.shape[0], nt * 64, -1)[:, :T])
+        t0 += nt
+    return np.concatenate(rows, axis=1).transpose(1, 0, 2)
+
+
+def _bf16_of_ints(c):
+    return (np.asarray(c, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _run_hybrid_prefill(c, with_lse=True):
+    w = c.w
+    k_mix = torch.zeros((w.ntok, w.Hkv, w.d), dtype=torch.bfloat16, device="cuda")
+    v_mix = torch.zeros_like(k_mix)
+    out = torch.full((w.ntok, w.Hq, w.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((w.Hq, w.ntok), dtype=torch.float32, device="cuda") if with_lse else None
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tra.hybrid_attention_prefill(c.shape, c.plan.hy, c.q, c.k, c.v, c.cache, k_mix, v_mix,
+                                 1.0 / math.sqrt(w.d), out, lse, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return k_mix, v_mix, out, lse
+
+
+HSMALL = SMALL + [
+    (wl.custom("hy_win100", [64 * 7 + 5, 129], 8, 2, 128, 85, "boundary"), 0.05, 100),
+    (wl.custom("hy_win300_d64", [900, 3], 4, 2, 64, 86, "boundary"), 0.1, 300),
+    (wl.custom("hy_win64_g8", [64 * 6], 8, 1, 128, 87, "boundary"), 0.05, 64),
+    # rows of one warp that meet their first keys in different entries (window edges)
+    (wl.custom("hy_win200", [64 * 7 + 5, 129], 8, 2, 128, 85, "boundary"), 0.05, 200),
+    (wl.custom("hy_win1", [64 * 5 + 9, 70], 4, 2, 128, 88, "boundary"), 0.0, 1),
+]
+
+
+@pytest.mark.parametrize("w,frac,window", HSMALL, ids=lambda x: getattr(x, "name", str(x)))
+def test_hybrid_prefill_matches_oracle(w, frac, window):
+    """Every row against the oracle (selection from the oracle, which the selection test
+    shows is the GPU's), and the mixed operands bit for bit: a selected token's bf16
+    row, else its INT4 codes from the oracle's quantiser as bf16 integers."""
+    c = HybridCase(w, frac, window, seed=9, need_q=True)
+    k_mix, v_mix, out, lse = _run_hybrid_prefill(c)
+    cu = w.cu_seqlens
+    kv = oracle.Quantised(None, c.kb, c.vb, cu)
+    sel = c.sel[:, :, None]
+    want_k = np.where(sel, c.kb, _bf16_of_ints(_tiles_to_tokens(_codes4(kv.k4), cu)))
+    want_v = np.where(sel, c.vb, _bf16_of_ints(_tiles_to_tokens(_codes4(kv.v4), cu)))
+    assert np.array_equal(wl.bf16_bits(k_mix), want_k)
+    assert np.array_equal(wl.bf16_bits(v_mix), want_v)
+    ref, ref_lse = oracle.hybrid_prefill(wl.bf16_bits(c.q), c.kb, c.vb, cu, kv, c.sel, window,
+                                         with_lse=True)
+    _assert_close(out.float().cpu().numpy(), ref, w.name)
+    assert np.max(np.abs(lse.cpu().numpy() - ref_lse)) <= LSE_TOL
+
+
+def test_hybrid_prefill_plan_end_to_end():
+    """HybridPrefillPlan (quantise K/V, select, attend) equals the calls made one by one."""
+    w, frac, window = HSMALL[0]
+    c = HybridCase(w, frac, window, seed=9, need_q=True)
+    _, _, out_ref, _ = _run_hybrid_prefill(c, with_lse=False)
+    plan = api.HybridPrefillPlan(c.shape, frac, window)
+    out = torch.zeros_like(out_ref)
+    plan.run(c.q, c.k, c.v, torch.from_numpy(c.imp).cuda(), out)
+    torch.cuda.synchronize()
+    assert int(plan.status.item()) == 0
+    assert torch.equal(out.view(torch.int16), out_ref.view(torch.int16))
+
+
+def test_hybrid_prefill_full_size_sampled():
+    """32K context, 32/8 heads, d 128, 5% selected, 128-token window (the benchmarked
+    hybrid prefill): sampled rows around tile and window edges against the oracle."""
+    w = wl.bitmask_32k()
+    c = HybridCase(w, 0.05, 128, seed=10, gen_device="cuda", need_q=True)
+    _, _, out, lse = _run_hybrid_prefill(c)
+    rows = np.array([0, 1, 63, 64, 127, 128, 129, 191, 192, 255, 1000, 4095, 4096, 16383,
+                     20000, 32766, 32767])
+    kv = oracle.Quantised(None, c.kb, c.vb, w.cu_seqlens)
+    ref, ref_lse = oracle.hybrid_prefill(wl.bf16_bits(c.q), c.kb, c.vb, w.cu_seqlens, kv, c.sel,
+                                         128, rows=rows, with_lse=True)
+    _assert_close(out.float().cpu().numpy()[rows], ref[rows], "hybrid prefill 32K")
+    assert np.max(np.abs(lse.cpu().numpy()[:, rows] - ref_lse[:, rows])) <= LSE_TOL

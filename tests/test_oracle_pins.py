@@ -618,6 +618,32 @@ def test_hybrid_prefill_mixes_per_key_and_rows_sum_to_one():
     assert diff[j + 16:300, heads].max() > 0.0
 
 
+def test_hybrid_prefill_row_subset_and_lse():
+    """A row subset is the same rows of the full computation; with every key in bf16 the
+    lse is scipy's logsumexp of the row's scaled causal scores, and nothing-in-bf16 moves
+    it only through the INT4 keys."""
+    from scipy.special import logsumexp
+    w, q, k, v, cu, kv = _hybrid_case()
+    sel = oracle.hybrid_select(wl.hybrid_importance(w, 8), cu, 0.05)
+    full, lse_full = oracle.hybrid_prefill(q, k, v, cu, kv, sel, 16, with_lse=True)
+    rows = np.array([0, 63, 64, 299, 300, 364, 365, 400, w.ntok - 1])
+    part, lse_part = oracle.hybrid_prefill(q, k, v, cu, kv, sel, 16, rows=rows, with_lse=True)
+    assert np.max(np.abs(part[rows] - full[rows])) < 1e-13
+    assert np.max(np.abs(lse_part[:, rows] - lse_full[:, rows])) < 1e-13
+    rest = np.setdiff1d(np.arange(w.ntok), rows)
+    assert not part[rest].any() and not lse_part[:, rest].any()
+    every = np.ones((w.ntok, w.Hkv), bool)
+    _, lse = oracle.hybrid_prefill(q, k, v, cu, kv, every, 0, with_lse=True)
+    qv, kvv = val_of(q), val_of(k)
+    g = w.Hq // w.Hkv
+    for b in range(len(cu) - 1):
+        s, e = int(cu[b]), int(cu[b + 1])
+        for i in range(s, e, 7):
+            for h in range(w.Hq):
+                sc = kvv[s:i + 1, h // g] @ qv[i, h] / np.sqrt(w.d)
+                assert abs(lse[h, i] - logsumexp(sc)) < 1e-12
+
+
 def test_hybrid_decode_reduces_to_dense_softmax():
     """One decode step: all prefix keys in bf16 gives the textbook softmax over the prefix
     plus the tail; none gives it over the INT4-dequantised prefix plus the tail."""

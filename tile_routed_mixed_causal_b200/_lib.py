@@ -87,8 +87,10 @@ def load():
         "tra_boundary_tile_counts": ([P, I32, I32, P, P], I32),
         "tra_allocate_boundaries": ([I32, I32, P, P, I64, P, P, P], I32),
         "tra_hybrid_capacity": ([P, ctypes.c_double], I32),
+        "tra_prefill_cost_model": ([P, P, P, ctypes.c_double, ctypes.c_double, I32, P, P], I32),
         "hybrid_select_tokens": ([P, P, ctypes.c_double, P, P, P, P], I32),
         "hybrid_attention_decode": ([P, P, P, P, P, P, P, P, P, I32, F, P, P, SZ, P, P], I32),
+        "hybrid_attention_prefill": ([P, P, P, P, P, P, P, P, F, P, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -323,12 +325,49 @@ def hybrid_attention_decode(shape: Shape, hy: Hybrid, q, k_new, v_new, cache: QT
         workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
 
 
+def hybrid_attention_prefill(shape: Shape, hy: Hybrid, q, k, v, kv: QTiles, k_mix, v_mix,
+                             softmax_scale, out, lse, status, stream=None):
+    _check(load().hybrid_attention_prefill(
+        shape.c, hy.c, _ptr(q), _ptr(k), _ptr(v), kv.c, _ptr(k_mix), _ptr(v_mix),
+        float(softmax_scale), _ptr(out), _ptr(lse) if lse is not None else None, _ptr(status),
+        _stream(stream)))
+
+
 def boundary_tile_counts(shape: Shape, b1: int, b2: int):
     """(INT8 tiles, INT4 tiles) of one head's boundary pair over the batch."""
     n8, n4 = ctypes.c_int64(), ctypes.c_int64()
     _check(load().tra_boundary_tile_counts(shape.c, int(b1), int(b2), ctypes.byref(n8),
                                            ctypes.byref(n4)))
     return n8.value, n4.value
+
+
+def prefill_cost_model(shape: Shape, b1, b2, dual_weight: float = 1.25, solo: float = 1.0,
+                       n_sm: int = 148):
+    """(makespan in entry units, total entries) of the prefill under boundaries b1 / b2
+    (host arrays [Hq]); see tra_prefill_cost_model in include/tra.h."""
+    b1 = np.ascontiguousarray(np.asarray(b1, np.int32))
+    b2 = np.ascontiguousarray(np.asarray(b2, np.int32))
+    ms, ne = ctypes.c_double(), ctypes.c_double()
+    _check(load().tra_prefill_cost_model(shape.c, _ptr(b1), _ptr(b2), float(dual_weight),
+                                         float(solo), int(n_sm), ctypes.byref(ms), ctypes.byref(ne)))
+    return ms.value, ne.value
+
+
+def fit_prefill_cost_model(shape: Shape, policies, times_ms, dual_weight: float = 1.25,
+                           n_sm: int = 148):
+    """Fit (entry_time_ms, fixed_ms, solo) of tra_prefill_cost_model to measured kernel times of
+    boundary policies [(b1, b2), ...]: least squares in the two linear constants for each
+    solo on a grid over (0, 1], keeping the best.  Host arithmetic only."""
+    best = None
+    y = np.asarray(times_ms, np.float64)
+    for solo in np.linspace(0.3, 1.0, 36):
+        X = np.array([[prefill_cost_model(shape, b1, b2, dual_weight, solo, n_sm)[0], 1.0]
+                      for b1, b2 in policies])
+        coef, *_ = np.linalg.lstsq(X, y, rcond=None)
+        res = float(np.sum((X @ coef - y) ** 2))
+        if best is None or res < best[0]:
+            best = (res, float(coef[0]), float(coef[1]), float(solo))
+    return best[1], best[2], best[3]
 
 
 def allocate_boundaries(err, cost, budget: int):

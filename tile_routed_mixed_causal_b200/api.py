@@ -6,6 +6,8 @@ per step, over the K/V tiles a PrefillPlan (or quantize_qkv_tiles) produced.
 ``HybridDecodePlan``: hybrid_select_tokens (once, over the prefix) ->
 hybrid_attention_decode per step (token-level hybrid: INT4 tiles plus bf16 selected
 and recent tokens).
+``HybridPrefillPlan``: quantize_qkv_tiles (K and V INT4 scales) ->
+hybrid_select_tokens -> hybrid_attention_prefill.
 Buffers are allocated once per plan; ``run``/``step`` only enqueue kernels.  The
 decode workspace is zero-filled once (the decode's arrival counters need that, and
 every step leaves them at zero).
@@ -103,3 +105,32 @@ class HybridDecodePlan:
         L.hybrid_attention_decode(self.shape, self.hy, q, k_new, v_new, self.cache, self.k_tail,
                                   self.v_tail, self.tail_len, scale, out, self.workspace,
                                   self.status, stream)
+
+
+class HybridPrefillPlan:
+    """Causal prefill of the token-level hybrid: keys outside the query's window are read
+    from their INT4 tile unless selected; the selection also serves a HybridDecodePlan."""
+
+    def __init__(self, shape: L.Shape, frac: float, window: int, device="cuda"):
+        self.shape = shape
+        self.tiles = L.QTiles(shape, L.FMT_K4 | L.FMT_V4, device)
+        self.hy = L.Hybrid(shape, frac, window, device)
+        ntok = int(shape.cu_host[-1])
+        self.k_mix = torch.zeros((max(ntok, 1), shape.Hkv, shape.d), dtype=torch.bfloat16,
+                                 device=device)
+        self.v_mix = torch.zeros_like(self.k_mix)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def prepare(self, k, v, importance, stream=None):
+        """Quantise K and V (INT4 scales) and select the bf16 tokens."""
+        L.quantize_qkv_tiles(self.shape, None, k, v, self.tiles, stream)
+        L.hybrid_select_tokens(self.shape, importance, self.hy.frac, k, v, self.hy, stream)
+
+    def attend(self, q, k, v, out, lse=None, scale=None, stream=None):
+        scale = 1.0 / math.sqrt(self.shape.d) if scale is None else scale
+        L.hybrid_attention_prefill(self.shape, self.hy, q, k, v, self.tiles, self.k_mix,
+                                   self.v_mix, scale, out, lse, self.status, stream)
+
+    def run(self, q, k, v, importance, out, lse=None, scale=None, stream=None):
+        self.prepare(k, v, importance, stream)
+        self.attend(q, k, v, out, lse, scale, stream)

@@ -468,8 +468,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 #pragma unroll
     for (int mq = 0; mq < C::kQM; ++mq)
       qsig[mq] = real[mq] ? ldexpf(1.0f, qe[tq + 4 * mq] - F) : 0.0f;
+    // hybrid: the selected-key mask of this warp's next tile, loaded a tile ahead
+    uint64_t hi_next = (HYB && warp < ntile)
+                           ? __ldg(p.sel_mask + (long long)kvh * p.ntiles + toff + my0 + warp) : 0ull;
     for (int i = warp; i < ntile; i += kConsumers) {
       const int s = i % kDecStages;
+      const uint64_t hi_sel = hi_next;
+      if (HYB && i + kConsumers < ntile)
+        hi_next = __ldg(p.sel_mask + (long long)kvh * p.ntiles + toff + my0 + i + kConsumers);
       // Stage s last held tile i - kDecStages, which another warp consumes.  A
       // parity wait only tells adjacent phases apart, so this warp first waits for
       // that tile's release (which the load of tile i needs anyway): only then is the
@@ -550,7 +556,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       if (HYB) {
         // selected keys and keys within the window of the query (position T + tl) are
         // read in bf16 by the row pass: masked out of their INT4 tile here
-        uint64_t hi = __ldg(p.sel_mask + tile);
+        uint64_t hi = hi_sel;
         const int wlo = T + tl - p.window + 1 - kt * kTile;  // first in-window key of the tile
         if (p.window > 0 && wlo < kTile) hi |= wlo <= 0 ? ~0ull : (~0ull << wlo);
         if (hi) {

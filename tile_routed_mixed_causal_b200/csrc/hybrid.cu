@@ -1,16 +1,22 @@
-// hybrid.cu -- token selection for the token-level hybrid (HyQuant Uses Hybrid
-// Precision to Compress LLM Attention, "The observation behind the method" and
-// "How HyQuant works": a small set of important key positions -- vertical lines
-// in the attention map -- and a recent window keep high precision, the rest of
-// the context is read from quantised storage).
+// hybrid.cu -- token selection and the prefill's mixed operands for the
+// token-level hybrid (HyQuant Uses Hybrid Precision to Compress LLM Attention,
+// "The observation behind the method" and "How HyQuant works": a small set of
+// important key positions -- vertical lines in the attention map -- and a recent
+// window keep high precision, the rest of the context is read from quantised
+// storage).
 //
-// One CTA per (sequence, KV head).  The n = ceil(frac * T) positions of largest
-// importance (ties to the earlier position) are found by a radix select over
-// unique 64-bit keys (orderable importance bits above the complemented
+// Selection: one CTA per (sequence, KV head).  The n = ceil(frac * T) positions of
+// largest importance (ties to the earlier position) are found by a radix select
+// over unique 64-bit keys (orderable importance bits above the complemented
 // position), then written in ascending order, as a 64-bit mask per 64-token tile,
 // and as a compact bf16 copy of their K and V rows; the last `window` prefix
 // tokens are copied too.  Together these are the high-precision side of the
 // hybrid KV cache that the decode reads beside the INT4 tiles.
+//
+// Mixed operands: one CTA per (tile, KV head) writes K and V rows that are the
+// bf16 row of a selected token and the INT4 code row of any other, the form in
+// which the hybrid prefill's tensor-core tiles read keys and values outside the
+// window.
 #include "tra_device.cuh"
 #include "tra_launch.h"
 
@@ -140,7 +146,67 @@ __global__ void __launch_bounds__(kSelThreads) hybrid_select_kernel(const Hybrid
   }
 }
 
+// One CTA per (tile, KV head): the tile's 64 rows of K and V, 16 bytes per load,
+// each row copied as is when its token is selected and otherwise replaced by its INT4
+// codes (exact small integers in bf16).  HBM-bound: 2 * 64 * d * 2 bytes in and out
+// per tile.
+template <int D>
+__global__ void __launch_bounds__(256) hybrid_mix_kernel(const HybridMixParams p) {
+  constexpr int kChunks = D / 8;                 // 16-byte chunks per row
+  constexpr int kPasses = kTile * kChunks / 256;  // chunks per thread
+  const int gt = blockIdx.x, h = blockIdx.y;
+  int b = 0, toff = 0;
+  for (;; ++b) {
+    const int nt = (__ldg(p.cu + b + 1) - __ldg(p.cu + b) + kTile - 1) / kTile;
+    if (gt < toff + nt) break;
+    toff += nt;
+  }
+  const int seq0 = __ldg(p.cu + b);
+  const int T = __ldg(p.cu + b + 1) - seq0;
+  const int tt = gt - toff;
+  const long long tile = (long long)h * p.ntiles + gt;
+  const float sk = __ldg(p.sk4 + tile), sv = __ldg(p.sv4 + tile);
+  const uint64_t sel = __ldg(reinterpret_cast<const unsigned long long*>(p.sel_mask) + tile);
+#pragma unroll
+  for (int i = 0; i < kPasses; ++i) {
+    const int f = i * 256 + threadIdx.x;
+    const int r = f / kChunks, c = f % kChunks;
+    const int tok = tt * kTile + r;
+    if (tok >= T) continue;
+    const long long off = ((long long)(seq0 + tok) * p.Hkv + h) * D + c * 8;
+    uint4 kk = __ldg(reinterpret_cast<const uint4*>(p.k + off));
+    uint4 vv = __ldg(reinterpret_cast<const uint4*>(p.v + off));
+    if (!((sel >> r) & 1ull)) {
+      auto codes = [](uint4 w, float s) {
+        uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float lo = __uint_as_float(a[j] << 16), hi = __uint_as_float(a[j] & 0xFFFF0000u);
+          const __nv_bfloat162 q2 = __floats2bfloat162_rn((float)quant_code(lo, s, 7),
+                                                          (float)quant_code(hi, s, 7));
+          a[j] = *reinterpret_cast<const uint32_t*>(&q2);
+        }
+        return make_uint4(a[0], a[1], a[2], a[3]);
+      };
+      kk = codes(kk, sk);
+      vv = codes(vv, sv);
+    }
+    *reinterpret_cast<uint4*>(p.k_mix + off) = kk;
+    *reinterpret_cast<uint4*>(p.v_mix + off) = vv;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_hybrid_mix(const HybridMixParams& p, cudaStream_t s) {
+  if (p.ntiles == 0 || p.Hkv == 0) return cudaSuccess;
+  dim3 grid(p.ntiles, p.Hkv);
+  if (p.d == 128)
+    hybrid_mix_kernel<128><<<grid, 256, 0, s>>>(p);
+  else
+    hybrid_mix_kernel<64><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_hybrid_select(const HybridSelectParams& p, cudaStream_t s) {
   dim3 grid(p.Hkv, p.B);

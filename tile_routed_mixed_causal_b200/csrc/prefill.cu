@@ -52,14 +52,19 @@ constexpr float kRescaleThreshold = 16.0f;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
 constexpr uint32_t kNoKt = 0x0FFFFFFFu;
 
+// Precision of a hybrid-prefill entry whose K and V come from the mixed operands
+// (bf16 rows of selected tokens, INT4 codes as bf16 integers for the others).
+constexpr int kPrecHyb = 4;
+
 template <int D, int MODE>
 struct Cfg {
+  static constexpr bool kHyb = MODE == kPrefillModeHybrid;        // token-level hybrid prefill
   static constexpr bool kHasBf16 = MODE != TRA_POLICY_BOUNDARY;  // bf16 Q and K operands
-  static constexpr bool kHasInt4 = MODE != TRA_POLICY_BITMASK;   // INT4 operands (int8 form)
+  static constexpr bool kHasInt4 = MODE != TRA_POLICY_BITMASK && !kHyb;  // INT4 operands (int8 form)
   // work units per CTA: two, or one under a mixed policy, whose operand buffers
   // (int8, INT4 and bf16 Q, bf16-sized K slots) do not fit twice
   static constexpr int kCtaUnits = MODE == TRA_POLICY_MIXED ? 1 : 2;
-  static constexpr int kQ8Bytes = 128 * D;                     // int8 Q codes
+  static constexpr int kQ8Bytes = kHyb ? 0 : 128 * D;          // int8 Q codes
   static constexpr int kQ4Bytes = kHasInt4 ? 128 * D : 0;      // INT4 Q codes as int8
   static constexpr int kQbBytes = kHasBf16 ? 128 * D * 2 : 0;  // bf16 Q
   static constexpr int kQUnitBytes = kQ8Bytes + kQ4Bytes + kQbBytes;
@@ -195,6 +200,59 @@ __device__ __forceinline__ KtMerge unit_merge(const PrefillParams& p, const Unit
   return c;
 }
 
+// The hybrid prefill's stream for one unit (q-tiles qt0, qt0 + 1): first every key
+// tile that holds, for some row of the unit, keys outside the row's window (kPrecHyb:
+// the mixed operands), then every tile that holds keys inside it (BF16: the original
+// K and V).  A tile on a window's edge appears in both, each entry keeping only its
+// own keys (the softmax masks by position).  Per q-tile qt: keys outside the window
+// lie in tiles kt <= hhi(qt) = floor((64 qt + 63 - window) / 64), keys inside it in
+// tiles wlo(qt) <= kt <= qt with wlo(qt) = max(0, floor((64 qt - window + 1) / 64)).
+struct HybStream {
+  int kt, hhi0, hhi1, wlo0, wlo1, qt0;
+  bool second, in_window, any_window;
+  __device__ __forceinline__ void init(const Unit& x, int window) {
+    qt0 = x.qt0;
+    second = x.valid && x.has_second;
+    any_window = x.valid && window > 0;
+    hhi0 = x.valid ? (64 * qt0 + 63 - window) >> 6 : -1;  // arithmetic shift: floor
+    hhi1 = second ? (64 * (qt0 + 1) + 63 - window) >> 6 : -1;
+    wlo0 = max(0, (64 * qt0 - window + 1) >> 6);
+    wlo1 = max(0, (64 * (qt0 + 1) - window + 1) >> 6);
+    kt = 0;
+    in_window = false;
+  }
+  __device__ __forceinline__ bool next(int& kt_, int& p0, int& p1) {
+    while (true) {
+      if (!in_window) {
+        if (kt <= max(hhi0, hhi1)) {
+          p0 = kt <= hhi0 ? kPrecHyb : 0;
+          p1 = kt <= hhi1 ? kPrecHyb : 0;
+          kt_ = kt++;
+          return true;
+        }
+        if (!any_window) return false;
+        in_window = true;
+        kt = second ? min(wlo0, wlo1) : wlo0;
+      }
+      const int kmax = second ? qt0 + 1 : qt0;
+      if (kt > kmax) return false;
+      p0 = (kt >= wlo0 && kt <= qt0) ? TRA_PREC_BF16 : 0;
+      p1 = (second && kt >= wlo1) ? TRA_PREC_BF16 : 0;
+      kt_ = kt++;
+      if (p0 | p1) return true;
+    }
+  }
+};
+
+__device__ __forceinline__ KtMerge unit_stream(const PrefillParams& p, const Unit& x, std::false_type) {
+  return unit_merge(p, x);
+}
+__device__ __forceinline__ HybStream unit_stream(const PrefillParams& p, const Unit& x, std::true_type) {
+  HybStream c;
+  c.init(x, p.window);
+  return c;
+}
+
 // The K tiles of an entry: one per distinct precision, q-tile 2j's first.
 __device__ __forceinline__ int entry_fills(int p0, int p1) { return (p0 && p1 && p0 != p1) ? 2 : 1; }
 __device__ __forceinline__ int entry_fill_prec(int p0, int p1, int f) {
@@ -327,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t qbytes = x.valid ? C::kQ8Bytes + (int4 ? C::kQ4Bytes : 0) + C::kQbBytes : 0u;
       mbar_arrive_expect_tx(bar_q, qbytes);
       if (x.valid) {
-        tma_load_2d(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
+        if (!C::kHyb) tma_load_2d(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
         if (int4) tma_load_2d(sQ4(u), &m.q4x, bar_q, 0, x.row0 * kTile);
         if (C::kHasBf16) {
           for (int sl = 0; sl < C::kSlabs; ++sl)
@@ -335,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         x.seq0 + x.qt0 * kTile);
         }
       }
-      KtMerge c = unit_merge(p, x);
+      auto c = unit_stream(p, x, std::bool_constant<C::kHyb>{});
       int kt, p0, p1;
       int nk = 0, nv = 0;  // fills issued so far into this unit's K and V rings
       while (c.next(kt, p0, p1)) {
@@ -351,10 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (use > 0 && !mbar_wait(bar_kfree(u, s), (use - 1) & 1, err)) { ok = false; break; }
           const uint32_t dst = sK(u, s);
           const int krow = (x.kvh * p.ntiles + x.toff + kt) * kTile;
-          if (prec == TRA_PREC_BF16) {
+          if (prec == TRA_PREC_BF16 || prec == kPrecHyb) {
+            const CUtensorMap* km = prec == kPrecHyb ? &m.kmix : &m.kb;
             mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D * 2);
             for (int sl = 0; sl < C::kSlabs; ++sl)
-              tma_load_3d(dst + sl * 64 * 128, &m.kb, bar_kfull(u, s), sl * 64, x.kvh,
+              tma_load_3d(dst + sl * 64 * 128, km, bar_kfull(u, s), sl * 64, x.kvh,
                           x.seq0 + kt * kTile);
           } else {
             mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D);
@@ -365,9 +424,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         const int sv = nv % NSV, usev = nv / NSV;  // the unit's V ring slot
         if (usev > 0 && !mbar_wait(bar_vfree(u, sv), (usev - 1) & 1, err)) break;
+        // V of the entry: the mixed operand for a hybrid entry, else bf16 V
+        const CUtensorMap* vm = (p0 == kPrecHyb || p1 == kPrecHyb) ? &m.vmix : &m.vb;
         mbar_arrive_expect_tx(bar_vfull(u, sv), 64 * D * 2);
         for (int sl = 0; sl < C::kSlabs; ++sl)
-          tma_load_3d(sV(u, sv) + sl * 64 * 128, &m.vb, bar_vfull(u, sv), sl * 64, x.kvh,
+          tma_load_3d(sV(u, sv) + sl * 64 * 128, vm, bar_vfull(u, sv), sl * 64, x.kvh,
                       x.seq0 + kt * kTile);
         ++nv;
       }
@@ -412,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         int nk = 0;  // this unit's K ring fills consumed so far
         int i = 0;   // entries of this unit issued so far
-        KtMerge c = unit_merge(p, mu ? un1 : un0);
+        auto c = unit_stream(p, mu ? un1 : un0, std::bool_constant<C::kHyb>{});
         int kt, p0, p1;
         while (c.next(kt, p0, p1)) {
           if ((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) {
@@ -435,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t msk[4] = {f == 1 ? keep : 0u, f == 1 ? keep : 0u, f == 0 ? keep : 0u,
                                      f == 0 ? keep : 0u};
             const uint32_t kb = sK(mu, s);
-            if (prec == TRA_PREC_BF16) {
+            if (prec == TRA_PREC_BF16 || prec == kPrecHyb) {
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const int sl = kk >> 2, off = (kk & 3) * 32;
@@ -478,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tq = qt * kTile + rr;              // query position in the sequence
     const bool row_valid = half_valid && tq < x.T;
     const long long qtile = (long long)x.h * p.ntiles + x.toff + qt;
-    const float sq8 = half_valid ? __ldg(p.sq8 + qtile) : 0.0f;
+    const float sq8 = (half_valid && !C::kHyb) ? __ldg(p.sq8 + qtile) : 0.0f;
     // INT4 operands are 16 x code, so INT4 accumulators are 256 x the code product:
     // the power of two goes into the row's INT4 scale (exact)
     const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) * (1.0f / 256.0f) : 0.0f;
@@ -487,23 +548,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     int i = 0;
-    KtMerge c = unit_merge(p, x);
+    auto c = unit_stream(p, x, std::bool_constant<C::kHyb>{});
     // the K-tile scale of this row's precision of an entry (1 for BF16), loaded one
     // entry ahead
     auto kscale = [&](int kt_, int pr) -> float {
       const long long t_ = (long long)x.kvh * p.ntiles + x.toff + kt_;
       if (pr == TRA_PREC_INT8) return __ldg(p.sk8 + t_);
       if (pr == TRA_PREC_INT4 && int4) return __ldg(p.sk4 + t_);
+      if (C::kHyb && pr == kPrecHyb) return __ldg(p.sk4 + t_);
       return 1.0f;
+    };
+    // hybrid entries: the tile's V INT4 scale and its 64-bit selection mask
+    auto hyb_tile = [&](int kt_, int pr, float& sv, uint2& sel) {
+      sv = 1.0f;
+      sel = make_uint2(0u, 0u);
+      if (C::kHyb && pr == kPrecHyb) {
+        const long long t_ = (long long)x.kvh * p.ntiles + x.toff + kt_;
+        sv = __ldg(p.sv4 + t_);
+        sel = __ldg(reinterpret_cast<const uint2*>(p.sel_mask) + t_);
+      }
     };
     int nkt = 0, np0 = 0, np1 = 0;
     bool have = c.next(nkt, np0, np1);
     float nsk = have ? kscale(nkt, half ? np1 : np0) : 0.0f;
+    float nsv = 1.0f;
+    uint2 nsel = make_uint2(0u, 0u);
+    if (C::kHyb && have) hyb_tile(nkt, half ? np1 : np0, nsv, nsel);
     for (; have; ++i) {
       const int kt = nkt, pa = np0, pb = np1;
       const float skt = nsk;
+      const float svt = nsv;
+      const uint2 selt = nsel;
       have = c.next(nkt, np0, np1);  // look-ahead: next entry and its scale
       if (have) nsk = kscale(nkt, half ? np1 : np0);
+      if (C::kHyb && have) hyb_tile(nkt, half ? np1 : np0, nsv, nsel);
       const int sb = i & 1;
       const uint32_t tS = tU + sb * 64;
       if (!mbar_wait(bar_sfull(u, sb), (i >> 1) & 1, err)) { ok = false; break; }
@@ -532,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tS + 32, hi);
         }
         tmem_wait_ld();
-        if (p.n_dump > 0 && row_valid && prec != TRA_PREC_BF16) {
+        if (!C::kHyb && p.n_dump > 0 && row_valid && prec != TRA_PREC_BF16) {
           for (int di = 0; di < p.n_dump; ++di) {
             const int* dc = p.dump_coords + di * 4;
             if (__ldg(dc) == x.b && __ldg(dc + 1) == x.h && __ldg(dc + 2) == qt &&
@@ -546,11 +624,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // log2-domain score = raw * f
         const float f = p.scale_log2 * skt *
                         (prec == TRA_PREC_INT8 ? sq8 : (prec == TRA_PREC_INT4 ? sq4 : 1.0f));
-        // valid keys of this tile for this row (causal and sequence end); only the
-        // diagonal tile and a sequence's last tile have fewer than 64
-        const int nvalid =
-            row_valid ? min(min(tq - kt * kTile + 1, x.T - kt * kTile), kTile) : 0;
-        const bool full = __all_sync(0xffffffffu, nvalid >= kTile);
+        // valid keys of this tile for this row, columns [clo, nvalid): causal and
+        // sequence end; only the diagonal tile and a sequence's last tile have fewer
+        // than 64.  Hybrid: a kPrecHyb entry keeps the keys at least `window`
+        // positions behind the query, a BF16 entry the causal keys closer than that.
+        int clo = 0;
+        int nvalid = row_valid ? min(min(tq - kt * kTile + 1, x.T - kt * kTile), kTile) : 0;
+        if (C::kHyb && row_valid) {
+          const int behind = tq - kt * kTile;  // query position minus the tile's first key
+          if (prec == kPrecHyb)
+            nvalid = min(min(behind - p.window + 1, x.T - kt * kTile), kTile);
+          else
+            clo = max(0, behind - p.window + 1);
+        }
+        const bool full = __all_sync(0xffffffffu, clo == 0 && nvalid >= kTile);
         // One row of the tile -> bf16 P and the online-softmax update.  Full
         // tiles (every key valid) take a copy with no per-column test; only
         // the diagonal tile and a sequence's last tile take the masked copy.
@@ -563,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < 64; ++cc) {
             xs[cc] = kInt ? (float)(int)sr[cc] : __uint_as_float(sr[cc]);
-            if (!kFull) xs[cc] = cc < nvalid ? xs[cc] : -INFINITY;
+            if (!kFull) xs[cc] = (cc >= clo && cc < nvalid) ? xs[cc] : -INFINITY;
           }
           float mx;
           if (kInt && kFull) {
@@ -592,9 +679,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float m_tile = mx == -INFINITY ? -INFINITY : mx * f;  // f > 0 keeps the argmax
           const float m_new = fmaxf(m_run, m_tile);
           const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
+          // once one row of the warp passes the threshold, every row whose max grew
+          // moves it too (one O pass for the warp); O is rescaled if one of those rows
+          // had seen keys (O rows that have seen none are exactly zero; the rows of a
+          // warp may meet their first keys in different entries)
           const bool warp_need = __any_sync(0xffffffffu, need);
-          // O rows that have seen no key yet are exactly zero: no rescale
-          warp_rescale_o = __any_sync(0xffffffffu, need && m_run != -INFINITY);
+          const bool grew = __any_sync(0xffffffffu, m_new > m_run && m_run != -INFINITY);
+          warp_rescale_o = warp_need && grew;
           if (warp_need && m_new > m_run) {
             alpha = ex2(m_run - m_new);  // m_run = -inf gives 0
             m_run = m_new;
@@ -611,8 +702,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float q0 = ex2(arg.x);
             float q1 = ex2(arg.y);
             if (!kFull) {  // masked columns of a row whose max is still -inf
-              q0 = cc < nvalid ? q0 : 0.0f;
-              q1 = cc + 1 < nvalid ? q1 : 0.0f;
+              q0 = (cc >= clo && cc < nvalid) ? q0 : 0.0f;
+              q1 = (cc + 1 >= clo && cc + 1 < nvalid) ? q1 : 0.0f;
             }
             const __nv_bfloat162 pbf = __floats2bfloat162_rn(q0, q1);
             const uint32_t w = *reinterpret_cast<const uint32_t*>(&pbf);
@@ -624,9 +715,74 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 l2 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
           l_run = l_run * alpha + (l2.x + l2.y);
         };
+        // A hybrid entry (mixed operands): column c of the tile is a selected token's
+        // bf16 key (log2 factor f) or an INT4 code row (factor f * sK), and P V
+        // reads that token's bf16 V row (P as is) or its INT4 code row (P * sV).
+        auto hyb_row = [&](auto full_tag) {
+          constexpr bool kFull = decltype(full_tag)::value;
+          const float fs = p.scale_log2, fc = p.scale_log2 * skt;
+          float xs[64];
+#pragma unroll
+          for (int cc = 0; cc < 64; ++cc) {
+            const bool sel = (((cc < 32 ? selt.x : selt.y) >> (cc & 31)) & 1u) != 0u;
+            xs[cc] = __uint_as_float(sr[cc]) * (sel ? fs : fc);
+            if (!kFull) xs[cc] = (cc >= clo && cc < nvalid) ? xs[cc] : -INFINITY;
+          }
+          float mx4[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(xs[k], xs[k + 4]);
+#pragma unroll
+          for (int cc = 8; cc < 64; cc += 8) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(mx4[k], fmaxf(xs[cc + k], xs[cc + k + 4]));
+          }
+          const float m_tile = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          const float m_new = fmaxf(m_run, m_tile);
+          const bool need = m_new > m_run + kRescaleThreshold;
+          const bool warp_need = __any_sync(0xffffffffu, need);
+          const bool grew = __any_sync(0xffffffffu, m_new > m_run && m_run != -INFINITY);
+          warp_rescale_o = warp_need && grew;
+          if (warp_need && m_new > m_run) {
+            alpha = ex2(m_run - m_new);
+            m_run = m_new;
+          }
+          // l adds what P V accumulates, divided by the column's factor: the bf16 P of
+          // a selected column, bf16(p * sV) / sV of a code column (an all-zero V tile,
+          // sV = 0, takes factor 1: its codes are 0)
+          const float gv = svt != 0.0f ? svt : 1.0f;
+#pragma unroll
+          for (int cc = 0; cc < 64; cc += 2) {
+            float q0 = ex2(xs[cc] - m_run);
+            float q1 = ex2(xs[cc + 1] - m_run);
+            if (!kFull) {
+              q0 = (cc >= clo && cc < nvalid) ? q0 : 0.0f;
+              q1 = (cc + 1 >= clo && cc + 1 < nvalid) ? q1 : 0.0f;
+            }
+            const uint32_t w = cc < 32 ? selt.x : selt.y;
+            const bool s0 = ((w >> (cc & 31)) & 1u) != 0u;
+            const bool s1 = ((w >> ((cc + 1) & 31)) & 1u) != 0u;
+            const __nv_bfloat162 pbf = __floats2bfloat162_rn(s0 ? q0 : q0 * gv, s1 ? q1 : q1 * gv);
+            pk[cc >> 1] = *reinterpret_cast<const uint32_t*>(&pbf);
+          }
+          // l from the bf16 P just written, each value divided by its column's factor
+          // (a pass of its own, once the scores are dead)
+          const float ig = 1.0f / gv;
+          float lt[2] = {0.0f, 0.0f};
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const uint32_t w = k < 16 ? selt.x : selt.y;
+            const float h0 = ((w >> ((2 * k) & 31)) & 1u) ? 1.0f : ig;
+            const float h1 = ((w >> ((2 * k + 1) & 31)) & 1u) ? 1.0f : ig;
+            lt[k & 1] = fmaf(__uint_as_float(pk[k] << 16), h0, lt[k & 1]);
+            lt[k & 1] = fmaf(__uint_as_float(pk[k] & 0xFFFF0000u), h1, lt[k & 1]);
+          }
+          l_run = l_run * alpha + (lt[0] + lt[1]);
+        };
         using T_ = std::true_type;
         using F_ = std::false_type;
-        if (prec == TRA_PREC_BF16) {
+        if (C::kHyb && prec == kPrecHyb) {
+          if (full) hyb_row(T_{}); else hyb_row(F_{});
+        } else if (prec == TRA_PREC_BF16) {
           if (full) softmax_row(F_{}, T_{}); else softmax_row(F_{}, F_{});
         } else {
           if (full) softmax_row(T_{}, T_{}); else softmax_row(T_{}, F_{});
@@ -712,6 +868,7 @@ template <int D>
 cudaError_t launch_d(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s) {
   if (p.mode == TRA_POLICY_BITMASK) return launch_one<D, TRA_POLICY_BITMASK>(p, m, s);
   if (p.mode == TRA_POLICY_MIXED) return launch_one<D, TRA_POLICY_MIXED>(p, m, s);
+  if (p.mode == kPrefillModeHybrid) return launch_one<D, kPrefillModeHybrid>(p, m, s);
   return launch_one<D, TRA_POLICY_BOUNDARY>(p, m, s);
 }
 

@@ -16,12 +16,6 @@
 namespace tra {
 namespace {
 
-__device__ __forceinline__ int quant_code(float x, float s, int qmax) {
-  if (s == 0.0f) return 0;
-  int c = __float2int_rn(__fdiv_rn(x, s));
-  return c > qmax ? qmax : (c < -qmax ? -qmax : c);
-}
-
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

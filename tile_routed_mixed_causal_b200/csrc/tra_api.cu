@@ -641,6 +641,74 @@ tra_status hybrid_attention_decode(const tra_shape* shape, const tra_hybrid* hy,
   return ok();
 }
 
+tra_status hybrid_attention_prefill(const tra_shape* shape, const tra_hybrid* hy, const uint16_t* q,
+                                    const uint16_t* k, const uint16_t* v, const tra_qtiles* kv,
+                                    uint16_t* k_mix, uint16_t* v_mix, float softmax_scale,
+                                    uint16_t* out, float* lse, int32_t* status_dev, void* stream) {
+  int64_t nt = 0, ntok = 0, nt_max = 0;
+  tra_status st = check_shape(shape, &nt, &ntok, &nt_max);
+  if (st != TRA_OK) return st;
+  if (!hy || !hy->sel_mask) return fail(TRA_ERR_INVALID, "the hybrid selection masks are required");
+  if (hy->window < 0) return fail(TRA_ERR_INVALID, "window must be >= 0 (got %d)", hy->window);
+  if (!q || !k || !v || !kv || !k_mix || !v_mix || !out || !status_dev)
+    return fail(TRA_ERR_INVALID, "q, k, v, kv, k_mix, v_mix, out and status are required");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_mix) || !aligned16(v_mix) ||
+      !aligned16(out) || !aligned16(hy->sel_mask) || (lse && !aligned16(lse)))
+    return fail(TRA_ERR_INVALID, "q/k/v/k_mix/v_mix/out/lse/sel_mask must be 16-byte aligned");
+  if (!(kv->formats & (TRA_FMT_K4 | TRA_FMT_K4X)) || !(kv->formats & TRA_FMT_V4) || !kv->sk4 ||
+      !kv->sv4)
+    return fail(TRA_ERR_INVALID, "the hybrid prefill needs the K and V INT4 tile scales (K4 or K4X, V4)");
+  if (nt_max >= (1ll << 24)) return fail(TRA_ERR_UNSUPPORTED, "a sequence has more than 2^24 tiles");
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
+    return fail(TRA_ERR_INVALID, "softmax_scale must be positive and finite");
+  if (ntok == 0 || nt == 0) return ok();
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  tra::HybridMixParams mp{};
+  mp.cu = shape->cu_seqlens_dev;
+  mp.B = shape->B;
+  mp.Hkv = shape->Hkv;
+  mp.d = shape->d;
+  mp.ntiles = (int)nt;
+  mp.k = k;
+  mp.v = v;
+  mp.sk4 = kv->sk4;
+  mp.sv4 = kv->sv4;
+  mp.sel_mask = hy->sel_mask;
+  mp.k_mix = k_mix;
+  mp.v_mix = v_mix;
+  cudaError_t e = tra::launch_hybrid_mix(mp, s);
+  if (e != cudaSuccess) return cuda_fail(e, "hybrid mix launch");
+  tra::PrefillParams p{};
+  p.cu = shape->cu_seqlens_dev;
+  p.B = shape->B;
+  p.Hq = shape->Hq;
+  p.Hkv = shape->Hkv;
+  p.d = shape->d;
+  p.ntiles = (int)nt;
+  p.mode = tra::kPrefillModeHybrid;
+  p.jmax = (int)((nt_max + 1) / 2);
+  p.sk4 = kv->sk4;
+  p.sv4 = kv->sv4;
+  p.sel_mask = hy->sel_mask;
+  p.window = hy->window;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  p.lse = lse;
+  p.status = status_dev;
+  tra::PrefillMaps m;
+  memset(&m, 0, sizeof m);
+  const int d = shape->d;
+  bool good = map_bf16(&m.qb, q, d, shape->Hq, ntok, 128) &&
+              map_bf16(&m.kb, k, d, shape->Hkv, ntok, 64) &&
+              map_bf16(&m.vb, v, d, shape->Hkv, ntok, 64) &&
+              map_bf16(&m.kmix, k_mix, d, shape->Hkv, ntok, 64) &&
+              map_bf16(&m.vmix, v_mix, d, shape->Hkv, ntok, 64);
+  if (!good) return fail(TRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  e = tra::launch_prefill(p, m, s);
+  if (e != cudaSuccess) return cuda_fail(e, "hybrid prefill launch");
+  return ok();
+}
+
 tra_status tra_boundary_tile_counts(const tra_shape* shape, int32_t b1, int32_t b2, int64_t* n8,
                                     int64_t* n4) {
   tra_status st = check_shape(shape, nullptr, nullptr, nullptr);
@@ -656,6 +724,66 @@ tra_status tra_boundary_tile_counts(const tra_shape* shape, int32_t b1, int32_t 
   }
   *n8 = kept8;
   *n4 = kept - kept8;
+  return ok();
+}
+
+tra_status tra_prefill_cost_model(const tra_shape* shape, const int32_t* b1, const int32_t* b2,
+                                  double dual_weight, double solo, int32_t n_sm, double* makespan,
+                                  double* entries) {
+  int64_t nt = 0, nt_max = 0;
+  tra_status st = check_shape(shape, &nt, nullptr, &nt_max);
+  if (st != TRA_OK) return st;
+  tra_policy pol{};
+  pol.mode = TRA_POLICY_BOUNDARY;
+  pol.b1 = b1;
+  pol.b2 = b2;
+  st = check_policy(shape, &pol, nt_max);
+  if (st != TRA_OK) return st;
+  if (!(dual_weight >= 1.0) || !(solo > 0.0 && solo <= 1.0) || n_sm < 1 || !makespan || !entries)
+    return fail(TRA_ERR_INVALID, "need dual_weight >= 1, 0 < solo <= 1, n_sm >= 1 and outputs");
+  const int32_t* cu = shape->cu_seqlens_host;
+  const int Hq = shape->Hq, B = shape->B;
+  const int64_t jmax = (nt_max + 1) / 2;
+  // precision a q-tile row gives k-tile kt under (b1, b2): 2 INT8, 1 INT4, 0 skipped
+  auto prec = [](int64_t qt, int64_t kt, int32_t lo1, int32_t lo2) -> int {
+    if (kt > qt || kt < 0) return 0;
+    const int64_t dist = qt - kt;
+    return dist < lo1 ? 2 : (dist < lo2 ? 1 : 0);
+  };
+  // work of unit id (launch order: q-tile pairs from the heaviest, then sequence, then head)
+  auto unit_work = [&](int64_t id, double* cnt) -> double {
+    const int h = (int)(id % Hq);
+    const int b = (int)((id / Hq) % B);
+    const int64_t j = jmax - 1 - id / ((int64_t)Hq * B);
+    const int64_t ntb = ceil_tiles(cu[b + 1] - cu[b]);
+    const int64_t q0 = 2 * j, q1 = 2 * j + 1;
+    if (q0 >= ntb) return 0.0;
+    const bool second = q1 < ntb;
+    double w = 0.0;
+    const int64_t lo = std::max<int64_t>(0, q0 - b2[h] + 1);
+    const int64_t hi = second ? q1 : q0;
+    for (int64_t kt = lo; kt <= hi; ++kt) {
+      const int pa = prec(q0, kt, b1[h], b2[h]);
+      const int pb = second ? prec(q1, kt, b1[h], b2[h]) : 0;
+      if (!pa && !pb) continue;
+      w += (pa && pb && pa != pb) ? dual_weight : 1.0;
+      *cnt += 1.0;
+    }
+    return w;
+  };
+  const int64_t units = jmax * B * Hq;
+  const int64_t ctas = (units + 1) / 2;
+  std::vector<double> sm((size_t)n_sm, 0.0);  // time each SM frees up
+  double total = 0.0;
+  for (int64_t c = 0; c < ctas; ++c) {
+    const double w0 = unit_work(2 * c, &total), w1 = unit_work(2 * c + 1, &total);
+    const double w = std::min(w0, w1) + solo * std::fabs(w0 - w1);
+    if (w == 0.0) continue;  // an empty CTA exits at once
+    auto it = std::min_element(sm.begin(), sm.end());
+    *it += w;
+  }
+  *makespan = *std::max_element(sm.begin(), sm.end());
+  *entries = total;
   return ok();
 }
 

@@ -258,6 +258,14 @@ __device__ __forceinline__ uint2 expand_int4x8(uint32_t w) {
 }
 
 // Tile offset of sequence b (tiles restart at each sequence): sum of ceil(T/64).
+// Symmetric quantisation code of x with scale s: clamp(rne(fl32(x / s)), -qmax, qmax)
+// with IEEE division; a zero scale (all-zero tile) gives code 0.
+__device__ __forceinline__ int quant_code(float x, float s, int qmax) {
+  if (s == 0.0f) return 0;
+  int c = __float2int_rn(__fdiv_rn(x, s));
+  return c > qmax ? qmax : (c < -qmax ? -qmax : c);
+}
+
 __device__ __forceinline__ int seq_tile_offset(const int32_t* cu, int b) {
   int off = 0;
   for (int i = 0; i < b; ++i) off += (cu[i + 1] - cu[i] + kTile - 1) / kTile;

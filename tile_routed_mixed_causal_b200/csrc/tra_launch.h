@@ -67,12 +67,22 @@ struct PrefillParams {
   int n_dump;
   int32_t* dump_out;
   int32_t* status;
+  // token-level hybrid prefill (mode kPrefillModeHybrid): INT4 scales of V, the
+  // per-tile selection masks [Hkv][ntiles] and the window (keys closer than it to
+  // the query are read in bf16)
+  const float* sv4;
+  const uint64_t* sel_mask;
+  int window;
 };
+
+// prefill mode of the token-level hybrid (beside the TRA_POLICY_* modes)
+constexpr int kPrefillModeHybrid = 3;
 
 struct PrefillMaps {
   CUtensorMap q8, k8;    // int8 tiles, 2-D (d bytes x rows)
   CUtensorMap q4x, k4x;  // expanded INT4 tiles (int8 16 x code), 2-D like q8 / k8
   CUtensorMap qb, kb, vb;  // bf16, 3-D (d, H, ntok)
+  CUtensorMap kmix, vmix;  // hybrid: mixed K / V operands, bf16 3-D like kb / vb
 };
 
 cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s);
@@ -135,6 +145,23 @@ struct HybridSelectParams {
 };
 
 cudaError_t launch_hybrid_select(const HybridSelectParams& p, cudaStream_t s);
+
+// Mixed K / V operands of the hybrid prefill: each key row is the token's bf16 row
+// when its tile's selection mask marks it, else its INT4 codes (the tile's INT4
+// scale, as the quantiser computes them) written as bf16 integers.
+struct HybridMixParams {
+  const int32_t* cu;
+  int B, Hkv, d, ntiles;
+  const uint16_t* k;         // [ntok][Hkv][d] bf16
+  const uint16_t* v;
+  const float* sk4;          // [Hkv][ntiles]
+  const float* sv4;
+  const uint64_t* sel_mask;  // [Hkv][ntiles]
+  uint16_t* k_mix;           // [ntok][Hkv][d] bf16
+  uint16_t* v_mix;
+};
+
+cudaError_t launch_hybrid_mix(const HybridMixParams& p, cudaStream_t s);
 
 int decode_splits(int B, int Hkv);
 cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t s);
