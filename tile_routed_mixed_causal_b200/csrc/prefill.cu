@@ -455,7 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // O += P(idx) V(idx): P from TMEM buffer idx & 1, V (MN-major) from the unit's
       // V ring, which holds one tile per entry of the unit, in order
-      auto issue_pv = [&](int idx) -> bool {
+      // hi_lo: a mixed-operand entry of the hybrid prefill, whose P is a bf16 pair
+      // (hi in the block's first 32 columns, lo in the next 32): both multiply V
+      auto issue_pv = [&](int idx, bool hi_lo) -> bool {
         const int pb = idx & 1, slot = idx % NSV;
         if (!mbar_wait(bar_pfull(mu, pb), (idx >> 1) & 1, err)) return false;
         if (!mbar_wait(bar_vfull(mu, slot), (idx / NSV) & 1, err)) return false;
@@ -466,6 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = smem_desc(vb + kk * 2048, 64 * 128, 1024, kSwz128);
           mma_bf16_ts(tU + 128, tU + pb * 64 + kk * 8, bd, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
         }
+        if (C::kHyb && hi_lo) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = smem_desc(vb + kk * 2048, 64 * 128, 1024, kSwz128);
+            mma_bf16_ts(tU + 128, tU + pb * 64 + 32 + kk * 8, bd, kIdPV, 1u);
+          }
+        }
         mma_commit(bar_ofull(mu));
         mma_commit(bar_vfree(mu, slot));
         return true;
@@ -473,6 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         int nk = 0;  // this unit's K ring fills consumed so far
         int i = 0;   // entries of this unit issued so far
+        bool hyb_prev = false;  // entry i - 1 reads the mixed operands
         auto c = unit_stream(p, mu ? un1 : un0, std::bool_constant<C::kHyb>{});
         int kt, p0, p1;
         while (c.next(kt, p0, p1)) {
@@ -518,10 +528,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           mma_commit(bar_sfull(mu, i & 1));
-          if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+          if (i >= 1 && !issue_pv(i - 1, hyb_prev)) { ok = false; break; }
+          hyb_prev = p0 == kPrecHyb || p1 == kPrecHyb;
           ++i;
         }
-        if (ok && i >= 1 && issue_pv(i - 1)) mma_commit(bar_ofinal(mu));
+        if (ok && i >= 1 && issue_pv(i - 1, hyb_prev)) mma_commit(bar_ofinal(mu));
       }
       // every MMA of this thread completes before TMEM is released
       mma_commit(bar_done);
@@ -596,6 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool half_applies = prec != 0 && half_valid;
       uint32_t pk[32];
       bool warp_rescale_o = false;
+      bool p_stored = false;  // a mixed-operand entry stores its P itself
       float alpha = 1.0f;
       if (!half_applies) {
 #pragma unroll
@@ -718,6 +730,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // A hybrid entry (mixed operands): column c of the tile is a selected token's
         // bf16 key (log2 factor f) or an INT4 code row (factor f * sK), and P V
         // reads that token's bf16 V row (P as is) or its INT4 code row (P * sV).
+        // An all-zero V tile (sV = 0) has codes 0: its P * sV = 0 adds nothing, as it
+        // should, while l still counts p.
         auto hyb_row = [&](auto full_tag) {
           constexpr bool kFull = decltype(full_tag)::value;
           const float fs = p.scale_log2, fc = p.scale_log2 * skt;
@@ -749,39 +763,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           // l adds what P V accumulates, divided by the column's factor: the bf16 P of
           // a selected column, bf16(p * sV) / sV of a code column (an all-zero V tile,
           // sV = 0, takes factor 1: its codes are 0)
-          const float gv = svt != 0.0f ? svt : 1.0f;
+          // P written as a bf16 pair hi + lo (lo = the rounding residual of hi), hi in
+          // the S block's first 32 columns and lo in the next 32, two halves at a time
+          // in pk; P V adds both, so P carries about 16 bits and l sums fp32 p
+          float2 ls = make_float2(0.0f, 0.0f);
+          // the mask through an opaque copy: the bit tests are recomputed here instead
+          // of 64 results being kept live from the score loop (they do not fit)
+          uint32_t sw0, sw1;
+          asm volatile("mov.b32 %0, %1;" : "=r"(sw0) : "r"(selt.x));
+          asm volatile("mov.b32 %0, %1;" : "=r"(sw1) : "r"(selt.y));
 #pragma unroll
-          for (int cc = 0; cc < 64; cc += 2) {
-            float q0 = ex2(xs[cc] - m_run);
-            float q1 = ex2(xs[cc + 1] - m_run);
-            if (!kFull) {
-              q0 = (cc >= clo && cc < nvalid) ? q0 : 0.0f;
-              q1 = (cc + 1 >= clo && cc + 1 < nvalid) ? q1 : 0.0f;
+          for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+            for (int cc = 32 * hh; cc < 32 * hh + 32; cc += 2) {
+              float q0 = ex2(xs[cc] - m_run);
+              float q1 = ex2(xs[cc + 1] - m_run);
+              if (!kFull) {
+                q0 = (cc >= clo && cc < nvalid) ? q0 : 0.0f;
+                q1 = (cc + 1 >= clo && cc + 1 < nvalid) ? q1 : 0.0f;
+              }
+              ls = __fadd2_rn(ls, make_float2(q0, q1));
+              const uint32_t w = cc < 32 ? sw0 : sw1;
+              const float g0 = ((w >> (cc & 31)) & 1u) ? q0 : q0 * svt;
+              const float g1 = ((w >> ((cc + 1) & 31)) & 1u) ? q1 : q1 * svt;
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(g0, g1);
+              const uint32_t hw = *reinterpret_cast<const uint32_t*>(&hb);
+              const __nv_bfloat162 lb = __floats2bfloat162_rn(g0 - __uint_as_float(hw << 16),
+                                                              g1 - __uint_as_float(hw & 0xFFFF0000u));
+              pk[((cc >> 1) & 15)] = hw;
+              pk[16 + ((cc >> 1) & 15)] = *reinterpret_cast<const uint32_t*>(&lb);
             }
-            const uint32_t w = cc < 32 ? selt.x : selt.y;
-            const bool s0 = ((w >> (cc & 31)) & 1u) != 0u;
-            const bool s1 = ((w >> ((cc + 1) & 31)) & 1u) != 0u;
-            const __nv_bfloat162 pbf = __floats2bfloat162_rn(s0 ? q0 : q0 * gv, s1 ? q1 : q1 * gv);
-            pk[cc >> 1] = *reinterpret_cast<const uint32_t*>(&pbf);
+            tmem_st16(tS + 16 * hh, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+            tmem_st16(tS + 32 + 16 * hh, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
           }
-          // l from the bf16 P just written, each value divided by its column's factor
-          // (a pass of its own, once the scores are dead)
-          const float ig = 1.0f / gv;
-          float lt[2] = {0.0f, 0.0f};
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const uint32_t w = k < 16 ? selt.x : selt.y;
-            const float h0 = ((w >> ((2 * k) & 31)) & 1u) ? 1.0f : ig;
-            const float h1 = ((w >> ((2 * k + 1) & 31)) & 1u) ? 1.0f : ig;
-            lt[k & 1] = fmaf(__uint_as_float(pk[k] << 16), h0, lt[k & 1]);
-            lt[k & 1] = fmaf(__uint_as_float(pk[k] & 0xFFFF0000u), h1, lt[k & 1]);
-          }
-          l_run = l_run * alpha + (lt[0] + lt[1]);
+          l_run = l_run * alpha + (ls.x + ls.y);
         };
         using T_ = std::true_type;
         using F_ = std::false_type;
         if (C::kHyb && prec == kPrecHyb) {
           if (full) hyb_row(T_{}); else hyb_row(F_{});
+          p_stored = true;
         } else if (prec == TRA_PREC_BF16) {
           if (full) softmax_row(F_{}, T_{}); else softmax_row(F_{}, F_{});
         } else {
@@ -804,7 +825,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(tO + col, o);
         }
       }
-      tmem_st32(tS, pk);  // P(i) over S(i), which this thread has read
+      if (!p_stored) {
+        tmem_st32(tS, pk);  // P(i) over S(i), which this thread has read
+        // a mixed-operand entry's P V also reads the lo half: zero for these rows too
+        if (C::kHyb && (pa == kPrecHyb || pb == kPrecHyb)) tmem_st32(tS + 32, pk);
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_pfull(u, sb));
