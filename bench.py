@@ -76,16 +76,19 @@ def parse():
 # each dominant kernel, keyed by the SHA-256 prefix of the kernel source that was captured; a
 # source that has changed since reports null.
 PROFILED_TRAFFIC = {
-    "prefill.cu": ("701cf6b01ac2f0b3", 3_403_118_848),
-    "decode.cu": ("681e247ef97b3884", 662_413_568),
+    # key: (source file, its sha256[:16] when captured, dram__bytes_read.sum + dram__bytes_write.sum
+    # of one launch in the ncu capture); reported only while the source is unchanged
+    "prefill_bitmask": ("prefill.cu", "f06f0ba6c946b8cd", 3_376_191_016),
+    "prefill_hybrid": ("prefill.cu", "f06f0ba6c946b8cd", 2_313_416_048),
+    "decode": ("decode.cu", "1fedbc1ad6951867", 666_226_944),
 }
 
 
-def profiled_traffic(src):
+def profiled_traffic(key):
     import hashlib
+    src, want, nbytes = PROFILED_TRAFFIC[key]
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "tile_routed_mixed_causal_b200",
                         "csrc", src)
-    want, nbytes = PROFILED_TRAFFIC[src]
     try:
         with open(path, "rb") as f:
             have = hashlib.sha256(f.read()).hexdigest()[:16]
@@ -488,7 +491,7 @@ def decode_bench(device, passes, stream, hbm_gbs):
         "passes": len(times), "pass_ms": [round(t, 3) for t in times], "stat": "median of passes",
         "bytes_per_step": int(pass_bytes / steps),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
-                     "frac": round(gbs / hbm_gbs, 4), "traffic": profiled_traffic("decode.cu"),
+                     "frac": round(gbs / hbm_gbs, 4), "traffic": profiled_traffic("decode"),
                      "kernel": "decode_split_kernel (one ABI call: the two- and three-limb launches, each group in one)"},
         "gpu_launches_per_step": 2,
     }
@@ -603,6 +606,7 @@ def hybrid_prefill_bench(device, stream, bf16_tflops, frac=0.05, window=128, rep
             "stat": "median of calls",
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_tflops,
                          "unit": "TFLOP/s", "frac": round(t_roof / (ms * 1e-3), 4),
+                         "traffic": profiled_traffic("prefill_hybrid"),
                          "kernel": "hybrid_mix_kernel + prefill_kernel<128, hybrid> (one ABI call)"}}
 
 
@@ -872,7 +876,7 @@ def main():
             "roofline": {
                 "bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak_eff, 2),
                 "unit": "TFLOP/s", "frac": round(achieved / peak_eff, 4),
-                "traffic": profiled_traffic("prefill.cu"),
+                "traffic": profiled_traffic("prefill_bitmask"),
                 "kernel": "prefill_kernel<128, bitmask>",
                 "peak_basis": f"tile-mix weighted: bf16 {bf16_tflops} TF/s ({peak_src}, burst), "
                               f"int8 = 2x bf16 (nominal ratio)",
