@@ -31,7 +31,7 @@ _lock = threading.Lock()
 _lib = None
 
 TILE = 64
-INT4, INT8, BF16 = 1, 2, 3
+INT4, INT8, BF16, FP8 = 1, 2, 3, 4
 
 
 def build(force: bool = False) -> str:
@@ -61,18 +61,25 @@ def _load():
             lib.orc_num_tiles.restype = L
             lib.orc_quantize.argtypes = [P, P, I, I, I, P, P, P, P]
             lib.orc_quantize.restype = I
-            lib.orc_lists_boundary.argtypes = [P, I, I, P, P, P, P]
+            lib.orc_e4m3_value.argtypes = [I]
+            lib.orc_e4m3_value.restype = D
+            lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.orc_e4m3_encode.restype = I
+            lib.orc_quantize_f8.argtypes = [P, P, I, I, I, P, P]
+            lib.orc_quantize_f8.restype = I
+            lib.orc_lists_boundary.argtypes = [P, I, I, P, P, P, P, P]
             lib.orc_lists_boundary.restype = L
             lib.orc_lists_bitmask.argtypes = [P, I, I, P, I, I, P, P]
             lib.orc_lists_bitmask.restype = L
             lib.orc_lists_mixed.argtypes = [P, I, I, P, P, P, I, I, P, P]
             lib.orc_lists_mixed.restype = L
-            lib.orc_lists_decode.argtypes = [P, I, I, I, I, P, P, P, P]
+            lib.orc_lists_decode.argtypes = [P, I, I, I, I, P, P, P, P, P]
             lib.orc_lists_decode.restype = L
             lib.orc_int_tile.argtypes = [I, I, P, P, P, P, P]
             lib.orc_int_tile.restype = I
             lib.orc_prefill_rows.argtypes = [P, P, P, P, I, I, I, I,
                                              P, P, P, P, P, P, P, P,
+                                             P, P, P, P,
                                              P, P, D, I, P, P, P]
             lib.orc_prefill_rows.restype = I
             lib.orc_decode_step.argtypes = [P, P, I, I, I, I,
@@ -123,19 +130,45 @@ def quantize(x_bits, cu_seqlens, want8=True, want4=True):
     return x8, x4, s8, s4
 
 
-def lists_boundary(cu_seqlens, b1, b2):
-    """Precision-grouped traversal rows (h, q-tile) from two diagonal boundaries."""
+def e4m3_value(code: int) -> float:
+    """Value of an FP8 E4M3 code (the format's definition)."""
+    return float(_load().orc_e4m3_value(int(code)))
+
+
+def e4m3_encode(r) -> int:
+    """E4M3 code of the fp32 value r: round to nearest, ties to even, saturating at 448."""
+    return int(_load().orc_e4m3_encode(float(np.float32(r))))
+
+
+def quantize_f8(x_bits, cu_seqlens):
+    """Per-(head, 64-token tile) FP8 E4M3 quantisation: (codes uint8 [H, ntiles, 64, d],
+    scales float32 [H, ntiles]) with sf = fl32(amax / 448), code = E4M3(fl32(x / sf))."""
+    x = _c(x_bits, np.uint16)
+    cu = _c(cu_seqlens, np.int32)
+    ntok, H, d = x.shape
+    nt = num_tiles(cu)
+    xf = np.zeros((H, nt, TILE, d), np.uint8)
+    sf = np.zeros((H, nt), np.float32)
+    if _load().orc_quantize_f8(_p(x), _p(cu), len(cu) - 1, H, d, _p(xf), _p(sf)) != 0:
+        raise ValueError("oracle FP8 quantize failed")
+    return xf, sf
+
+
+def lists_boundary(cu_seqlens, b1, b2, b8=None):
+    """Precision-grouped traversal rows (h, q-tile) from two diagonal boundaries, with an
+    optional FP8 band [b1, b8) between the INT8 and INT4 regions."""
     cu = _c(cu_seqlens, np.int32)
     b1 = _c(b1, np.int32)
     b2 = _c(b2, np.int32)
+    b8 = None if b8 is None else _c(b8, np.int32)
     lib = _load()
     B, Hq = len(cu) - 1, len(b1)
-    nnz = lib.orc_lists_boundary(_p(cu), B, Hq, _p(b1), _p(b2), None, None)
+    nnz = lib.orc_lists_boundary(_p(cu), B, Hq, _p(b1), _p(b8), _p(b2), None, None)
     if nnz < 0:
         raise ValueError("invalid boundaries")
     row_ptr = np.zeros(Hq * num_tiles(cu) + 1, np.int32)
     entries = np.zeros(max(nnz, 1), np.uint32)
-    lib.orc_lists_boundary(_p(cu), B, Hq, _p(b1), _p(b2), _p(row_ptr), _p(entries))
+    lib.orc_lists_boundary(_p(cu), B, Hq, _p(b1), _p(b8), _p(b2), _p(row_ptr), _p(entries))
     return row_ptr, entries[:nnz]
 
 
@@ -174,20 +207,23 @@ def lists_mixed(cu_seqlens, b1, b2, bitmask, G):
     return row_ptr, entries[:nnz]
 
 
-def lists_decode(cu_seqlens, Hq, Hkv, b1=None, b2=None):
-    """Decode-cache rows (b, kv-head); boundary mode if b1/b2 given, else all INT8."""
+def lists_decode(cu_seqlens, Hq, Hkv, b1=None, b2=None, b8=None):
+    """Decode-cache rows (b, kv-head); boundary mode if b1/b2 given (an FP8-band tile is
+    cached as INT8), else all INT8."""
     cu = _c(cu_seqlens, np.int32)
     mode = 1 if b1 is None else 0
     b1a = _c(b1 if b1 is not None else np.zeros(Hq), np.int32)
     b2a = _c(b2 if b2 is not None else np.zeros(Hq), np.int32)
+    b8a = None if b8 is None else _c(b8, np.int32)
     lib = _load()
     B = len(cu) - 1
-    nnz = lib.orc_lists_decode(_p(cu), B, Hq, Hkv, mode, _p(b1a), _p(b2a), None, None)
+    nnz = lib.orc_lists_decode(_p(cu), B, Hq, Hkv, mode, _p(b1a), _p(b8a), _p(b2a), None, None)
     if nnz < 0:
         raise ValueError("invalid decode policy")
     row_ptr = np.zeros(B * Hkv + 1, np.int32)
     entries = np.zeros(max(nnz, 1), np.uint32)
-    lib.orc_lists_decode(_p(cu), B, Hq, Hkv, mode, _p(b1a), _p(b2a), _p(row_ptr), _p(entries))
+    lib.orc_lists_decode(_p(cu), B, Hq, Hkv, mode, _p(b1a), _p(b8a), _p(b2a), _p(row_ptr),
+                         _p(entries))
     return row_ptr, entries[:nnz]
 
 
@@ -207,7 +243,7 @@ def int_tile(prec, q8t=None, q4t=None, k8t=None, k4t=None, d=None):
 class Quantised:
     """Oracle-side quantised tensors of one prefill (its own, never the GPU's)."""
 
-    def __init__(self, q_bits, k_bits, v_bits, cu_seqlens):
+    def __init__(self, q_bits, k_bits, v_bits, cu_seqlens, want_f8=False):
         none = (None, None, None, None)
         self.q8, self.q4, self.sq8, self.sq4 = (
             quantize(q_bits, cu_seqlens) if q_bits is not None else none)
@@ -215,6 +251,11 @@ class Quantised:
             quantize(k_bits, cu_seqlens) if k_bits is not None else none)
         self.v8, self.v4, self.sv8, self.sv4 = (
             quantize(v_bits, cu_seqlens) if v_bits is not None else none)
+        self.qf = self.sqf = self.kf = self.skf = None
+        if want_f8 and q_bits is not None:
+            self.qf, self.sqf = quantize_f8(q_bits, cu_seqlens)
+        if want_f8 and k_bits is not None:
+            self.kf, self.skf = quantize_f8(k_bits, cu_seqlens)
 
 
 def prefill_rows(q_bits, k_bits, v_bits, cu_seqlens, qz: Quantised, row_ptr, entries,
@@ -234,6 +275,7 @@ def prefill_rows(q_bits, k_bits, v_bits, cu_seqlens, qz: Quantised, row_ptr, ent
         _p(q), _p(k), _p(v), _p(cu), len(cu) - 1, Hq, Hkv, d,
         _p(qz.q8), _p(qz.q4), _p(qz.sq8), _p(qz.sq4),
         _p(qz.k8), _p(qz.k4), _p(qz.sk8), _p(qz.sk4),
+        _p(qz.qf), _p(qz.sqf), _p(qz.kf), _p(qz.skf),
         _p(rp), _p(en), float(scale), len(rows), _p(rows), _p(out), _p(lse))
     if rc != 0:
         raise ValueError(f"oracle prefill failed ({rc})")

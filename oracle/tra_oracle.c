@@ -50,6 +50,12 @@
  *  - decode cache precision of a k-tile is the highest precision any query
  *    head of the GQA group gives it at dist = (last prefill tile) - kt; in
  *    bitmask mode every cached tile is INT8.
+ *  - FP8 middle band (an extension the pages do not describe: an FP8 score
+ *    tier between INT8 and INT4): a third boundary b8 with b1 <= b8 <= b2;
+ *    b1 <= dist < b8 -> FP8 (E4M3) instead of INT4; per (head, tile) scale
+ *    sf = fl32(amax/448) and code = E4M3 round-to-nearest-even of fl32(x/sf),
+ *    saturating at +-448; precision code 4, listed after the other groups;
+ *    the decode cache keeps an FP8-band tile as INT8.
  */
 #include <math.h>
 #include <omp.h>
@@ -62,6 +68,7 @@
 #define ORC_INT4 1
 #define ORC_INT8 2
 #define ORC_BF16 3
+#define ORC_FP8 4
 
 /* bf16 bit pattern -> double; exact (bf16 is the top half of an fp32). */
 static double bf16_val(uint16_t bits) {
@@ -173,6 +180,74 @@ static int int4_code(const uint8_t* row, int c) {
 }
 
 /* ---------------------------------------------------------------------------
+ * FP8 E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; code 0x7F / 0xFF is NaN, so the largest finite magnitude is
+ * 1.75 * 2^8 = 448).  Magnitude code c = (e << 3) | m:
+ *   e = 0: m/8 * 2^-6 (subnormal);  e >= 1: (1 + m/8) * 2^(e - 7).
+ * ------------------------------------------------------------------------- */
+double orc_e4m3_value(int code) {
+  int e = (code >> 3) & 0xF, m = code & 7;
+  double mag = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return (code & 0x80) ? -mag : mag;
+}
+
+/* Round-to-nearest-even of r onto the finite E4M3 values, saturating at +-448:
+ * the nearest of the 127 non-negative finite magnitudes (a sorted table, binary
+ * search, then the closer neighbour), a tie going to the even code (mantissa LSB
+ * 0); the sign bit is r's own (so -0 and small negatives give 0x80). */
+int orc_e4m3_encode(float r) {
+  double a = fabs((double)r);
+  int lo = 0, hi = 126;                       /* magnitude codes 0x00 .. 0x7E */
+  if (a >= orc_e4m3_value(126)) {
+    lo = 126;
+  } else {
+    while (hi - lo > 1) {                     /* value(lo) <= a < value(hi) */
+      int mid = (lo + hi) / 2;
+      if (orc_e4m3_value(mid) <= a) lo = mid; else hi = mid;
+    }
+    double dl = a - orc_e4m3_value(lo), dh = orc_e4m3_value(hi) - a;
+    if (dh < dl || (dh == dl && (hi & 1) == 0)) lo = hi;
+  }
+  return (signbit(r) ? 0x80 : 0) | lo;
+}
+
+/* FP8 quantisation of one tensor: xf [H][ntiles][64][d] E4M3 codes, sf [H][ntiles]. */
+int orc_quantize_f8(const uint16_t* x, const int32_t* cu, int B, int H, int d, uint8_t* xf,
+                    float* sf) {
+  int64_t* off = (int64_t*)malloc(sizeof(int64_t) * (size_t)(B + 1));
+  int64_t ntiles = tile_offsets(cu, B, off);
+  for (int h = 0; h < H; ++h)
+    for (int b = 0; b < B; ++b) {
+      int T = cu[b + 1] - cu[b];
+      int nt = ceil_tiles(T);
+      for (int t = 0; t < nt; ++t) {
+        int64_t gt = off[b] + t;
+        float amax = 0.0f;
+        for (int r = 0; r < ORC_TILE && t * ORC_TILE + r < T; ++r) {
+          const uint16_t* row = x + ((int64_t)(cu[b] + t * ORC_TILE + r) * H + h) * d;
+          for (int c = 0; c < d; ++c) {
+            float a = fabsf(bf16_f32(row[c]));
+            if (a > amax) amax = a;
+          }
+        }
+        float s = amax / 448.0f;              /* IEEE fp32 divide */
+        sf[(int64_t)h * ntiles + gt] = s;
+        for (int r = 0; r < ORC_TILE; ++r) {
+          int tok = t * ORC_TILE + r;
+          uint8_t* o = xf + (((int64_t)h * ntiles + gt) * ORC_TILE + r) * d;
+          for (int c = 0; c < d; ++c) {
+            if (tok >= T || s == 0.0f) { o[c] = 0; continue; }
+            float xv = bf16_f32(x[((int64_t)(cu[b] + tok) * H + h) * d + c]);
+            o[c] = (uint8_t)orc_e4m3_encode(xv / s);
+          }
+        }
+      }
+    }
+  free(off);
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
  * Traversal lists.  Rows: prefill rows are (h, global q-tile) in h-major order;
  * decode-cache rows are (b, kv-head) in b-major order.
  * Pass row_ptr/entries NULL to only count; returns nnz (or -1 on error).
@@ -183,10 +258,18 @@ static int boundary_prec(int dist, int b1, int b2) {
   return ORC_SKIP;
 }
 
+/* with the FP8 middle band [b1, b8) */
+static int boundary_prec3(int dist, int b1, int b8, int b2) {
+  if (dist < b1) return ORC_INT8;
+  if (dist < b8) return ORC_FP8;
+  if (dist < b2) return ORC_INT4;
+  return ORC_SKIP;
+}
+
 /* Emit one row's entries from a per-k-tile precision array, grouped. */
 static int64_t emit_row(const int* prec, int n, uint32_t* entries, int64_t pos) {
-  static const int order[3] = {ORC_INT4, ORC_INT8, ORC_BF16};
-  for (int g = 0; g < 3; ++g)
+  static const int order[4] = {ORC_INT4, ORC_INT8, ORC_BF16, ORC_FP8};
+  for (int g = 0; g < 4; ++g)
     for (int kt = 0; kt < n; ++kt)
       if (prec[kt] == order[g]) {
         if (entries) entries[pos] = ((uint32_t)order[g] << 28) | (uint32_t)kt;
@@ -195,20 +278,23 @@ static int64_t emit_row(const int* prec, int n, uint32_t* entries, int64_t pos) 
   return pos;
 }
 
+/* b8 may be NULL (no FP8 band, b8 = b1). */
 int64_t orc_lists_boundary(const int32_t* cu, int B, int Hq, const int32_t* b1,
-                           const int32_t* b2, int32_t* row_ptr, uint32_t* entries) {
+                           const int32_t* b8, const int32_t* b2, int32_t* row_ptr,
+                           uint32_t* entries) {
   int64_t ntiles = orc_num_tiles(cu, B);
   int64_t pos = 0, row = 0;
   int nt_max = 0;
   for (int b = 0; b < B; ++b) if (ceil_tiles(cu[b + 1] - cu[b]) > nt_max) nt_max = ceil_tiles(cu[b + 1] - cu[b]);
   int* prec = (int*)malloc(sizeof(int) * (size_t)(nt_max + 1));
   for (int h = 0; h < Hq; ++h) {
-    if (b1[h] < 1 || b2[h] < b1[h]) { free(prec); return -1; }
+    const int bm = b8 ? b8[h] : b1[h];
+    if (b1[h] < 1 || bm < b1[h] || b2[h] < bm) { free(prec); return -1; }
     for (int b = 0; b < B; ++b) {
       int nt = ceil_tiles(cu[b + 1] - cu[b]);
       for (int qt = 0; qt < nt; ++qt, ++row) {
         if (row_ptr) row_ptr[row] = (int32_t)pos;
-        for (int kt = 0; kt <= qt; ++kt) prec[kt] = boundary_prec(qt - kt, b1[h], b2[h]);
+        for (int kt = 0; kt <= qt; ++kt) prec[kt] = boundary_prec3(qt - kt, b1[h], bm, b2[h]);
         pos = emit_row(prec, qt + 1, entries, pos);
       }
     }
@@ -293,7 +379,7 @@ int64_t orc_lists_mixed(const int32_t* cu, int B, int Hq, const int32_t* b1, con
 /* Decode-cache lists: rows (b, kvh).  mode 0 = boundary (b1,b2 per q head),
  * mode 1 = bitmask (every prefill tile cached as INT8). */
 int64_t orc_lists_decode(const int32_t* cu, int B, int Hq, int Hkv, int mode,
-                         const int32_t* b1, const int32_t* b2,
+                         const int32_t* b1, const int32_t* b8, const int32_t* b2,
                          int32_t* row_ptr, uint32_t* entries) {
   if (Hkv <= 0 || Hq % Hkv) return -1;
   int grp = Hq / Hkv;
@@ -312,7 +398,9 @@ int64_t orc_lists_decode(const int32_t* cu, int B, int Hq, int Hkv, int mode,
         } else {
           for (int j = 0; j < grp; ++j) {
             int h = kvh * grp + j;
-            int p = boundary_prec((nt - 1) - kt, b1[h], b2[h]);
+            /* an FP8-band tile is cached as INT8 */
+            int p = boundary_prec3((nt - 1) - kt, b1[h], b8 ? b8[h] : b1[h], b2[h]);
+            if (p == ORC_FP8) p = ORC_INT8;
             if (p > best) best = p;
           }
         }
@@ -365,6 +453,7 @@ int orc_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      const int32_t* cu, int B, int Hq, int Hkv, int d,
                      const int8_t* q8, const uint8_t* q4, const float* sq8, const float* sq4,
                      const int8_t* k8, const uint8_t* k4, const float* sk8, const float* sk4,
+                     const uint8_t* qf, const float* sqf, const uint8_t* kf, const float* skf,
                      const int32_t* row_ptr, const uint32_t* entries, double scale,
                      int nrows, const int64_t* rows, double* out, double* lse) {
   if (Hkv <= 0 || Hq % Hkv) return -1;
@@ -409,6 +498,14 @@ int orc_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
             double acc = 0.0;
             for (int ch = 0; ch < d; ++ch) acc += bf16_val(qr[ch]) * bf16_val(kr[ch]);
             sc = acc * scale;
+          } else if (prec == ORC_FP8) {
+            /* E4M3 values are exact in double, and so is the sum of their products */
+            const uint8_t* qr = qf + (((int64_t)h * ntiles + gq) * ORC_TILE + r) * d;
+            const uint8_t* kr = kf + (((int64_t)kvh * ntiles + gk) * ORC_TILE + c) * d;
+            double acc = 0.0;
+            for (int ch = 0; ch < d; ++ch) acc += orc_e4m3_value(qr[ch]) * orc_e4m3_value(kr[ch]);
+            sc = acc * (double)sqf[(int64_t)h * ntiles + gq] * (double)skf[(int64_t)kvh * ntiles + gk] *
+                 scale;
           } else {
             int64_t acc = 0;
             if (prec == ORC_INT8) {

@@ -668,3 +668,169 @@ def test_hybrid_decode_reduces_to_dense_softmax():
                 sc = keys @ val_of(qd[b, h]) / np.sqrt(d)
                 p = np.exp(sc - sc.max())
                 assert np.max(np.abs(got[b, h] - p @ vals / p.sum())) < 1e-12
+
+
+# --------------------------------------------------------------------------- FP8 middle band
+def _torch_e4m3(codes) -> np.ndarray:
+    """Values of E4M3 codes decoded by torch's float8_e4m3fn (an implementation of the
+    format independent of the oracle)."""
+    c = torch.from_numpy(np.asarray(codes, np.uint8).copy())
+    return c.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_values_match_the_format():
+    """Every finite code decodes as torch does; spot values of the format (largest finite
+    448, smallest normal 2^-6, smallest subnormal 2^-9, 1.0, 1.875, -1.0)."""
+    codes = [c for c in range(256) if c & 0x7F != 0x7F]
+    ours = np.array([oracle.e4m3_value(c) for c in codes])
+    assert np.array_equal(ours, _torch_e4m3(codes))
+    for c, v in ((0x7E, 448.0), (0x08, 2.0 ** -6), (0x01, 2.0 ** -9), (0x38, 1.0), (0x3F, 1.875),
+                 (0xB8, -1.0), (0x00, 0.0)):
+        assert oracle.e4m3_value(c) == v
+
+
+def test_e4m3_encode_round_to_nearest_even_and_saturation():
+    """Round to the nearest finite E4M3 value (torch's conversion agrees on every value in
+    range, midpoints included: ties to the even code), saturate beyond 448, keep the sign
+    of zero; every code's own value encodes back to it."""
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([
+        rng.uniform(-448, 448, 4000), rng.standard_normal(4000) * 3.0,
+        np.exp2(rng.uniform(-14, 8.8, 2000)) * rng.choice([-1, 1], 2000)]).astype(np.float32)
+    finite = np.array([oracle.e4m3_value(c) for c in range(0x7F)])
+    mids = ((finite[:-1] + finite[1:]) / 2).astype(np.float32)     # exact in fp32
+    vals = np.concatenate([vals, mids, -mids]).astype(np.float32)
+    vals = vals[np.abs(vals) <= 448]
+    ours = np.array([oracle.e4m3_encode(x) for x in vals], np.uint8)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+    for c in range(0x7F):
+        assert oracle.e4m3_encode(finite[c]) == c
+        assert oracle.e4m3_encode(-finite[c]) == 0x80 | c
+    assert oracle.e4m3_encode(500.0) == 0x7E and oracle.e4m3_encode(-1e9) == 0xFE
+    assert oracle.e4m3_encode(464.0) == 0x7E                        # past the last midpoint
+    assert oracle.e4m3_encode(-0.0) == 0x80 and oracle.e4m3_encode(-1e-9) == 0x80
+
+
+def test_quantize_f8_invariants():
+    """sf = fl32(amax / 448); the tile's largest magnitude maps to +-448; every code is the
+    nearest E4M3 value to fl32(x / sf); zero tiles give sf = 0 and codes 0; rows past the
+    sequence end are 0."""
+    w = wl.custom("f8q", [130, 64, 1], 2, 2, 64, 21, "boundary")
+    q, _, _ = _inputs(w)
+    q[64:128, 1] = 0                                                 # an all-zero tile of head 1
+    cu = w.cu_seqlens
+    xf, sf = oracle.quantize_f8(q, cu)
+    x = val_of(q).astype(np.float32)
+    gt = 0
+    for b in range(len(cu) - 1):
+        L = cu[b + 1] - cu[b]
+        for t in range((L + 63) // 64):
+            n = min(64, L - t * 64)
+            for h in range(w.Hq):
+                tile = x[cu[b] + t * 64: cu[b] + t * 64 + n, h]
+                amax = np.float32(np.abs(tile).max())
+                assert sf[h, gt] == np.float32(amax / np.float32(448.0))
+                codes = xf[h, gt, :n]
+                assert not xf[h, gt, n:].any()
+                if amax == 0:
+                    assert not codes.any()
+                    continue
+                r = (tile / sf[h, gt]).astype(np.float32)
+                assert np.all(np.abs(r) <= np.float32(448.0) * (1 + 2 ** -20))
+                ref = torch.from_numpy(np.clip(r, -448, 448)).to(torch.float8_e4m3fn)
+                assert np.array_equal(codes, ref.view(torch.uint8).numpy())
+                peak = codes.reshape(-1)[np.abs(tile).reshape(-1).argmax()]
+                assert peak & 0x7F == 0x7E
+            gt += 1
+
+
+def test_lists_fp8_band_closed_form():
+    """With the band [b1, b8): per row qt, FP8 tiles are min(qt+1, b8) - min(qt+1, b1), listed
+    after the INT8 group with precision code 4; b8 = b1 gives the two-boundary lists exactly;
+    the decode cache keeps a band tile as INT8, i.e. equals the cache of b1 := b8."""
+    cu = np.array([0, 700, 700 + 190], np.int32)
+    b1 = np.array([1, 3, 2, 5])
+    b8 = np.array([4, 3, 9, 5])
+    b2 = np.array([6, 7, 9, 11])
+    rp, en = oracle.lists_boundary(cu, b1, b2, b8=b8)
+    rp0, en0 = oracle.lists_boundary(cu, b1, b2)
+    rpe, ene = oracle.lists_boundary(cu, b1, b2, b8=b1)
+    assert np.array_equal(rp0, rpe) and np.array_equal(en0, ene)
+    nts = [(int(cu[i + 1] - cu[i]) + 63) // 64 for i in range(len(cu) - 1)]
+    row = 0
+    for h in range(len(b1)):
+        for nt in nts:
+            for qt in range(nt):
+                e = en[rp[row]:rp[row + 1]]
+                prec, kt = e >> 28, e & 0x0FFFFFFF
+                n8 = min(qt + 1, b1[h])
+                nf = min(qt + 1, b8[h]) - n8
+                n4 = min(qt + 1, b2[h]) - n8 - nf
+                assert (prec == oracle.INT8).sum() == n8 and (prec == oracle.FP8).sum() == nf
+                assert (prec == oracle.INT4).sum() == n4
+                assert list(prec) == sorted(prec, key=lambda p: [1, 2, 3, 4].index(p))
+                for p, k in zip(prec, kt):
+                    dist = qt - k
+                    want = 2 if dist < b1[h] else 4 if dist < b8[h] else 1
+                    assert p == want
+                row += 1
+    drp, den = oracle.lists_decode(cu, 4, 2, b1, b2, b8=b8)
+    drp1, den1 = oracle.lists_decode(cu, 4, 2, b8, b2)
+    assert np.array_equal(drp, drp1) and np.array_equal(den, den1)
+
+
+def test_prefill_fp8_band_brute_force():
+    """Every query/key pair through the routing rule with the band, scores from the codes
+    (FP8 codes decoded by torch, INT8 and INT4 codes as integers) times the two scales,
+    fp64 softmax and P V with bf16 V: the oracle's prefill agrees to 1e-12; b8 = b1
+    reproduces the two-boundary prefill."""
+    w = wl.custom("f8p", [200, 64, 1], 4, 2, 64, 23, "boundary", b1=[1, 2, 1, 3], b2=[4, 4, 2, 4])
+    b8 = np.array([3, 2, 2, 4])
+    q, k, v = _inputs(w)
+    cu = w.cu_seqlens
+    qz = oracle.Quantised(q, k, None, cu, want_f8=True)
+    rp, en = oracle.lists_boundary(cu, w.b1, w.b2, b8=b8)
+    rows = np.arange(len(rp) - 1)
+    out, lse = oracle.prefill_rows(q, k, v, cu, qz, rp, en, rows)
+    got = oracle.gather_rows(out, cu, rows, w.Hq)
+    d, grp = w.d, w.Hq // w.Hkv
+    vv = val_of(v)
+
+    def tok(codes, b, t):          # tile-major [H][nt][64][..] -> (global tile, row)
+        off = sum((cu[i + 1] - cu[i] + 63) // 64 for i in range(b))
+        return off + t // 64, t % 64
+
+    qf = _torch_e4m3(qz.qf.reshape(-1)).reshape(qz.qf.shape)
+    kf = _torch_e4m3(qz.kf.reshape(-1)).reshape(qz.kf.shape)
+    q4, k4 = _unpack4(qz.q4), _unpack4(qz.k4)
+    for b in range(len(cu) - 1):
+        T = cu[b + 1] - cu[b]
+        for h in range(w.Hq):
+            kh = h // grp
+            for i in range(T):
+                gq, rq = tok(None, b, i)
+                sc, vals = [], []
+                for j in range(i + 1):
+                    gk, rk = tok(None, b, j)
+                    dist = i // 64 - j // 64
+                    if dist < w.b1[h]:
+                        s = float(qz.q8[h, gq, rq].astype(np.int64) @ qz.k8[kh, gk, rk].astype(np.int64))
+                        s *= float(qz.sq8[h, gq]) * float(qz.sk8[kh, gk])
+                    elif dist < b8[h]:
+                        s = float(qf[h, gq, rq] @ kf[kh, gk, rk]) * float(qz.sqf[h, gq]) * float(qz.skf[kh, gk])
+                    elif dist < w.b2[h]:
+                        s = float(q4[h, gq, rq] @ k4[kh, gk, rk]) * float(qz.sq4[h, gq]) * float(qz.sk4[kh, gk])
+                    else:
+                        continue
+                    sc.append(s / np.sqrt(d))
+                    vals.append(vv[cu[b] + j, kh])
+                sc = np.array(sc)
+                p = np.exp(sc - sc.max())
+                ref = (p / p.sum()) @ np.array(vals)
+                assert np.max(np.abs(got[(h, cu[b] + i)] - ref)) < 1e-12
+    rp0, en0 = oracle.lists_boundary(cu, w.b1, w.b2)
+    out0, _ = oracle.prefill_rows(q, k, v, cu, qz, rp0, en0, rows)
+    rpe, ene = oracle.lists_boundary(cu, w.b1, w.b2, b8=w.b1)
+    oute, _ = oracle.prefill_rows(q, k, v, cu, qz, rpe, ene, rows)
+    assert np.array_equal(out0, oute)
