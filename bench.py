@@ -21,7 +21,8 @@ For N > 1 launch with torch.distributed.run; every rank runs an independent
 replica (the method has no cross-GPU exchange) and rank 0 prints one JSON line.
 
 Reduced lines (--only): "prefill" times one prefill workload (--workload
-bitmask_32k | llama8b_8k | varlen_8 | mixed_8k), "decode" the decode alone,
+bitmask_32k | llama8b_8k | varlen_8 | mixed_8k | llama8b_8k_fp8, the last with an
+FP8 band halfway between each head's b1 and b2), "decode" the decode alone,
 "allocate" fits the complete-tile cost model and runs the boundary allocator on
 synthetic error tables, then times the allocated policy; "hybrid" times the
 token-level hybrid decode and prefill.
@@ -65,7 +66,8 @@ def parse():
     ap.add_argument("--only", choices=["prefill", "decode", "allocate", "hybrid"], default=None,
                     help="run one part only (used for profiler captures); prints a reduced line. "
                          "allocate: measured complete-tile cost model + boundary allocator demo")
-    ap.add_argument("--workload", choices=["bitmask_32k", "llama8b_8k", "varlen_8", "mixed_8k"],
+    ap.add_argument("--workload", choices=["bitmask_32k", "llama8b_8k", "varlen_8", "mixed_8k",
+                                           "llama8b_8k_fp8"],
                     default="bitmask_32k",
                     help="prefill workload for --only prefill (the full bench line always uses "
                          "bitmask_32k)")
@@ -159,7 +161,8 @@ def prefill_setup(device, workload="bitmask_32k"):
     from tile_routed_mixed_causal_b200 import api
     from tile_routed_mixed_causal_b200 import workloads as wl
 
-    w = getattr(wl, workload)()
+    fp8 = workload.endswith("_fp8")  # the same workload with an FP8 band between b1 and b2
+    w = getattr(wl, workload[:-4] if fp8 else workload)()
     t = wl.make_inputs(w, device)
     q, k, v = t["q"], t["k"], t["v"]
     shape = tra.Shape(w.cu_seqlens, w.Hq, w.Hkv, w.d, device=device)
@@ -171,7 +174,7 @@ def prefill_setup(device, workload="bitmask_32k"):
         pol = tra.Policy.mixed(w.b1, w.b2, bitmask, w.G)
     else:
         bitmask = torch.zeros(1, dtype=torch.int32, device=device)
-        pol = tra.Policy.boundary(w.b1, w.b2)
+        pol = tra.Policy.boundary(w.b1, w.b2, b8=(w.b1 + w.b2) // 2 if fp8 else None)
     plan = api.PrefillPlan(shape, pol, device=device)
     out = torch.empty_like(q)
     plan.lists()
@@ -180,8 +183,10 @@ def prefill_setup(device, workload="bitmask_32k"):
     n16 = int(np.sum(prec == tra.PREC_BF16))
     n8 = int(np.sum(prec == tra.PREC_INT8))
     n4 = int(np.sum(prec == tra.PREC_INT4))
-    return dict(w=w, q=q, k=k, v=v, shape=shape, bitmask=bitmask, pol=pol, plan=plan, out=out,
-                tiles=plan.nnz, n16=n16, n8=n8, n4=n4)
+    nf = int(np.sum(prec == tra.PREC_FP8))
+    name = w.name + ("_fp8band" if fp8 else "")
+    return dict(w=w, name=name, q=q, k=k, v=v, shape=shape, bitmask=bitmask, pol=pol, plan=plan,
+                out=out, tiles=plan.nnz, n16=n16, n8=n8, n4=n4, nf=nf)
 
 
 def prefill_ops(S):
@@ -190,11 +195,13 @@ def prefill_ops(S):
 
 
 def roofline_time(S, bf16_tflops):
-    """Tile-mix-weighted tensor roofline: INT8/INT4 QK at 2x the bf16 rate (the nominal
-    4.5 / 2.25 PFLOP/s ratio), BF16 QK and all P*V at the bf16 rate."""
+    """Tile-mix-weighted tensor roofline: INT8/INT4/FP8 QK at 2x the bf16 rate (the nominal
+    4.5 / 2.25 PFLOP/s ratio of the int8 and fp8 kinds), BF16 QK and all P*V at the bf16
+    rate."""
     per = TILE_OPS_PER_GEMM * S["w"].d
     bf = bf16_tflops * 1e12
-    return (S["n8"] + S["n4"]) * per / (2 * bf) + S["n16"] * per / bf + S["tiles"] * per / bf
+    return ((S["n8"] + S["n4"] + S["nf"]) * per / (2 * bf) + S["n16"] * per / bf
+            + S["tiles"] * per / bf)
 
 
 def run_prefill_bench(S, steps, warmup, stream):
@@ -317,7 +324,8 @@ def quantize_bench(S, stream, reps=20):
     return {"ms": round(ms, 4), "bytes": int(bytes_), "GB/s": round(bytes_ / (ms * 1e-3) / 1e9, 1)}
 
 
-def workload_records(device, stream, bf16_tflops, names=("llama8b_8k", "varlen_8", "mixed_8k"),
+def workload_records(device, stream, bf16_tflops,
+                     names=("llama8b_8k", "varlen_8", "mixed_8k", "llama8b_8k_fp8"),
                      steps=10, warmup=3):
     """The other prefill configurations: kernel time, TOPS and tile-mix roofline fraction."""
     recs = {}
@@ -327,12 +335,13 @@ def workload_records(device, stream, bf16_tflops, names=("llama8b_8k", "varlen_8
         ops = prefill_ops(S)
         kern = statistics.median(attn_ms)
         t_roof = roofline_time(S, bf16_tflops)
-        recs[name] = {"workload": S["w"].name, "prefill_kernel_ms": round(kern, 4),
+        recs[name] = {"workload": S["name"], "prefill_kernel_ms": round(kern, 4),
                       "ms_per_step": round(total_ms / steps, 4),
                       "kernel_TOPS": round(ops / (kern * 1e-3) / 1e12, 2),
                       "roofline_frac": round(t_roof / (kern * 1e-3), 4),
                       "tiles": S["tiles"], "bf16_tiles": S["n16"], "int8_tiles": S["n8"],
-                      "int4_tiles": S["n4"], "prep_ms": round(statistics.median(prep_ms), 4)}
+                      "int4_tiles": S["n4"], "fp8_tiles": S["nf"],
+                      "prep_ms": round(statistics.median(prep_ms), 4)}
         del S
         torch.cuda.empty_cache()
     return recs
@@ -784,13 +793,13 @@ def main():
             ops = prefill_ops(S)
             kern = sum(attn_ms) / len(attn_ms)
             t_roof = roofline_time(S, bf16_tflops)
-            print(json.dumps({"only": "prefill", "workload": S["w"].name,
+            print(json.dumps({"only": "prefill", "workload": S["name"],
                               "ms_per_step": total_ms / args.steps, "prefill_kernel_ms": kern,
                               "TOPS": ops / (total_ms / args.steps * 1e-3) / 1e12,
                               "kernel_TOPS": ops / (kern * 1e-3) / 1e12,
                               "roofline_frac": t_roof / (kern * 1e-3),
                               "tiles": S["tiles"], "bf16_tiles": S["n16"], "int8_tiles": S["n8"],
-                              "int4_tiles": S["n4"]}), flush=True)
+                              "int4_tiles": S["n4"], "fp8_tiles": S["nf"]}), flush=True)
         return
     S = prefill_setup(device)
     ops = prefill_ops(S)

@@ -89,6 +89,10 @@ typedef enum {
 #define TRA_PREC_INT4 1
 #define TRA_PREC_INT8 2
 #define TRA_PREC_BF16 3
+/* FP8 (E4M3) score tiles of the optional middle band of a boundary policy (tra_policy.b8):
+ * an extension the pages do not describe (an FP8 tier between INT8 and INT4), run on the
+ * fp8 tensor-core kind at the INT8 rate.  Listed after the other groups of a row. */
+#define TRA_PREC_FP8 4
 
 #define TRA_POLICY_BOUNDARY 0
 #define TRA_POLICY_BITMASK 1
@@ -117,6 +121,12 @@ typedef enum {
  * The packed Q4 / K4 formats stay the compact cache for decoding. */
 #define TRA_FMT_Q4X 0x40u
 #define TRA_FMT_K4X 0x80u
+/* FP8 E4M3 codes of Q / K [H][ntiles][64][d] (one byte per value, row-major) with one
+ * scale per (head, tile): sf = fl32(amax / 448), code = E4M3 round-to-nearest-even of
+ * fl32(x / sf) saturating at +-448 (the sign of a zero kept); amax = 0 gives sf = 0 and
+ * codes 0.  Needed by the prefill when a boundary policy has an FP8 band (b8 > b1). */
+#define TRA_FMT_Q8F 0x100u
+#define TRA_FMT_K8F 0x200u
 
 /* device status word bits */
 #define TRA_DEV_TIMEOUT 0x1      /* a bounded pipeline wait expired */
@@ -142,6 +152,9 @@ typedef struct {
   const uint32_t* bitmask_dev;      /* device [Hq][ntiles][W] (bitmask and mixed modes) */
   int32_t G;                        /* k-tiles per bit (bitmask and mixed modes), >= 1 */
   int32_t W;                        /* words per bitmask row, W*32*G >= max nt */
+  /* boundary mode only, optional (NULL: no FP8 band): host [Hq] with b1 <= b8 <= b2;
+   * b1 <= dist < b8 -> FP8 instead of INT4.  Decode caches keep a band tile as INT8. */
+  const int32_t* b8;
 } tra_policy;
 
 typedef struct {
@@ -153,6 +166,8 @@ typedef struct {
   float* sv8;  float* sv4;
   uint32_t formats;                 /* TRA_FMT_* bits: which fields are present */
   int8_t* q4x; int8_t* k4x;         /* [Hq|Hkv][ntiles][64][d]: 16 x INT4 code (TRA_FMT_Q4X/K4X) */
+  uint8_t* q8f; uint8_t* k8f;       /* [Hq|Hkv][ntiles][64][d]: FP8 E4M3 codes (TRA_FMT_Q8F/K8F) */
+  float* sqf; float* skf;           /* [Hq|Hkv][ntiles]: their scales */
 } tra_qtiles;
 /* Code layout.  Rows are tokens of a 64-token tile; INT8 rows hold channel c in byte c,
  * as two's complement for Q8 and K8 and offset-binary (code + 128) for V8, which only
@@ -227,14 +242,16 @@ TRA_API tra_status build_tile_lists(const tra_shape* shape, const tra_policy* po
  * TileMix abstract: the high- and low-precision paths share one online-softmax
  * state.)
  * q/k/v: device bf16 as above; tiles: output of quantize_qkv_tiles (Q8/K8
- * always, Q4X/K4X and the INT4 scales when the policy has INT4 tiles);
- * row_ptr/entries: prefill
+ * always, Q4X/K4X and the INT4 scales when the policy has INT4 tiles, Q8F/K8F
+ * when a boundary policy has an FP8 band: its tiles score on FP8 E4M3 codes with
+ * fp32 accumulation, rescaled by sQ*sK); row_ptr/entries: prefill
  * lists; out: device bf16 [ntok][Hq][d]; lse: device float [Hq][ntok] natural-
  * log logsumexp of the scaled scores, or NULL.
  * Integer-accumulator dump (debug; n_dump = 0 disables): dump_coords device
  * int32 [n_dump][4] = (b, h, qt, kt); for each listed INT8/INT4 tile the raw
  * int32 Q-code x K-code^T accumulators go to dump_out [n_dump][64][64]
- * (row = query within the tile, column = key).  n_dump <= TRA_MAX_DUMP.
+ * (row = query within the tile, column = key; BF16 and FP8 tiles, whose
+ * accumulators are fp32, are not dumped).  n_dump <= TRA_MAX_DUMP.
  * status_dev: device int32, receives TRA_DEV_* bits.
  */
 TRA_API tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* policy,

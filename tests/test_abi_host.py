@@ -261,3 +261,38 @@ def test_hybrid_capacity_and_validation(lib):
     args = [s.c, ctypes.byref(hy), FAKE, FAKE, FAKE, ctypes.byref(qt), FAKE, FAKE, FAKE, 4, 0.1,
             FAKE, FAKE, 1 << 30, FAKE, None]
     assert lib.hybrid_attention_decode(*args) == 1 and b"K4" in lib.tra_last_error()
+
+
+def test_fp8_band_validation_and_sizes(lib):
+    """b8 must lie in [b1, b2]; only boundary policies take it; an FP8 band relabels kept
+    tiles, so list sizes equal the oracle's (with and without a band); the prefill asks for
+    the FP8 tiles before any launch; Q8F / K8F sizes."""
+    s = _shape([1000, 64, 1], Hq=4, Hkv=2)
+    b1, b2 = [1, 2, 3, 1], [4, 5, 9, 40]
+    for bad in ([0, 2, 3, 1], [5, 2, 3, 1]):          # below b1, above b2
+        with pytest.raises(L.TraError) as e:
+            L.tile_lists_size(s, L.Policy.boundary(b1, b2, b8=bad))
+        assert e.value.status == 1
+    b8 = [3, 2, 9, 20]
+    pol = L.Policy.boundary(b1, b2, b8=b8)
+    assert pol.has_fp8 and pol.has_int4
+    assert not L.Policy.boundary(b1, b2, b8=b1).has_fp8
+    assert not L.Policy.boundary([1, 1], [4, 4], b8=[4, 4]).has_int4
+    for kind, ref in ((L.LISTS_PREFILL, oracle.lists_boundary(s.cu_host, b1, b2, b8=b8)),
+                      (L.LISTS_DECODE_CACHE, oracle.lists_decode(s.cu_host, 4, 2, b1, b2, b8=b8))):
+        rows, nnz = L.tile_lists_size(s, pol, kind)
+        assert rows == len(ref[0]) - 1 and nnz == len(ref[1])
+    mixed = L.Policy(L.POLICY_MIXED, b1=b1, b2=b2, G=1, b8=b8)
+    mixed._c.W = 1
+    with pytest.raises(L.TraError) as e:
+        L.tile_lists_size(s, mixed)
+    assert e.value.status == 2
+    qt = L._QTiles()
+    qt.formats = L.FMT_Q8 | L.FMT_K8 | L.FMT_Q4X | L.FMT_K4X
+    for f in ("q8", "k8", "sq8", "sk8", "q4x", "k4x", "sq4", "sk4"):
+        setattr(qt, f, FAKE.value)
+    st = lib.routed_attention_prefill(s.c, pol.c, FAKE, FAKE, FAKE, ctypes.byref(qt), FAKE, FAKE,
+                                      ctypes.c_float(0.1), FAKE, None, None, 0, None, FAKE, None)
+    assert st == 1 and b"Q8F" in lib.tra_last_error()
+    nt = lib.tra_num_tiles(s.c)
+    assert lib.tra_qtiles_bytes(s.c, L.FMT_Q8F) == 4 * nt * 64 * 128 + ((4 * nt * 4 + 255) // 256) * 256

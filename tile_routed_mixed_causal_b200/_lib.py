@@ -18,11 +18,12 @@ LIB_PATH = os.path.join(_PKG, "libtra.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "tra.h")
 
 TILE = 64
-PREC_INT4, PREC_INT8, PREC_BF16 = 1, 2, 3
+PREC_INT4, PREC_INT8, PREC_BF16, PREC_FP8 = 1, 2, 3, 4
 POLICY_BOUNDARY, POLICY_BITMASK, POLICY_MIXED = 0, 1, 2
 LISTS_PREFILL, LISTS_DECODE_CACHE = 0, 1
 FMT_Q8, FMT_Q4, FMT_K8, FMT_K4, FMT_V8, FMT_V4 = 0x1, 0x2, 0x4, 0x8, 0x10, 0x20
 FMT_Q4X, FMT_K4X = 0x40, 0x80
+FMT_Q8F, FMT_K8F = 0x100, 0x200
 DEV_TIMEOUT, DEV_TAIL_FULL, DEV_BAD_LIST = 0x1, 0x2, 0x4
 STATUS = {0: "TRA_OK", 1: "TRA_ERR_INVALID", 2: "TRA_ERR_UNSUPPORTED", 3: "TRA_ERR_BUFFER",
           4: "TRA_ERR_CUDA", 5: "TRA_ERR_TIMEOUT"}
@@ -42,7 +43,8 @@ class _Shape(ctypes.Structure):
 
 class _Policy(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("b1", ctypes.c_void_p), ("b2", ctypes.c_void_p),
-                ("bitmask_dev", ctypes.c_void_p), ("G", ctypes.c_int32), ("W", ctypes.c_int32)]
+                ("bitmask_dev", ctypes.c_void_p), ("G", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("b8", ctypes.c_void_p)]
 
 
 class _Hybrid(ctypes.Structure):
@@ -54,7 +56,9 @@ class _Hybrid(ctypes.Structure):
 class _QTiles(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("q8", "q4", "k8", "k4", "v8", "v4", "sq8", "sq4", "sk8", "sk4", "sv8", "sv4")] + \
-               [("formats", ctypes.c_uint32), ("q4x", ctypes.c_void_p), ("k4x", ctypes.c_void_p)]
+               [("formats", ctypes.c_uint32), ("q4x", ctypes.c_void_p), ("k4x", ctypes.c_void_p),
+                ("q8f", ctypes.c_void_p), ("k8f", ctypes.c_void_p), ("sqf", ctypes.c_void_p),
+                ("skf", ctypes.c_void_p)]
 
 
 _lib = None
@@ -159,13 +163,15 @@ class Shape:
 
 
 class Policy:
-    """Boundary policy (host b1/b2 per head), bitmask policy (device words, G), or
-    both at once (mixed: boundaries decide skip / INT4 / INT8, a set bit BF16)."""
+    """Boundary policy (host b1/b2 per head, optionally an FP8 band [b1, b8)), bitmask
+    policy (device words, G), or both at once (mixed: boundaries decide skip / INT4 /
+    INT8, a set bit BF16)."""
 
-    def __init__(self, mode, b1=None, b2=None, bitmask=None, G=1):
+    def __init__(self, mode, b1=None, b2=None, bitmask=None, G=1, b8=None):
         self.mode = mode
         self.b1 = None if b1 is None else np.ascontiguousarray(np.asarray(b1, np.int32))
         self.b2 = None if b2 is None else np.ascontiguousarray(np.asarray(b2, np.int32))
+        self.b8 = None if b8 is None else np.ascontiguousarray(np.asarray(b8, np.int32))
         self.bitmask = bitmask
         self.G = int(G)
         self.W = int(bitmask.shape[-1]) if bitmask is not None else 0
@@ -173,11 +179,12 @@ class Policy:
                           self.b1.ctypes.data if self.b1 is not None else None,
                           self.b2.ctypes.data if self.b2 is not None else None,
                           bitmask.data_ptr() if isinstance(bitmask, torch.Tensor) else None,
-                          self.G, self.W)
+                          self.G, self.W,
+                          self.b8.ctypes.data if self.b8 is not None else None)
 
     @classmethod
-    def boundary(cls, b1, b2):
-        return cls(POLICY_BOUNDARY, b1=b1, b2=b2)
+    def boundary(cls, b1, b2, b8=None):
+        return cls(POLICY_BOUNDARY, b1=b1, b2=b2, b8=b8)
 
     @classmethod
     def from_bitmask(cls, bitmask: torch.Tensor, G: int):
@@ -193,7 +200,12 @@ class Policy:
 
     @property
     def has_int4(self) -> bool:
-        return self.mode != POLICY_BITMASK and bool(np.any(self.b2 > self.b1))
+        lo = self.b8 if self.b8 is not None else self.b1
+        return self.mode != POLICY_BITMASK and bool(np.any(self.b2 > lo))
+
+    @property
+    def has_fp8(self) -> bool:
+        return self.mode == POLICY_BOUNDARY and self.b8 is not None and bool(np.any(self.b8 > self.b1))
 
 
 class QTiles:
@@ -215,10 +227,14 @@ class QTiles:
                 self.t[name + "4x"] = torch.zeros((H, nt, TILE, d), dtype=torch.int8, device=device)
             if formats & ((FMT_Q4 << (2 * i)) | x4):
                 self.t["s" + name + "4"] = torch.zeros((H, nt), dtype=torch.float32, device=device)
+            if formats & {"q": FMT_Q8F, "k": FMT_K8F}.get(name, 0):
+                self.t[name + "8f"] = torch.zeros((H, nt, TILE, d), dtype=torch.uint8, device=device)
+                self.t["s" + name + "f"] = torch.zeros((H, nt), dtype=torch.float32, device=device)
         ptr = lambda n: self.t[n].data_ptr() if n in self.t else None
         self._c = _QTiles(*[ptr(n) for n in ("q8", "q4", "k8", "k4", "v8", "v4",
                                              "sq8", "sq4", "sk8", "sk4", "sv8", "sv4")],
-                          formats, ptr("q4x"), ptr("k4x"))
+                          formats, ptr("q4x"), ptr("k4x"), ptr("q8f"), ptr("k8f"), ptr("sqf"),
+                          ptr("skf"))
 
     def __getitem__(self, k):
         return self.t[k]

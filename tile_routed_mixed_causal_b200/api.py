@@ -28,6 +28,8 @@ class PrefillPlan:
         fm = L.FMT_Q8 | L.FMT_K8
         if policy.has_int4:
             fm |= L.FMT_Q4X | L.FMT_K4X     # INT4 codes in the tensor-core operand form
+        if policy.has_fp8:
+            fm |= L.FMT_Q8F | L.FMT_K8F     # FP8 E4M3 codes of the FP8 band
         if keep_v_cache:
             fm |= L.FMT_K4 | L.FMT_V8 | L.FMT_V4
         self.tiles = L.QTiles(shape, fm, device)

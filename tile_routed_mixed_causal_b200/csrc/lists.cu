@@ -75,12 +75,20 @@ __global__ void __launch_bounds__(256) lists_kernel(const ListParams p) {
     if (lane == 0) p.row_ptr[row] = (int32_t)off;
     uint32_t* e = p.entries + off;
     if (p.mode == TRA_POLICY_BOUNDARY) {
+      // the kept tiles qt-n+1 .. qt in distance bands: INT4 (farthest), then FP8, then
+      // INT8 (nearest); written as the INT4 group, the INT8 group, the FP8 group
       const int n = min(qt + 1, p.b2[h]);
       const int n8 = min(qt + 1, p.b1[h]);
-      const int n4 = n - n8;
+      const int nf = min(qt + 1, p.b8[h]) - n8;
+      const int n4 = n - n8 - nf;
       for (int i = lane; i < n; i += 32) {
-        const uint32_t prec = i < n4 ? TRA_PREC_INT4 : TRA_PREC_INT8;
-        e[i] = (prec << 28) | (uint32_t)(qt - n + 1 + i);
+        const uint32_t kt = (uint32_t)(qt - n + 1 + i);
+        if (i < n4)
+          e[i] = ((uint32_t)TRA_PREC_INT4 << 28) | kt;
+        else if (i < n4 + nf)
+          e[n4 + n8 + (i - n4)] = ((uint32_t)TRA_PREC_FP8 << 28) | kt;
+        else
+          e[n4 + (i - n4 - nf)] = ((uint32_t)TRA_PREC_INT8 << 28) | kt;
       }
     } else if (p.mode == TRA_POLICY_MIXED) {
       // kept tiles qt-n+1 .. qt as under boundaries; a set bit promotes one to BF16.
@@ -169,9 +177,9 @@ __global__ void __launch_bounds__(256) lists_kernel(const ListParams p) {
   const int b = (int)(row / p.Hkv), kvh = (int)(row % p.Hkv);
   const int nt = seq_tiles(p.cu, b);
   uint32_t* e = p.entries + off;
-  if (p.mode != TRA_POLICY_BITMASK) {  // boundaries (mixed policies too)
+  if (p.mode != TRA_POLICY_BITMASK) {  // boundaries (mixed policies too); an FP8-band tile is cached as INT8
     const int n = min(nt, group_max_b(p.b2, kvh, grp));
-    const int n8 = min(nt, group_max_b(p.b1, kvh, grp));
+    const int n8 = min(nt, group_max_b(p.b8, kvh, grp));
     for (int i = lane; i < n; i += 32) {
       const uint32_t prec = i < n - n8 ? TRA_PREC_INT4 : TRA_PREC_INT8;
       e[i] = (prec << 28) | (uint32_t)(nt - n + i);

@@ -54,20 +54,23 @@ constexpr uint32_t kNoKt = 0x0FFFFFFFu;
 
 // Precision of a hybrid-prefill entry whose K and V come from the mixed operands
 // (bf16 rows of selected tokens, INT4 codes as bf16 integers for the others).
-constexpr int kPrecHyb = 4;
+constexpr int kPrecHyb = 5;
 
 template <int D, int MODE>
 struct Cfg {
   static constexpr bool kHyb = MODE == kPrefillModeHybrid;        // token-level hybrid prefill
-  static constexpr bool kHasBf16 = MODE != TRA_POLICY_BOUNDARY;  // bf16 Q and K operands
+  static constexpr bool kHasF8 = MODE == kPrefillModeBoundaryF8;   // FP8 band of a boundary policy
+  static constexpr bool kHasBf16 = MODE != TRA_POLICY_BOUNDARY && !kHasF8;  // bf16 Q and K operands
   static constexpr bool kHasInt4 = MODE != TRA_POLICY_BITMASK && !kHyb;  // INT4 operands (int8 form)
+  static constexpr int kRuns = kHasF8 ? 4 : 3;  // precision runs of a traversal row
   // work units per CTA: two, or one under a mixed policy, whose operand buffers
   // (int8, INT4 and bf16 Q, bf16-sized K slots) do not fit twice
   static constexpr int kCtaUnits = MODE == TRA_POLICY_MIXED ? 1 : 2;
   static constexpr int kQ8Bytes = kHyb ? 0 : 128 * D;          // int8 Q codes
   static constexpr int kQ4Bytes = kHasInt4 ? 128 * D : 0;      // INT4 Q codes as int8
   static constexpr int kQbBytes = kHasBf16 ? 128 * D * 2 : 0;  // bf16 Q
-  static constexpr int kQUnitBytes = kQ8Bytes + kQ4Bytes + kQbBytes;
+  static constexpr int kQfBytes = kHasF8 ? 128 * D : 0;        // FP8 E4M3 Q codes
+  static constexpr int kQUnitBytes = kQ8Bytes + kQ4Bytes + kQbBytes + kQfBytes;
   // K slot: one K tile, BF16 or int8 codes (INT8 or INT4 in int8 form)
   static constexpr int kKBytes = kHasBf16 ? 64 * D * 2 : 64 * D;
   static constexpr int kVBytes = 64 * D * 2;
@@ -99,14 +102,15 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = 512;
 };
 
-// The two q-tiles' rows of a unit merged in ascending kt.  A row lists its INT4,
-// INT8 and BF16 tiles as three ascending runs (sorted as whole entries); next()
-// yields each kt of either row once with the precision each row gives it (0: the
-// row does not list it).
+// The two q-tiles' rows of a unit merged in ascending kt.  A row lists its tiles
+// as NR ascending runs, one per precision (INT4, INT8, BF16 and, with an FP8 band,
+// FP8; sorted as whole entries); next() yields each kt of either row once with the
+// precision each row gives it (0: the row does not list it).
+template <int NR>
 struct KtMerge {
   const uint32_t* e;
-  int pos[2][3], end[2][3];
-  uint32_t head[2][3];  // current kt of each run, kNoKt when exhausted
+  int pos[2][NR], end[2][NR];
+  uint32_t head[2][NR];  // current kt of each run, kNoKt when exhausted
 
   __device__ __forceinline__ void load(int r, int g) {
     head[r][g] = pos[r][g] < end[r][g] ? (__ldg(e + pos[r][g]) & kNoKt) : kNoKt;
@@ -123,13 +127,16 @@ struct KtMerge {
     e = entries;
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int b8 = lower_bound(e, rs[r], re[r], (uint32_t)TRA_PREC_INT8 << 28);
-      const int bb = lower_bound(e, b8, re[r], (uint32_t)TRA_PREC_BF16 << 28);
-      pos[r][0] = rs[r]; end[r][0] = b8;
-      pos[r][1] = b8;    end[r][1] = bb;
-      pos[r][2] = bb;    end[r][2] = re[r];
+      int lo = rs[r];
 #pragma unroll
-      for (int g = 0; g < 3; ++g) load(r, g);
+      for (int g = 0; g < NR; ++g) {  // run g holds precision g + 1
+        const int hi = g + 1 < NR ? lower_bound(e, lo, re[r], (uint32_t)(g + 2) << 28) : re[r];
+        pos[r][g] = lo;
+        end[r][g] = hi;
+        lo = hi;
+      }
+#pragma unroll
+      for (int g = 0; g < NR; ++g) load(r, g);
     }
   }
   // next entry: kt and each row's precision (TRA_PREC_*, or 0)
@@ -138,15 +145,15 @@ struct KtMerge {
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int g = 0; g < 3; ++g) k = min(k, head[r][g]);
+      for (int g = 0; g < NR; ++g) k = min(k, head[r][g]);
     if (k == kNoKt) return false;
     int pr[2] = {0, 0};
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int g = 0; g < 3; ++g)
+      for (int g = 0; g < NR; ++g)
         if (head[r][g] == k) {
-          pr[r] = g + 1;  // TRA_PREC_INT4 = 1, INT8 = 2, BF16 = 3
+          pr[r] = g + 1;  // TRA_PREC_INT4 = 1, INT8 = 2, BF16 = 3, FP8 = 4
           ++pos[r][g];
           load(r, g);
         }
@@ -188,8 +195,9 @@ __device__ __forceinline__ Unit make_unit(const PrefillParams& p, long long id) 
   return x;
 }
 
-__device__ __forceinline__ KtMerge unit_merge(const PrefillParams& p, const Unit& x) {
-  KtMerge c;
+template <int NR>
+__device__ __forceinline__ KtMerge<NR> unit_merge(const PrefillParams& p, const Unit& x) {
+  KtMerge<NR> c;
   int rs[2] = {0, 0}, re[2] = {0, 0};
   if (x.valid) {
     rs[0] = __ldg(p.row_ptr + x.row0);
@@ -244,13 +252,16 @@ struct HybStream {
   }
 };
 
-__device__ __forceinline__ KtMerge unit_stream(const PrefillParams& p, const Unit& x, std::false_type) {
-  return unit_merge(p, x);
-}
-__device__ __forceinline__ HybStream unit_stream(const PrefillParams& p, const Unit& x, std::true_type) {
-  HybStream c;
-  c.init(x, p.window);
-  return c;
+// the entry stream of a unit: the merged traversal rows, or the hybrid's own
+template <class C>
+__device__ __forceinline__ auto unit_stream(const PrefillParams& p, const Unit& x) {
+  if constexpr (C::kHyb) {
+    HybStream c;
+    c.init(x, p.window);
+    return c;
+  } else {
+    return unit_merge<C::kRuns>(p, x);
+  }
 }
 
 // The K tiles of an entry: one per distinct precision, q-tile 2j's first.
@@ -282,6 +293,16 @@ __device__ __forceinline__ void mma_bf16_mask(uint32_t d_tmem, uint64_t a, uint6
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(m[0]), "r"(m[1]), "r"(m[2]), "r"(m[3])
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_f8_mask(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate, const uint32_t (&m)[4]) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(m[0]), "r"(m[1]), "r"(m[2]), "r"(m[3])
       : "memory");
 }
@@ -321,6 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sQ8 = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes; };
   auto sQ4 = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes; };
   auto sQb = [&](int u) { return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes + C::kQ4Bytes; };
+  auto sQf = [&](int u) {
+    return base + C::kOffQ + u * C::kQUnitBytes + C::kQ8Bytes + C::kQ4Bytes + C::kQbBytes;
+  };
   auto sK = [&](int u, int s) { return base + C::kOffK + (u * NSK + s) * C::kKBytes; };
   auto sV = [&](int u, int s) { return base + C::kOffV + (u * NSV + s) * C::kVBytes; };
   const uint32_t bars = base + C::kOffBar;
@@ -382,22 +406,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const int u = warp >> 1;
       const Unit x = u ? un1 : un0;
-      const uint32_t qbytes = x.valid ? C::kQ8Bytes + (int4 ? C::kQ4Bytes : 0) + C::kQbBytes : 0u;
+      const uint32_t qbytes =
+          x.valid ? C::kQ8Bytes + (int4 ? C::kQ4Bytes : 0) + C::kQbBytes + C::kQfBytes : 0u;
       mbar_arrive_expect_tx(bar_q, qbytes);
       if (x.valid) {
         if (!C::kHyb) tma_load_2d(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
         if (int4) tma_load_2d(sQ4(u), &m.q4x, bar_q, 0, x.row0 * kTile);
+        if (C::kHasF8) tma_load_2d(sQf(u), &m.qf8, bar_q, 0, x.row0 * kTile);
         if (C::kHasBf16) {
           for (int sl = 0; sl < C::kSlabs; ++sl)
             tma_load_3d(sQb(u) + sl * 128 * 128, &m.qb, bar_q, sl * 64, x.h,
                         x.seq0 + x.qt0 * kTile);
         }
       }
-      auto c = unit_stream(p, x, std::bool_constant<C::kHyb>{});
+      auto c = unit_stream<C>(p, x);
       int kt, p0, p1;
       int nk = 0, nv = 0;  // fills issued so far into this unit's K and V rings
       while (c.next(kt, p0, p1)) {
-        if ((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) {
+        if (((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) ||
+            (!C::kHasF8 && (p0 == TRA_PREC_FP8 || p1 == TRA_PREC_FP8))) {
           *err = TRA_DEV_BAD_LIST;
           break;
         }
@@ -417,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                           x.seq0 + kt * kTile);
           } else {
             mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D);
-            tma_load_2d(dst, prec == TRA_PREC_INT8 ? &m.k8 : &m.k4x, bar_kfull(u, s), 0, krow);
+            tma_load_2d(dst, prec == TRA_PREC_INT8 ? &m.k8 : prec == TRA_PREC_FP8 ? &m.kf8 : &m.k4x,
+                        bar_kfull(u, s), 0, krow);
           }
           ++nk;
         }
@@ -449,6 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mu = warp >> 1;  // the unit this thread issues for
       constexpr uint32_t kIdI8 = instr_desc(2, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdQK16 = instr_desc(1, 1, 0, 0, 64, 128);
+      constexpr uint32_t kIdF8 = instr_desc(1, 0, 0, 0, 64, 128);  // f32 <- E4M3 x E4M3
       constexpr uint32_t kIdPV = instr_desc(1, 1, 0, 1, D, 128);
       const uint32_t tU = tmem + mu * 256;
       bool ok = mbar_wait(bar_q, 0, err);
@@ -483,10 +512,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int nk = 0;  // this unit's K ring fills consumed so far
         int i = 0;   // entries of this unit issued so far
         bool hyb_prev = false;  // entry i - 1 reads the mixed operands
-        auto c = unit_stream(p, mu ? un1 : un0, std::bool_constant<C::kHyb>{});
+        auto c = unit_stream<C>(p, mu ? un1 : un0);
         int kt, p0, p1;
         while (c.next(kt, p0, p1)) {
-          if ((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) {
+          if (((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) ||
+              (!C::kHasF8 && (p0 == TRA_PREC_FP8 || p1 == TRA_PREC_FP8))) {
             *err = TRA_DEV_BAD_LIST;
             ok = false;
             break;
@@ -513,6 +543,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t a = smem_desc(sQb(mu) + sl * 128 * 128 + off, 16, 1024, kSwz128);
                 const uint64_t bd = smem_desc(kb + sl * 64 * 128 + off, 16, 1024, kSwz128);
                 mma_bf16_mask(tSb, a, bd, kIdQK16, kk > 0 ? 1u : 0u, msk);
+              }
+            } else if (C::kHasF8 && prec == TRA_PREC_FP8) {
+              // E4M3 x E4M3 -> fp32; operands laid out like the int8 codes (32 bytes of K
+              // per MMA)
+#pragma unroll
+              for (int kk = 0; kk < D / 32; ++kk) {
+                const uint64_t a = smem_desc(sQf(mu) + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
+                const uint64_t bd = smem_desc(kb + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
+                mma_f8_mask(tSb, a, bd, kIdF8, kk > 0 ? 1u : 0u, msk);
               }
             } else {
               const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(mu) : sQ4(mu);
@@ -554,12 +593,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // INT4 operands are 16 x code, so INT4 accumulators are 256 x the code product:
     // the power of two goes into the row's INT4 scale (exact)
     const float sq4 = (half_valid && int4) ? __ldg(p.sq4 + qtile) * (1.0f / 256.0f) : 0.0f;
+    const float sqf = (half_valid && C::kHasF8) ? __ldg(p.sqf + qtile) : 0.0f;
     const uint32_t lane_addr = ((uint32_t)(q4 * 32) << 16) + (uint32_t)(u * 256);
     const uint32_t tU = tmem + lane_addr, tO = tU + 128;  // S/P buffer b at tU + 64 * b
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     int i = 0;
-    auto c = unit_stream(p, x, std::bool_constant<C::kHyb>{});
+    auto c = unit_stream<C>(p, x);
     // the K-tile scale of this row's precision of an entry (1 for BF16), loaded one
     // entry ahead
     auto kscale = [&](int kt_, int pr) -> float {
@@ -567,6 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (pr == TRA_PREC_INT8) return __ldg(p.sk8 + t_);
       if (pr == TRA_PREC_INT4 && int4) return __ldg(p.sk4 + t_);
       if (C::kHyb && pr == kPrecHyb) return __ldg(p.sk4 + t_);
+      if (C::kHasF8 && pr == TRA_PREC_FP8) return __ldg(p.skf + t_);
       return 1.0f;
     };
     // hybrid entries: the tile's V INT4 scale and its 64-bit selection mask
@@ -596,7 +637,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sb = i & 1;
       const uint32_t tS = tU + sb * 64;
       if (!mbar_wait(bar_sfull(u, sb), (i >> 1) & 1, err)) { ok = false; break; }
-      if ((pa == TRA_PREC_INT4 || pb == TRA_PREC_INT4) && !int4) {
+      if (((pa == TRA_PREC_INT4 || pb == TRA_PREC_INT4) && !int4) ||
+          (!C::kHasF8 && (pa == TRA_PREC_FP8 || pb == TRA_PREC_FP8))) {
         *err = TRA_DEV_BAD_LIST;
         ok = false;
         break;
@@ -622,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tS + 32, hi);
         }
         tmem_wait_ld();
-        if (!C::kHyb && p.n_dump > 0 && row_valid && prec != TRA_PREC_BF16) {
+        if (!C::kHyb && p.n_dump > 0 && row_valid && (prec == TRA_PREC_INT8 || prec == TRA_PREC_INT4)) {
           for (int di = 0; di < p.n_dump; ++di) {
             const int* dc = p.dump_coords + di * 4;
             if (__ldg(dc) == x.b && __ldg(dc + 1) == x.h && __ldg(dc + 2) == qt &&
@@ -635,7 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // log2-domain score = raw * f
         const float f = p.scale_log2 * skt *
-                        (prec == TRA_PREC_INT8 ? sq8 : (prec == TRA_PREC_INT4 ? sq4 : 1.0f));
+                        (prec == TRA_PREC_INT8 ? sq8
+                         : prec == TRA_PREC_INT4 ? sq4
+                         : (C::kHasF8 && prec == TRA_PREC_FP8) ? sqf : 1.0f);
         // valid keys of this tile for this row, columns [clo, nvalid): causal and
         // sequence end; only the diagonal tile and a sequence's last tile have fewer
         // than 64.  Hybrid: a kPrecHyb entry keeps the keys at least `window`
@@ -803,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (C::kHyb && prec == kPrecHyb) {
           if (full) hyb_row(T_{}); else hyb_row(F_{});
           p_stored = true;
-        } else if (prec == TRA_PREC_BF16) {
+        } else if (prec == TRA_PREC_BF16 || (C::kHasF8 && prec == TRA_PREC_FP8)) {
           if (full) softmax_row(F_{}, T_{}); else softmax_row(F_{}, F_{});
         } else {
           if (full) softmax_row(T_{}, T_{}); else softmax_row(T_{}, F_{});
@@ -894,6 +938,7 @@ cudaError_t launch_d(const PrefillParams& p, const PrefillMaps& m, cudaStream_t 
   if (p.mode == TRA_POLICY_BITMASK) return launch_one<D, TRA_POLICY_BITMASK>(p, m, s);
   if (p.mode == TRA_POLICY_MIXED) return launch_one<D, TRA_POLICY_MIXED>(p, m, s);
   if (p.mode == kPrefillModeHybrid) return launch_one<D, kPrefillModeHybrid>(p, m, s);
+  if (p.mode == kPrefillModeBoundaryF8) return launch_one<D, kPrefillModeBoundaryF8>(p, m, s);
   return launch_one<D, TRA_POLICY_BOUNDARY>(p, m, s);
 }
 

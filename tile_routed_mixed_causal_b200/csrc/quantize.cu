@@ -1,15 +1,17 @@
-// quantize.cu -- per-(head, 64-token tile) symmetric INT8/INT4 quantisation of
+// quantize.cu -- per-(head, 64-token tile) symmetric INT8/INT4 (and FP8 E4M3) quantisation of
 // Q, K and V (TriAttention abstract: the prefill prepares quantised keys and
 // values; TileMix abstract: INT8 score tiles and INT8 K/V caches).
 //
 // One CTA per (tensor, head, tile): the 64 x d bf16 tile is read once with
 // 16-byte loads into registers, the absolute maximum is reduced with warp
 // shuffles, and the INT8 codes, packed INT4 codes, INT4 codes expanded to the
-// int8 operand form (16 x code) and both scales are written tile-major.
-// HBM-bound: 2*64*d bytes in, per requested format 64*d (INT8, expanded INT4) or
-// 64*d/2 (packed INT4) bytes + 4 (scale) out.
+// int8 operand form (16 x code), FP8 E4M3 codes and their scales are written
+// tile-major.  HBM-bound: 2*64*d bytes in, per requested format 64*d (INT8,
+// expanded INT4, FP8) or 64*d/2 (packed INT4) bytes + 4 (scale) out.
 // Arithmetic: s = fl32(amax / qmax) and code = rne(fl32(x / s)) with IEEE
-// division (__fdiv_rn) and round-half-even conversion (__float2int_rn).
+// division (__fdiv_rn) and round-half-even conversion (__float2int_rn); FP8:
+// sf = fl32(amax / 448) and the hardware's round-to-nearest-even, saturating
+// conversion of fl32(x / sf) to E4M3.
 #include "tra_device.cuh"
 #include "tra_launch.h"
 
@@ -17,6 +19,14 @@ namespace tra {
 namespace {
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+
+// Two fp32 values to FP8 E4M3 codes (round to nearest even, saturating at +-448):
+// byte 0 = lo, byte 1 = hi.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  unsigned short r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 template <int D>
@@ -75,10 +85,12 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p) {
 
   const float s8 = __fdiv_rn(amax, 127.0f);
   const float s4 = __fdiv_rn(amax, 7.0f);
+  const float sf = __fdiv_rn(amax, 448.0f);  // FP8 E4M3: largest finite magnitude 448
   const long long tile_base = (long long)h * p.ntiles + gt;
   if (threadIdx.x == 0) {
     if (t.s8) t.s8[tile_base] = s8;
     if (t.s4) t.s4[tile_base] = s4;
+    if (t.sf) t.sf[tile_base] = sf;
   }
 #pragma unroll
   for (int i = 0; i < kPasses; ++i) {
@@ -108,6 +120,15 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p) {
       for (int j = 0; j < 8; ++j)
         o[j >> 2] |= (uint32_t)((quant_code(x[j], s4, 7) * 16) & 0xFF) << ((j & 3) * 8);
       *reinterpret_cast<uint2*>(t.x4x + (tile_base * kTile + r) * D + c * 8) = make_uint2(o[0], o[1]);
+    }
+    if (t.xf) {  // E4M3 of fl32(x / sf); a zero scale (all-zero tile) gives codes 0
+      uint32_t o[2] = {0, 0};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t w2 = sf == 0.0f ? 0u : e4m3x2(__fdiv_rn(x[2 * j], sf), __fdiv_rn(x[2 * j + 1], sf));
+        o[j >> 1] |= w2 << ((j & 1) * 16);
+      }
+      *reinterpret_cast<uint2*>(t.xf + (tile_base * kTile + r) * D + c * 8) = make_uint2(o[0], o[1]);
     }
     if (t.x4) {
       uint32_t o = 0;  // byte jj: channels 8c + 2jj (low nibble) and 8c + 2jj + 1

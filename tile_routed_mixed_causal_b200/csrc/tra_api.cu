@@ -84,6 +84,14 @@ tra_status check_policy(const tra_shape* s, const tra_policy* p, int64_t nt_max)
       if (p->b2[h] < p->b1[h]) return fail(TRA_ERR_INVALID, "b2[%d] = %d < b1 = %d", h, p->b2[h], p->b1[h]);
     }
   }
+  if (p->b8) {
+    if (p->mode != TRA_POLICY_BOUNDARY)
+      return fail(TRA_ERR_UNSUPPORTED, "the FP8 band (b8) is supported under boundary policies only");
+    for (int h = 0; h < s->Hq; ++h)
+      if (p->b8[h] < p->b1[h] || p->b8[h] > p->b2[h])
+        return fail(TRA_ERR_INVALID, "need b1 <= b8 <= b2 (head %d: %d, %d, %d)", h, p->b1[h],
+                    p->b8[h], p->b2[h]);
+  }
   if (uses_bitmask(p)) {
     if (p->G < 1) return fail(TRA_ERR_INVALID, "G must be >= 1 (got %d)", p->G);
     if (p->W < 1) return fail(TRA_ERR_INVALID, "W must be >= 1");
@@ -97,7 +105,14 @@ tra_status check_policy(const tra_shape* s, const tra_policy* p, int64_t nt_max)
 bool policy_has_int4(const tra_shape* s, const tra_policy* p) {
   if (!uses_boundaries(p)) return false;
   for (int h = 0; h < s->Hq; ++h)
-    if (p->b2[h] > p->b1[h]) return true;
+    if (p->b2[h] > (p->b8 ? p->b8[h] : p->b1[h])) return true;
+  return false;
+}
+
+bool policy_has_fp8(const tra_shape* s, const tra_policy* p) {
+  if (p->mode != TRA_POLICY_BOUNDARY || !p->b8) return false;
+  for (int h = 0; h < s->Hq; ++h)
+    if (p->b8[h] > p->b1[h]) return true;
   return false;
 }
 
@@ -176,7 +191,7 @@ size_t tra_qtiles_bytes(const tra_shape* shape, uint32_t formats) {
   size_t total = 0;
   // codes of each format; scales once per (tensor, precision): Q4X / K4X share the
   // INT4 scales of Q4 / K4
-  const struct { uint32_t bit, scale_bits; int H; size_t per_row; } f[8] = {
+  const struct { uint32_t bit, scale_bits; int H; size_t per_row; } f[10] = {
       {TRA_FMT_Q8, TRA_FMT_Q8, shape->Hq, d},
       {TRA_FMT_Q4, TRA_FMT_Q4 | TRA_FMT_Q4X, shape->Hq, d / 2},
       {TRA_FMT_K8, TRA_FMT_K8, shape->Hkv, d},
@@ -184,7 +199,9 @@ size_t tra_qtiles_bytes(const tra_shape* shape, uint32_t formats) {
       {TRA_FMT_V8, TRA_FMT_V8, shape->Hkv, d},
       {TRA_FMT_V4, TRA_FMT_V4, shape->Hkv, d / 2},
       {TRA_FMT_Q4X, 0, shape->Hq, d},
-      {TRA_FMT_K4X, 0, shape->Hkv, d}};
+      {TRA_FMT_K4X, 0, shape->Hkv, d},
+      {TRA_FMT_Q8F, TRA_FMT_Q8F, shape->Hq, d},
+      {TRA_FMT_K8F, TRA_FMT_K8F, shape->Hkv, d}};
   for (const auto& x : f) {
     if (formats & x.bit) total += round256((size_t)x.H * nt * TRA_TILE * x.per_row);
     if (formats & x.scale_bits) total += round256((size_t)x.H * nt * 4);
@@ -199,7 +216,7 @@ tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const u
   if (st != TRA_OK) return st;
   if (!out) return fail(TRA_ERR_INVALID, "out is NULL");
   const uint32_t f = out->formats;
-  if (f & ~0xFFu) return fail(TRA_ERR_INVALID, "unknown format bits 0x%x", f);
+  if (f & ~0x3FFu) return fail(TRA_ERR_INVALID, "unknown format bits 0x%x", f);
   tra::QuantParams p{};
   const uint16_t* src[3] = {q, k, v};
   const int H[3] = {shape->Hq, shape->Hkv, shape->Hkv};
@@ -207,6 +224,9 @@ tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const u
   uint8_t* o4[3] = {out->q4, out->k4, out->v4};
   int8_t* o4x[3] = {out->q4x, out->k4x, nullptr};
   const uint32_t fx[3] = {TRA_FMT_Q4X, TRA_FMT_K4X, 0u};
+  uint8_t* of[3] = {out->q8f, out->k8f, nullptr};
+  float* sfp[3] = {out->sqf, out->skf, nullptr};
+  const uint32_t ff[3] = {TRA_FMT_Q8F, TRA_FMT_K8F, 0u};
   float* s8[3] = {out->sq8, out->sk8, out->sv8};
   float* s4[3] = {out->sq4, out->sk4, out->sv4};
   const char* nm[3] = {"q", "k", "v"};
@@ -216,9 +236,10 @@ tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const u
     const bool wantp = f & (TRA_FMT_Q4 << (2 * i));  // packed INT4
     const bool wantx = (f & fx[i]) != 0;              // INT4 as int8 16 x code
     const bool want4 = wantp || wantx;
+    const bool wantf = (f & ff[i]) != 0;             // FP8 E4M3
     tra::QuantTensor& t = p.t[i];
     t = tra::QuantTensor{};
-    if (want8 || want4) {
+    if (want8 || want4 || wantf) {
       if (!src[i]) return fail(TRA_ERR_INVALID, "%s is NULL but its formats are requested", nm[i]);
       if (!aligned16(src[i])) return fail(TRA_ERR_INVALID, "%s not 16-byte aligned", nm[i]);
       if (want8 && (!o8[i] || !s8[i] || !aligned16(o8[i]) || !aligned16(s8[i])))
@@ -229,6 +250,8 @@ tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const u
         return fail(TRA_ERR_INVALID, "%s4 codes missing or misaligned", nm[i]);
       if (wantx && (!o4x[i] || !aligned16(o4x[i])))
         return fail(TRA_ERR_INVALID, "%s4x codes missing or misaligned", nm[i]);
+      if (wantf && (!of[i] || !sfp[i] || !aligned16(of[i]) || !aligned16(sfp[i])))
+        return fail(TRA_ERR_INVALID, "%s8f codes/scales missing or misaligned", nm[i]);
       t.x = src[i];
       t.H = H[i];
       t.x8 = want8 ? o8[i] : nullptr;
@@ -238,6 +261,8 @@ tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const u
       t.perm4 = i == 2;  // V4 is read only by the decode, in its MMA fragment order
       t.bias8 = i == 2;  // so is V8, kept offset-binary for its f16 conversion
       t.s4 = want4 ? s4[i] : nullptr;
+      t.xf = wantf ? of[i] : nullptr;
+      t.sf = wantf ? sfp[i] : nullptr;
     }
     p.cta_begin[i + 1] = p.cta_begin[i] + (t.x ? (long long)t.H * nt : 0);
   }
@@ -326,6 +351,7 @@ tra_status build_tile_lists(const tra_shape* shape, const tra_policy* policy, in
     for (int h = 0; h < shape->Hq; ++h) {
       p.b1[h] = policy->b1[h];
       p.b2[h] = policy->b2[h];
+      p.b8[h] = policy->b8 ? policy->b8[h] : policy->b1[h];
     }
   cudaError_t e = tra::launch_lists(p, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lists launch");
@@ -359,6 +385,13 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
                   "the policy has INT4 tiles: Q4X and K4X tiles (INT4 as int8 operands) are required");
     if (!aligned16(tiles->q4x) || !aligned16(tiles->k4x)) return fail(TRA_ERR_INVALID, "Q4X/K4X misaligned");
   }
+  const bool hasf = policy_has_fp8(shape, policy);
+  if (hasf) {
+    const uint32_t needf = TRA_FMT_Q8F | TRA_FMT_K8F;
+    if ((tiles->formats & needf) != needf || !tiles->q8f || !tiles->k8f || !tiles->sqf || !tiles->skf)
+      return fail(TRA_ERR_INVALID, "the policy has an FP8 band: Q8F and K8F tiles are required");
+    if (!aligned16(tiles->q8f) || !aligned16(tiles->k8f)) return fail(TRA_ERR_INVALID, "Q8F/K8F misaligned");
+  }
   if (nt_max >= (1ll << 24)) return fail(TRA_ERR_UNSUPPORTED, "a sequence has more than 2^24 tiles");
   if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
     return fail(TRA_ERR_INVALID, "softmax_scale must be positive and finite");
@@ -372,7 +405,7 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
   p.Hkv = shape->Hkv;
   p.d = shape->d;
   p.ntiles = (int)nt;
-  p.mode = policy->mode;
+  p.mode = hasf ? tra::kPrefillModeBoundaryF8 : policy->mode;
   p.has_int4 = policy_has_int4(shape, policy) ? 1 : 0;
   p.jmax = (int)((nt_max + 1) / 2);
   p.row_ptr = row_ptr;
@@ -381,6 +414,8 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
   p.sq4 = tiles->sq4;
   p.sk8 = tiles->sk8;
   p.sk4 = tiles->sk4;
+  p.sqf = hasf ? tiles->sqf : nullptr;
+  p.skf = hasf ? tiles->skf : nullptr;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.out = out;
   p.lse = lse;
@@ -397,7 +432,9 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
                          map_i8(&m.k4x, tiles->k4x, d, krows, 64))) &&
               map_bf16(&m.qb, q, d, shape->Hq, ntok, 128) &&
               map_bf16(&m.kb, k, d, shape->Hkv, ntok, 64) &&
-              map_bf16(&m.vb, v, d, shape->Hkv, ntok, 64);
+              map_bf16(&m.vb, v, d, shape->Hkv, ntok, 64) &&
+              (!hasf || (map_i8(&m.qf8, tiles->q8f, d, qrows, 128) &&
+                         map_i8(&m.kf8, tiles->k8f, d, krows, 64)));
   if (!good) return fail(TRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
   cudaError_t e = tra::launch_prefill(p, m, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");

@@ -21,6 +21,8 @@ struct QuantTensor {
   float* s4;
   int perm4;           // x4 in the decode's V fragment order (V), else row-major
   int bias8;           // x8 codes stored offset-binary, code + 128 (V), else two's complement
+  uint8_t* xf;         // nullable: FP8 E4M3 codes, row-major
+  float* sf;           // their scales
 };
 
 struct QuantParams {
@@ -43,6 +45,7 @@ struct ListParams {
   long long rows;
   int32_t b1[TRA_MAX_HEADS];
   int32_t b2[TRA_MAX_HEADS];
+  int32_t b8[TRA_MAX_HEADS];  // FP8 band [b1, b8) of a boundary policy (b8 = b1: none)
 };
 
 cudaError_t launch_lists(const ListParams& p, cudaStream_t s);
@@ -73,16 +76,22 @@ struct PrefillParams {
   const float* sv4;
   const uint64_t* sel_mask;
   int window;
+  // FP8 band (mode kPrefillModeBoundaryF8): scales of the E4M3 Q and K tiles
+  const float* sqf;
+  const float* skf;
 };
 
-// prefill mode of the token-level hybrid (beside the TRA_POLICY_* modes)
+// prefill modes beside the TRA_POLICY_* ones: the token-level hybrid, and a boundary
+// policy with an FP8 band
 constexpr int kPrefillModeHybrid = 3;
+constexpr int kPrefillModeBoundaryF8 = 4;
 
 struct PrefillMaps {
   CUtensorMap q8, k8;    // int8 tiles, 2-D (d bytes x rows)
   CUtensorMap q4x, k4x;  // expanded INT4 tiles (int8 16 x code), 2-D like q8 / k8
   CUtensorMap qb, kb, vb;  // bf16, 3-D (d, H, ntok)
   CUtensorMap kmix, vmix;  // hybrid: mixed K / V operands, bf16 3-D like kb / vb
+  CUtensorMap qf8, kf8;    // FP8 E4M3 tiles, 2-D like q8 / k8
 };
 
 cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s);
