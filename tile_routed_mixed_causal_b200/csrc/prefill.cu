@@ -62,7 +62,11 @@ struct Cfg {
   static constexpr bool kHasF8 = MODE == kPrefillModeBoundaryF8;   // FP8 band of a boundary policy
   static constexpr bool kHasBf16 = MODE != TRA_POLICY_BOUNDARY && !kHasF8;  // bf16 Q and K operands
   static constexpr bool kHasInt4 = MODE != TRA_POLICY_BITMASK && !kHyb;  // INT4 operands (int8 form)
-  static constexpr int kRuns = kHasF8 ? 4 : 3;  // precision runs of a traversal row
+  static constexpr int kMode = MODE;
+  // fp32 score tiles (BF16, FP8, hybrid) occur: otherwise their softmax code is not
+  // generated (the integer path stays in every mode: the hybrid's register allocation
+  // spills without it)
+  static constexpr bool kFloatScores = kHasBf16 || kHasF8;
   // work units per CTA: two, or one under a mixed policy, whose operand buffers
   // (int8, INT4 and bf16 Q, bf16-sized K slots) do not fit twice
   static constexpr int kCtaUnits = MODE == TRA_POLICY_MIXED ? 1 : 2;
@@ -103,11 +107,17 @@ struct Cfg {
 };
 
 // The two q-tiles' rows of a unit merged in ascending kt.  A row lists its tiles
-// as NR ascending runs, one per precision (INT4, INT8, BF16 and, with an FP8 band,
-// FP8; sorted as whole entries); next() yields each kt of either row once with the
+// as ascending runs, one per precision, in increasing precision code (entries are
+// sorted as whole words); PR are the precisions a mode's lists can hold, so the
+// merge walks only those runs.  next() yields each kt of either row once with the
 // precision each row gives it (0: the row does not list it).
-template <int NR>
+template <int... PR>
 struct KtMerge {
+  static constexpr int NR = sizeof...(PR);
+  __host__ __device__ static constexpr int prec(int g) {
+    constexpr int a[NR] = {PR...};
+    return a[g];
+  }
   const uint32_t* e;
   int pos[2][NR], end[2][NR];
   uint32_t head[2][NR];  // current kt of each run, kNoKt when exhausted
@@ -122,15 +132,21 @@ struct KtMerge {
     }
     return lo;
   }
-  // rows [rs[r], re[r]) of the entry array; an absent row is empty
-  __device__ __forceinline__ void init(const uint32_t* entries, const int (&rs)[2], const int (&re)[2]) {
+  // rows [rs[r], re[r]) of the entry array; an absent row is empty.  len[r][g]: the
+  // length of run g when the policy fixes it (boundary rows), or -1 to find the run's
+  // end by binary search; a length is clamped to the row.
+  __device__ __forceinline__ void init(const uint32_t* entries, const int (&rs)[2], const int (&re)[2],
+                                       const int (&len)[2][NR]) {
     e = entries;
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       int lo = rs[r];
 #pragma unroll
-      for (int g = 0; g < NR; ++g) {  // run g holds precision g + 1
-        const int hi = g + 1 < NR ? lower_bound(e, lo, re[r], (uint32_t)(g + 2) << 28) : re[r];
+      for (int g = 0; g < NR; ++g) {  // run g holds precision prec(g)
+        int hi = re[r];
+        if (g + 1 < NR)
+          hi = len[r][g] >= 0 ? min(lo + len[r][g], re[r])
+                              : lower_bound(e, lo, re[r], (uint32_t)prec(g + 1) << 28);
         pos[r][g] = lo;
         end[r][g] = hi;
         lo = hi;
@@ -153,7 +169,7 @@ struct KtMerge {
 #pragma unroll
       for (int g = 0; g < NR; ++g)
         if (head[r][g] == k) {
-          pr[r] = g + 1;  // TRA_PREC_INT4 = 1, INT8 = 2, BF16 = 3, FP8 = 4
+          pr[r] = prec(g);
           ++pos[r][g];
           load(r, g);
         }
@@ -195,16 +211,44 @@ __device__ __forceinline__ Unit make_unit(const PrefillParams& p, long long id) 
   return x;
 }
 
-template <int NR>
-__device__ __forceinline__ KtMerge<NR> unit_merge(const PrefillParams& p, const Unit& x) {
-  KtMerge<NR> c;
+// the precisions each prefill mode's traversal rows can hold
+template <int MODE> struct MergeOf { using T = KtMerge<TRA_PREC_INT4, TRA_PREC_INT8>; };
+template <> struct MergeOf<TRA_POLICY_BITMASK> { using T = KtMerge<TRA_PREC_INT8, TRA_PREC_BF16>; };
+template <> struct MergeOf<TRA_POLICY_MIXED> {
+  using T = KtMerge<TRA_PREC_INT4, TRA_PREC_INT8, TRA_PREC_BF16>;
+};
+template <> struct MergeOf<kPrefillModeBoundaryF8> {
+  using T = KtMerge<TRA_PREC_INT4, TRA_PREC_INT8, TRA_PREC_FP8>;
+};
+
+template <class M, bool kClosedForm>
+__device__ __forceinline__ M unit_merge(const PrefillParams& p, const Unit& x) {
+  M c;
   int rs[2] = {0, 0}, re[2] = {0, 0};
   if (x.valid) {
     rs[0] = __ldg(p.row_ptr + x.row0);
     re[0] = rs[1] = __ldg(p.row_ptr + x.row0 + 1);
     re[1] = x.has_second ? __ldg(p.row_ptr + x.row0 + 2) : rs[1];
   }
-  c.init(p.entries, rs, re);
+  int len[2][M::NR];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int g = 0; g < M::NR; ++g) len[r][g] = -1;
+  if constexpr (kClosedForm) {
+    // boundary rows in closed form: the row keeps n = min(qt + 1, b2) tiles, the
+    // nearest min(qt + 1, b1) INT8, then min(qt + 1, b8) - that FP8, the rest INT4,
+    // written as the INT4 run, the INT8 run, the FP8 run
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int qt = x.qt0 + r;
+      const int n8 = min(qt + 1, p.b1[x.h]);
+      const int nf = min(qt + 1, p.b8[x.h]) - n8;
+      len[r][0] = max(0, re[r] - rs[r] - n8 - nf);  // INT4
+      if (M::NR > 2) len[r][1] = n8;                 // INT8 (before FP8)
+    }
+  }
+  c.init(p.entries, rs, re, len);
   return c;
 }
 
@@ -260,7 +304,8 @@ __device__ __forceinline__ auto unit_stream(const PrefillParams& p, const Unit& 
     c.init(x, p.window);
     return c;
   } else {
-    return unit_merge<C::kRuns>(p, x);
+    return unit_merge<typename MergeOf<C::kMode>::T,
+                      C::kMode == TRA_POLICY_BOUNDARY || C::kMode == kPrefillModeBoundaryF8>(p, x);
   }
 }
 
@@ -436,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (use > 0 && !mbar_wait(bar_kfree(u, s), (use - 1) & 1, err)) { ok = false; break; }
           const uint32_t dst = sK(u, s);
           const int krow = (x.kvh * p.ntiles + x.toff + kt) * kTile;
-          if (prec == TRA_PREC_BF16 || prec == kPrecHyb) {
+          if (C::kHasBf16 && (prec == TRA_PREC_BF16 || prec == kPrecHyb)) {
             const CUtensorMap* km = prec == kPrecHyb ? &m.kmix : &m.kb;
             mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D * 2);
             for (int sl = 0; sl < C::kSlabs; ++sl)
@@ -536,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t msk[4] = {f == 1 ? keep : 0u, f == 1 ? keep : 0u, f == 0 ? keep : 0u,
                                      f == 0 ? keep : 0u};
             const uint32_t kb = sK(mu, s);
-            if (prec == TRA_PREC_BF16 || prec == kPrecHyb) {
+            if (C::kHasBf16 && (prec == TRA_PREC_BF16 || prec == kPrecHyb)) {
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const int sl = kk >> 2, off = (kk & 3) * 32;
@@ -847,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (C::kHyb && prec == kPrecHyb) {
           if (full) hyb_row(T_{}); else hyb_row(F_{});
           p_stored = true;
-        } else if (prec == TRA_PREC_BF16 || (C::kHasF8 && prec == TRA_PREC_FP8)) {
+        } else if (C::kFloatScores && (prec == TRA_PREC_BF16 || (C::kHasF8 && prec == TRA_PREC_FP8))) {
           if (full) softmax_row(F_{}, T_{}); else softmax_row(F_{}, F_{});
         } else {
           if (full) softmax_row(T_{}, T_{}); else softmax_row(T_{}, F_{});
@@ -916,6 +961,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
   if (threadIdx.x == 0 && *err) atomicOr(p.status, *err);
 }
+
+// the launch parameters stay within the classic 4 KB kernel-parameter space
+static_assert(sizeof(PrefillParams) + sizeof(PrefillMaps) <= 4096, "prefill launch parameters");
 
 template <int D, int MODE>
 cudaError_t launch_one(const PrefillParams& p, const PrefillMaps& m, cudaStream_t s) {

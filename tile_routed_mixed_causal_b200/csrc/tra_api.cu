@@ -416,6 +416,11 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
   p.sk4 = tiles->sk4;
   p.sqf = hasf ? tiles->sqf : nullptr;
   p.skf = hasf ? tiles->skf : nullptr;
+  if (policy->mode == TRA_POLICY_BOUNDARY)
+    for (int h = 0; h < shape->Hq; ++h) {
+      p.b1[h] = policy->b1[h];
+      p.b8[h] = policy->b8 ? policy->b8[h] : policy->b1[h];
+    }
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.out = out;
   p.lse = lse;

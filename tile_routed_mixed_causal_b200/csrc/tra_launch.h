@@ -79,6 +79,10 @@ struct PrefillParams {
   // FP8 band (mode kPrefillModeBoundaryF8): scales of the E4M3 Q and K tiles
   const float* sqf;
   const float* skf;
+  // boundary policies: b1 and b8 (b8 = b1 without an FP8 band) per query head, which fix
+  // the lengths of a traversal row's precision runs
+  int32_t b1[TRA_MAX_HEADS];
+  int32_t b8[TRA_MAX_HEADS];
 };
 
 // prefill modes beside the TRA_POLICY_* ones: the token-level hybrid, and a boundary
