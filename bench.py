@@ -400,6 +400,10 @@ def allocate_bench(device, stream, budget_frac=0.5, units=4096, seed=7):
     w8 = (meas["int8_all"] - meas["int8_half"]) / (cnt["int8_all"][0] - cnt["int8_half"][0])
     t0 = meas["int8_all"] - cnt["int8_all"][0] * w8
     w4 = (meas["int4_all"] - t0 - cnt["int4_all"][0] * w8) / cnt["int4_all"][1]
+    # a per-tile time fitted from noisy (e.g. profiled, serialised) launches can come out
+    # at or below zero: the costs the allocator takes must stay positive
+    w8 = max(w8, 1e-9)
+    w4 = max(w4, 0.0)
 
     # candidates: b1 in powers of two, b2 in b1 x powers of two, up to nt
     cands = [(b1, b2) for b1 in [1 << i for i in range(8) if (1 << i) <= nt]

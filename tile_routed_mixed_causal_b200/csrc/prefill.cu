@@ -63,9 +63,7 @@ struct Cfg {
   static constexpr bool kHasBf16 = MODE != TRA_POLICY_BOUNDARY && !kHasF8;  // bf16 Q and K operands
   static constexpr bool kHasInt4 = MODE != TRA_POLICY_BITMASK && !kHyb;  // INT4 operands (int8 form)
   static constexpr int kMode = MODE;
-  // fp32 score tiles (BF16, FP8, hybrid) occur: otherwise their softmax code is not
-  // generated (the integer path stays in every mode: the hybrid's register allocation
-  // spills without it)
+  // fp32 score tiles (BF16, FP8, hybrid) occur beside the integer ones
   static constexpr bool kFloatScores = kHasBf16 || kHasF8;
   // work units per CTA: two, or one under a mixed policy, whose operand buffers
   // (int8, INT4 and bf16 Q, bf16-sized K slots) do not fit twice
@@ -743,16 +741,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tiles (every key valid) take a copy with no per-column test; only
         // the diagonal tile and a sequence's last tile take the masked copy.
         // Raw scores as floats: fp32 accumulators as they are, int32 ones
-        // converted (exact: |S| < 2^24).
-        auto softmax_row = [&](auto int_tag, auto full_tag) {
+        // converted (exact: |S| < 2^24).  A mode whose tiles are all integer
+        // (kInt) takes the row max on the raw int32 values; where fp32 and int32
+        // tiles alternate, both share one body (is_int selects the conversion),
+        // which keeps the softmax's hot code in one piece.
+        auto softmax_row = [&](auto int_tag, auto full_tag, bool is_int) {
           constexpr bool kInt = decltype(int_tag)::value;
           constexpr bool kFull = decltype(full_tag)::value;
           float xs[64];
+          if (kInt || is_int) {
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc) {
-            xs[cc] = kInt ? (float)(int)sr[cc] : __uint_as_float(sr[cc]);
-            if (!kFull) xs[cc] = (cc >= clo && cc < nvalid) ? xs[cc] : -INFINITY;
+            for (int cc = 0; cc < 64; ++cc) xs[cc] = (float)(int)sr[cc];
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < 64; ++cc) xs[cc] = __uint_as_float(sr[cc]);
           }
+#pragma unroll
+          for (int cc = 0; cc < 64; ++cc)
+            if (!kFull) xs[cc] = (cc >= clo && cc < nvalid) ? xs[cc] : -INFINITY;
           float mx;
           if (kInt && kFull) {
             // integer row max on the raw accumulators, independent of the conversions
@@ -892,10 +898,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (C::kHyb && prec == kPrecHyb) {
           if (full) hyb_row(T_{}); else hyb_row(F_{});
           p_stored = true;
-        } else if (C::kFloatScores && (prec == TRA_PREC_BF16 || (C::kHasF8 && prec == TRA_PREC_FP8))) {
-          if (full) softmax_row(F_{}, T_{}); else softmax_row(F_{}, F_{});
+        } else if (C::kFloatScores) {
+          const bool is_int = !(prec == TRA_PREC_BF16 || (C::kHasF8 && prec == TRA_PREC_FP8));
+          if (full) softmax_row(F_{}, T_{}, is_int); else softmax_row(F_{}, F_{}, is_int);
         } else {
-          if (full) softmax_row(T_{}, T_{}); else softmax_row(T_{}, F_{});
+          if (full) softmax_row(T_{}, T_{}, true); else softmax_row(T_{}, F_{}, true);
         }
       }
       if (warp_rescale_o && i >= 1) {
