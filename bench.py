@@ -80,8 +80,8 @@ def parse():
 PROFILED_TRAFFIC = {
     # key: (source file, its sha256[:16] when captured, dram__bytes_read.sum + dram__bytes_write.sum
     # of one launch in the ncu capture); reported only while the source is unchanged
-    "prefill_bitmask": ("prefill.cu", "f06f0ba6c946b8cd", 3_376_191_016),
-    "prefill_hybrid": ("prefill.cu", "f06f0ba6c946b8cd", 2_313_416_048),
+    "prefill_bitmask": ("prefill.cu", "37f5befbc60ef1f8", 2_870_104_576),
+    "prefill_hybrid": ("prefill.cu", "37f5befbc60ef1f8", 2_311_292_672),
     "decode": ("decode.cu", "1fedbc1ad6951867", 666_226_944),
 }
 
