@@ -320,22 +320,25 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // tcgen05.mma with an output-lane mask: lanes whose bit is set in m0..m3 (lane
-// 32 w + i <-> bit i of m_w) keep their contents.
+// 32 w + i <-> bit i of m_w) keep their contents.  Issued by one elected lane of a
+// converged warp (all lanes pass the same operands).
 __device__ __forceinline__ void mma_i8_mask(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                             uint32_t accumulate, const uint32_t (&m)[4]) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(m[0]), "r"(m[1]), "r"(m[2]), "r"(m[3])
       : "memory");
 }
 __device__ __forceinline__ void mma_bf16_mask(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                               uint32_t accumulate, const uint32_t (&m)[4]) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(m[0]), "r"(m[1]), "r"(m[2]), "r"(m[3])
       : "memory");
 }
@@ -343,20 +346,22 @@ __device__ __forceinline__ void mma_bf16_mask(uint32_t d_tmem, uint64_t a, uint6
 __device__ __forceinline__ void mma_f8_mask(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                             uint32_t accumulate, const uint32_t (&m)[4]) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(m[0]), "r"(m[1]), "r"(m[2]), "r"(m[3])
       : "memory");
 }
 
-// O += P V with the 128 x 16 bf16 A operand (P) read from TMEM.
+// O += P V with the 128 x 16 bf16 A operand (P) read from TMEM (elected lane).
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -443,23 +448,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // a wait left by the whole (converged) warp together: true when every lane saw
+  // the phase complete
+  auto wwait = [&](uint32_t bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, err));
+  };
+
   if (warp == 0 || warp == 2) {
     // ================================================================ TMA producers
-    // one per unit, each walking its own unit's merged stream into its own rings
-    if (lane == 0) {
+    // one warp per unit, each walking its own unit's merged stream into its own
+    // rings.  The whole warp runs it with warp-uniform values; one elected lane
+    // issues each copy and arrive, and a wait is left by all lanes together.
+    {
       const int u = warp >> 1;
       const Unit x = u ? un1 : un0;
       const uint32_t qbytes =
           x.valid ? C::kQ8Bytes + (int4 ? C::kQ4Bytes : 0) + C::kQbBytes + C::kQfBytes : 0u;
-      mbar_arrive_expect_tx(bar_q, qbytes);
+      mbar_arrive_expect_tx_e(bar_q, qbytes);
       if (x.valid) {
-        if (!C::kHyb) tma_load_2d(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
-        if (int4) tma_load_2d(sQ4(u), &m.q4x, bar_q, 0, x.row0 * kTile);
-        if (C::kHasF8) tma_load_2d(sQf(u), &m.qf8, bar_q, 0, x.row0 * kTile);
+        if (!C::kHyb) tma_load_2d_e(sQ8(u), &m.q8, bar_q, 0, x.row0 * kTile);
+        if (int4) tma_load_2d_e(sQ4(u), &m.q4x, bar_q, 0, x.row0 * kTile);
+        if (C::kHasF8) tma_load_2d_e(sQf(u), &m.qf8, bar_q, 0, x.row0 * kTile);
         if (C::kHasBf16) {
           for (int sl = 0; sl < C::kSlabs; ++sl)
-            tma_load_3d(sQb(u) + sl * 128 * 128, &m.qb, bar_q, sl * 64, x.h,
-                        x.seq0 + x.qt0 * kTile);
+            tma_load_3d_e(sQb(u) + sl * 128 * 128, &m.qb, bar_q, sl * 64, x.h,
+                          x.seq0 + x.qt0 * kTile);
         }
       }
       auto c = unit_stream<C>(p, x);
@@ -476,37 +489,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int f = 0; f < nf; ++f) {
           const int prec = entry_fill_prec(p0, p1, f);
           const int s = nk % NSK, use = nk / NSK;  // the unit's K ring slot
-          if (use > 0 && !mbar_wait(bar_kfree(u, s), (use - 1) & 1, err)) { ok = false; break; }
+          if (use > 0 && !wwait(bar_kfree(u, s), (use - 1) & 1)) { ok = false; break; }
           const uint32_t dst = sK(u, s);
           const int krow = (x.kvh * p.ntiles + x.toff + kt) * kTile;
           if (C::kHasBf16 && (prec == TRA_PREC_BF16 || prec == kPrecHyb)) {
             const CUtensorMap* km = prec == kPrecHyb ? &m.kmix : &m.kb;
-            mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D * 2);
+            mbar_arrive_expect_tx_e(bar_kfull(u, s), 64 * D * 2);
             for (int sl = 0; sl < C::kSlabs; ++sl)
-              tma_load_3d(dst + sl * 64 * 128, km, bar_kfull(u, s), sl * 64, x.kvh,
-                          x.seq0 + kt * kTile);
+              tma_load_3d_e(dst + sl * 64 * 128, km, bar_kfull(u, s), sl * 64, x.kvh,
+                            x.seq0 + kt * kTile);
           } else {
-            mbar_arrive_expect_tx(bar_kfull(u, s), 64 * D);
-            tma_load_2d(dst, prec == TRA_PREC_INT8 ? &m.k8 : prec == TRA_PREC_FP8 ? &m.kf8 : &m.k4x,
-                        bar_kfull(u, s), 0, krow);
+            mbar_arrive_expect_tx_e(bar_kfull(u, s), 64 * D);
+            tma_load_2d_e(dst, prec == TRA_PREC_INT8 ? &m.k8 : prec == TRA_PREC_FP8 ? &m.kf8 : &m.k4x,
+                          bar_kfull(u, s), 0, krow);
           }
           ++nk;
         }
         if (!ok) break;
         const int sv = nv % NSV, usev = nv / NSV;  // the unit's V ring slot
-        if (usev > 0 && !mbar_wait(bar_vfree(u, sv), (usev - 1) & 1, err)) break;
+        if (usev > 0 && !wwait(bar_vfree(u, sv), (usev - 1) & 1)) break;
         // V of the entry: the mixed operand for a hybrid entry, else bf16 V
         const CUtensorMap* vm = (p0 == kPrecHyb || p1 == kPrecHyb) ? &m.vmix : &m.vb;
-        mbar_arrive_expect_tx(bar_vfull(u, sv), 64 * D * 2);
+        mbar_arrive_expect_tx_e(bar_vfull(u, sv), 64 * D * 2);
         for (int sl = 0; sl < C::kSlabs; ++sl)
-          tma_load_3d(sV(u, sv) + sl * 64 * 128, vm, bar_vfull(u, sv), sl * 64, x.kvh,
-                      x.seq0 + kt * kTile);
+          tma_load_3d_e(sV(u, sv) + sl * 64 * 128, vm, bar_vfull(u, sv), sl * 64, x.kvh,
+                        x.seq0 + kt * kTile);
         ++nv;
       }
       if (*err) {
-        // an abandoned traversal: every load this thread issued lands before the
-        // CTA can exit. Only this thread arrives on a full barrier, so the last
-        // fill of each slot completes its phase as soon as its bytes are in.
+        // an abandoned traversal: every load this warp issued lands before the CTA
+        // can exit. Only this warp arrives on a full barrier, so the last fill of
+        // each slot completes its phase as soon as its bytes are in.
         mbar_wait_drain(bar_q, 0);
         for (int s = 0; s < NSK && s < nk; ++s)
           mbar_wait_drain(bar_kfull(u, s), (uint32_t)(((nk - 1 - s) / NSK) & 1));
@@ -516,14 +529,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 || warp == 3) {
     // ================================================================ MMA issuers
-    if (lane == 0) {
-      const int mu = warp >> 1;  // the unit this thread issues for
+    // The whole warp runs the issuer with warp-uniform values; one elected lane
+    // issues each MMA and commit.
+    {
+      const int mu = warp >> 1;  // the unit this warp issues for
       constexpr uint32_t kIdI8 = instr_desc(2, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdQK16 = instr_desc(1, 1, 0, 0, 64, 128);
       constexpr uint32_t kIdF8 = instr_desc(1, 0, 0, 0, 64, 128);  // f32 <- E4M3 x E4M3
       constexpr uint32_t kIdPV = instr_desc(1, 1, 0, 1, D, 128);
       const uint32_t tU = tmem + mu * 256;
-      bool ok = mbar_wait(bar_q, 0, err);
+      // Operand descriptors, built once: a K step (or a block of V rows) moves only
+      // the start address, the descriptor's low bits in 16-byte units
+      const uint64_t dQ8 = smem_desc(sQ8(mu), 16, C::kI8Sbo, C::kI8Layout);
+      const uint64_t dQ4 = smem_desc(sQ4(mu), 16, C::kI8Sbo, C::kI8Layout);
+      const uint64_t dQf = smem_desc(sQf(mu), 16, C::kI8Sbo, C::kI8Layout);
+      const uint64_t dQb = smem_desc(sQb(mu), 16, 1024, kSwz128);
+      bool ok = wwait(bar_q, 0);
       tc_fence_after();
       // O += P(idx) V(idx): P from TMEM buffer idx & 1, V (MN-major) from the unit's
       // V ring, which holds one tile per entry of the unit, in order
@@ -531,24 +552,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (hi in the block's first 32 columns, lo in the next 32): both multiply V
       auto issue_pv = [&](int idx, bool hi_lo) -> bool {
         const int pb = idx & 1, slot = idx % NSV;
-        if (!mbar_wait(bar_pfull(mu, pb), (idx >> 1) & 1, err)) return false;
-        if (!mbar_wait(bar_vfull(mu, slot), (idx / NSV) & 1, err)) return false;
+        if (!wwait(bar_pfull(mu, pb), (idx >> 1) & 1)) return false;
+        if (!wwait(bar_vfull(mu, slot), (idx / NSV) & 1)) return false;
         tc_fence_after();
-        const uint32_t vb = sV(mu, slot);
+        const uint64_t dV = smem_desc(sV(mu, slot), 64 * 128, 1024, kSwz128);  // 16 V rows: +2048 B
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc(vb + kk * 2048, 64 * 128, 1024, kSwz128);
-          mma_bf16_ts(tU + 128, tU + pb * 64 + kk * 8, bd, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ts(tU + 128, tU + pb * 64 + kk * 8, dV + kk * 128, kIdPV, (idx > 0 || kk > 0) ? 1u : 0u);
         if (C::kHyb && hi_lo) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = smem_desc(vb + kk * 2048, 64 * 128, 1024, kSwz128);
-            mma_bf16_ts(tU + 128, tU + pb * 64 + 32 + kk * 8, bd, kIdPV, 1u);
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tU + 128, tU + pb * 64 + 32 + kk * 8, dV + kk * 128, kIdPV, 1u);
         }
-        mma_commit(bar_ofull(mu));
-        mma_commit(bar_vfree(mu, slot));
+        mma_commit_e(bar_ofull(mu));
+        mma_commit_e(bar_vfree(mu, slot));
         return true;
       };
       if (ok) {
@@ -571,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int f = 0; f < nf; ++f) {
             const int prec = entry_fill_prec(p0, p1, f);
             const int s = nk % NSK;
-            if (!mbar_wait(bar_kfull(mu, s), (uint32_t)((nk / NSK) & 1), err)) { ok = false; break; }
+            if (!wwait(bar_kfull(mu, s), (uint32_t)((nk / NSK) & 1))) { ok = false; break; }
             tc_fence_after();
             // lanes written: all for a single-precision entry; for two precisions the
             // first MMA writes q-tile 2j's lanes 0-63, the second q-tile 2j+1's 64-127
@@ -580,45 +597,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      f == 0 ? keep : 0u};
             const uint32_t kb = sK(mu, s);
             if (C::kHasBf16 && (prec == TRA_PREC_BF16 || prec == kPrecHyb)) {
+              // 16 elements of K per MMA: 32 bytes within a 128-byte slab, slabs of 128
+              // Q rows (16 KB) and 64 K rows (8 KB)
+              const uint64_t dK = smem_desc(kb, 16, 1024, kSwz128);
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const int sl = kk >> 2, off = (kk & 3) * 32;
-                const uint64_t a = smem_desc(sQb(mu) + sl * 128 * 128 + off, 16, 1024, kSwz128);
-                const uint64_t bd = smem_desc(kb + sl * 64 * 128 + off, 16, 1024, kSwz128);
-                mma_bf16_mask(tSb, a, bd, kIdQK16, kk > 0 ? 1u : 0u, msk);
-              }
+              for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16_mask(tSb, dQb + (kk >> 2) * 1024 + (kk & 3) * 2, dK + (kk >> 2) * 512 + (kk & 3) * 2,
+                              kIdQK16, kk > 0 ? 1u : 0u, msk);
             } else if (C::kHasF8 && prec == TRA_PREC_FP8) {
               // E4M3 x E4M3 -> fp32; operands laid out like the int8 codes (32 bytes of K
               // per MMA)
+              const uint64_t dK = smem_desc(kb, 16, C::kI8Sbo, C::kI8Layout);
 #pragma unroll
-              for (int kk = 0; kk < D / 32; ++kk) {
-                const uint64_t a = smem_desc(sQf(mu) + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
-                const uint64_t bd = smem_desc(kb + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
-                mma_f8_mask(tSb, a, bd, kIdF8, kk > 0 ? 1u : 0u, msk);
-              }
+              for (int kk = 0; kk < D / 32; ++kk)
+                mma_f8_mask(tSb, dQf + kk * 2, dK + kk * 2, kIdF8, kk > 0 ? 1u : 0u, msk);
             } else {
-              const uint32_t qa = prec == TRA_PREC_INT8 ? sQ8(mu) : sQ4(mu);
+              const uint64_t dA = prec == TRA_PREC_INT8 ? dQ8 : dQ4;
+              const uint64_t dK = smem_desc(kb, 16, C::kI8Sbo, C::kI8Layout);
 #pragma unroll
-              for (int kk = 0; kk < D / 32; ++kk) {
-                const uint64_t a = smem_desc(qa + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
-                const uint64_t bd = smem_desc(kb + kk * 32, 16, C::kI8Sbo, C::kI8Layout);
-                mma_i8_mask(tSb, a, bd, kIdI8, kk > 0 ? 1u : 0u, msk);
-              }
+              for (int kk = 0; kk < D / 32; ++kk)
+                mma_i8_mask(tSb, dA + kk * 2, dK + kk * 2, kIdI8, kk > 0 ? 1u : 0u, msk);
             }
-            mma_commit(bar_kfree(mu, s));
+            mma_commit_e(bar_kfree(mu, s));
             ++nk;
           }
           if (!ok) break;
-          mma_commit(bar_sfull(mu, i & 1));
+          mma_commit_e(bar_sfull(mu, i & 1));
           if (i >= 1 && !issue_pv(i - 1, hyb_prev)) { ok = false; break; }
           hyb_prev = p0 == kPrecHyb || p1 == kPrecHyb;
           ++i;
         }
-        if (ok && i >= 1 && issue_pv(i - 1, hyb_prev)) mma_commit(bar_ofinal(mu));
+        if (ok && i >= 1 && issue_pv(i - 1, hyb_prev)) mma_commit_e(bar_ofinal(mu));
       }
-      // every MMA of this thread completes before TMEM is released
-      mma_commit(bar_done);
+      // every MMA of this warp completes before TMEM is released
+      mma_commit_e(bar_done);
       mbar_wait_drain(bar_done, 0);
+      __syncwarp();
     }
   } else if (warp >= 4 && warp < 12) {
     // ================================================================ softmax / epilogue
