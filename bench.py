@@ -80,8 +80,8 @@ def parse():
 PROFILED_TRAFFIC = {
     # key: (source file, its sha256[:16] when captured, dram__bytes_read.sum + dram__bytes_write.sum
     # of one launch in the ncu capture); reported only while the source is unchanged
-    "prefill_bitmask": ("prefill.cu", "37f5befbc60ef1f8", 2_870_104_576),
-    "prefill_hybrid": ("prefill.cu", "37f5befbc60ef1f8", 2_311_292_672),
+    "prefill_bitmask": ("prefill.cu", "aad8d0c1d81ef06e", 2_870_809_600),
+    "prefill_hybrid": ("prefill.cu", "aad8d0c1d81ef06e", 2_318_178_304),
     "decode": ("decode.cu", "1fedbc1ad6951867", 666_226_944),
 }
 
