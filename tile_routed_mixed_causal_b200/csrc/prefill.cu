@@ -30,6 +30,9 @@
 //               online softmax with lazy rescaling of O -> bf16 P into TMEM;
 //               finally O / l.  With two S blocks, QK(i+1) runs while entry i is
 //               in the softmax.
+// The producer and MMA warps run converged, every lane computing the same
+// (warp-uniform) operands; elect.sync picks the one lane that issues each TMA
+// copy, MMA, commit and arrive, and waits are left by the warp as a whole.
 // Every ring belongs to one unit: one filler and one consumer, both taking its
 // slots in order, so no parity wait can alias a phase two uses away.  All waits
 // are bounded (2 s); on expiry a role records TRA_DEV_TIMEOUT and all drain.
