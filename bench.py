@@ -233,9 +233,9 @@ def run_prefill_bench(S, steps, warmup, stream):
 
 def run_prefill_e2e(S, steps, stream):
     """Same path with pinned-host inputs copied in and the output copied out every step.
-    Copies run on their own streams and are double-buffered, so step i's output copy and
-    step i+1's input copy overlap step i's and i+1's kernels; the timed region spans the
-    first input copy to the last output copy."""
+    Copies run on their own streams and are double-buffered: step i+1's input copy overlaps
+    step i's kernels and step i-1's output copy; the timed region spans the first input
+    copy to the last output copy."""
     plan = S["plan"]
     hq = S["q"].cpu().pin_memory()
     hk = S["k"].cpu().pin_memory()
@@ -252,14 +252,15 @@ def run_prefill_e2e(S, steps, stream):
 
     def run(nsteps):
         loaded = [None, None]      # set i: its inputs are in
-        computed = [None, None]    # set i: its kernels are done
-        drained = [ev(), ev()]     # set i: its output copy is done (inputs free again)
+        computed = [None, None]    # set i: its kernels are done (its inputs free again)
+        drained = [ev(), ev()]     # set i: its output copy is done (its output free again)
         for e in drained:
             e.record(s_out)
         for i in range(nsteps):
             b = i % 2
             st = sets[b]
-            s_in.wait_event(drained[b])
+            # the input copy waits only for the set's previous kernels, so it overlaps the
+            # previous output copy (the other direction) as well as the other set's kernels
             if computed[b] is not None:
                 s_in.wait_event(computed[b])
             with torch.cuda.stream(s_in):
@@ -271,6 +272,7 @@ def run_prefill_e2e(S, steps, stream):
             loaded[b] = ev()
             loaded[b].record(s_in)
             stream.wait_event(loaded[b])
+            stream.wait_event(drained[b])  # the set's output buffer has been copied out
             plan.run(st["q"], st["k"], st["v"], st["out"], stream=stream)
             computed[b] = ev()
             computed[b].record(stream)
