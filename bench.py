@@ -81,8 +81,8 @@ def parse():
 PROFILED_TRAFFIC = {
     # key: (source file, its sha256[:16] when captured, dram__bytes_read.sum + dram__bytes_write.sum
     # of one launch in the ncu capture); reported only while the source is unchanged
-    "prefill_bitmask": ("prefill.cu", "c3c58e614db91cca", 2_870_809_600),
-    "prefill_hybrid": ("prefill.cu", "c3c58e614db91cca", 2_318_178_304),
+    "prefill_bitmask": ("prefill.cu", "8de08c900e5c3099", 2_870_786_560),
+    "prefill_hybrid": ("prefill.cu", "8de08c900e5c3099", 2_237_638_144),
     "decode": ("decode.cu", "1fedbc1ad6951867", 666_226_944),
 }
 

@@ -716,14 +716,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 32; ++k) pk[k] = 0u;
       } else {
         tc_fence_after();
+        // S in two halves.  Hybrid prefill: columns 32-63 load while columns 0-31 take
+        // their per-column selection work (every reader of sr[32..63] waits for the
+        // second load first; where both loads are already waited for, that wait is
+        // a no-op).  The routed modes gained nothing from the split and wait once.
         uint32_t sr[64];
         {
           uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
           uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
           tmem_ld32(tS, lo);
+          if (C::kHyb) tmem_wait_ld();
           tmem_ld32(tS + 32, hi);
+          if (!C::kHyb) tmem_wait_ld();
         }
-        tmem_wait_ld();
+        if (!C::kHyb && p.n_dump > 0) tmem_wait_ld();
         if (!C::kHyb && p.n_dump > 0 && row_valid && (prec == TRA_PREC_INT8 || prec == TRA_PREC_INT4)) {
           for (int di = 0; di < p.n_dump; ++di) {
             const int* dc = p.dump_coords + di * 4;
@@ -766,40 +772,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           constexpr bool kInt = decltype(int_tag)::value;
           constexpr bool kFull = decltype(full_tag)::value;
           float xs[64];
-          if (kInt || is_int) {
+          // integer row max on the raw accumulators (kInt), else on the converted scores
+          int mi4[4];
+          float mx4[4];
 #pragma unroll
-            for (int cc = 0; cc < 64; ++cc) xs[cc] = (float)(int)sr[cc];
-          } else {
+          for (int hf = 0; hf < 2; ++hf) {
+            if (hf == 1) tmem_wait_ld();  // columns 32-63 are in
+            const int c0 = 32 * hf;
+            if (kInt || is_int) {
 #pragma unroll
-            for (int cc = 0; cc < 64; ++cc) xs[cc] = __uint_as_float(sr[cc]);
-          }
+              for (int cc = c0; cc < c0 + 32; ++cc) xs[cc] = (float)(int)sr[cc];
+            } else {
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc)
-            if (!kFull) xs[cc] = (cc >= clo && cc < nvalid) ? xs[cc] : -INFINITY;
-          float mx;
-          if (kInt && kFull) {
-            // integer row max on the raw accumulators, independent of the conversions
-            int mi4[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) mi4[k] = max((int)sr[k], (int)sr[k + 4]);
-#pragma unroll
-            for (int cc = 8; cc < 64; cc += 8) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mi4[k] = __vimax3_s32(mi4[k], (int)sr[cc + k], (int)sr[cc + k + 4]);
+              for (int cc = c0; cc < c0 + 32; ++cc) xs[cc] = __uint_as_float(sr[cc]);
             }
-            mx = (float)max(max(mi4[0], mi4[1]), max(mi4[2], mi4[3]));
-          } else {
-            float mx4[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(xs[k], xs[k + 4]);
+            for (int cc = c0; cc < c0 + 32; ++cc)
+              if (!kFull) xs[cc] = (cc >= clo && cc < nvalid) ? xs[cc] : -INFINITY;
+            if (kInt && kFull) {
 #pragma unroll
-            for (int cc = 8; cc < 64; cc += 8) {
+              for (int cc = c0; cc < c0 + 32; cc += 8) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(mx4[k], fmaxf(xs[cc + k], xs[cc + k + 4]));
+                for (int k = 0; k < 4; ++k)
+                  mi4[k] = cc == 0 ? max((int)sr[k], (int)sr[k + 4])
+                                   : __vimax3_s32(mi4[k], (int)sr[cc + k], (int)sr[cc + k + 4]);
+              }
+            } else {
+#pragma unroll
+              for (int cc = c0; cc < c0 + 32; cc += 8) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  mx4[k] = cc == 0 ? fmaxf(xs[k], xs[k + 4])
+                                   : fmaxf(mx4[k], fmaxf(xs[cc + k], xs[cc + k + 4]));
+              }
             }
-            mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
           }
+          const float mx = kInt && kFull ? (float)max(max(mi4[0], mi4[1]), max(mi4[2], mi4[3]))
+                                         : fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
           const float m_tile = mx == -INFINITY ? -INFINITY : mx * f;  // f > 0 keeps the argmax
           const float m_new = fmaxf(m_run, m_tile);
           const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first finite max
@@ -850,6 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float xs[64];
 #pragma unroll
           for (int cc = 0; cc < 64; ++cc) {
+            if (cc == 32) tmem_wait_ld();  // columns 32-63 are in
             const bool sel = (((cc < 32 ? selt.x : selt.y) >> (cc & 31)) & 1u) != 0u;
             xs[cc] = __uint_as_float(sr[cc]) * (sel ? fs : fc);
             if (!kFull) xs[cc] = (cc >= clo && cc < nvalid) ? xs[cc] : -INFINITY;
