@@ -725,11 +725,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
           uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
           tmem_ld32(tS, lo);
-          if (C::kHyb) tmem_wait_ld();
+          if (C::kHyb) {
+            tmem_wait_ld();
+            tmem_reg_fence(lo);
+          }
           tmem_ld32(tS + 32, hi);
-          if (!C::kHyb) tmem_wait_ld();
+          if (!C::kHyb) {
+            tmem_wait_ld();
+            tmem_reg_fence(lo);
+            tmem_reg_fence(hi);
+          }
         }
-        if (!C::kHyb && p.n_dump > 0) tmem_wait_ld();
+        uint32_t (&s_hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        if (!C::kHyb && p.n_dump > 0) {
+          tmem_wait_ld();
+          tmem_reg_fence(s_hi);
+        }
         if (!C::kHyb && p.n_dump > 0 && row_valid && (prec == TRA_PREC_INT8 || prec == TRA_PREC_INT4)) {
           for (int di = 0; di < p.n_dump; ++di) {
             const int* dc = p.dump_coords + di * 4;
@@ -777,7 +788,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float mx4[4];
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            if (hf == 1) tmem_wait_ld();  // columns 32-63 are in
+            if (hf == 1) {  // columns 32-63 are in
+              tmem_wait_ld();
+              tmem_reg_fence(s_hi);
+            }
             const int c0 = 32 * hf;
             if (kInt || is_int) {
 #pragma unroll
@@ -859,7 +873,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float xs[64];
 #pragma unroll
           for (int cc = 0; cc < 64; ++cc) {
-            if (cc == 32) tmem_wait_ld();  // columns 32-63 are in
+            if (cc == 32) {  // columns 32-63 are in
+              tmem_wait_ld();
+              tmem_reg_fence(s_hi);
+            }
             const bool sel = (((cc < 32 ? selt.x : selt.y) >> (cc & 31)) & 1u) != 0u;
             xs[cc] = __uint_as_float(sr[cc]) * (sel ? fs : fc);
             if (!kFull) xs[cc] = (cc >= clo && cc < nvalid) ? xs[cc] : -INFINITY;
@@ -943,6 +960,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t o[32];
           tmem_ld32(tO + col, o);
           tmem_wait_ld();
+          tmem_reg_fence(o);
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
           tmem_st32(tO + col, o);
@@ -969,6 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t o[32];
         tmem_ld32(tO + col, o);
         tmem_wait_ld();
+        tmem_reg_fence(o);
         if (row_valid) {
 #pragma unroll
           for (int k = 0; k < 32; k += 8) {
