@@ -11,7 +11,10 @@ usable:
   end with TRA_DEV_TIMEOUT;
 * traversal lists built for a boundary policy with an INT4 region, handed to
   the fused prefill under a policy without one (so no INT4 tiles are bound),
-  must end with TRA_DEV_BAD_LIST rather than read a missing operand.
+  must end with TRA_DEV_BAD_LIST rather than read a missing operand;
+* a list entry whose key tile lies past its work unit's last causal tile must
+  end with TRA_DEV_BAD_LIST: no copy is issued for it and no per-tile scale is
+  read at its index (the prefill's own range check, so the input cannot fault).
 """
 import math
 
@@ -74,6 +77,32 @@ def test_prefill_int4_list_without_int4_tiles_reports_bad_list():
     assert not st & tra.DEV_TIMEOUT, f"status {st:#x}: the error path itself timed out"
     # the context is intact and the kernel deterministic: the correct call again
     # reproduces the first output bit for bit
+    plan.status.zero_()
+    out2 = torch.zeros_like(q)
+    plan.attend(q, k, v, out2)
+    torch.cuda.synchronize()
+    assert int(plan.status.item()) == 0
+    assert torch.equal(out2.view(torch.int16), out_ref.view(torch.int16))
+
+
+def test_prefill_out_of_range_key_tile_reports_bad_list():
+    w, shape, q, k, v = _prefill_case()
+    pol = tra.Policy.boundary(w.b1, w.b2)
+    plan, out_ref = _good_prefill(shape, pol, q, k, v)
+    # one entry of a row gets a key tile far past every sequence (precision kept)
+    bad = plan.entries.clone()
+    e = plan.nnz // 2
+    word = int(bad[e].item()) & 0xFFFFFFFF
+    bad[e] = np.int64((word & 0xF0000000) | 0x0FFFFF00).astype(np.int32).item()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out_bad = torch.zeros_like(q)
+    L.routed_attention_prefill(shape, pol, q, k, v, plan.tiles, plan.row_ptr, bad,
+                               1.0 / math.sqrt(w.d), out_bad, None, status=status)
+    torch.cuda.synchronize()
+    st = int(status.item())
+    assert st & tra.DEV_BAD_LIST, f"status {st:#x}"
+    assert not st & tra.DEV_TIMEOUT, f"status {st:#x}: the error path itself timed out"
+    # the context is intact: the unmodified lists reproduce the first output bit for bit
     plan.status.zero_()
     out2 = torch.zeros_like(q)
     plan.attend(q, k, v, out2)

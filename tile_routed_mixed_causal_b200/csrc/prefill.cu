@@ -212,6 +212,11 @@ __device__ __forceinline__ Unit make_unit(const PrefillParams& p, long long id) 
   return x;
 }
 
+// The last key tile a unit's causal rows can list (its second q-tile's diagonal).
+// A list entry beyond it is reported as a bad list: no copy is issued for it and
+// no per-tile array is indexed with it.
+__device__ __forceinline__ int unit_kt_max(const Unit& x) { return x.qt0 + (x.has_second ? 1 : 0); }
+
 // the precisions each prefill mode's traversal rows can hold
 template <int MODE> struct MergeOf { using T = KtMerge<TRA_PREC_INT4, TRA_PREC_INT8>; };
 template <> struct MergeOf<TRA_POLICY_BITMASK> { using T = KtMerge<TRA_PREC_INT8, TRA_PREC_BF16>; };
@@ -483,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int nk = 0, nv = 0;  // fills issued so far into this unit's K and V rings
       while (c.next(kt, p0, p1)) {
         if (((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) ||
-            (!C::kHasF8 && (p0 == TRA_PREC_FP8 || p1 == TRA_PREC_FP8))) {
+            (!C::kHasF8 && (p0 == TRA_PREC_FP8 || p1 == TRA_PREC_FP8)) || kt > unit_kt_max(x)) {
           *err = TRA_DEV_BAD_LIST;
           break;
         }
@@ -579,7 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int kt, p0, p1;
         while (c.next(kt, p0, p1)) {
           if (((p0 == TRA_PREC_INT4 || p1 == TRA_PREC_INT4) && !int4) ||
-              (!C::kHasF8 && (p0 == TRA_PREC_FP8 || p1 == TRA_PREC_FP8))) {
+              (!C::kHasF8 && (p0 == TRA_PREC_FP8 || p1 == TRA_PREC_FP8)) ||
+              kt > unit_kt_max(mu ? un1 : un0)) {
             *err = TRA_DEV_BAD_LIST;
             ok = false;
             break;
@@ -661,9 +667,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int i = 0;
     auto c = unit_stream<C>(p, x);
     // the K-tile scale of this row's precision of an entry (1 for BF16), loaded one
-    // entry ahead
+    // entry ahead (an out-of-range kt, reported by the producer, reads the last
+    // in-range tile's scale instead of memory past the sequence)
+    const int kt_max = unit_kt_max(x);
     auto kscale = [&](int kt_, int pr) -> float {
-      const long long t_ = (long long)x.kvh * p.ntiles + x.toff + kt_;
+      const long long t_ = (long long)x.kvh * p.ntiles + x.toff + min(kt_, kt_max);
       if (pr == TRA_PREC_INT8) return __ldg(p.sk8 + t_);
       if (pr == TRA_PREC_INT4 && int4) return __ldg(p.sk4 + t_);
       if (C::kHyb && pr == kPrecHyb) return __ldg(p.sk4 + t_);
@@ -675,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sv = 1.0f;
       sel = make_uint2(0u, 0u);
       if (C::kHyb && pr == kPrecHyb) {
-        const long long t_ = (long long)x.kvh * p.ntiles + x.toff + kt_;
+        const long long t_ = (long long)x.kvh * p.ntiles + x.toff + min(kt_, kt_max);
         sv = __ldg(p.sv4 + t_);
         sel = __ldg(reinterpret_cast<const uint2*>(p.sel_mask) + t_);
       }
@@ -698,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tS = tU + sb * 64;
       if (!mbar_wait(bar_sfull(u, sb), (i >> 1) & 1, err)) { ok = false; break; }
       if (((pa == TRA_PREC_INT4 || pb == TRA_PREC_INT4) && !int4) ||
-          (!C::kHasF8 && (pa == TRA_PREC_FP8 || pb == TRA_PREC_FP8))) {
+          (!C::kHasF8 && (pa == TRA_PREC_FP8 || pb == TRA_PREC_FP8)) || kt > kt_max) {
         *err = TRA_DEV_BAD_LIST;
         ok = false;
         break;
