@@ -131,7 +131,7 @@ typedef enum {
 /* device status word bits */
 #define TRA_DEV_TIMEOUT 0x1      /* a bounded pipeline wait expired */
 #define TRA_DEV_TAIL_FULL 0x2    /* decode: tail_len reached tail_cap */
-#define TRA_DEV_BAD_LIST 0x4     /* prefill: an INT4 list entry but no INT4 tiles */
+#define TRA_DEV_BAD_LIST 0x4     /* prefill: a list entry whose precision has no tiles bound, or whose key tile is past its rows' last causal tile */
 
 #define TRA_MAX_HEADS 256        /* Hq limit (policies travel as launch params) */
 #define TRA_MAX_DUMP 64          /* max tiles per integer-accumulator dump */
@@ -252,7 +252,11 @@ TRA_API tra_status build_tile_lists(const tra_shape* shape, const tra_policy* po
  * int32 Q-code x K-code^T accumulators go to dump_out [n_dump][64][64]
  * (row = query within the tile, column = key; BF16 and FP8 tiles, whose
  * accumulators are fp32, are not dumped).  n_dump <= TRA_MAX_DUMP.
- * status_dev: device int32, receives TRA_DEV_* bits.
+ * status_dev: device int32, receives TRA_DEV_* bits.  row_ptr must be as
+ * build_tile_lists wrote it (entries are read over [row_ptr[r], row_ptr[r+1]));
+ * an entry the kernel cannot use (a precision with no tiles bound, a key tile past
+ * its rows' last causal tile) sets TRA_DEV_BAD_LIST, no copy is issued for it, and
+ * out is then undefined.
  */
 TRA_API tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* policy,
                                     const uint16_t* q, const uint16_t* k, const uint16_t* v,
