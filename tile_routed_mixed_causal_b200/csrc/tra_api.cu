@@ -13,10 +13,27 @@
 #include <string>
 #include <vector>
 
+#ifndef TRA_NO_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 #include "../../include/tra.h"
 #include "tra_launch.h"
 
 namespace {
+
+// A named NVTX range around an ABI call (what a profiler timeline shows for it);
+// free when no profiler is attached.  Build with -DTRA_NO_NVTX to leave it out.
+struct CallRange {
+#ifndef TRA_NO_NVTX
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+#else
+  explicit CallRange(const char*) {}
+#endif
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 thread_local std::string g_last_error;
 
@@ -211,6 +228,7 @@ size_t tra_qtiles_bytes(const tra_shape* shape, uint32_t formats) {
 
 tra_status quantize_qkv_tiles(const tra_shape* shape, const uint16_t* q, const uint16_t* k,
                               const uint16_t* v, const tra_qtiles* out, void* stream) {
+  const CallRange range("tra::quantize_qkv_tiles");
   int64_t nt = 0, ntok = 0;
   tra_status st = check_shape(shape, &nt, &ntok, nullptr);
   if (st != TRA_OK) return st;
@@ -319,6 +337,7 @@ tra_status tra_tile_lists_size(const tra_shape* shape, const tra_policy* policy,
 tra_status build_tile_lists(const tra_shape* shape, const tra_policy* policy, int32_t list_kind,
                             int32_t* row_ptr, int64_t row_ptr_len, uint32_t* entries,
                             int64_t entries_cap, void* stream) {
+  const CallRange range("tra::build_tile_lists");
   int64_t rows = 0, nnz = 0;
   tra_status st = tra_tile_lists_size(shape, policy, list_kind, &rows, &nnz);
   if (st != TRA_OK) return st;
@@ -364,6 +383,7 @@ tra_status routed_attention_prefill(const tra_shape* shape, const tra_policy* po
                                     const uint32_t* entries, float softmax_scale, uint16_t* out,
                                     float* lse, const int32_t* dump_coords, int32_t n_dump,
                                     int32_t* dump_out, int32_t* status_dev, void* stream) {
+  const CallRange range("tra::routed_attention_prefill");
   int64_t nt = 0, ntok = 0, nt_max = 0;
   tra_status st = check_shape(shape, &nt, &ntok, &nt_max);
   if (st != TRA_OK) return st;
@@ -469,6 +489,7 @@ tra_status routed_attention_decode(const tra_shape* shape, const tra_policy* pol
                                    int32_t* tail_len_dev, int32_t tail_cap, float softmax_scale,
                                    uint16_t* out, void* workspace, size_t workspace_bytes,
                                    int32_t* status_dev, void* stream) {
+  const CallRange range("tra::routed_attention_decode");
   int64_t nt = 0, ntok = 0, nt_max = 0;
   tra_status st = check_shape(shape, &nt, &ntok, &nt_max);
   if (st != TRA_OK) return st;
@@ -572,6 +593,7 @@ static tra_status check_hybrid(const tra_shape* shape, const tra_hybrid* hy, int
 tra_status hybrid_select_tokens(const tra_shape* shape, const float* importance, double frac,
                                 const uint16_t* k, const uint16_t* v, const tra_hybrid* hy,
                                 void* stream) {
+  const CallRange range("tra::hybrid_select_tokens");
   int64_t nt = 0, ntok = 0;
   tra_status st = check_shape(shape, &nt, &ntok, nullptr);
   if (st != TRA_OK) return st;
@@ -614,6 +636,7 @@ tra_status hybrid_attention_decode(const tra_shape* shape, const tra_hybrid* hy,
                                    int32_t* tail_len_dev, int32_t tail_cap, float softmax_scale,
                                    uint16_t* out, void* workspace, size_t workspace_bytes,
                                    int32_t* status_dev, void* stream) {
+  const CallRange range("tra::hybrid_attention_decode");
   int64_t nt = 0, ntok = 0, nt_max = 0;
   tra_status st = check_shape(shape, &nt, &ntok, &nt_max);
   if (st != TRA_OK) return st;
@@ -687,6 +710,7 @@ tra_status hybrid_attention_prefill(const tra_shape* shape, const tra_hybrid* hy
                                     const uint16_t* k, const uint16_t* v, const tra_qtiles* kv,
                                     uint16_t* k_mix, uint16_t* v_mix, float softmax_scale,
                                     uint16_t* out, float* lse, int32_t* status_dev, void* stream) {
+  const CallRange range("tra::hybrid_attention_prefill");
   int64_t nt = 0, ntok = 0, nt_max = 0;
   tra_status st = check_shape(shape, &nt, &ntok, &nt_max);
   if (st != TRA_OK) return st;
